@@ -1,0 +1,158 @@
+/*
+ * qsa_oracle.c -- FP64 CPU oracle for QSA top-K sparse-attention prefill.
+ *
+ * TEST INFRASTRUCTURE ONLY (see qsa_oracle.h).  Written directly from the
+ * definition on page "Qwen4-Exp QSA llega al Ascend de Huawei", section
+ * "Lo que realmente añade la pull request": attention restricted to the
+ * cache rows named by the token's selected-slot list, softmax with the model's
+ * D256 scale.  Nothing here is blocked, fused or reordered beyond the plain
+ * definition; threads only split the independent query tokens.
+ */
+#include "qsa_oracle.h"
+
+#include <math.h>
+#include <pthread.h>
+#include <stdlib.h>
+#include <string.h>
+
+double qsa_oracle_bf16_to_double(uint16_t bits) {
+  /* BF16 is the top half of an IEEE binary32; the widening is exact. */
+  uint32_t w = ((uint32_t)bits) << 16;
+  float f;
+  memcpy(&f, &w, sizeof f);
+  return (double)f;
+}
+
+typedef struct {
+  const qsa_oracle_args* a;
+  const int64_t* tokens;
+  int64_t n_tokens;
+  double* out;
+  double* lse;
+  int64_t next;      /* shared work counter */
+  int64_t oob;       /* out-of-range entries seen */
+  int error;
+} job_t;
+
+/* One (token, query head) row, following the definition step by step. */
+static int64_t one_row(const qsa_oracle_args* a, int64_t t, int64_t h,
+                       double* out_row, double* lse_out, int64_t* sel,
+                       double* s) {
+  const int64_t D = a->head_dim;
+  const int64_t G = a->num_q_heads / a->num_kv_heads;
+  const int64_t g = h / G; /* contiguous GQA grouping */
+  const double scale = a->scale > 0.0 ? a->scale : 1.0 / sqrt((double)D);
+  int64_t oob = 0;
+
+  /* Step 1: the selected entries J.  n_valid and negative ids both mask. */
+  int64_t n_list = a->topk;
+  if (a->n_valid) {
+    int64_t nv = a->n_valid[t * a->num_kv_heads + g];
+    if (nv < n_list) n_list = nv;
+    if (n_list < 0) n_list = 0;
+  }
+  const int32_t* list = a->idx + t * a->idx_stride_tok + g * a->idx_stride_head;
+  int64_t n = 0;
+  for (int64_t j = 0; j < n_list; ++j) {
+    int64_t slot = list[j];
+    if (slot < 0) continue;
+    if (slot >= a->num_slots) {
+      if (h % G == 0) ++oob; /* count each list entry once, not per head */
+      continue;
+    }
+    sel[n++] = slot;
+  }
+
+  /* Empty selection: zero output, lse = -inf. */
+  if (n == 0) {
+    for (int64_t d = 0; d < D; ++d) out_row[d] = 0.0;
+    *lse_out = -INFINITY;
+    return oob;
+  }
+
+  /* Step 2: scores s_j = scale * <q, k_j>. */
+  const uint16_t* q = a->q + t * a->q_stride_tok + h * a->q_stride_head;
+  for (int64_t j = 0; j < n; ++j) {
+    const uint16_t* kr = a->k + sel[j] * a->kv_stride_slot + g * a->kv_stride_head;
+    double dot = 0.0;
+    for (int64_t d = 0; d < D; ++d)
+      dot += qsa_oracle_bf16_to_double(q[d]) * qsa_oracle_bf16_to_double(kr[d]);
+    s[j] = scale * dot;
+  }
+
+  /* Step 3: softmax with the maximum subtracted (exact in real arithmetic). */
+  double m = s[0];
+  for (int64_t j = 1; j < n; ++j) if (s[j] > m) m = s[j];
+  double l = 0.0;
+  for (int64_t j = 0; j < n; ++j) { s[j] = exp(s[j] - m); l += s[j]; }
+
+  /* Step 4: weighted sum of the selected V rows, normalised by l. */
+  for (int64_t d = 0; d < D; ++d) out_row[d] = 0.0;
+  for (int64_t j = 0; j < n; ++j) {
+    const uint16_t* vr = a->v + sel[j] * a->kv_stride_slot + g * a->kv_stride_head;
+    const double p = s[j];
+    for (int64_t d = 0; d < D; ++d) out_row[d] += p * qsa_oracle_bf16_to_double(vr[d]);
+  }
+  for (int64_t d = 0; d < D; ++d) out_row[d] /= l;
+  *lse_out = m + log(l);
+  return oob;
+}
+
+static void* worker(void* arg) {
+  job_t* job = (job_t*)arg;
+  const qsa_oracle_args* a = job->a;
+  const int64_t Hq = a->num_q_heads, D = a->head_dim;
+  const int64_t cap = a->topk > 0 ? a->topk : 1;
+  int64_t* sel = (int64_t*)malloc((size_t)cap * sizeof(int64_t));
+  double* s = (double*)malloc((size_t)cap * sizeof(double));
+  if (!sel || !s) {
+    free(sel); free(s);
+    __atomic_store_n(&job->error, 1, __ATOMIC_RELAXED);
+    return NULL;
+  }
+  int64_t oob = 0;
+  for (;;) {
+    int64_t i = __atomic_fetch_add(&job->next, 1, __ATOMIC_RELAXED);
+    if (i >= job->n_tokens) break;
+    const int64_t t = job->tokens[i];
+    for (int64_t h = 0; h < Hq; ++h)
+      oob += one_row(a, t, h, job->out + (i * Hq + h) * D, job->lse + i * Hq + h, sel, s);
+  }
+  __atomic_fetch_add(&job->oob, oob, __ATOMIC_RELAXED);
+  free(sel); free(s);
+  return NULL;
+}
+
+int64_t qsa_oracle_fwd(const qsa_oracle_args* a, const int64_t* tokens,
+                       int64_t n_tokens, int n_threads, double* out,
+                       double* lse) {
+  if (!a || n_tokens < 0 || (n_tokens > 0 && (!tokens || !out || !lse))) return -1;
+  if (a->num_kv_heads <= 0 || a->num_q_heads <= 0 || a->head_dim <= 0 ||
+      a->num_q_heads % a->num_kv_heads != 0 || a->topk < 0 || a->num_slots < 0)
+    return -1;
+  if (n_tokens > 0 && (!a->q || (a->topk > 0 && (!a->idx || !a->k || !a->v)))) return -1;
+  for (int64_t i = 0; i < n_tokens; ++i)
+    if (tokens[i] < 0 || tokens[i] >= a->num_tokens) return -1;
+
+  job_t job;
+  memset(&job, 0, sizeof job);
+  job.a = a; job.tokens = tokens; job.n_tokens = n_tokens; job.out = out; job.lse = lse;
+
+  if (n_threads <= 1 || n_tokens <= 1) {
+    worker(&job);
+  } else {
+    if (n_threads > n_tokens) n_threads = (int)n_tokens;
+    pthread_t* th = (pthread_t*)malloc((size_t)n_threads * sizeof(pthread_t));
+    if (!th) return -1;
+    int started = 0;
+    for (int i = 0; i < n_threads; ++i) {
+      if (pthread_create(&th[i], NULL, worker, &job) != 0) break;
+      ++started;
+    }
+    if (started == 0) worker(&job);
+    for (int i = 0; i < started; ++i) pthread_join(th[i], NULL);
+    free(th);
+  }
+  if (job.error) return -1;
+  return job.oob;
+}

@@ -1,0 +1,241 @@
+"""Checks that pin the FP64 oracle to facts other than itself.
+
+Each check takes an oracle handle (``oracle.Oracle``) so that the same checks
+also run against copies of the oracle with a planted mistake, which must fail
+at least one of them (tests/test_oracle_mutants.py).
+
+Pins (what the pages and the mathematics fix):
+* dense_causal  -- when a list holds every causal slot 0..t, sparse attention
+  is dense causal attention: torch's scaled_dot_product_attention and
+  logsumexp in float64 (library routines) must agree.
+* packing       -- the layout identity of page "Qwen4-Exp QSA llega al Ascend
+  de Huawei", section "Lo que realmente añade la pull request":
+  softmax(scale [Q,0][K,V]^T)[K,V] = [P K, P V] with the D256 scale.
+* permutation   -- the result does not depend on list order or interleaved
+  -1 padding (same page, "Nueve pruebas": unordered physical slots).
+* head_padding  -- padding the group with extra query heads (12->16, 6->8,
+  3->4; same page, "Formas de cabeza") leaves the real heads unchanged.
+* closed_forms  -- zero queries give the mean of the selected V rows with
+  lse = ln n; one entry gives that V row with lse = its score; an empty row
+  gives exact zeros with lse = -inf ("Límites de tamaño"); duplicates count
+  twice; out-of-range slots are reported and ignored.
+* brute_force   -- an independent numpy evaluation without the max trick.
+* worked_example -- the hand-derived fixture in tests/golden.
+"""
+from __future__ import annotations
+
+import json
+import math
+import os
+
+import numpy as np
+import torch
+
+from top_sparse_attention_qsa_b200 import workloads as W
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+TOL = dict(rtol=1e-12, atol=1e-12)
+
+
+def _np64(x):
+    return x.to(torch.float64).numpy()
+
+
+def _expand_kv(x, G):
+    # [S, Hkv, D] -> [Hq, S, D] with head h reading KV head h // G
+    return x.to(torch.float64).permute(1, 0, 2).repeat_interleave(G, dim=0)
+
+
+def check_bf16_widening(orc):
+    bits = torch.arange(0, 1 << 16, dtype=torch.int32)
+    keep = ((bits >> 7) & 0xFF) != 0xFF                   # drop inf/nan exponents
+    bits = bits[keep][::37]
+    want = bits.to(torch.int16).view(torch.bfloat16).to(torch.float64).numpy()
+    got = np.array([orc.bf16_to_double(int(b) & 0xFFFF) for b in bits.tolist()])
+    np.testing.assert_array_equal(got, want)
+
+
+def check_dense_causal(orc, shapes=((3, 1), (6, 1), (12, 1), (16, 2), (24, 2)), T=24, seed=11):
+    for i, (Hq, Hkv) in enumerate(shapes):
+        G = Hq // Hkv
+        gen = torch.Generator().manual_seed(seed + i)
+        D = W.HEAD_DIM
+        q = W.normal_bf16((T, Hq, D), gen, "cpu")
+        k = W.normal_bf16((T, Hkv, D), gen, "cpu", std=2.0)
+        v = W.normal_bf16((T, Hkv, D), gen, "cpu")
+        K = T + 5
+        idx = torch.full((T, Hkv, K), -1, dtype=torch.int32)
+        for t in range(T):
+            for g in range(Hkv):
+                perm = torch.randperm(t + 1, generator=gen).to(torch.int32)
+                slots = torch.randperm(K, generator=gen)[: t + 1]
+                idx[t, g, slots] = perm          # every causal slot, scattered
+        for scale in (0.0, 0.037):
+            out, lse, oob = orc.sparse_prefill(q, k, v, idx, None, scale)
+            assert oob == 0
+            sc = scale if scale > 0 else 1.0 / math.sqrt(D)
+            qd = q.to(torch.float64).permute(1, 0, 2)[None]          # [1,Hq,T,D]
+            kd = _expand_kv(k, G)[None]
+            vd = _expand_kv(v, G)[None]
+            ref = torch.nn.functional.scaled_dot_product_attention(qd, kd, vd, is_causal=True, scale=sc)
+            ref = ref[0].permute(1, 0, 2).numpy()
+            scores = (qd @ kd.transpose(-1, -2)) * sc
+            mask = torch.ones(T, T, dtype=torch.bool).tril()
+            scores = scores.masked_fill(~mask, float("-inf"))
+            ref_lse = torch.logsumexp(scores, dim=-1)[0].permute(1, 0).numpy()
+            np.testing.assert_allclose(out, ref, **TOL)
+            np.testing.assert_allclose(lse, ref_lse, **TOL)
+
+
+def _small_case(Hq, Hkv, T=6, S=40, K=9, seed=3):
+    return W.generic_case(T, S, Hq, Hkv, K, seed)
+
+
+def check_packing(orc, shapes=((3, 1), (16, 2))):
+    for Hq, Hkv in shapes:
+        w = _small_case(Hq, Hkv)
+        scale = 1.0 / 16                      # the original D256 scale is kept
+        C = torch.cat([w.k_cache, w.v_cache], dim=-1)          # [S, Hkv, 512]
+        Qp = torch.cat([w.q, torch.zeros_like(w.q)], dim=-1)   # [T, Hq, 512]
+        packed, lse_p, _ = orc.sparse_prefill(Qp, C, C, w.topk_idx, None, scale)
+        pv, lse, _ = orc.sparse_prefill(w.q, w.k_cache, w.v_cache, w.topk_idx, None, scale)
+        pk, _, _ = orc.sparse_prefill(w.q, w.k_cache, w.k_cache, w.topk_idx, None, scale)
+        np.testing.assert_allclose(packed[..., 256:], pv, **TOL)
+        np.testing.assert_allclose(packed[..., :256], pk, **TOL)
+        np.testing.assert_allclose(lse_p, lse, **TOL)
+
+
+def check_permutation(orc, shapes=((6, 1), (24, 2))):
+    for j, (Hq, Hkv) in enumerate(shapes):
+        w = _small_case(Hq, Hkv, K=13, seed=5 + j)
+        gen = torch.Generator().manual_seed(99 + j)
+        T, _, K = w.topk_idx.shape
+        K2 = K + 7
+        idx2 = torch.full((T, Hkv, K2), -1, dtype=torch.int32)
+        for t in range(T):
+            for g in range(Hkv):
+                pos = torch.randperm(K2, generator=gen)[:K]
+                idx2[t, g, pos] = w.topk_idx[t, g, torch.randperm(K, generator=gen)]
+        a = orc.sparse_prefill(w.q, w.k_cache, w.v_cache, w.topk_idx)
+        b = orc.sparse_prefill(w.q, w.k_cache, w.v_cache, idx2)
+        np.testing.assert_allclose(b[0], a[0], **TOL)
+        np.testing.assert_allclose(b[1], a[1], **TOL)
+        # n_valid masks the tail exactly like -1 does, whatever the tail holds
+        nv = torch.randint(0, K + 1, (T, Hkv), generator=gen, dtype=torch.int32)
+        ar = torch.arange(K)[None, None, :]
+        masked = torch.where(ar < nv[:, :, None], w.topk_idx, torch.full_like(w.topk_idx, -1))
+        c = orc.sparse_prefill(w.q, w.k_cache, w.v_cache, w.topk_idx, nv)
+        d = orc.sparse_prefill(w.q, w.k_cache, w.v_cache, masked)
+        np.testing.assert_array_equal(c[0], d[0])
+        np.testing.assert_array_equal(c[1], d[1])
+
+
+def check_head_padding(orc, pad=((12, 1, 16), (6, 1, 8), (3, 1, 4), (24, 2, 16))):
+    for Hq, Hkv, Gp in pad:
+        w = _small_case(Hq, Hkv, seed=17)
+        G = Hq // Hkv
+        T, _, D = w.q.shape
+        gen = torch.Generator().manual_seed(5)
+        qp = W.normal_bf16((T, Hkv * Gp, D), gen, "cpu", std=3.0)   # garbage heads
+        real = [g * Gp + r for g in range(Hkv) for r in range(G)]
+        qp[:, real] = w.q
+        a = orc.sparse_prefill(w.q, w.k_cache, w.v_cache, w.topk_idx)
+        b = orc.sparse_prefill(qp, w.k_cache, w.v_cache, w.topk_idx)
+        np.testing.assert_allclose(b[0][:, real], a[0], **TOL)
+        np.testing.assert_allclose(b[1][:, real], a[1], **TOL)
+
+
+def check_closed_forms(orc):
+    D = W.HEAD_DIM
+    w = _small_case(12, 1, T=5, S=30, K=7, seed=23)
+    S = 30
+    # zero queries: uniform weights -> mean of the selected rows, lse = ln n
+    q0 = torch.zeros_like(w.q)
+    nv = torch.tensor([[7], [3], [1], [5], [2]], dtype=torch.int32)
+    out, lse, _ = orc.sparse_prefill(q0, w.k_cache, w.v_cache, w.topk_idx, nv)
+    vd = _np64(w.v_cache)
+    for t in range(5):
+        n = int(nv[t, 0])
+        rows = w.topk_idx[t, 0, :n].long().numpy()
+        mean = vd[rows, 0, :].mean(axis=0)
+        for h in range(12):
+            np.testing.assert_allclose(out[t, h], mean, **TOL)
+            np.testing.assert_allclose(lse[t, h], math.log(n), **TOL)
+    # one entry: that V row exactly, lse = scale * q.k
+    one = w.topk_idx[:, :, :1].contiguous()
+    out, lse, _ = orc.sparse_prefill(w.q, w.k_cache, w.v_cache, one)
+    qd, kd = _np64(w.q), _np64(w.k_cache)
+    for t in range(5):
+        s = int(one[t, 0, 0])
+        np.testing.assert_array_equal(out[t], np.broadcast_to(vd[s, 0], (12, D)))
+        np.testing.assert_allclose(lse[t], (qd[t] @ kd[s, 0]) / 16.0, **TOL)
+    # duplicates: [a, a] -> v_a, lse = s_a + ln 2
+    dup = torch.cat([one, one], dim=2)
+    out2, lse2, _ = orc.sparse_prefill(w.q, w.k_cache, w.v_cache, dup)
+    np.testing.assert_allclose(out2, out, **TOL)
+    np.testing.assert_allclose(lse2, lse + math.log(2.0), **TOL)
+    # empty rows (all -1, n_valid = 0, K = 0): exact +0.0 and -inf
+    empty = torch.full((5, 1, 4), -1, dtype=torch.int32)
+    for args in ((empty, None), (w.topk_idx, torch.zeros((5, 1), dtype=torch.int32)),
+                 (torch.empty((5, 1, 0), dtype=torch.int32), None)):
+        out, lse, _ = orc.sparse_prefill(w.q, w.k_cache, w.v_cache, *args)
+        assert np.all(out == 0.0) and not np.any(np.signbit(out))
+        assert np.all(np.isneginf(lse))
+    # an out-of-range slot is reported and ignored
+    bad = w.topk_idx.clone()
+    bad[:, :, 0] = S + 3
+    out_b, lse_b, oob = orc.sparse_prefill(w.q, w.k_cache, w.v_cache, bad)
+    assert oob == 5
+    out_r, lse_r, _ = orc.sparse_prefill(w.q, w.k_cache, w.v_cache, w.topk_idx[:, :, 1:].contiguous())
+    np.testing.assert_allclose(out_b, out_r, **TOL)
+    np.testing.assert_allclose(lse_b, lse_r, **TOL)
+
+
+def check_brute_force(orc, shapes=((3, 1), (16, 2))):
+    for Hq, Hkv in shapes:
+        w = _small_case(Hq, Hkv, T=7, S=50, K=11, seed=31)
+        G = Hq // Hkv
+        qd, kd, vd = _np64(w.q), _np64(w.k_cache), _np64(w.v_cache)
+        idx = w.topk_idx.numpy()
+        ref = np.zeros(qd.shape)
+        ref_lse = np.zeros(qd.shape[:2])
+        for t in range(qd.shape[0]):
+            for h in range(Hq):
+                rows = idx[t, h // G]
+                e = np.exp(np.array([qd[t, h] @ kd[r, h // G] for r in rows]) / 16.0)
+                ref[t, h] = (e[:, None] * vd[rows, h // G]).sum(0) / e.sum()
+                ref_lse[t, h] = np.log(e.sum())
+        out, lse, _ = orc.sparse_prefill(w.q, w.k_cache, w.v_cache, w.topk_idx)
+        np.testing.assert_allclose(out, ref, rtol=1e-11, atol=1e-12)
+        np.testing.assert_allclose(lse, ref_lse, rtol=1e-11, atol=1e-12)
+
+
+def check_worked_example(orc):
+    with open(os.path.join(GOLDEN, "worked_example_three_keys.json")) as f:
+        ex = json.load(f)
+    D, S = ex["head_dim"], ex["num_slots"]
+    q = torch.zeros((1, 1, D))
+    for d, x in ex["q_nonzero"].items():
+        q[0, 0, int(d)] = x
+    k = torch.full((S, 1, D), ex["filler_value"])
+    v = torch.full((S, 1, D), ex["filler_value"])
+    for s, row in ex["k_rows"].items():
+        k[int(s), 0] = 0
+        for d, x in row.items():
+            k[int(s), 0, int(d)] = x
+    for s, row in ex["v_rows"].items():
+        v[int(s), 0] = 0
+        for d, x in row.items():
+            v[int(s), 0, int(d)] = x
+    idx = torch.tensor(ex["list"], dtype=torch.int32).view(1, 1, -1)
+    out, lse, _ = orc.sparse_prefill(q.to(torch.bfloat16), k.to(torch.bfloat16),
+                                     v.to(torch.bfloat16), idx, None, ex["scale"])
+    want = np.zeros(D)
+    for d, x in ex["expected_out_nonzero"].items():
+        want[int(d)] = float(x)
+    np.testing.assert_allclose(out[0, 0], want, rtol=1e-14, atol=1e-15)
+    np.testing.assert_allclose(lse[0, 0], float(ex["expected_lse"]), rtol=1e-14)
+
+
+ALL_CHECKS = [check_bf16_widening, check_dense_causal, check_packing, check_permutation,
+              check_head_padding, check_closed_forms, check_brute_force, check_worked_example]
