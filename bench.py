@@ -1,0 +1,457 @@
+#!/usr/bin/env python
+"""QSA sparse-attention prefill benchmark (one JSON line on rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload c5] [--impl cuda|reference]
+
+A step is one pass of the whole hot path -- index load/mask, KV gather,
+scores, online softmax, PV, epilogue: one launch of the sparse-prefill
+kernel -- over one batch of synthetic input already resident in HBM.  The
+default workload is the chunked long prefill: 8192 new query tokens at
+positions 122880..131071 over a 131072-slot cache, heads (24,2), D=256,
+top-K=2048 (256 local + 1792 random earlier slots, unsorted).
+
+value  = query tokens/s over all ranks (each rank runs its own replica; the
+         path has no exchange step, so scaling is weak).
+e2e    = the same metric through the host-buffer C-ABI entry point: every
+         step copies Q, both caches, the lists and n_valid host->device and
+         the output and lse device->host inside the timed region.
+roofline: algorithmic bytes per launch (1024 B of K+V rows and 4 B of list
+         entry per live entry, plus Q and out rows and the lse) over the
+         kernel's mean event-timed duration, against the measured HBM copy
+         bandwidth.
+cpu_baseline: the FP64 oracle on a bounded token sample (rank 0, N=1).
+--impl reference: times only the FP64 oracle (the CPU reference arm).
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import glob
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+METRIC = "QSA sparse prefill query-tokens/s and gathered-KV GB/s (% of B200 roofline)"
+UNIT = "tokens/s"
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["cuda", "reference"], default="cuda")
+    ap.add_argument("--workload", default="c5",
+                    choices=["tiny", "c2", "c3", "c4", "c5", "pages_long"])
+    ap.add_argument("--secondary", default="c4",
+                    help="second workload reported under 'secondary' ('' to skip)")
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=12.0,
+                    help="seconds of oracle work for the cpu_baseline sample")
+    ap.add_argument("--profile", action="store_true",
+                    help="minimal run for ncu: no clocks, e2e, cpu baseline or secondary")
+    return ap.parse_args()
+
+
+# ---------------------------------------------------------------- helpers
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, "fallback"
+
+
+def workload_accounting(w):
+    """Live list entries and the algorithmic bytes / FLOPs of one launch."""
+    s = w.shape
+    idx = w.topk_idx
+    live = (idx >= 0) & (idx < s["S"])
+    if w.n_valid is not None:
+        ar = torch.arange(s["K"], device=idx.device)
+        live &= ar[None, None, :] < w.n_valid[:, :, None]
+    entries = int(live.sum().item())
+    G = s["Hq"] // s["Hkv"]
+    gathered = entries * 2 * s["D"] * 2
+    algo = gathered + entries * 4 + s["T"] * s["Hq"] * s["D"] * 2 * 2 + s["T"] * s["Hq"] * 4
+    flops = entries * 4 * G * s["D"]
+    return dict(entries=entries, gathered_bytes=gathered, algo_bytes=algo, flops=flops)
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    pkg = os.path.join(ROOT, "top_sparse_attention_qsa_b200", "csrc")
+    for p in sorted(glob.glob(os.path.join(pkg, "*.cu")) + glob.glob(os.path.join(pkg, "*.cuh"))):
+        with open(p, "rb") as f:
+            h.update(os.path.basename(p).encode())
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload, units):
+    """DRAM bytes per launch from a committed ncu summary, when it was taken
+    on the current kernel sources (else None).  The summary records
+    dram bytes for a capture of `units_captured` (token, KV head) units;
+    the figure is scaled to `units` when the summary says it scales."""
+    path = os.path.join(ROOT, "profiles", f"traffic_{workload}.txt")
+    if not os.path.exists(path):
+        return None
+    kv = {}
+    with open(path) as f:
+        for line in f:
+            if ":" in line and not line.startswith("#"):
+                k, v = line.split(":", 1)
+                kv[k.strip()] = v.strip()
+    if kv.get("kernel_source_sha256_16") != kernel_source_hash():
+        return None
+    try:
+        b = float(kv["dram_bytes_per_launch"])
+        cap = float(kv.get("units_captured", units))
+    except (KeyError, ValueError):
+        return None
+    return b * units / cap
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 100 ms."""
+
+    FIELDS = ["timestamp", "index", "clocks.sm", "clocks.max.sm", "power.draw",
+              "clocks_event_reasons.active", "clocks_event_reasons.hw_slowdown",
+              "clocks_event_reasons.hw_thermal_slowdown",
+              "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
+
+    def __init__(self, device_index):
+        self.proc = None
+        self.path = None
+        try:
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            sel = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+        except Exception:
+            sel = str(device_index)
+        self.sel = sel
+
+    def start(self):
+        try:
+            os.makedirs(os.path.join(ROOT, "gpurun_out"), exist_ok=True)
+            self.path = os.path.join(ROOT, "gpurun_out", f"clocks_{os.getpid()}.csv")
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.sel, "--query-gpu=" + ",".join(self.FIELDS),
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.fh, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self, t0, t1):
+        if self.proc is None:
+            return {"unavailable": "nvidia-smi could not be started"}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.fh.close()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) != len(self.FIELDS):
+                    continue
+                try:
+                    ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                except ValueError:
+                    continue
+                rows.append((ts, parts))
+        inside = [p for ts, p in rows if t0 - 0.05 <= ts <= t1 + 0.15]
+        if not inside:
+            inside = [p for _, p in rows[-3:]]
+        if not inside:
+            return {"unavailable": "no nvidia-smi samples"}
+        sm = [float(p[2]) for p in inside if p[2].replace(".", "").isdigit()]
+        reasons = []
+        for name, col in (("hw_slowdown", 6), ("hw_thermal_slowdown", 7),
+                          ("sw_thermal_slowdown", 8), ("sw_power_cap", 9)):
+            if any(p[col] == "Active" for p in inside):
+                reasons.append(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": float(inside[0][3]) if inside[0][3].replace(".", "").isdigit() else None,
+                "reasons": reasons, "samples": len(inside)}
+
+
+def time_launches(fn, steps, warmup, barrier):
+    for _ in range(warmup):
+        fn()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    barrier()
+    torch.cuda.synchronize()
+    t0 = time.time()
+    for i in range(steps):
+        starts[i].record()
+        fn()
+        ends[i].record()
+    torch.cuda.synchronize()
+    t1 = time.time()
+    barrier()
+    per = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    total = starts[0].elapsed_time(ends[-1])
+    return total, per, (t0, t1)
+
+
+def time_oracle(w, budget_s, min_tokens=1):
+    """FP64 oracle over a bounded sample of the workload's tokens (host copies)."""
+    import numpy as np
+
+    import oracle
+    q, k, v = w.q.cpu(), w.k_cache.cpu(), w.v_cache.cpu()
+    idx = w.topk_idx.cpu()
+    nv = w.n_valid.cpu() if w.n_valid is not None else None
+    T = q.shape[0]
+    cores = os.cpu_count() or 1
+    rng = np.random.default_rng(0)
+    probe = np.sort(rng.choice(T, size=min(T, max(cores, min_tokens)), replace=False))
+    t = time.perf_counter()
+    oracle.sparse_prefill(q, k, v, idx, nv, w.scale, tokens=probe, n_threads=cores)
+    dt = time.perf_counter() - t
+    per_tok = dt / len(probe)
+    n = int(min(T, max(len(probe), budget_s / max(per_tok, 1e-9))))
+    sample = np.sort(rng.choice(T, size=n, replace=False))
+    t = time.perf_counter()
+    oracle.sparse_prefill(q, k, v, idx, nv, w.scale, tokens=sample, n_threads=cores)
+    dt = time.perf_counter() - t
+    return dict(value=n / dt, unit=UNIT, cores=cores, kind="oracle",
+                sample=f"{n} of {T} query tokens (all heads), uniform without replacement, seed 0; "
+                       f"{dt:.1f} s on {cores} threads")
+
+
+def make_workload(name, device):
+    from top_sparse_attention_qsa_b200 import workloads as W
+    return W.make(name, device=device)
+
+
+def config_of(w, acct):
+    s = w.shape
+    return {"workload": w.name, "desc": w.description, "T": s["T"], "S": s["S"],
+            "heads": [s["Hq"], s["Hkv"]], "head_dim": s["D"], "topk": s["K"],
+            "live_entries": acct["entries"],
+            "l2": "inputs exceed L2 (126 MB): %.0f MB resident per rank" % (
+                (w.q.numel() * 2 + w.k_cache.numel() * 4 + w.topk_idx.numel() * 4) / 1e6)}
+
+
+# ---------------------------------------------------------------- arms
+
+def run_reference(args):
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    w = make_workload(args.workload, dev)
+    acct = workload_accounting(w)
+    import numpy as np
+
+    import oracle
+    q, k, v = w.q.cpu(), w.k_cache.cpu(), w.v_cache.cpu()
+    idx = w.topk_idx.cpu()
+    nv = w.n_valid.cpu() if w.n_valid is not None else None
+    T = q.shape[0]
+    cores = os.cpu_count() or 1
+    rng = np.random.default_rng(1)
+    # calibrate the per-step sample so the whole run stays within ~2 minutes
+    probe = np.sort(rng.choice(T, size=min(T, cores), replace=False))
+    t = time.perf_counter()
+    oracle.sparse_prefill(q, k, v, idx, nv, w.scale, tokens=probe, n_threads=cores)
+    per_tok = (time.perf_counter() - t) / len(probe)
+    step_budget = 120.0 / max(1, args.steps + args.warmup)
+    n = int(min(T, max(len(probe), cores * max(1, int(step_budget / max(per_tok * cores, 1e-9))))))
+    times = []
+    for i in range(args.warmup + args.steps):
+        sample = np.sort(rng.choice(T, size=n, replace=False))
+        t = time.perf_counter()
+        oracle.sparse_prefill(q, k, v, idx, nv, w.scale, tokens=sample, n_threads=cores)
+        if i >= args.warmup:
+            times.append(time.perf_counter() - t)
+    total = sum(times)
+    value = n * len(times) / total
+    sample_desc = f"{n} of {T} query tokens per step (all heads), uniform without replacement"
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / len(times),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": config_of(w, acct), "impl": "reference",
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "sample": sample_desc},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_cuda(args):
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", device_id=dev, timeout=datetime.timedelta(seconds=120))
+        pg = dist
+
+    def barrier():
+        if pg is not None:
+            pg.barrier()
+
+    def max_over_ranks(x):
+        if pg is None:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        return float(t.item())
+
+    from top_sparse_attention_qsa_b200 import _capi
+    from top_sparse_attention_qsa_b200 import workloads as W
+
+    seed_off = 1000 * rank
+    w = W.make(args.workload, device=dev, seed=W.CONFIG_SEED_BASE + {"tiny": 1, "c2": 2, "c3": 3, "c4": 4,
+                                                                       "c5": 5, "pages_long": 6}[args.workload] + seed_off)
+    acct = workload_accounting(w)
+    out = torch.empty_like(w.q)
+    lse = torch.empty(w.q.shape[:2], dtype=torch.float32, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+
+    def step():
+        _capi.sparse_prefill_fwd(w.q, w.k_cache, w.v_cache, w.topk_idx, w.n_valid, w.scale,
+                                 out=out, lse=lse, status=status)
+
+    sampler = None
+    if not args.profile:
+        sampler = ClockSampler(local)
+        sampler.start()
+        time.sleep(0.3)
+    total_ms, per_ms, (t0, t1) = time_launches(step, args.steps, args.warmup, barrier)
+    clocks = sampler.stop(t0, t1) if sampler is not None else None
+    total_ms = max_over_ranks(total_ms)
+    T = w.shape["T"]
+    value = T * args.steps * world / (total_ms / 1e3)
+    mean_launch_ms = statistics.mean(per_ms)
+    hbm, bf16, peak_src = measured_peaks()
+    achieved = acct["algo_bytes"] / (mean_launch_ms / 1e3) / 1e9
+    units = T * w.shape["Hkv"]
+    traffic = profiled_traffic(args.workload, units)
+    roof = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+            "frac": achieved / hbm, "traffic": traffic,
+            "peak_source": peak_src + " (hbm_gbs, STREAM-style copy)",
+            "kernel": "qsa_prefill_mma_kernel", "algo_bytes_per_launch": acct["algo_bytes"],
+            "mean_launch_ms": mean_launch_ms}
+    gathered_gbs = acct["gathered_bytes"] / (mean_launch_ms / 1e3) / 1e9
+    tflops = acct["flops"] / (mean_launch_ms / 1e3) / 1e12
+    roof_time_ms = 1e3 * max(acct["gathered_bytes"] / (hbm * 1e9), acct["flops"] / (bf16 * 1e12))
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": config_of(w, acct), "gpu_launches": args.steps,
+            "gathered_kv_gbs": gathered_gbs, "effective_tflops": tflops,
+            "roofline_time_ms": roof_time_ms, "frac_of_roofline_time": roof_time_ms / mean_launch_ms,
+            "roofline": roof, "clocks": clocks}
+    if int(status.item()) != 0:
+        line["status_word"] = int(status.item())
+
+    if not args.no_e2e and not args.profile:
+        line["e2e"] = run_e2e(w, args, barrier, max_over_ranks, world, dev)
+    if args.secondary and not args.profile and args.secondary != args.workload:
+        line["secondary"] = run_secondary(args.secondary, dev, barrier, max_over_ranks, world, hbm, bf16)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.profile:
+        line["cpu_baseline"] = time_oracle(w, args.cpu_budget)
+    elif not args.profile:
+        line["cpu_baseline"] = None
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if pg is not None:
+        pg.barrier()
+        pg.destroy_process_group()
+    return 0
+
+
+def run_e2e(w, args, barrier, max_over_ranks, world, dev):
+    from top_sparse_attention_qsa_b200 import _capi
+    hq = w.q.cpu().pin_memory()
+    hk = w.k_cache.cpu().pin_memory()
+    hv = w.v_cache.cpu().pin_memory()
+    hi = w.topk_idx.cpu().pin_memory()
+    hn = w.n_valid.cpu().pin_memory() if w.n_valid is not None else None
+    ho = torch.empty(w.q.shape, dtype=torch.bfloat16).pin_memory()
+    hl = torch.empty(w.q.shape[:2], dtype=torch.float32).pin_memory()
+    bufs = dict(q=torch.empty_like(w.q), k_cache=torch.empty_like(w.k_cache),
+                v_cache=torch.empty_like(w.v_cache), topk_idx=torch.empty_like(w.topk_idx),
+                n_valid=torch.empty_like(w.n_valid) if hn is not None else None,
+                out=torch.empty_like(w.q), lse=torch.empty(w.q.shape[:2], device=dev),
+                status=torch.zeros(1, dtype=torch.int32, device=dev))
+
+    def step():
+        _capi.sparse_prefill_fwd_host(hq, hk, hv, hi, hn, w.scale, ho, hl, bufs)
+
+    steps = max(1, args.e2e_steps)
+    total_ms, _, _ = time_launches(step, steps, 2, barrier)
+    total_ms = max_over_ranks(total_ms)
+    h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv, hi) + ((hn,) if hn is not None else ()))
+    d2h = ho.numel() * 2 + hl.numel() * 4
+    T = w.shape["T"]
+    return {"value": T * steps * world / (total_ms / 1e3), "unit": UNIT,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "ms_per_step": total_ms / steps, "steps": steps,
+            "api": "qsa_sparse_prefill_fwd_host (pinned host buffers)"}
+
+
+def run_secondary(name, dev, barrier, max_over_ranks, world, hbm, bf16):
+    from top_sparse_attention_qsa_b200 import _capi
+    w = make_workload(name, dev)
+    acct = workload_accounting(w)
+    out = torch.empty_like(w.q)
+    lse = torch.empty(w.q.shape[:2], dtype=torch.float32, device=dev)
+
+    def step():
+        _capi.sparse_prefill_fwd(w.q, w.k_cache, w.v_cache, w.topk_idx, w.n_valid, w.scale,
+                                 out=out, lse=lse)
+
+    steps = 20
+    total_ms, per_ms, _ = time_launches(step, steps, 3, barrier)
+    total_ms = max_over_ranks(total_ms)
+    ms = statistics.mean(per_ms)
+    roof_ms = 1e3 * max(acct["gathered_bytes"] / (hbm * 1e9), acct["flops"] / (bf16 * 1e12))
+    return {"workload": w.name, "tokens_per_s": w.shape["T"] * steps * world / (total_ms / 1e3),
+            "mean_launch_ms": ms, "gathered_kv_gbs": acct["gathered_bytes"] / (ms / 1e3) / 1e9,
+            "effective_tflops": acct["flops"] / (ms / 1e3) / 1e12,
+            "algo_gbs": acct["algo_bytes"] / (ms / 1e3) / 1e9,
+            "frac_of_roofline_time": roof_ms / ms, "steps": steps}
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_cuda(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,155 @@
+/*
+ * qsa.h -- C ABI of the B200 (sm_100a) QSA top-K sparse-attention prefill.
+ *
+ * The operation (page "Qwen4-Exp QSA llega al Ascend de Huawei", section
+ * "Lo que realmente añade la pull request", and its bullets "Hardware y tipo
+ * de dato", "Formas de cabeza", "Límites de tamaño"): for every query token t
+ * and KV head g, with G = Hq / Hkv query heads per KV head (query head h uses
+ * KV head h / G), attention restricted to the cache rows named by the
+ * token's selected-slot list:
+ *
+ *   J        = { j < n_valid[t,g] (K when n_valid is NULL) : 0 <= idx[t,g,j] < S }
+ *   s_j      = scale * < q[t,h,:], k_cache[idx[t,g,j], g, :] >
+ *   out[t,h] = sum_{j in J} softmax_J(s)_j * v_cache[idx[t,g,j], g, :]
+ *   lse[t,h] = log( sum_{j in J} exp(s_j) )           (natural log, FP32)
+ *
+ * The Q and K inputs are already rotated (RoPE applied); list order does not
+ * matter, -1 marks an empty entry anywhere in a list (interior -1 included);
+ * a row with an empty J gets out = +0.0 exactly and lse = -inf.  The default
+ * scale is 1/sqrt(head_dim) = 1/16 (the model's D256 scale).
+ *
+ * Support set: BF16 Q/K/V/out, head_dim = 256, G in 1..16 (covers the local
+ * head shapes (16,2), (24,2), (12,1), (6,1), (3,1)).  Anything else returns
+ * QSA_ERR_UNSUPPORTED; there is no fallback path.
+ *
+ * Conventions for every entry point:
+ *  - Device pointers unless stated; the caller owns every buffer.  The
+ *    device entry points allocate nothing, free nothing and never
+ *    synchronise the host; all work is enqueued on `stream` (a cudaStream_t
+ *    passed as void*, NULL = legacy default stream).
+ *  - Host-detectable errors are returned before anything is enqueued.
+ *    QSA_ERR_CUDA means a CUDA runtime call failed (the launch itself, or a
+ *    copy in the host-buffer variant).
+ *  - A slot id >= num_slots is treated as empty and sets bit 0 of *status
+ *    (a device int32 the caller zeroes; NULL disables the report).  The
+ *    kernels never trap.
+ *  - All strides are in elements.  Rows of Q, the caches and out must start on
+ *    16-byte boundaries: base pointers 16-byte aligned and every stride other
+ *    than the innermost a multiple of 8 elements (QSA_ERR_ALIGN otherwise).
+ */
+#ifndef QSA_H
+#define QSA_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define QSA_ABI_VERSION 1
+
+typedef enum {
+  QSA_OK = 0,
+  QSA_ERR_NULL = 1,        /* a required pointer is NULL */
+  QSA_ERR_SHAPE = 2,       /* inconsistent sizes or strides */
+  QSA_ERR_UNSUPPORTED = 3, /* head_dim != 256, G > 16, ... */
+  QSA_ERR_ALIGN = 4,       /* a row is not 16-byte aligned */
+  QSA_ERR_CUDA = 5         /* a CUDA runtime call failed */
+} qsa_status_t;
+
+/* Bits of the device status word. */
+#define QSA_STATUS_OOB_SLOT 1 /* some list entry named a slot >= num_slots */
+
+typedef struct {
+  int64_t num_tokens;     /* T >= 0: query tokens, packed over all sequences
+                             (varlen needs no cu_seqlens: ids are physical) */
+  int32_t num_q_heads;    /* Hq >= 1 */
+  int32_t num_kv_heads;   /* Hkv >= 1, Hq % Hkv == 0 */
+  int32_t head_dim;       /* D, must be 256 */
+  int32_t topk;           /* K >= 0 entries per list (K == 0: every row empty) */
+  int64_t num_slots;      /* S: cache rows; ids outside [0, S) are empty */
+  int64_t q_stride_tok, q_stride_head;     /* q       [T, Hq, D]  */
+  int64_t kv_stride_slot, kv_stride_head;  /* k_cache, v_cache [S, Hkv, D],
+                                              both with these strides */
+  int64_t idx_stride_tok, idx_stride_head; /* topk_idx [T, Hkv, K], entries
+                                              contiguous; head stride may be 0
+                                              (one list shared by all heads) */
+  int64_t o_stride_tok, o_stride_head;     /* out     [T, Hq, D]  */
+  int64_t lse_stride_tok;                  /* lse     [T, Hq], head stride 1 */
+} qsa_shape_t;
+
+/*
+ * Sparse prefill forward.
+ *   q, k_cache, v_cache : BF16 (__nv_bfloat16 bits), device, layouts above.
+ *   topk_idx            : int32 device [T, Hkv, K] physical slot ids, -1 empty.
+ *   n_valid             : int32 device [T, Hkv] contiguous (entries at
+ *                         positions >= n_valid are empty), or NULL (= K).
+ *   scale               : softmax scale; <= 0 selects 1/sqrt(head_dim).
+ *   out                 : BF16 device [T, Hq, D] (round to nearest even).
+ *   lse                 : FP32 device [T, Hq] natural-log LSE, or NULL.
+ *   status              : int32 device word (bit 0: out-of-range id), or NULL.
+ *   stream              : cudaStream_t.
+ * Enqueues one kernel launch.  Graph-capturable (no sync, no allocation).
+ */
+qsa_status_t qsa_sparse_prefill_fwd(const qsa_shape_t* shape, const void* q,
+                                    const void* k_cache, const void* v_cache,
+                                    const int32_t* topk_idx,
+                                    const int32_t* n_valid, float scale,
+                                    void* out, float* lse, int32_t* status,
+                                    void* stream);
+
+/*
+ * Debug variant of the same kernel: runs the identical gather stage (same
+ * index load, masking and copy addresses) and additionally writes, for
+ * every list entry, the slot id of the row the gather actually copied into
+ * shared memory (derived from the copy's source address), or -1 where the
+ * entry was masked and zero-filled.  gathered_ids is int32 device
+ * [T, Hkv, K] contiguous.  out/lse are written as by the forward call.
+ */
+qsa_status_t qsa_sparse_prefill_debug_gather(
+    const qsa_shape_t* shape, const void* q, const void* k_cache,
+    const void* v_cache, const int32_t* topk_idx, const int32_t* n_valid,
+    float scale, void* out, float* lse, int32_t* status,
+    int32_t* gathered_ids, void* stream);
+
+/* Device staging buffers for the host-buffer entry point (caller-owned,
+ * sized for the layouts of `shape`; n_valid / lse / status may be NULL when
+ * the matching host pointer is NULL). */
+typedef struct {
+  void* q;
+  void* k_cache;
+  void* v_cache;
+  int32_t* topk_idx;
+  int32_t* n_valid;
+  void* out;
+  float* lse;
+  int32_t* status;
+} qsa_device_buffers_t;
+
+/*
+ * Host-buffer variant: enqueues on `stream` one host->device cudaMemcpyAsync
+ * per input (q, k_cache, v_cache, topk_idx, n_valid), the forward kernel,
+ * and one device->host cudaMemcpyAsync per output (out, lse), then returns.
+ * Host pointers address buffers laid out exactly like the device ones with
+ * the strides of `shape` (each copied as one contiguous span from the first
+ * to the last element); page-locked host memory keeps the copies
+ * asynchronous.  The caller synchronises `stream` before reading out/lse.
+ * The status word (dev->status) is zeroed on the stream before the launch.
+ */
+qsa_status_t qsa_sparse_prefill_fwd_host(
+    const qsa_shape_t* shape, const void* q_host, const void* k_cache_host,
+    const void* v_cache_host, const int32_t* topk_idx_host,
+    const int32_t* n_valid_host, float scale, void* out_host,
+    float* lse_host, const qsa_device_buffers_t* dev, void* stream);
+
+/* Static description of a status code. */
+const char* qsa_status_string(qsa_status_t status);
+
+/* QSA_ABI_VERSION of the built library. */
+int32_t qsa_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QSA_H */

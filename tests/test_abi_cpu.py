@@ -1,0 +1,113 @@
+"""The C-ABI library loads and exports what include/qsa.h declares; host-side
+argument validation answers before anything touches a device (CPU only:
+no call here reaches a kernel)."""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "qsa.h")
+
+
+@pytest.fixture(scope="module")
+def capi():
+    from top_sparse_attention_qsa_b200 import build
+    build.build()
+    from top_sparse_attention_qsa_b200 import _capi
+    return _capi
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(qsa_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_header_declares_expected_entry_points():
+    names = declared_functions()
+    assert "qsa_sparse_prefill_fwd" in names
+    assert "qsa_sparse_prefill_debug_gather" in names
+
+
+def test_library_exports_every_declared_symbol(capi):
+    lib = capi.library()
+    for name in declared_functions():
+        assert hasattr(lib, name), f"libqsa.so does not export {name}"
+    assert sorted(capi.EXPORTS) == declared_functions()
+
+
+def test_library_is_sm100a_only_and_static_runtime(capi):
+    # the build flags the driver checks: one sm_100a target, static cudart
+    from top_sparse_attention_qsa_b200 import build
+    flags = " ".join(build.NVCC_FLAGS)
+    assert "arch=compute_100a,code=sm_100a" in flags
+    assert flags.count("-gencode") == 1
+
+
+def test_abi_version_and_status_strings(capi):
+    m = re.search(r"#define QSA_ABI_VERSION (\d+)", open(HEADER).read())
+    assert capi.abi_version() == int(m.group(1))
+    for code in range(6):
+        assert capi.status_string(code)
+    assert capi.status_string(99) == "unknown status"
+
+
+def _shape(capi, **kw):
+    base = dict(num_tokens=4, num_q_heads=12, num_kv_heads=1, head_dim=256, topk=8,
+                num_slots=64, q_stride_tok=12 * 256, q_stride_head=256, kv_stride_slot=256,
+                kv_stride_head=256, idx_stride_tok=8, idx_stride_head=8, o_stride_tok=12 * 256,
+                o_stride_head=256, lse_stride_tok=12)
+    base.update(kw)
+    return capi.Shape(**base)
+
+
+# Fake, 16-byte-aligned addresses: every case below is rejected by the host
+# checks before any CUDA call, so nothing is ever dereferenced.
+P = 0x10000
+
+
+def _fwd(capi, shape, q=P, k=P, v=P, idx=P, out=P, lse=None, nv=None):
+    return capi.library().qsa_sparse_prefill_fwd(ctypes.byref(shape) if shape is not None else None,
+                                                 q, k, v, idx, nv, 0.0, out, lse, None, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(head_dim=128), 3),
+    (dict(num_q_heads=34, num_kv_heads=2), 3),      # G = 17
+    (dict(num_q_heads=7, num_kv_heads=2), 2),       # Hq % Hkv != 0
+    (dict(num_tokens=-1), 2),
+    (dict(topk=-3), 2),
+    (dict(q_stride_head=260), 4),                   # rows not 16-byte aligned
+    (dict(kv_stride_slot=-256), 2),
+    (dict(kv_stride_slot=0), 2),
+])
+def test_shape_validation(capi, kw, code):
+    assert _fwd(capi, _shape(capi, **kw)) == code
+
+
+def test_null_and_alignment_checks(capi):
+    s = _shape(capi)
+    assert _fwd(capi, None) == 1
+    assert _fwd(capi, s, q=None) == 1
+    assert _fwd(capi, s, idx=None) == 1
+    assert _fwd(capi, s, out=P + 8) == 4
+    assert _fwd(capi, s, k=P + 2) == 4
+    # with K == 0 the caches and lists are never read: NULL is fine there,
+    # and T == 0 is a no-op that returns before any CUDA call
+    assert _fwd(capi, _shape(capi, num_tokens=0), q=None, out=None) == 0
+    lib = capi.library()
+    assert lib.qsa_sparse_prefill_debug_gather(ctypes.byref(s), P, P, P, P, None, 0.0, P, None,
+                                               None, None, None) == 1
+
+
+def test_binding_rejects_host_tensors(capi):
+    q = torch.zeros(2, 3, 256, dtype=torch.bfloat16)
+    k = torch.zeros(8, 1, 256, dtype=torch.bfloat16)
+    idx = torch.zeros(2, 1, 4, dtype=torch.int32)
+    with pytest.raises(ValueError):
+        capi.sparse_prefill_fwd(q, k, k, idx)
+    with pytest.raises(TypeError):
+        capi.sparse_prefill_fwd(q.float(), k, k, idx)

@@ -1,0 +1,21 @@
+"""QSA top-K sparse-attention prefill for B200 (sm_100a).
+
+The compute path is libqsa.so (hand-written CUDA kernels behind the C ABI of
+include/qsa.h); ``_capi`` is its ctypes binding.  The kernel entry points
+are loaded on first use, so ``workloads`` (the seeded input generator)
+imports without the library; using a kernel entry point without a built
+libqsa.so raises ImportError (there is no fallback).
+"""
+
+_API = ("sparse_prefill_fwd", "sparse_prefill_debug_gather", "sparse_prefill_fwd_host",
+        "status_string", "abi_version", "QSAError", "STATUS_OOB_SLOT")
+
+
+def __getattr__(name):
+    if name in _API:
+        from . import _capi
+        return getattr(_capi, name)
+    raise AttributeError(name)
+
+
+__all__ = list(_API)

@@ -1,0 +1,230 @@
+"""ctypes binding of libqsa.so (include/qsa.h).
+
+Argument marshalling only: tensors become pointers, sizes and strides; every
+step of the computation runs in the library's CUDA kernels.  Importing this
+module fails loudly when libqsa.so has not been built; there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libqsa.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing: build it with `python -m top_sparse_attention_qsa_b200.build` "
+        "(the QSA kernels have no CPU or Python fallback)")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+QSA_OK, QSA_ERR_NULL, QSA_ERR_SHAPE, QSA_ERR_UNSUPPORTED, QSA_ERR_ALIGN, QSA_ERR_CUDA = range(6)
+STATUS_OOB_SLOT = 1
+HEAD_DIM = 256
+
+# Every symbol include/qsa.h declares.
+EXPORTS = ("qsa_sparse_prefill_fwd", "qsa_sparse_prefill_debug_gather",
+           "qsa_sparse_prefill_fwd_host", "qsa_status_string", "qsa_abi_version")
+
+
+class Shape(ctypes.Structure):
+    _fields_ = [
+        ("num_tokens", ctypes.c_int64),
+        ("num_q_heads", ctypes.c_int32),
+        ("num_kv_heads", ctypes.c_int32),
+        ("head_dim", ctypes.c_int32),
+        ("topk", ctypes.c_int32),
+        ("num_slots", ctypes.c_int64),
+        ("q_stride_tok", ctypes.c_int64),
+        ("q_stride_head", ctypes.c_int64),
+        ("kv_stride_slot", ctypes.c_int64),
+        ("kv_stride_head", ctypes.c_int64),
+        ("idx_stride_tok", ctypes.c_int64),
+        ("idx_stride_head", ctypes.c_int64),
+        ("o_stride_tok", ctypes.c_int64),
+        ("o_stride_head", ctypes.c_int64),
+        ("lse_stride_tok", ctypes.c_int64),
+    ]
+
+
+class DeviceBuffers(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in
+                ("q", "k_cache", "v_cache", "topk_idx", "n_valid", "out", "lse", "status")]
+
+
+_vp = ctypes.c_void_p
+_lib.qsa_sparse_prefill_fwd.restype = ctypes.c_int
+_lib.qsa_sparse_prefill_fwd.argtypes = [ctypes.POINTER(Shape), _vp, _vp, _vp, _vp, _vp,
+                                        ctypes.c_float, _vp, _vp, _vp, _vp]
+_lib.qsa_sparse_prefill_debug_gather.restype = ctypes.c_int
+_lib.qsa_sparse_prefill_debug_gather.argtypes = [ctypes.POINTER(Shape), _vp, _vp, _vp, _vp, _vp,
+                                                 ctypes.c_float, _vp, _vp, _vp, _vp, _vp]
+_lib.qsa_sparse_prefill_fwd_host.restype = ctypes.c_int
+_lib.qsa_sparse_prefill_fwd_host.argtypes = [ctypes.POINTER(Shape), _vp, _vp, _vp, _vp, _vp,
+                                             ctypes.c_float, _vp, _vp,
+                                             ctypes.POINTER(DeviceBuffers), _vp]
+_lib.qsa_status_string.restype = ctypes.c_char_p
+_lib.qsa_status_string.argtypes = [ctypes.c_int]
+_lib.qsa_abi_version.restype = ctypes.c_int32
+_lib.qsa_abi_version.argtypes = []
+
+
+class QSAError(RuntimeError):
+    def __init__(self, code: int):
+        super().__init__(f"qsa status {code}: {status_string(code)}")
+        self.code = code
+
+
+def status_string(code: int) -> str:
+    return _lib.qsa_status_string(int(code)).decode()
+
+
+def abi_version() -> int:
+    return int(_lib.qsa_abi_version())
+
+
+def library():
+    return _lib
+
+
+def _ptr(x: Optional[torch.Tensor]):
+    return None if x is None else x.data_ptr()
+
+
+def _need(x: torch.Tensor, name: str, dtype, device=None, host=False):
+    if not isinstance(x, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if x.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {x.dtype}")
+    if host:
+        if x.device.type != "cpu":
+            raise ValueError(f"{name} must be a host tensor")
+    elif x.device.type != "cuda" or (device is not None and x.device != device):
+        raise ValueError(f"{name} must be a CUDA tensor on {device}")
+
+
+def make_shape(q, k_cache, topk_idx, out, lse=None) -> Shape:
+    """Shape/stride descriptor of a call (no checks beyond ranks: the library
+    validates sizes, strides and alignment itself)."""
+    if q.dim() != 3 or k_cache.dim() != 3 or topk_idx.dim() != 3 or out.dim() != 3:
+        raise ValueError("q, caches, topk_idx and out must be 3-d")
+    T, Hq, D = q.shape
+    S, Hkv, _ = k_cache.shape
+    K = topk_idx.shape[2]
+    if topk_idx.shape[0] != T or topk_idx.shape[1] != Hkv:
+        raise ValueError("topk_idx must be [T, Hkv, K]")
+    if tuple(out.shape) != (T, Hq, D):
+        raise ValueError("out must be [T, Hq, D]")
+    if q.stride(2) != 1 or k_cache.stride(2) != 1 or out.stride(2) != 1 or (K > 1 and topk_idx.stride(2) != 1):
+        raise ValueError("innermost dimensions must be contiguous")
+    if lse is not None and (tuple(lse.shape) != (T, Hq) or (Hq > 1 and lse.stride(1) != 1)):
+        raise ValueError("lse must be [T, Hq] with unit head stride")
+    return Shape(T, Hq, Hkv, D, K, S,
+                 q.stride(0), q.stride(1), k_cache.stride(0), k_cache.stride(1),
+                 topk_idx.stride(0), topk_idx.stride(1), out.stride(0), out.stride(1),
+                 lse.stride(0) if lse is not None else Hq)
+
+
+def _check_kv(k_cache, v_cache):
+    if tuple(v_cache.shape) != tuple(k_cache.shape) or v_cache.stride() != k_cache.stride():
+        raise ValueError("k_cache and v_cache must have the same shape and strides")
+
+
+def _raise(rc: int):
+    if rc != QSA_OK:
+        raise QSAError(rc)
+
+
+def sparse_prefill_fwd(q, k_cache, v_cache, topk_idx, n_valid=None, scale: float = 0.0,
+                       out=None, lse=None, status=None, stream=None, want_lse: bool = True):
+    """QSA sparse prefill on the GPU.  Returns (out [T,Hq,D] bf16, lse [T,Hq] fp32 or None)."""
+    dev = q.device
+    _need(q, "q", torch.bfloat16, dev)
+    _need(k_cache, "k_cache", torch.bfloat16, dev)
+    _need(v_cache, "v_cache", torch.bfloat16, dev)
+    _need(topk_idx, "topk_idx", torch.int32, dev)
+    _check_kv(k_cache, v_cache)
+    if n_valid is not None:
+        _need(n_valid, "n_valid", torch.int32, dev)
+        if not n_valid.is_contiguous() or tuple(n_valid.shape) != tuple(topk_idx.shape[:2]):
+            raise ValueError("n_valid must be a contiguous [T, Hkv] tensor")
+    if out is None:
+        out = torch.empty(q.shape, dtype=torch.bfloat16, device=dev)
+    _need(out, "out", torch.bfloat16, dev)
+    if lse is None and want_lse:
+        lse = torch.empty(q.shape[:2], dtype=torch.float32, device=dev)
+    if lse is not None:
+        _need(lse, "lse", torch.float32, dev)
+    if status is not None:
+        _need(status, "status", torch.int32, dev)
+    shape = make_shape(q, k_cache, topk_idx, out, lse)
+    if stream is None:
+        stream = torch.cuda.current_stream(dev).cuda_stream
+    rc = _lib.qsa_sparse_prefill_fwd(ctypes.byref(shape), _ptr(q), _ptr(k_cache), _ptr(v_cache),
+                                     _ptr(topk_idx), _ptr(n_valid), float(scale), _ptr(out),
+                                     _ptr(lse), _ptr(status), stream)
+    _raise(rc)
+    return out, lse
+
+
+def sparse_prefill_debug_gather(q, k_cache, v_cache, topk_idx, n_valid=None, scale: float = 0.0,
+                                status=None, stream=None):
+    """Same kernel with the gather dump: returns (out, lse, gathered_ids [T,Hkv,K] int32)."""
+    dev = q.device
+    _need(q, "q", torch.bfloat16, dev)
+    _need(k_cache, "k_cache", torch.bfloat16, dev)
+    _need(v_cache, "v_cache", torch.bfloat16, dev)
+    _need(topk_idx, "topk_idx", torch.int32, dev)
+    _check_kv(k_cache, v_cache)
+    if n_valid is not None:
+        _need(n_valid, "n_valid", torch.int32, dev)
+    out = torch.empty(q.shape, dtype=torch.bfloat16, device=dev)
+    lse = torch.empty(q.shape[:2], dtype=torch.float32, device=dev)
+    ids = torch.empty(topk_idx.shape, dtype=torch.int32, device=dev)
+    shape = make_shape(q, k_cache, topk_idx, out, lse)
+    if stream is None:
+        stream = torch.cuda.current_stream(dev).cuda_stream
+    rc = _lib.qsa_sparse_prefill_debug_gather(ctypes.byref(shape), _ptr(q), _ptr(k_cache),
+                                              _ptr(v_cache), _ptr(topk_idx), _ptr(n_valid),
+                                              float(scale), _ptr(out), _ptr(lse), _ptr(status),
+                                              _ptr(ids), stream)
+    _raise(rc)
+    return out, lse, ids
+
+
+def sparse_prefill_fwd_host(q, k_cache, v_cache, topk_idx, n_valid, scale, out, lse,
+                            dev_bufs: dict, stream=None):
+    """Host-buffer entry point: host tensors in and out (pinned for async copies),
+    device staging tensors in `dev_bufs` (keys as in qsa_device_buffers_t).
+    Enqueues copies + kernel + copies on `stream`; the caller synchronises."""
+    for name, x, dt in (("q", q, torch.bfloat16), ("k_cache", k_cache, torch.bfloat16),
+                        ("v_cache", v_cache, torch.bfloat16), ("topk_idx", topk_idx, torch.int32),
+                        ("out", out, torch.bfloat16)):
+        _need(x, name, dt, host=True)
+    _check_kv(k_cache, v_cache)
+    if n_valid is not None:
+        _need(n_valid, "n_valid", torch.int32, host=True)
+    if lse is not None:
+        _need(lse, "lse", torch.float32, host=True)
+    dev = dev_bufs["q"].device
+    host = {"q": q, "k_cache": k_cache, "v_cache": v_cache, "topk_idx": topk_idx, "out": out}
+    for name, h in host.items():
+        d = dev_bufs[name]
+        _need(d, "dev." + name, h.dtype, dev)
+        if d.stride() != h.stride() or d.shape != h.shape:
+            raise ValueError(f"dev.{name} must match the host tensor's shape and strides")
+    db = DeviceBuffers(*[_ptr(dev_bufs.get(n)) for n in
+                         ("q", "k_cache", "v_cache", "topk_idx", "n_valid", "out", "lse", "status")])
+    shape = make_shape(q, k_cache, topk_idx, out, lse)
+    if stream is None:
+        stream = torch.cuda.current_stream(dev).cuda_stream
+    rc = _lib.qsa_sparse_prefill_fwd_host(ctypes.byref(shape), _ptr(q), _ptr(k_cache),
+                                          _ptr(v_cache), _ptr(topk_idx), _ptr(n_valid),
+                                          float(scale), _ptr(out), _ptr(lse), ctypes.byref(db),
+                                          stream)
+    _raise(rc)
+    return out, lse

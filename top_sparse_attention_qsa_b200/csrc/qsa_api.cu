@@ -1,0 +1,210 @@
+// qsa_api.cu -- C ABI of the QSA sparse-attention prefill library (sm_100a).
+//
+// Host-side argument validation, kernel selection and launch.  See
+// include/qsa.h for the contract of every entry point.
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cstdint>
+#include <cstring>
+
+#include "qsa.h"
+#include "qsa_prefill_mma.cuh"
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Validates `s` and the pointers of a forward call.  Returns QSA_OK or the
+// first error found; never touches device memory.
+qsa_status_t validate(const qsa_shape_t* s, const void* q, const void* k, const void* v,
+                      const int32_t* idx, const void* out) {
+  if (s == nullptr) return QSA_ERR_NULL;
+  if (s->num_tokens < 0 || s->topk < 0 || s->num_slots < 0 || s->num_q_heads <= 0 ||
+      s->num_kv_heads <= 0)
+    return QSA_ERR_SHAPE;
+  if (s->num_q_heads % s->num_kv_heads != 0) return QSA_ERR_SHAPE;
+  if (s->head_dim != qsa::kHeadDim) return QSA_ERR_UNSUPPORTED;
+  const int G = s->num_q_heads / s->num_kv_heads;
+  if (G > 16) return QSA_ERR_UNSUPPORTED;
+  if (s->num_kv_heads > 65535 || s->num_tokens > 0x7fffffffLL) return QSA_ERR_UNSUPPORTED;
+  if (s->num_tokens == 0) return QSA_OK;
+  if (q == nullptr || out == nullptr) return QSA_ERR_NULL;
+  const bool reads_cache = s->topk > 0;
+  if (reads_cache && (k == nullptr || v == nullptr || idx == nullptr)) return QSA_ERR_NULL;
+  // strides: non-negative, rows 16-byte aligned
+  const int64_t st[] = {s->q_stride_tok, s->q_stride_head, s->o_stride_tok, s->o_stride_head,
+                        s->kv_stride_slot, s->kv_stride_head};
+  for (int64_t x : st)
+    if (x < 0) return QSA_ERR_SHAPE;
+  if (s->idx_stride_tok < 0 || s->idx_stride_head < 0 || s->lse_stride_tok < 0) return QSA_ERR_SHAPE;
+  if (reads_cache && s->num_slots > 0 && s->kv_stride_slot == 0) return QSA_ERR_SHAPE;
+  for (int64_t x : st)
+    if (x % 8 != 0) return QSA_ERR_ALIGN;
+  if (!aligned16(q) || !aligned16(out)) return QSA_ERR_ALIGN;
+  if (reads_cache && (!aligned16(k) || !aligned16(v))) return QSA_ERR_ALIGN;
+  if (reads_cache && (reinterpret_cast<uintptr_t>(idx) & 3u)) return QSA_ERR_ALIGN;
+  if (s->num_slots > 0x80000000LL) return QSA_ERR_UNSUPPORTED;  // int32 slot ids
+  return QSA_OK;
+}
+
+template <typename Kernel>
+cudaError_t set_smem_once(Kernel kernel, int bytes, std::atomic<int>* done) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  if (done[dev].load(std::memory_order_acquire)) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) done[dev].store(1, std::memory_order_release);
+  return e;
+}
+
+template <int NT, bool kDump>
+cudaError_t launch_mma(const qsa::PrefillParams& p, cudaStream_t stream) {
+  using C = qsa::MmaCfg<NT>;
+  static std::atomic<int> done[kMaxDevices];
+  auto kernel = qsa::qsa_prefill_mma_kernel<NT, kDump>;
+  cudaError_t e = set_smem_once(kernel, C::SMEM, done);
+  if (e != cudaSuccess) return e;
+  dim3 grid(static_cast<unsigned>(p.T), static_cast<unsigned>(p.Hkv));
+  kernel<<<grid, C::THREADS, C::SMEM, stream>>>(p);
+  return cudaGetLastError();
+}
+
+qsa_status_t run_forward(const qsa_shape_t* s, const void* q, const void* k, const void* v,
+                         const int32_t* idx, const int32_t* n_valid, float scale, void* out,
+                         float* lse, int32_t* status, int32_t* gathered, void* stream) {
+  qsa_status_t rc = validate(s, q, k, v, idx, out);
+  if (rc != QSA_OK) return rc;
+  if (gathered != nullptr && s->topk > 0 && (reinterpret_cast<uintptr_t>(gathered) & 3u))
+    return QSA_ERR_ALIGN;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (s->num_tokens == 0) return QSA_OK;
+  if (gathered != nullptr && s->topk > 0) {
+    const size_t n = static_cast<size_t>(s->num_tokens) * s->num_kv_heads * s->topk;
+    if (cudaMemsetAsync(gathered, 0xff, n * sizeof(int32_t), st) != cudaSuccess) return QSA_ERR_CUDA;
+  }
+  qsa::PrefillParams p;
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.k = static_cast<const __nv_bfloat16*>(k);
+  p.v = static_cast<const __nv_bfloat16*>(v);
+  p.idx = idx;
+  p.n_valid = n_valid;
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.lse = lse;
+  p.status = status;
+  p.gathered = gathered;
+  p.T = s->num_tokens;
+  p.Hkv = s->num_kv_heads;
+  p.G = s->num_q_heads / s->num_kv_heads;
+  p.K = s->topk;
+  p.S = s->num_slots;
+  p.q_st = s->q_stride_tok;
+  p.q_sh = s->q_stride_head;
+  p.kv_ss = s->kv_stride_slot;
+  p.kv_sh = s->kv_stride_head;
+  p.idx_st = s->idx_stride_tok;
+  p.idx_sh = s->idx_stride_head;
+  p.o_st = s->o_stride_tok;
+  p.o_sh = s->o_stride_head;
+  p.lse_st = s->lse_stride_tok;
+  const float sc = scale > 0.f ? scale : 0.0625f;  // 1/sqrt(256)
+  p.scale_log2 = sc * 1.4426950408889634f;
+  cudaError_t e;
+  const bool dump = gathered != nullptr;
+  if (p.G <= 8)
+    e = dump ? launch_mma<1, true>(p, st) : launch_mma<1, false>(p, st);
+  else
+    e = dump ? launch_mma<2, true>(p, st) : launch_mma<2, false>(p, st);
+  return e == cudaSuccess ? QSA_OK : QSA_ERR_CUDA;
+}
+
+// Bytes spanned by a strided [n0, n1, inner] layout (first to last element).
+size_t span_bytes(int64_t n0, int64_t s0, int64_t n1, int64_t s1, int64_t inner, size_t elem) {
+  if (n0 <= 0 || n1 <= 0 || inner <= 0) return 0;
+  return static_cast<size_t>((n0 - 1) * s0 + (n1 - 1) * s1 + inner) * elem;
+}
+
+}  // namespace
+
+extern "C" {
+
+qsa_status_t qsa_sparse_prefill_fwd(const qsa_shape_t* shape, const void* q, const void* k_cache,
+                                    const void* v_cache, const int32_t* topk_idx,
+                                    const int32_t* n_valid, float scale, void* out, float* lse,
+                                    int32_t* status, void* stream) {
+  return run_forward(shape, q, k_cache, v_cache, topk_idx, n_valid, scale, out, lse, status,
+                     nullptr, stream);
+}
+
+qsa_status_t qsa_sparse_prefill_debug_gather(const qsa_shape_t* shape, const void* q,
+                                             const void* k_cache, const void* v_cache,
+                                             const int32_t* topk_idx, const int32_t* n_valid,
+                                             float scale, void* out, float* lse, int32_t* status,
+                                             int32_t* gathered_ids, void* stream) {
+  if (gathered_ids == nullptr) return QSA_ERR_NULL;
+  return run_forward(shape, q, k_cache, v_cache, topk_idx, n_valid, scale, out, lse, status,
+                     gathered_ids, stream);
+}
+
+qsa_status_t qsa_sparse_prefill_fwd_host(const qsa_shape_t* s, const void* q_host,
+                                         const void* k_cache_host, const void* v_cache_host,
+                                         const int32_t* topk_idx_host, const int32_t* n_valid_host,
+                                         float scale, void* out_host, float* lse_host,
+                                         const qsa_device_buffers_t* dev, void* stream) {
+  if (s == nullptr || dev == nullptr) return QSA_ERR_NULL;
+  qsa_status_t rc = validate(s, dev->q, dev->k_cache, dev->v_cache, dev->topk_idx, dev->out);
+  if (rc != QSA_OK) return rc;
+  if (s->num_tokens == 0) return QSA_OK;
+  const int64_t T = s->num_tokens, Hq = s->num_q_heads, Hkv = s->num_kv_heads, D = s->head_dim;
+  const int64_t K = s->topk, S = s->num_slots;
+  if (q_host == nullptr || out_host == nullptr) return QSA_ERR_NULL;
+  if (K > 0 && (k_cache_host == nullptr || v_cache_host == nullptr || topk_idx_host == nullptr))
+    return QSA_ERR_NULL;
+  if ((n_valid_host != nullptr) != (dev->n_valid != nullptr)) return QSA_ERR_NULL;
+  if (lse_host != nullptr && dev->lse == nullptr) return QSA_ERR_NULL;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  auto h2d = [&](void* d, const void* h, size_t n) {
+    return n == 0 || cudaMemcpyAsync(d, h, n, cudaMemcpyHostToDevice, st) == cudaSuccess;
+  };
+  auto d2h = [&](void* h, const void* d, size_t n) {
+    return n == 0 || cudaMemcpyAsync(h, d, n, cudaMemcpyDeviceToHost, st) == cudaSuccess;
+  };
+  bool ok = h2d(dev->q, q_host, span_bytes(T, s->q_stride_tok, Hq, s->q_stride_head, D, 2));
+  if (K > 0) {
+    const size_t kv = span_bytes(S, s->kv_stride_slot, Hkv, s->kv_stride_head, D, 2);
+    ok = ok && h2d(dev->k_cache, k_cache_host, kv) && h2d(dev->v_cache, v_cache_host, kv);
+    ok = ok && h2d(dev->topk_idx, topk_idx_host,
+                   span_bytes(T, s->idx_stride_tok, Hkv, s->idx_stride_head, K, 4));
+  }
+  if (n_valid_host != nullptr)
+    ok = ok && h2d(dev->n_valid, n_valid_host, static_cast<size_t>(T * Hkv) * 4);
+  if (dev->status != nullptr) ok = ok && cudaMemsetAsync(dev->status, 0, 4, st) == cudaSuccess;
+  if (!ok) return QSA_ERR_CUDA;
+  rc = run_forward(s, dev->q, dev->k_cache, dev->v_cache, dev->topk_idx, dev->n_valid, scale,
+                   dev->out, lse_host != nullptr ? dev->lse : nullptr, dev->status, nullptr, stream);
+  if (rc != QSA_OK) return rc;
+  ok = d2h(out_host, dev->out, span_bytes(T, s->o_stride_tok, Hq, s->o_stride_head, D, 2));
+  if (lse_host != nullptr)
+    ok = ok && d2h(lse_host, dev->lse, span_bytes(T, s->lse_stride_tok, 1, 0, Hq, 4));
+  return ok ? QSA_OK : QSA_ERR_CUDA;
+}
+
+const char* qsa_status_string(qsa_status_t status) {
+  switch (status) {
+    case QSA_OK: return "ok";
+    case QSA_ERR_NULL: return "a required pointer is NULL";
+    case QSA_ERR_SHAPE: return "inconsistent sizes or strides";
+    case QSA_ERR_UNSUPPORTED: return "unsupported configuration (needs BF16, head_dim 256, G <= 16)";
+    case QSA_ERR_ALIGN: return "rows must start on 16-byte boundaries";
+    case QSA_ERR_CUDA: return "a CUDA runtime call failed";
+  }
+  return "unknown status";
+}
+
+int32_t qsa_abi_version(void) { return QSA_ABI_VERSION; }
+
+}  // extern "C"
