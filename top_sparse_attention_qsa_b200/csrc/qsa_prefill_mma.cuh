@@ -252,11 +252,12 @@ __global__ void __launch_bounds__(MmaCfg<NT>::THREADS, 1)
         const float m_use = m_new == -INFINITY ? 0.f : m_new;
         alpha[nt][e] = ex2(m_run[nt][e] - m_use);
         m_run[nt][e] = m_new;
-        const __nv_bfloat16 p0 = __float2bfloat16_rn(ex2(s[nt][e] - m_use));
-        const __nv_bfloat16 p1 = __float2bfloat16_rn(ex2(s[nt][2 + e] - m_use));
-        l_run[nt][e] = l_run[nt][e] * alpha[nt][e] + __bfloat162float(p0) + __bfloat162float(p1);
-        p_s[h * C::P_STRIDE + key0] = p0;
-        p_s[h * C::P_STRIDE + key1] = p1;
+        const float p0 = ex2(s[nt][e] - m_use);
+        const float p1 = ex2(s[nt][2 + e] - m_use);
+        // the row sum keeps FP32 precision (it sets lse); P enters PV as BF16
+        l_run[nt][e] = l_run[nt][e] * alpha[nt][e] + p0 + p1;
+        p_s[h * C::P_STRIDE + key0] = __float2bfloat16_rn(p0);
+        p_s[h * C::P_STRIDE + key1] = __float2bfloat16_rn(p1);
       }
     __syncthreads();
 
