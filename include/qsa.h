@@ -59,6 +59,9 @@ typedef enum {
 
 /* Bits of the device status word. */
 #define QSA_STATUS_OOB_SLOT 1 /* some list entry named a slot >= num_slots */
+#define QSA_STATUS_TIMEOUT 2  /* a pipeline wait inside the kernel exceeded its
+                                 2 s bound; the kernel stopped early and its
+                                 outputs are not valid */
 
 typedef struct {
   int64_t num_tokens;     /* T >= 0: query tokens, packed over all sequences
@@ -89,7 +92,8 @@ typedef struct {
  *   lse                 : FP32 device [T, Hq] natural-log LSE, or NULL.
  *   status              : int32 device word (bit 0: out-of-range id), or NULL.
  *   stream              : cudaStream_t.
- * Enqueues one kernel launch.  Graph-capturable (no sync, no allocation).
+ * Enqueues one kernel launch (QSA_KERNEL_AUTO choice, see below).
+ * Graph-capturable (no sync, no allocation).
  */
 qsa_status_t qsa_sparse_prefill_fwd(const qsa_shape_t* shape, const void* q,
                                     const void* k_cache, const void* v_cache,
@@ -98,8 +102,28 @@ qsa_status_t qsa_sparse_prefill_fwd(const qsa_shape_t* shape, const void* q,
                                     void* out, float* lse, int32_t* status,
                                     void* stream);
 
+/* Kernel choice for qsa_sparse_prefill_fwd_with. */
+typedef enum {
+  QSA_KERNEL_AUTO = 0,      /* TMA + tcgen05 kernel when TMA descriptors can express
+                               the layout (Hkv <= 16, slot stride >= 256 elements,
+                               K > 0, 0 < S < 2^31 - 1), otherwise the warp-MMA kernel */
+  QSA_KERNEL_TCGEN05 = 1,   /* persistent TMA-gather + tcgen05/TMEM kernel only
+                               (QSA_ERR_UNSUPPORTED when the layout does not fit) */
+  QSA_KERNEL_WARP_MMA = 2   /* cp.async-gather + mma.sync kernel (any valid layout) */
+} qsa_kernel_t;
+
+/* Same contract as qsa_sparse_prefill_fwd, with an explicit kernel choice.
+ * qsa_sparse_prefill_fwd is this call with QSA_KERNEL_AUTO. */
+qsa_status_t qsa_sparse_prefill_fwd_with(const qsa_shape_t* shape, const void* q,
+                                         const void* k_cache, const void* v_cache,
+                                         const int32_t* topk_idx,
+                                         const int32_t* n_valid, float scale,
+                                         void* out, float* lse, int32_t* status,
+                                         qsa_kernel_t kernel, void* stream);
+
 /*
- * Debug variant of the same kernel: runs the identical gather stage (same
+ * Debug variant of the same kernel (the one QSA_KERNEL_AUTO picks): runs
+ * the identical gather stage (same
  * index load, masking and copy addresses) and additionally writes, for
  * every list entry, the slot id of the row the gather actually copied into
  * shared memory (derived from the copy's source address), or -1 where the

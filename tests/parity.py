@@ -21,9 +21,10 @@ PAGES_ATOL = PAGES_RTOL = 0.025
 PAGES_REL_L2 = 0.008
 
 
-def run_gpu(w, **kw):
+def run_gpu(w, kernel="auto", **kw):
     from top_sparse_attention_qsa_b200 import _capi
-    return _capi.sparse_prefill_fwd(w.q, w.k_cache, w.v_cache, w.topk_idx, w.n_valid, w.scale, **kw)
+    return _capi.sparse_prefill_fwd(w.q, w.k_cache, w.v_cache, w.topk_idx, w.n_valid, w.scale,
+                                    kernel=kernel, **kw)
 
 
 def host(x):

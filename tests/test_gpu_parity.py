@@ -19,6 +19,7 @@ pytestmark = [pytest.mark.gpu,
               pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA device")]
 
 DEV = "cuda"
+KERNELS = ["tcgen05", "warp_mma"]
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -26,15 +27,15 @@ def _lib():
     from top_sparse_attention_qsa_b200 import _capi  # noqa: F401  (fails loudly if unbuilt)
 
 
-def check_all(w, label):
-    out, lse = run_gpu(w)
+def check_all(w, label, kernel="auto"):
+    out, lse = run_gpu(w, kernel)
     torch.cuda.synchronize()
     ref_out, ref_lse, _ = run_oracle(w)
     return compare(host(out), host(lse), ref_out, ref_lse, label)
 
 
-def check_sampled(w, label, tokens):
-    out, lse = run_gpu(w)
+def check_sampled(w, label, tokens, kernel="auto"):
+    out, lse = run_gpu(w, kernel)
     torch.cuda.synchronize()
     o, ls = host(out), host(lse)
     # properties that hold at any size: every row finite, empty rows exact
@@ -46,21 +47,23 @@ def check_sampled(w, label, tokens):
 
 # --- the five configurations ------------------------------------------------
 
+@pytest.mark.parametrize("kernel", KERNELS)
 @pytest.mark.parametrize("name", ["tiny", "c2"])
-def test_config_full(name):
+def test_config_full(name, kernel):
     w = W.make(name, device=DEV)
-    print(name, check_all(w, name))
+    print(name, kernel, check_all(w, name, kernel))
 
 
+@pytest.mark.parametrize("kernel", KERNELS)
 @pytest.mark.parametrize("name", ["c3", "c4", "c5"])
-def test_config_sampled(name):
+def test_config_sampled(name, kernel):
     w = W.make(name, device=DEV)
     s = w.shape
     extra = []
     if name == "c3":
         extra = [8190, 8191, 8192, 8193, 8192 + 1023, 8192 + 1024]   # second sequence start
     tokens = sample_tokens(s["T"], s["K"], n_random=48, seed=len(name), extra=extra)
-    print(name, check_sampled(w, name, tokens))
+    print(name, kernel, check_sampled(w, name, tokens, kernel))
 
 
 def test_pages_long_prefill():
@@ -87,18 +90,20 @@ def test_gather_dump_bit_exact(name):
 
 # --- the pages' operator cases ------------------------------------------------
 
-@pytest.mark.parametrize("K", [1, 63, 64, 65, 2051])
+@pytest.mark.parametrize("kernel", KERNELS)
+@pytest.mark.parametrize("K", [1, 63, 64, 65, 127, 128, 129, 2051])
 @pytest.mark.parametrize("heads", [(12, 1), (24, 2)])
-def test_widths_unordered(K, heads):
+def test_widths_unordered(K, heads, kernel):
     w = W.generic_case(T=19, S=4096, Hq=heads[0], Hkv=heads[1], K=K, seed=K, device=DEV)
-    check_all(w, f"width{K}")
+    check_all(w, f"width{K}", kernel)
 
 
+@pytest.mark.parametrize("kernel", KERNELS)
 @pytest.mark.parametrize("heads", W.HEAD_SHAPES)
 @pytest.mark.parametrize("T", [1, 257])
-def test_head_shapes_rows(heads, T):
+def test_head_shapes_rows(heads, T, kernel):
     w = W.generic_case(T=T, S=3000, Hq=heads[0], Hkv=heads[1], K=130, seed=T + heads[0], device=DEV)
-    check_all(w, f"heads{heads}T{T}")
+    check_all(w, f"heads{heads}T{T}", kernel)
 
 
 @pytest.mark.parametrize("scale", [0.0, 1.0 / 16, 0.037, 0.25])
@@ -115,7 +120,8 @@ def test_default_scale_is_d256():
     assert torch.equal(a, b) and torch.equal(la, lb)
 
 
-def test_masked_rows_and_interior_padding():
+@pytest.mark.parametrize("kernel", KERNELS)
+def test_masked_rows_and_interior_padding(kernel):
     w = W.generic_case(T=40, S=1000, Hq=24, Hkv=2, K=96, seed=5, device=DEV)
     idx = w.topk_idx.clone()
     idx[3] = -1                                # fully masked token, both heads
@@ -129,7 +135,7 @@ def test_masked_rows_and_interior_padding():
     nv[22] = 65                                # tail beyond n_valid holds live ids but is ignored
     nv[23] = 200                               # n_valid > K clamps to K
     w.topk_idx, w.n_valid = idx.contiguous(), nv
-    st = check_all(w, "masked")
+    st = check_all(w, "masked", kernel)
     assert st["empty_rows"] >= 24 + 12 + 24
 
 

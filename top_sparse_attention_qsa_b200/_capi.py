@@ -24,10 +24,13 @@ _lib = ctypes.CDLL(LIB_PATH)
 
 QSA_OK, QSA_ERR_NULL, QSA_ERR_SHAPE, QSA_ERR_UNSUPPORTED, QSA_ERR_ALIGN, QSA_ERR_CUDA = range(6)
 STATUS_OOB_SLOT = 1
+STATUS_TIMEOUT = 2
+KERNEL_AUTO, KERNEL_TCGEN05, KERNEL_WARP_MMA = 0, 1, 2
+KERNELS = {"auto": KERNEL_AUTO, "tcgen05": KERNEL_TCGEN05, "warp_mma": KERNEL_WARP_MMA}
 HEAD_DIM = 256
 
 # Every symbol include/qsa.h declares.
-EXPORTS = ("qsa_sparse_prefill_fwd", "qsa_sparse_prefill_debug_gather",
+EXPORTS = ("qsa_sparse_prefill_fwd", "qsa_sparse_prefill_fwd_with", "qsa_sparse_prefill_debug_gather",
            "qsa_sparse_prefill_fwd_host", "qsa_status_string", "qsa_abi_version")
 
 
@@ -60,6 +63,9 @@ _vp = ctypes.c_void_p
 _lib.qsa_sparse_prefill_fwd.restype = ctypes.c_int
 _lib.qsa_sparse_prefill_fwd.argtypes = [ctypes.POINTER(Shape), _vp, _vp, _vp, _vp, _vp,
                                         ctypes.c_float, _vp, _vp, _vp, _vp]
+_lib.qsa_sparse_prefill_fwd_with.restype = ctypes.c_int
+_lib.qsa_sparse_prefill_fwd_with.argtypes = [ctypes.POINTER(Shape), _vp, _vp, _vp, _vp, _vp,
+                                             ctypes.c_float, _vp, _vp, _vp, ctypes.c_int, _vp]
 _lib.qsa_sparse_prefill_debug_gather.restype = ctypes.c_int
 _lib.qsa_sparse_prefill_debug_gather.argtypes = [ctypes.POINTER(Shape), _vp, _vp, _vp, _vp, _vp,
                                                  ctypes.c_float, _vp, _vp, _vp, _vp, _vp]
@@ -140,8 +146,10 @@ def _raise(rc: int):
 
 
 def sparse_prefill_fwd(q, k_cache, v_cache, topk_idx, n_valid=None, scale: float = 0.0,
-                       out=None, lse=None, status=None, stream=None, want_lse: bool = True):
-    """QSA sparse prefill on the GPU.  Returns (out [T,Hq,D] bf16, lse [T,Hq] fp32 or None)."""
+                       out=None, lse=None, status=None, stream=None, want_lse: bool = True,
+                       kernel: str = "auto"):
+    """QSA sparse prefill on the GPU.  Returns (out [T,Hq,D] bf16, lse [T,Hq] fp32 or None).
+    kernel: "auto" | "tcgen05" | "warp_mma" (see qsa_kernel_t)."""
     dev = q.device
     _need(q, "q", torch.bfloat16, dev)
     _need(k_cache, "k_cache", torch.bfloat16, dev)
@@ -164,9 +172,10 @@ def sparse_prefill_fwd(q, k_cache, v_cache, topk_idx, n_valid=None, scale: float
     shape = make_shape(q, k_cache, topk_idx, out, lse)
     if stream is None:
         stream = torch.cuda.current_stream(dev).cuda_stream
-    rc = _lib.qsa_sparse_prefill_fwd(ctypes.byref(shape), _ptr(q), _ptr(k_cache), _ptr(v_cache),
-                                     _ptr(topk_idx), _ptr(n_valid), float(scale), _ptr(out),
-                                     _ptr(lse), _ptr(status), stream)
+    rc = _lib.qsa_sparse_prefill_fwd_with(ctypes.byref(shape), _ptr(q), _ptr(k_cache),
+                                          _ptr(v_cache), _ptr(topk_idx), _ptr(n_valid),
+                                          float(scale), _ptr(out), _ptr(lse), _ptr(status),
+                                          KERNELS[kernel], stream)
     _raise(rc)
     return out, lse
 

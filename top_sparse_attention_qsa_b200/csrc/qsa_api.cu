@@ -2,14 +2,17 @@
 //
 // Host-side argument validation, kernel selection and launch.  See
 // include/qsa.h for the contract of every entry point.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <atomic>
 #include <cstdint>
 #include <cstring>
+#include <mutex>
 
 #include "qsa.h"
 #include "qsa_prefill_mma.cuh"
+#include "qsa_prefill_tc.cuh"
 
 namespace {
 
@@ -74,9 +77,106 @@ cudaError_t launch_mma(const qsa::PrefillParams& p, cudaStream_t stream) {
   return cudaGetLastError();
 }
 
+// ---------------------------------------------------------------- TMA path
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(f);
+  });
+  return fn;
+}
+
+int sm_count() {
+  static std::atomic<int> cache[kMaxDevices];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 0;
+  int n = cache[dev].load(std::memory_order_relaxed);
+  if (n == 0) {
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    cache[dev].store(n, std::memory_order_relaxed);
+  }
+  return n;
+}
+
+// Fills the tensor maps of the TMA kernel.  Returns false when a TMA
+// descriptor cannot express the layout (the warp-MMA kernel takes those).
+bool make_tc_params(const qsa_shape_t* s, const void* q, const void* k, const void* v,
+                    qsa::tc::TcParams* tp) {
+  using namespace qsa::tc;
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr) return false;
+  if (s->num_kv_heads > kMaxKvHeads || s->topk <= 0 || s->num_slots <= 0 ||
+      s->num_slots >= 0x7fffffffLL)
+    return false;
+  const uint64_t row_bytes = static_cast<uint64_t>(s->kv_stride_slot) * 2;
+  if (s->num_slots > 1 && row_bytes < 512) return false;
+  const cuuint32_t elem_str[3] = {1, 1, 1};
+  for (int g = 0; g < s->num_kv_heads; ++g) {
+    const cuuint64_t dims[2] = {256, static_cast<cuuint64_t>(s->num_slots)};
+    const cuuint64_t strides[1] = {s->num_slots > 1 ? row_bytes : 512};
+    const cuuint32_t box[2] = {64, 1};
+    for (int which = 0; which < 2; ++which) {
+      const char* base = static_cast<const char*>(which == 0 ? k : v) +
+                         static_cast<int64_t>(g) * s->kv_stride_head * 2;
+      CUtensorMap* m = which == 0 ? &tp->tm_k[g] : &tp->tm_v[g];
+      if (enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<char*>(base), dims, strides, box,
+              elem_str, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return false;
+    }
+  }
+  const uint64_t hq = static_cast<uint64_t>(s->num_q_heads);
+  uint64_t st_h = static_cast<uint64_t>(s->q_stride_head) * 2;
+  if (hq == 1 || st_h < 512) {
+    if (hq > 1) return false;
+    st_h = 512;
+  }
+  uint64_t st_t = static_cast<uint64_t>(s->q_stride_tok) * 2;
+  if (s->num_tokens == 1 || st_t < st_h * hq) {
+    if (s->num_tokens > 1) return false;
+    st_t = st_h * hq;
+  }
+  const cuuint64_t qdims[3] = {256, hq, static_cast<cuuint64_t>(s->num_tokens)};
+  const cuuint64_t qstr[2] = {st_h, st_t};
+  const cuuint32_t qbox[3] = {64, static_cast<cuuint32_t>(kGp), 1};
+  if (enc(&tp->tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(q), qdims, qstr, qbox,
+          elem_str, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return false;
+  return true;
+}
+
+template <bool kDump>
+cudaError_t launch_tc(const qsa::tc::TcParams& tp, cudaStream_t stream) {
+  static std::atomic<int> done[kMaxDevices];
+  auto kernel = qsa::tc::qsa_prefill_tc_kernel<kDump>;
+  cudaError_t e = set_smem_once(kernel, qsa::tc::SMEM_BYTES, done);
+  if (e != cudaSuccess) return e;
+  const int64_t units = tp.T * tp.Hkv;
+  int nsm = sm_count();
+  if (nsm <= 0) return cudaErrorInvalidDevice;
+  const unsigned grid = static_cast<unsigned>(units < nsm ? units : nsm);
+  kernel<<<grid, qsa::tc::kThreads, qsa::tc::SMEM_BYTES, stream>>>(tp);
+  return cudaGetLastError();
+}
+
 qsa_status_t run_forward(const qsa_shape_t* s, const void* q, const void* k, const void* v,
                          const int32_t* idx, const int32_t* n_valid, float scale, void* out,
-                         float* lse, int32_t* status, int32_t* gathered, void* stream) {
+                         float* lse, int32_t* status, int32_t* gathered, void* stream,
+                         qsa_kernel_t which = QSA_KERNEL_AUTO) {
+  if (which != QSA_KERNEL_AUTO && which != QSA_KERNEL_TCGEN05 && which != QSA_KERNEL_WARP_MMA)
+    return QSA_ERR_UNSUPPORTED;
   qsa_status_t rc = validate(s, q, k, v, idx, out);
   if (rc != QSA_OK) return rc;
   if (gathered != nullptr && s->topk > 0 && (reinterpret_cast<uintptr_t>(gathered) & 3u))
@@ -115,7 +215,29 @@ qsa_status_t run_forward(const qsa_shape_t* s, const void* q, const void* k, con
   p.scale_log2 = sc * 1.4426950408889634f;
   cudaError_t e;
   const bool dump = gathered != nullptr;
-  if (p.G <= 8)
+  static thread_local qsa::tc::TcParams tp;
+  const bool use_tc = which != QSA_KERNEL_WARP_MMA && make_tc_params(s, q, k, v, &tp);
+  if (which == QSA_KERNEL_TCGEN05 && !use_tc) return QSA_ERR_UNSUPPORTED;
+  if (use_tc) {
+    tp.idx = idx;
+    tp.n_valid = n_valid;
+    tp.out = p.out;
+    tp.lse = lse;
+    tp.status = status;
+    tp.gathered = gathered;
+    tp.T = p.T;
+    tp.idx_st = p.idx_st;
+    tp.idx_sh = p.idx_sh;
+    tp.o_st = p.o_st;
+    tp.o_sh = p.o_sh;
+    tp.lse_st = p.lse_st;
+    tp.Hkv = p.Hkv;
+    tp.G = p.G;
+    tp.K = p.K;
+    tp.S = static_cast<int32_t>(p.S);
+    tp.scale_log2 = p.scale_log2;
+    e = dump ? launch_tc<true>(tp, st) : launch_tc<false>(tp, st);
+  } else if (p.G <= 8)
     e = dump ? launch_mma<1, true>(p, st) : launch_mma<1, false>(p, st);
   else
     e = dump ? launch_mma<2, true>(p, st) : launch_mma<2, false>(p, st);
@@ -138,6 +260,15 @@ qsa_status_t qsa_sparse_prefill_fwd(const qsa_shape_t* shape, const void* q, con
                                     int32_t* status, void* stream) {
   return run_forward(shape, q, k_cache, v_cache, topk_idx, n_valid, scale, out, lse, status,
                      nullptr, stream);
+}
+
+qsa_status_t qsa_sparse_prefill_fwd_with(const qsa_shape_t* shape, const void* q,
+                                         const void* k_cache, const void* v_cache,
+                                         const int32_t* topk_idx, const int32_t* n_valid,
+                                         float scale, void* out, float* lse, int32_t* status,
+                                         qsa_kernel_t kernel, void* stream) {
+  return run_forward(shape, q, k_cache, v_cache, topk_idx, n_valid, scale, out, lse, status,
+                     nullptr, stream, kernel);
 }
 
 qsa_status_t qsa_sparse_prefill_debug_gather(const qsa_shape_t* shape, const void* q,

@@ -1,0 +1,579 @@
+// qsa_prefill_tc.cuh -- QSA top-K sparse-attention prefill, TMA-gather +
+// tcgen05 (TMEM) kernel for sm_100a.
+//
+// The operation (page "Qwen4-Exp QSA llega al Ascend de Huawei", section
+// "Lo que realmente añade la pull request"; bullets "Formas de cabeza" and
+// "Límites de tamaño"): for each (query token t, KV head g) unit, the G query
+// heads of the group attend to the cache rows named by the token's list,
+// softmax(scale q K_sel^T) V_sel, -1 / n_valid masking, zeros for empty rows.
+//
+// Persistent CTAs (one per SM) walk the units in KV-head-major order.  Six
+// warps with fixed roles, synchronised only through mbarriers:
+//   warp 0      producer: reads 128 list entries per tile and issues TMA
+//               tile::gather4 loads (4 rows x 128 B per instruction, 128-byte
+//               swizzle) of the K and V rows into a ring of six 32 KB slots
+//               (K dims 0-127, K dims 128-255, V dims 0-127, V dims 128-255);
+//               masked entries use an out-of-range row so the TMA zero-fills
+//               them without reading memory.  Also loads the 16 Q rows of
+//               the unit (TMA, double-buffered).
+//   warp 1      one thread issues tcgen05.mma:
+//                 scores  S^T[128 keys x 16 heads] = K_tile . Q^T  (M=128,
+//                         N=16, K-major operands) into a TMEM double buffer;
+//                 PV      O^T[256 x 16] += V_tile^T . P^T  (two M=128 halves,
+//                         V read MN-major from the same slots) into TMEM.
+//   warps 2-5   softmax: thread k owns TMEM lane k = key k of the tile; tile
+//               max per head by a transposing shuffle reduction and a 4-warp
+//               exchange; exponentials in base 2; P^T written MN-major to
+//               shared memory; the running max is only raised (with an O
+//               rescale in TMEM) when a head's max grows by more than 2^8,
+//               which keeps every p <= 256 and the result exact up to rounding.
+//               Epilogue: lse = m + ln l, O / l -> BF16 rows, zeros for empty rows.
+// Every wait (all on mbarriers, including the exchanges inside the softmax
+// group) is bounded by 2 s of %globaltimer; on expiry the kernel raises status
+// bit 1, every role stops, in-flight copies and MMAs are drained and the TMEM
+// is released.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include <cstdint>
+
+#include "qsa_ptx.cuh"
+#include "qsa_tc_ptx.cuh"
+
+namespace qsa {
+namespace tc {
+
+constexpr int kKeys = 128;                 // list entries per tile (M of the score MMA)
+constexpr int kGp = 16;                    // query heads per group, padded (N)
+constexpr int kSlotBytes = 32768;          // 128 rows x 128 dims x 2 B
+constexpr int kSlots = 6;
+constexpr int kBlockBytes = 16384;         // 128 rows x 64 dims (one 128-byte swizzle column block)
+constexpr int kQBytes = kGp * 512;         // 16 rows x 256 dims x 2 B
+constexpr int kPBytes = kKeys * kGp * 2;   // 128 keys x 16 heads x 2 B
+constexpr int kMaxKvHeads = 16;
+constexpr int kThreads = 192;
+constexpr int kTmemCols = 64;              // S double buffer (2 x 16) + O (2 halves x 16)
+constexpr float kRescaleLog2 = 8.f;        // lazy-rescale threshold (p <= 2^8)
+
+constexpr int OFF_RING = 0;
+constexpr int OFF_Q = OFF_RING + kSlots * kSlotBytes;
+constexpr int OFF_P = OFF_Q + 2 * kQBytes;
+constexpr int OFF_RED = OFF_P + 2 * kPBytes;     // max[2][4][16] + sum[2][4][16] floats
+constexpr int OFF_BAR = OFF_RED + 1024;
+// barrier indices
+constexpr int B_FULL = 0, B_EMPTY = 6, B_SFULL = 12, B_SFREE = 14, B_PFULL = 16, B_PEMPTY = 18,
+              B_QFULL = 20, B_QEMPTY = 22, B_OFULL = 24, B_OEMPTY = 25, B_RMAX = 26, B_RSUM = 28,
+              B_DONE = 30, NUM_BARS = 31;
+constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;  // tmem base, abort flag
+constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + slack for 1024-byte alignment
+
+constexpr uint32_t kStatusOob = 1u, kStatusTimeout = 2u;
+
+struct TcParams {
+  CUtensorMap tm_q;                 // Q as [T][Hq][256], box 16 heads x 64 dims
+  CUtensorMap tm_k[kMaxKvHeads];    // per KV head: cache rows [S][256], box 1 x 64
+  CUtensorMap tm_v[kMaxKvHeads];
+  const int32_t* idx;
+  const int32_t* n_valid;
+  __nv_bfloat16* out;
+  float* lse;
+  int32_t* status;
+  int32_t* gathered;                // debug dump [T][Hkv][K] or nullptr
+  int64_t T;
+  int64_t idx_st, idx_sh, o_st, o_sh, lse_st;
+  int32_t Hkv, G, K, S;
+  float scale_log2;
+};
+
+// Instruction descriptors (kind::f16): FP32 accumulator, BF16 A and B,
+// N = 16 (bits 17-22 hold N/8), M = 128 (bits 24-28 hold M/16).
+constexpr uint32_t kIdescQK = (1u << 4) | (1u << 7) | (1u << 10) | (2u << 17) | (8u << 24);
+// PV: both operands MN-major (bits 15 and 16).
+constexpr uint32_t kIdescPV = kIdescQK | (1u << 15) | (1u << 16);
+
+struct Sync {
+  uint32_t bars;
+  volatile uint32_t* abort_flag;
+  int32_t* status;
+
+  __device__ uint32_t bar(int i) const { return bars + 8u * i; }
+
+  __device__ bool aborted() const { return *abort_flag != 0; }
+
+  __device__ void raise_abort() const {
+    *abort_flag = 1u;
+    if (status != nullptr) atomicOr(status, static_cast<int32_t>(kStatusTimeout));
+  }
+
+  // Bounded wait for the phase of parity `parity` of barrier i.
+  __device__ bool wait(int i, uint32_t parity) const {
+    const uint32_t b = bar(i);
+    if (mbar_try_wait(b, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    for (uint32_t it = 1;; ++it) {
+      if (mbar_try_wait(b, parity)) return true;
+      if ((it & 63u) == 0u) {
+        if (aborted()) return false;
+        if (globaltimer_ns() - t0 > 2000000000ull) {
+          raise_abort();
+          return false;
+        }
+      }
+    }
+  }
+
+  // Bounded wait that ignores the abort flag (used to drain in-flight copies).
+  __device__ void drain(int i, uint32_t parity) const {
+    const uint32_t b = bar(i);
+    const uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait(b, parity))
+      if (globaltimer_ns() - t0 > 2000000000ull) return;
+  }
+};
+
+struct Unit {
+  int64_t t;
+  int g;
+  int n_eff;
+  int n_tiles;
+};
+
+__device__ __forceinline__ Unit decode_unit(const TcParams& p, int64_t u) {
+  Unit r;
+  r.g = static_cast<int>(u / p.T);
+  r.t = u - static_cast<int64_t>(r.g) * p.T;
+  int n = p.K;
+  if (p.n_valid != nullptr) n = min(n, max(__ldg(p.n_valid + r.t * p.Hkv + r.g), 0));
+  r.n_eff = n;
+  r.n_tiles = (n + kKeys - 1) / kKeys;
+  return r;
+}
+
+// Reduce 16 per-lane values across the 32 lanes of a warp by exchanging
+// halves (16 shuffles instead of 80).  Lane l ends with the result for head
+// (l >> 1) & 15.
+template <bool kMax>
+__device__ __forceinline__ float xreduce16(const float (&v)[16], int lane) {
+  auto op = [](float a, float b) { return kMax ? fmaxf(a, b) : a + b; };
+  float a[8], b[4], c[2];
+  bool up = (lane & 16) != 0;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const float send = up ? v[j] : v[8 + j];
+    const float keep = up ? v[8 + j] : v[j];
+    a[j] = op(keep, __shfl_xor_sync(0xffffffffu, send, 16));
+  }
+  up = (lane & 8) != 0;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const float send = up ? a[j] : a[4 + j];
+    const float keep = up ? a[4 + j] : a[j];
+    b[j] = op(keep, __shfl_xor_sync(0xffffffffu, send, 8));
+  }
+  up = (lane & 4) != 0;
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+    const float send = up ? b[j] : b[2 + j];
+    const float keep = up ? b[2 + j] : b[j];
+    c[j] = op(keep, __shfl_xor_sync(0xffffffffu, send, 4));
+  }
+  up = (lane & 2) != 0;
+  float d = op(up ? c[1] : c[0], __shfl_xor_sync(0xffffffffu, up ? c[0] : c[1], 2));
+  d = op(d, __shfl_xor_sync(0xffffffffu, d, 1));
+  return d;
+}
+
+// ------------------------------------------------------------------ producer
+
+template <bool kDump>
+__device__ void producer_role(const TcParams& p, const Sync& sy, uint32_t sb, int lane) {
+  uint32_t c_slot = 0, c_unit = 0;
+  // per-slot / per-Q-buffer parity of the latest issued load, for draining
+  uint32_t pend_slot = 0, pend_par = 0, pend_q = 0, pend_qpar = 0;
+  const int64_t units = p.T * p.Hkv;
+  bool ok = true;
+  for (int64_t u = blockIdx.x; u < units && ok; u += gridDim.x) {
+    const Unit un = decode_unit(p, u);
+    const uint32_t qb = c_unit & 1u;
+    if (lane == 0) {
+      ok = sy.wait(B_QEMPTY + qb, ((c_unit >> 1) & 1u) ^ 1u);
+      if (ok) {
+        mbar_arrive_expect_tx(sy.bar(B_QFULL + qb), kQBytes);
+#pragma unroll
+        for (int b = 0; b < 4; ++b)
+          tma_load_3d(sb + OFF_Q + qb * kQBytes + b * (kQBytes / 4), &p.tm_q, b * 64, un.g * p.G,
+                      static_cast<int32_t>(un.t), sy.bar(B_QFULL + qb));
+        pend_q |= 1u << qb;
+        pend_qpar = (pend_qpar & ~(1u << qb)) | (((c_unit >> 1) & 1u) << qb);
+      }
+    }
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    ++c_unit;
+    const int32_t* list = p.idx + un.t * p.idx_st + static_cast<int64_t>(un.g) * p.idx_sh;
+    const CUtensorMap* mk = &p.tm_k[un.g];
+    const CUtensorMap* mv = &p.tm_v[un.g];
+    for (int i = 0; i < un.n_tiles && ok; ++i) {
+      // rows 4*lane .. 4*lane+3 of the tile
+      int32_t y[4];
+      bool bad_any = false;
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const int j = i * kKeys + 4 * lane + r;
+        const int32_t id = j < un.n_eff ? __ldg(list + j) : -1;
+        const bool bad = id >= p.S;
+        bad_any |= bad;
+        y[r] = (id < 0 || bad) ? p.S : id;  // row S is out of range: zero fill
+        if (kDump && j < p.K)
+          p.gathered[(un.t * p.Hkv + un.g) * static_cast<int64_t>(p.K) + j] = y[r] < p.S ? y[r] : -1;
+      }
+      if (bad_any && p.status != nullptr) atomicOr(p.status, static_cast<int32_t>(kStatusOob));
+#pragma unroll 1
+      for (int h = 0; h < 4 && ok; ++h) {
+        const uint32_t slot = c_slot % kSlots;
+        const uint32_t round = c_slot / kSlots;
+        if (lane == 0) {
+          ok = sy.wait(B_EMPTY + slot, (round & 1u) ^ 1u);
+          if (ok) mbar_arrive_expect_tx(sy.bar(B_FULL + slot), kSlotBytes);
+        }
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) break;
+        const CUtensorMap* map = h < 2 ? mk : mv;
+        const int cb0 = (h & 1) * 2;  // first 64-dim column block of this half
+#pragma unroll
+        for (int b = 0; b < 2; ++b)
+          tma_gather4(sb + OFF_RING + slot * kSlotBytes + b * kBlockBytes + lane * 4 * 128, map,
+                      (cb0 + b) * 64, y[0], y[1], y[2], y[3], sy.bar(B_FULL + slot));
+        pend_slot |= 1u << slot;
+        pend_par = (pend_par & ~(1u << slot)) | ((round & 1u) << slot);
+        ++c_slot;
+      }
+    }
+  }
+  if (!ok && lane == 0) {
+    // stop cleanly: wait (bounded) for every load this warp issued
+    for (int s = 0; s < kSlots; ++s)
+      if (pend_slot & (1u << s)) sy.drain(B_FULL + s, (pend_par >> s) & 1u);
+    for (int q = 0; q < 2; ++q)
+      if (pend_q & (1u << q)) sy.drain(B_QFULL + q, (pend_qpar >> q) & 1u);
+  }
+}
+
+// ------------------------------------------------------------------ MMA issuer
+
+__device__ void mma_role(const TcParams& p, const Sync& sy, uint32_t sb, uint32_t tmem) {
+  uint32_t c_slot = 0, c_tile = 0, c_unit = 0;
+  const int64_t units = p.T * p.Hkv;
+  bool ok = true;
+  const uint32_t t_s = tmem;          // S buffers: columns 0-15, 16-31
+  const uint32_t t_o = tmem + 32;     // O halves: columns 32-47, 48-63
+
+  // PV for tile index `c` (ring slots start at c_slot0), first = first tile of the unit.
+  auto pv = [&](uint32_t c, uint32_t slot0, bool first, uint32_t unit_idx) -> bool {
+    const uint32_t pb = c & 1u;
+    if (!sy.wait(B_PFULL + pb, (c >> 1) & 1u)) return false;
+    if (first && !sy.wait(B_OEMPTY, (unit_idx & 1u) ^ 1u)) return false;
+#pragma unroll 1
+    for (int mh = 0; mh < 2; ++mh) {
+      const uint32_t cv = slot0 + 2 + mh;
+      const uint32_t slot = cv % kSlots;
+      if (!sy.wait(B_FULL + slot, (cv / kSlots) & 1u)) return false;
+      tc_fence_after();
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        // A = V^T: MN-major, 128-byte swizzle; the two 64-dim blocks of the
+        // half are 16 KB apart (LBO), groups of 8 keys 1 KB apart (SBO).
+        const uint64_t a = smem_desc(sb + OFF_RING + slot * kSlotBytes + kk * 2048, kBlockBytes, 1024, 2);
+        // B = P^T: MN-major, no swizzle; 8x8 core matrices, keys groups 128 B
+        // apart (LBO), head groups 2 KB apart (SBO).
+        const uint64_t b = smem_desc(sb + OFF_P + pb * kPBytes + kk * 256, 128, 2048, 0);
+        umma_f16_ss(t_o + mh * 16, a, b, kIdescPV, (first && kk == 0) ? 0u : 1u);
+      }
+      umma_commit(sy.bar(B_EMPTY + slot));
+    }
+    umma_commit(sy.bar(B_PEMPTY + pb));
+    return true;
+  };
+
+  for (int64_t u = blockIdx.x; u < units && ok; u += gridDim.x) {
+    const Unit un = decode_unit(p, u);
+    const uint32_t qb = c_unit & 1u;
+    ok = sy.wait(B_QFULL + qb, (c_unit >> 1) & 1u);
+    if (!ok) break;
+    if (un.n_tiles == 0) {
+      mbar_arrive(sy.bar(B_QEMPTY + qb));
+      ok = sy.wait(B_OEMPTY, (c_unit & 1u) ^ 1u);
+      if (ok) mbar_arrive(sy.bar(B_OFULL));
+      ++c_unit;
+      continue;
+    }
+    const uint32_t qaddr = sb + OFF_Q + qb * kQBytes;
+    for (int i = 0; i < un.n_tiles && ok; ++i) {
+      const uint32_t c = c_tile + i;
+      const uint32_t sbuf = c & 1u;
+      const uint32_t slot0 = c_slot + 4u * i;
+      ok = sy.wait(B_SFREE + sbuf, ((c >> 1) & 1u) ^ 1u);
+      for (int h = 0; h < 2 && ok; ++h) {
+        const uint32_t ck = slot0 + h;
+        const uint32_t slot = ck % kSlots;
+        ok = sy.wait(B_FULL + slot, (ck / kSlots) & 1u);
+        if (!ok) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const int ks = h * 8 + kk;
+          // A = K tile, B = Q: K-major, 128-byte swizzle, 8-row groups 1 KB
+          // apart; a 16-dim step advances 32 B inside the swizzle atom.
+          const uint64_t a = smem_desc(
+              sb + OFF_RING + slot * kSlotBytes + (kk >> 2) * kBlockBytes + (kk & 3) * 32, 16, 1024, 2);
+          const uint64_t b = smem_desc(qaddr + (ks >> 2) * (kQBytes / 4) + (ks & 3) * 32, 16, 1024, 2);
+          umma_f16_ss(t_s + sbuf * 16, a, b, kIdescQK, ks > 0 ? 1u : 0u);
+        }
+        umma_commit(sy.bar(B_EMPTY + slot));
+      }
+      if (!ok) break;
+      umma_commit(sy.bar(B_SFULL + sbuf));
+      if (i == un.n_tiles - 1) umma_commit(sy.bar(B_QEMPTY + qb));
+      if (i > 0) ok = pv(c - 1, slot0 - 4, i == 1, c_unit);
+    }
+    if (ok) ok = pv(c_tile + un.n_tiles - 1, c_slot + 4u * (un.n_tiles - 1), un.n_tiles == 1, c_unit);
+    if (ok) umma_commit(sy.bar(B_OFULL));
+    c_tile += un.n_tiles;
+    c_slot += 4u * un.n_tiles;
+    ++c_unit;
+  }
+  // no tensor-core operation may still be running when the CTA releases TMEM
+  umma_commit(sy.bar(B_DONE));
+  sy.drain(B_DONE, 0);
+}
+
+// ------------------------------------------------------------------ softmax
+
+__device__ void softmax_role(const TcParams& p, const Sync& sy, uint32_t sb, uint8_t* sp,
+                             uint32_t tmem, int warp, int lane) {
+  const int wq = warp & 3;                       // TMEM lane quadrant of this warp
+  const int key = wq * 32 + lane;                // TMEM lane = key row of the tile
+  const uint32_t tl = tmem + (static_cast<uint32_t>(wq * 32) << 16);
+  float* red_max = reinterpret_cast<float*>(sp + OFF_RED);        // [2][4][16]
+  float* red_sum = red_max + 128;                                  // [2][4][16]
+  uint32_t c_tile = 0, c_unit = 0;
+  const int64_t units = p.T * p.Hkv;
+  const int G = p.G;
+  bool ok = true;
+  for (int64_t u = blockIdx.x; u < units && ok; u += gridDim.x) {
+    const Unit un = decode_unit(p, u);
+    const int32_t* list = p.idx + un.t * p.idx_st + static_cast<int64_t>(un.g) * p.idx_sh;
+    float m_run[kGp], l_part[kGp];
+#pragma unroll
+    for (int h = 0; h < kGp; ++h) {
+      m_run[h] = -INFINITY;
+      l_part[h] = 0.f;
+    }
+    for (int i = 0; i < un.n_tiles; ++i) {
+      const uint32_t c = c_tile + i;
+      const uint32_t buf = c & 1u;
+      const int j = i * kKeys + key;
+      const int32_t id = j < un.n_eff ? __ldg(list + j) : -1;
+      const bool valid = id >= 0 && id < p.S;
+      ok = sy.wait(B_SFULL + buf, (c >> 1) & 1u);
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t r[16];
+      tmem_ld16(tl + buf * 16, r);
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(sy.bar(B_SFREE + buf));
+      float s[kGp];
+#pragma unroll
+      for (int h = 0; h < kGp; ++h)
+        s[h] = (valid && h < G) ? __uint_as_float(r[h]) * p.scale_log2 : -INFINITY;
+      // tile max per head over the 128 keys
+      const float wmax = xreduce16<true>(s, lane);
+      float* rm = red_max + buf * 64;
+      if ((lane & 1) == 0) rm[wq * 16 + ((lane >> 1) & 15)] = wmax;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(sy.bar(B_RMAX + buf));
+      ok = sy.wait(B_RMAX + buf, (c >> 1) & 1u);  // all four warps' maxima are in
+      if (!ok) break;
+      float tmax[kGp];
+#pragma unroll
+      for (int h = 0; h < kGp; ++h)
+        tmax[h] = fmaxf(fmaxf(rm[h], rm[16 + h]), fmaxf(rm[32 + h], rm[48 + h]));
+      bool need = false;
+#pragma unroll
+      for (int h = 0; h < kGp; ++h)
+        need |= (m_run[h] != -INFINITY) && (tmax[h] > m_run[h] + kRescaleLog2);
+      if (need) {
+        // raise the running max: O (TMEM) and the partial sums scale by 2^(m_old - m_new)
+        if (i > 0) {
+          const uint32_t cp = c - 1;
+          ok = sy.wait(B_PEMPTY + (cp & 1u), (cp >> 1) & 1u);  // the previous PV has finished
+          if (!ok) break;
+        }
+        tc_fence_after();
+        float alpha[kGp];
+#pragma unroll
+        for (int h = 0; h < kGp; ++h) {
+          const float mn = fmaxf(m_run[h], tmax[h]);
+          alpha[h] = m_run[h] == -INFINITY ? 1.f : ex2(m_run[h] - mn);
+          m_run[h] = mn;
+          l_part[h] *= alpha[h];
+        }
+        if (i > 0) {
+#pragma unroll
+          for (int half = 0; half < 2; ++half) {
+            uint32_t o[16];
+            tmem_ld16(tl + 32 + half * 16, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int h = 0; h < kGp; ++h) o[h] = __float_as_uint(__uint_as_float(o[h]) * alpha[h]);
+            tmem_st16(tl + 32 + half * 16, o);
+          }
+          tmem_wait_st();
+        }
+      } else {
+#pragma unroll
+        for (int h = 0; h < kGp; ++h)
+          if (m_run[h] == -INFINITY) m_run[h] = tmax[h];
+      }
+      uint32_t pk[8];
+#pragma unroll
+      for (int h = 0; h < kGp; h += 2) {
+        const float p0 = ex2(s[h] - (m_run[h] == -INFINITY ? 0.f : m_run[h]));
+        const float p1 = ex2(s[h + 1] - (m_run[h + 1] == -INFINITY ? 0.f : m_run[h + 1]));
+        l_part[h] += p0;
+        l_part[h + 1] += p1;
+        pk[h >> 1] = pack_bf16x2(p0, p1);
+      }
+      ok = sy.wait(B_PEMPTY + buf, ((c >> 1) & 1u) ^ 1u);
+      if (!ok) break;
+      // P^T row of this key: heads 0-7 in the first 8x8 core-matrix column,
+      // heads 8-15 in the second (2 KB further)
+      const uint32_t pa = sb + OFF_P + buf * kPBytes + (key >> 3) * 128 + (key & 7) * 16;
+      st_shared_v4(pa, pk[0], pk[1], pk[2], pk[3]);
+      st_shared_v4(pa + 2048, pk[4], pk[5], pk[6], pk[7]);
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(sy.bar(B_PFULL + buf));
+    }
+    if (!ok) break;
+    // epilogue: l per head over the 128 threads
+    const float wsum = xreduce16<false>(l_part, lane);
+    float* rs = red_sum + (c_unit & 1u) * 64;
+    if ((lane & 1) == 0) rs[wq * 16 + ((lane >> 1) & 15)] = wsum;
+    __syncwarp();
+    if (lane == 0) mbar_arrive(sy.bar(B_RSUM + (c_unit & 1u)));
+    ok = sy.wait(B_RSUM + (c_unit & 1u), (c_unit >> 1) & 1u);
+    if (!ok) break;
+    float l_tot[kGp];
+#pragma unroll
+    for (int h = 0; h < kGp; ++h) l_tot[h] = (rs[h] + rs[16 + h]) + (rs[32 + h] + rs[48 + h]);
+    ok = sy.wait(B_OFULL, c_unit & 1u);
+    if (!ok) break;
+    tc_fence_after();
+    uint32_t o0[16] = {}, o1[16] = {};
+    if (un.n_tiles > 0) {
+      tmem_ld16(tl + 32, o0);
+      tmem_ld16(tl + 48, o1);
+      tmem_wait_ld();
+    }
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(sy.bar(B_OEMPTY));
+    __nv_bfloat16* orow = p.out + un.t * p.o_st + static_cast<int64_t>(un.g) * G * p.o_sh;
+#pragma unroll
+    for (int h = 0; h < kGp; ++h) {
+      if (h < G) {
+        const bool live = l_tot[h] > 0.f;
+        const float inv = live ? 1.f / l_tot[h] : 0.f;
+        const float v0 = live ? __uint_as_float(o0[h]) * inv : 0.f;
+        const float v1 = live ? __uint_as_float(o1[h]) * inv : 0.f;
+        orow[h * p.o_sh + key] = __float2bfloat16_rn(v0);
+        orow[h * p.o_sh + 128 + key] = __float2bfloat16_rn(v1);
+      }
+    }
+    if (p.lse != nullptr && key < G) {
+      float mk = 0.f, lk = 0.f;
+#pragma unroll
+      for (int h = 0; h < kGp; ++h)
+        if (h == key) {
+          mk = m_run[h];
+          lk = l_tot[h];
+        }
+      p.lse[un.t * p.lse_st + static_cast<int64_t>(un.g) * G + key] =
+          lk > 0.f ? (mk + lg2(lk)) * 0.69314718055994531f : -INFINITY;
+    }
+    c_tile += un.n_tiles;
+    ++c_unit;
+  }
+}
+
+// ------------------------------------------------------------------ kernel
+
+template <bool kDump>
+__global__ void __launch_bounds__(kThreads, 1) qsa_prefill_tc_kernel(const __grid_constant__ TcParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t sb = (raw + 1023u) & ~1023u;
+  uint8_t* sp = smem_raw + (sb - raw);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  Sync sy;
+  sy.bars = sb + OFF_BAR;
+  sy.abort_flag = reinterpret_cast<volatile uint32_t*>(sp + OFF_MISC + 4);
+  sy.status = p.status;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kSlots; ++s) {
+      mbar_init(sy.bar(B_FULL + s), 1);
+      mbar_init(sy.bar(B_EMPTY + s), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(sy.bar(B_SFULL + b), 1);
+      mbar_init(sy.bar(B_SFREE + b), 4);
+      mbar_init(sy.bar(B_PFULL + b), 4);
+      mbar_init(sy.bar(B_PEMPTY + b), 1);
+      mbar_init(sy.bar(B_QFULL + b), 1);
+      mbar_init(sy.bar(B_QEMPTY + b), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(sy.bar(B_RMAX + b), 4);
+      mbar_init(sy.bar(B_RSUM + b), 4);
+    }
+    mbar_init(sy.bar(B_OFULL), 1);
+    mbar_init(sy.bar(B_OEMPTY), 4);
+    mbar_init(sy.bar(B_DONE), 1);
+    *sy.abort_flag = 0u;
+    mbar_fence_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tensormap(&p.tm_q);
+  }
+  if (warp == 1) {
+    tmem_alloc(sb + OFF_MISC, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(sp + OFF_MISC);
+
+  if (warp == 0) {
+    producer_role<kDump>(p, sy, sb, lane);
+  } else if (warp == 1) {
+    if (lane == 0) mma_role(p, sy, sb, tmem);
+    __syncwarp();
+  } else {
+    softmax_role(p, sy, sb, sp, tmem, warp, lane);
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, kTmemCols);
+}
+
+}  // namespace tc
+}  // namespace qsa
