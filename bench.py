@@ -44,6 +44,8 @@ METRIC = "QSA sparse prefill query-tokens/s and gathered-KV GB/s (% of B200 roof
 UNIT = "tokens/s"
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
+KERNEL_NAMES = {"auto": "qsa_prefill_tc_kernel", "tcgen05": "qsa_prefill_tc_kernel",
+                "warp_mma": "qsa_prefill_mma_kernel"}
 
 
 def parse_args():
@@ -56,6 +58,9 @@ def parse_args():
                     choices=["tiny", "c2", "c3", "c4", "c5", "pages_long"])
     ap.add_argument("--secondary", default="c4",
                     help="second workload reported under 'secondary' ('' to skip)")
+    ap.add_argument("--kernel", default="auto", choices=["auto", "tcgen05", "warp_mma"])
+    ap.add_argument("--compare", default="warp_mma",
+                    help="second kernel timed on the same workload ('' to skip)")
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -355,7 +360,7 @@ def run_cuda(args):
 
     def step():
         _capi.sparse_prefill_fwd(w.q, w.k_cache, w.v_cache, w.topk_idx, w.n_valid, w.scale,
-                                 out=out, lse=lse, status=status)
+                                 out=out, lse=lse, status=status, kernel=args.kernel)
 
     sampler = None
     if not args.profile:
@@ -375,7 +380,7 @@ def run_cuda(args):
     roof = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
             "frac": achieved / hbm, "traffic": traffic,
             "peak_source": peak_src + " (hbm_gbs, STREAM-style copy)",
-            "kernel": "qsa_prefill_mma_kernel", "algo_bytes_per_launch": acct["algo_bytes"],
+            "kernel": KERNEL_NAMES[args.kernel], "algo_bytes_per_launch": acct["algo_bytes"],
             "mean_launch_ms": mean_launch_ms}
     gathered_gbs = acct["gathered_bytes"] / (mean_launch_ms / 1e3) / 1e9
     tflops = acct["flops"] / (mean_launch_ms / 1e3) / 1e12
@@ -390,10 +395,22 @@ def run_cuda(args):
     if int(status.item()) != 0:
         line["status_word"] = int(status.item())
 
+    if args.compare and not args.profile and args.compare != args.kernel:
+        def step_cmp():
+            _capi.sparse_prefill_fwd(w.q, w.k_cache, w.v_cache, w.topk_idx, w.n_valid, w.scale,
+                                     out=out, lse=lse, kernel=args.compare)
+        cmp_ms, cmp_per, _ = time_launches(step_cmp, min(args.steps, 20), 3, barrier, "compare")
+        cmp_ms = max_over_ranks(cmp_ms)
+        n_cmp = min(args.steps, 20)
+        line["compare"] = {"kernel": KERNEL_NAMES[args.compare],
+                           "tokens_per_s": T * n_cmp * world / (cmp_ms / 1e3),
+                           "mean_launch_ms": statistics.mean(cmp_per),
+                           "algo_gbs": acct["algo_bytes"] / (statistics.mean(cmp_per) / 1e3) / 1e9}
     if not args.no_e2e and not args.profile:
         line["e2e"] = run_e2e(w, args, barrier, max_over_ranks, world, dev)
     if args.secondary and not args.profile and args.secondary != args.workload:
-        line["secondary"] = run_secondary(args.secondary, dev, barrier, max_over_ranks, world, hbm, bf16)
+        line["secondary"] = run_secondary(args.secondary, dev, barrier, max_over_ranks, world, hbm,
+                                          bf16, args.kernel)
     if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.profile:
         line["cpu_baseline"] = time_oracle(w, args.cpu_budget)
     elif not args.profile:
@@ -436,7 +453,7 @@ def run_e2e(w, args, barrier, max_over_ranks, world, dev):
             "api": "qsa_sparse_prefill_fwd_host (pinned host buffers)"}
 
 
-def run_secondary(name, dev, barrier, max_over_ranks, world, hbm, bf16):
+def run_secondary(name, dev, barrier, max_over_ranks, world, hbm, bf16, kernel="auto"):
     from top_sparse_attention_qsa_b200 import _capi
     w = make_workload(name, dev)
     acct = workload_accounting(w)
@@ -445,7 +462,7 @@ def run_secondary(name, dev, barrier, max_over_ranks, world, hbm, bf16):
 
     def step():
         _capi.sparse_prefill_fwd(w.q, w.k_cache, w.v_cache, w.topk_idx, w.n_valid, w.scale,
-                                 out=out, lse=lse)
+                                 out=out, lse=lse, kernel=kernel)
 
     steps = 20
     total_ms, per_ms, _ = time_launches(step, steps, 3, barrier, "secondary")

@@ -104,11 +104,11 @@ qsa_status_t qsa_sparse_prefill_fwd(const qsa_shape_t* shape, const void* q,
 
 /* Kernel choice for qsa_sparse_prefill_fwd_with. */
 typedef enum {
-  QSA_KERNEL_AUTO = 0,      /* TMA + tcgen05 kernel when TMA descriptors can express
-                               the layout (Hkv <= 16, slot stride >= 256 elements,
-                               K > 0, 0 < S < 2^31 - 1), otherwise the warp-MMA kernel */
-  QSA_KERNEL_TCGEN05 = 1,   /* persistent TMA-gather + tcgen05/TMEM kernel only
-                               (QSA_ERR_UNSUPPORTED when the layout does not fit) */
+  QSA_KERNEL_AUTO = 0,      /* the tcgen05 kernel when a TMA descriptor can express the
+                               Q layout and there is something to gather (K > 0,
+                               0 < S < 2^31 - 1), otherwise the warp-MMA kernel */
+  QSA_KERNEL_TCGEN05 = 1,   /* persistent warp-specialised cp.async-gather + tcgen05/TMEM
+                               kernel only (QSA_ERR_UNSUPPORTED when the layout does not fit) */
   QSA_KERNEL_WARP_MMA = 2   /* cp.async-gather + mma.sync kernel (any valid layout) */
 } qsa_kernel_t;
 

@@ -109,33 +109,15 @@ int sm_count() {
   return n;
 }
 
-// Fills the tensor maps of the TMA kernel.  Returns false when a TMA
-// descriptor cannot express the layout (the warp-MMA kernel takes those).
-bool make_tc_params(const qsa_shape_t* s, const void* q, const void* k, const void* v,
-                    qsa::tc::TcParams* tp) {
+// Fills the Q tensor map of the tcgen05 kernel.  Returns false when a TMA
+// descriptor cannot express the Q layout or there is nothing to gather (the
+// warp-MMA kernel takes those calls).
+bool make_tc_params(const qsa_shape_t* s, const void* q, qsa::tc::TcParams* tp) {
   using namespace qsa::tc;
   EncodeTiledFn enc = encode_fn();
   if (enc == nullptr) return false;
-  if (s->num_kv_heads > kMaxKvHeads || s->topk <= 0 || s->num_slots <= 0 ||
-      s->num_slots >= 0x7fffffffLL)
-    return false;
-  const uint64_t row_bytes = static_cast<uint64_t>(s->kv_stride_slot) * 2;
-  if (s->num_slots > 1 && row_bytes < 512) return false;
+  if (s->topk <= 0 || s->num_slots <= 0 || s->num_slots >= 0x7fffffffLL) return false;
   const cuuint32_t elem_str[3] = {1, 1, 1};
-  for (int g = 0; g < s->num_kv_heads; ++g) {
-    const cuuint64_t dims[2] = {256, static_cast<cuuint64_t>(s->num_slots)};
-    const cuuint64_t strides[1] = {s->num_slots > 1 ? row_bytes : 512};
-    const cuuint32_t box[2] = {64, 1};
-    for (int which = 0; which < 2; ++which) {
-      const char* base = static_cast<const char*>(which == 0 ? k : v) +
-                         static_cast<int64_t>(g) * s->kv_stride_head * 2;
-      CUtensorMap* m = which == 0 ? &tp->tm_k[g] : &tp->tm_v[g];
-      if (enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<char*>(base), dims, strides, box,
-              elem_str, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-        return false;
-    }
-  }
   const uint64_t hq = static_cast<uint64_t>(s->num_q_heads);
   uint64_t st_h = static_cast<uint64_t>(s->q_stride_head) * 2;
   if (hq == 1 || st_h < 512) {
@@ -150,11 +132,9 @@ bool make_tc_params(const qsa_shape_t* s, const void* q, const void* k, const vo
   const cuuint64_t qdims[3] = {256, hq, static_cast<cuuint64_t>(s->num_tokens)};
   const cuuint64_t qstr[2] = {st_h, st_t};
   const cuuint32_t qbox[3] = {64, static_cast<cuuint32_t>(kGp), 1};
-  if (enc(&tp->tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(q), qdims, qstr, qbox,
-          elem_str, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-    return false;
-  return true;
+  return enc(&tp->tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(q), qdims, qstr, qbox,
+             elem_str, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 template <bool kDump>
@@ -216,11 +196,15 @@ qsa_status_t run_forward(const qsa_shape_t* s, const void* q, const void* k, con
   cudaError_t e;
   const bool dump = gathered != nullptr;
   static thread_local qsa::tc::TcParams tp;
-  const bool use_tc = which != QSA_KERNEL_WARP_MMA && make_tc_params(s, q, k, v, &tp);
+  const bool use_tc = which != QSA_KERNEL_WARP_MMA && make_tc_params(s, q, &tp);
   if (which == QSA_KERNEL_TCGEN05 && !use_tc) return QSA_ERR_UNSUPPORTED;
   if (use_tc) {
     tp.idx = idx;
     tp.n_valid = n_valid;
+    tp.kraw = k;
+    tp.vraw = v;
+    tp.kv_ss = s->kv_stride_slot;
+    tp.kv_sh = s->kv_stride_head;
     tp.out = p.out;
     tp.lse = lse;
     tp.status = status;

@@ -7,20 +7,24 @@
 // heads of the group attend to the cache rows named by the token's list,
 // softmax(scale q K_sel^T) V_sel, -1 / n_valid masking, zeros for empty rows.
 //
-// Persistent CTAs (one per SM) walk the units in KV-head-major order.  Six
+// Persistent CTAs (one per SM) walk the units in KV-head-major order.  Seven
 // warps with fixed roles, synchronised only through mbarriers:
-//   warp 0      producer: reads 128 list entries per tile and issues TMA
-//               tile::gather4 loads (4 rows x 128 B per instruction, 128-byte
-//               swizzle) of the K and V rows into a ring of six 32 KB slots
-//               (K dims 0-127, K dims 128-255, V dims 0-127, V dims 128-255);
-//               masked entries use an out-of-range row so the TMA zero-fills
-//               them without reading memory.  Also loads the 16 Q rows of
-//               the unit (TMA, double-buffered).
-//   warp 1      one thread issues tcgen05.mma:
-//                 scores  S^T[128 keys x 16 heads] = K_tile . Q^T  (M=128,
-//                         N=16, K-major operands) into a TMEM double buffer;
-//                 PV      O^T[256 x 16] += V_tile^T . P^T  (two M=128 halves,
-//                         V read MN-major from the same slots) into TMEM.
+//   warp 0      producer: reads the 128 list entries of a tile two tiles
+//               ahead of its loads and asks L2 for those K and V rows (bulk
+//               prefetch), so the loads into shared memory meet L2 latency;
+//               then issues TMA tile::gather4 loads (4 rows x 128 B per
+//               instruction, 128-byte swizzle) of the K and V rows into a ring
+//               of six 32 KB slots (K dims 0-127, K dims 128-255, V dims 0-127,
+//               V dims 128-255); masked entries use an out-of-range row so the
+//               TMA zero-fills them without reading memory.  Also loads the 16
+//               Q rows of the unit (TMA, double-buffered).
+//   warp 1      one thread issues the score MMAs (tcgen05.mma, kind::f16):
+//               S^T[128 keys x 16 heads] = K_tile . Q^T (M=128, N=16, K-major
+//               operands) into a TMEM double buffer.
+//   warp 6      one thread issues the PV MMAs: O^T[256 x 16] += V_tile^T . P^T
+//               (two M=128 halves, V read MN-major from the same slots) into
+//               TMEM.  Two issuers keep PV of tile i from queueing behind the
+//               scores of tile i+1.
 //   warps 2-5   softmax: thread k owns TMEM lane k = key k of the tile; tile
 //               max per head by a transposing shuffle reduction and a 4-warp
 //               exchange; exponentials in base 2; P^T written MN-major to
@@ -52,8 +56,9 @@ constexpr int kSlots = 6;
 constexpr int kBlockBytes = 16384;         // 128 rows x 64 dims (one 128-byte swizzle column block)
 constexpr int kQBytes = kGp * 512;         // 16 rows x 256 dims x 2 B
 constexpr int kPBytes = kKeys * kGp * 2;   // 128 keys x 16 heads x 2 B
-constexpr int kMaxKvHeads = 16;
-constexpr int kThreads = 192;
+constexpr int kProducerWarps = 4;
+constexpr int kWarpQK = kProducerWarps, kWarpPV = kProducerWarps + 1, kWarpSoftmax0 = kProducerWarps + 2;
+constexpr int kThreads = 32 * (kProducerWarps + 6);
 constexpr int kTmemCols = 64;              // S double buffer (2 x 16) + O (2 halves x 16)
 constexpr float kRescaleLog2 = 8.f;        // lazy-rescale threshold (p <= 2^8)
 
@@ -65,7 +70,7 @@ constexpr int OFF_BAR = OFF_RED + 1024;
 // barrier indices
 constexpr int B_FULL = 0, B_EMPTY = 6, B_SFULL = 12, B_SFREE = 14, B_PFULL = 16, B_PEMPTY = 18,
               B_QFULL = 20, B_QEMPTY = 22, B_OFULL = 24, B_OEMPTY = 25, B_RMAX = 26, B_RSUM = 28,
-              B_DONE = 30, NUM_BARS = 31;
+              B_DONE = 30, NUM_BARS = 32;
 constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;  // tmem base, abort flag
 constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + slack for 1024-byte alignment
 
@@ -73,16 +78,16 @@ constexpr uint32_t kStatusOob = 1u, kStatusTimeout = 2u;
 
 struct TcParams {
   CUtensorMap tm_q;                 // Q as [T][Hq][256], box 16 heads x 64 dims
-  CUtensorMap tm_k[kMaxKvHeads];    // per KV head: cache rows [S][256], box 1 x 64
-  CUtensorMap tm_v[kMaxKvHeads];
   const int32_t* idx;
   const int32_t* n_valid;
+  const void* kraw;                 // K and V cache base pointers
+  const void* vraw;
   __nv_bfloat16* out;
   float* lse;
   int32_t* status;
   int32_t* gathered;                // debug dump [T][Hkv][K] or nullptr
   int64_t T;
-  int64_t idx_st, idx_sh, o_st, o_sh, lse_st;
+  int64_t idx_st, idx_sh, o_st, o_sh, lse_st, kv_ss, kv_sh;
   int32_t Hkv, G, K, S;
   float scale_log2;
 };
@@ -187,135 +192,107 @@ __device__ __forceinline__ float xreduce16(const float (&v)[16], int lane) {
 
 // ------------------------------------------------------------------ producer
 
+// kProducerWarps warps gather the K and V rows of each tile with 16-byte
+// cp.async copies written straight into the 128-byte-swizzled K-major layout
+// the tensor core reads.  Warp w owns rows 32w .. 32w+31 of every tile; one
+// warp instruction moves the 256-byte half rows of two keys (16 lanes each).
+// Masked entries are zero-filled without a global read.  Every lane signals
+// the slot's full barrier when its own copies land (cp.async.mbarrier.arrive).
 template <bool kDump>
-__device__ void producer_role(const TcParams& p, const Sync& sy, uint32_t sb, int lane) {
+__device__ void producer_role(const TcParams& p, const Sync& sy, uint32_t sb, int pw, int lane) {
   uint32_t c_slot = 0, c_unit = 0;
-  // per-slot / per-Q-buffer parity of the latest issued load, for draining
-  uint32_t pend_slot = 0, pend_par = 0, pend_q = 0, pend_qpar = 0;
   const int64_t units = p.T * p.Hkv;
+  const int cc = lane & 15;                          // 16-byte chunk of the half row
+  const int rsel = lane >> 4;                        // which of the two rows of an instruction
+  const uint32_t dchunk = static_cast<uint32_t>((cc >> 3) * kBlockBytes);
   bool ok = true;
   for (int64_t u = blockIdx.x; u < units && ok; u += gridDim.x) {
     const Unit un = decode_unit(p, u);
-    const uint32_t qb = c_unit & 1u;
-    if (lane == 0) {
-      ok = sy.wait(B_QEMPTY + qb, ((c_unit >> 1) & 1u) ^ 1u);
-      if (ok) {
-        mbar_arrive_expect_tx(sy.bar(B_QFULL + qb), kQBytes);
+    if (pw == 0) {
+      const uint32_t qb = c_unit & 1u;
+      if (lane == 0) {
+        ok = sy.wait(B_QEMPTY + qb, ((c_unit >> 1) & 1u) ^ 1u);
+        if (ok) {
+          mbar_arrive_expect_tx(sy.bar(B_QFULL + qb), kQBytes);
 #pragma unroll
-        for (int b = 0; b < 4; ++b)
-          tma_load_3d(sb + OFF_Q + qb * kQBytes + b * (kQBytes / 4), &p.tm_q, b * 64, un.g * p.G,
-                      static_cast<int32_t>(un.t), sy.bar(B_QFULL + qb));
-        pend_q |= 1u << qb;
-        pend_qpar = (pend_qpar & ~(1u << qb)) | (((c_unit >> 1) & 1u) << qb);
+          for (int b = 0; b < 4; ++b)
+            tma_load_3d(sb + OFF_Q + qb * kQBytes + b * (kQBytes / 4), &p.tm_q, b * 64, un.g * p.G,
+                        static_cast<int32_t>(un.t), sy.bar(B_QFULL + qb));
+        }
       }
+      ok = __shfl_sync(0xffffffffu, ok, 0);
     }
-    ok = __shfl_sync(0xffffffffu, ok, 0);
     ++c_unit;
+    if (!ok) break;
     const int32_t* list = p.idx + un.t * p.idx_st + static_cast<int64_t>(un.g) * p.idx_sh;
-    const CUtensorMap* mk = &p.tm_k[un.g];
-    const CUtensorMap* mv = &p.tm_v[un.g];
+    const char* kbase = reinterpret_cast<const char*>(p.kraw) + static_cast<int64_t>(un.g) * p.kv_sh * 2 + cc * 16;
+    const char* vbase = reinterpret_cast<const char*>(p.vraw) + static_cast<int64_t>(un.g) * p.kv_sh * 2 + cc * 16;
+    const int64_t row_bytes = p.kv_ss * 2;
+    // list entry of row 32*pw + lane, one tile ahead
+    const int jr = 32 * pw + lane;
+    int32_t id_next = (un.n_tiles > 0 && jr < un.n_eff) ? __ldg(list + jr) : -1;
     for (int i = 0; i < un.n_tiles && ok; ++i) {
-      // rows 4*lane .. 4*lane+3 of the tile
-      int32_t y[4];
-      bool bad_any = false;
-#pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        const int j = i * kKeys + 4 * lane + r;
-        const int32_t id = j < un.n_eff ? __ldg(list + j) : -1;
-        const bool bad = id >= p.S;
-        bad_any |= bad;
-        y[r] = (id < 0 || bad) ? p.S : id;  // row S is out of range: zero fill
-        if (kDump && j < p.K)
-          p.gathered[(un.t * p.Hkv + un.g) * static_cast<int64_t>(p.K) + j] = y[r] < p.S ? y[r] : -1;
+      int32_t id = id_next;
+      const int jn = (i + 1) * kKeys + jr;
+      id_next = (i + 1 < un.n_tiles && jn < un.n_eff) ? __ldg(list + jn) : -1;
+      const bool bad = id >= p.S;
+      if (bad) {
+        id = -1;
+        if (p.status != nullptr) atomicOr(p.status, static_cast<int32_t>(kStatusOob));
       }
-      if (bad_any && p.status != nullptr) atomicOr(p.status, static_cast<int32_t>(kStatusOob));
+      if (kDump) {
+        const int j = i * kKeys + jr;
+        if (j < p.K) p.gathered[(un.t * p.Hkv + un.g) * static_cast<int64_t>(p.K) + j] = id < 0 ? -1 : id;
+      }
 #pragma unroll 1
-      for (int h = 0; h < 4 && ok; ++h) {
+      for (int h = 0; h < 4; ++h) {
         const uint32_t slot = c_slot % kSlots;
         const uint32_t round = c_slot / kSlots;
-        if (lane == 0) {
-          ok = sy.wait(B_EMPTY + slot, (round & 1u) ^ 1u);
-          if (ok) mbar_arrive_expect_tx(sy.bar(B_FULL + slot), kSlotBytes);
-        }
-        ok = __shfl_sync(0xffffffffu, ok, 0);
+        ok = sy.wait(B_EMPTY + slot, (round & 1u) ^ 1u);
         if (!ok) break;
-        const CUtensorMap* map = h < 2 ? mk : mv;
-        const int cb0 = (h & 1) * 2;  // first 64-dim column block of this half
+        const char* src0 = (h < 2 ? kbase : vbase) + (h & 1) * 256;
+        const uint32_t dst0 = sb + OFF_RING + slot * kSlotBytes + dchunk;
 #pragma unroll
-        for (int b = 0; b < 2; ++b)
-          tma_gather4(sb + OFF_RING + slot * kSlotBytes + b * kBlockBytes + lane * 4 * 128, map,
-                      (cb0 + b) * 64, y[0], y[1], y[2], y[3], sy.bar(B_FULL + slot));
-        pend_slot |= 1u << slot;
-        pend_par = (pend_par & ~(1u << slot)) | ((round & 1u) << slot);
+        for (int k = 0; k < 16; ++k) {
+          const int r = 32 * pw + 2 * k + rsel;                   // row of the tile
+          const int32_t rid = __shfl_sync(0xffffffffu, id, 2 * k + rsel);
+          const bool live = rid >= 0;
+          const char* src = live ? src0 + static_cast<int64_t>(rid) * row_bytes : src0;
+          cp_async_16(dst0 + r * 128 + (((cc & 7) ^ (r & 7)) << 4), src, live ? 16 : 0);
+        }
+        cp_async_mbar_arrive(sy.bar(B_FULL + slot));
         ++c_slot;
       }
     }
   }
-  if (!ok && lane == 0) {
-    // stop cleanly: wait (bounded) for every load this warp issued
-    for (int s = 0; s < kSlots; ++s)
-      if (pend_slot & (1u << s)) sy.drain(B_FULL + s, (pend_par >> s) & 1u);
-    for (int q = 0; q < 2; ++q)
-      if (pend_q & (1u << q)) sy.drain(B_QFULL + q, (pend_qpar >> q) & 1u);
-  }
+  // every copy this lane issued has landed before the CTA can exit
+  asm volatile("cp.async.wait_all;\n" ::: "memory");
 }
 
-// ------------------------------------------------------------------ MMA issuer
+// ------------------------------------------------------------------ MMA issuers
 
-__device__ void mma_role(const TcParams& p, const Sync& sy, uint32_t sb, uint32_t tmem) {
-  uint32_t c_slot = 0, c_tile = 0, c_unit = 0;
+// Scores: S^T[c & 1] = K_tile(c) . Q^T for every tile c of the CTA.
+__device__ void qk_role(const TcParams& p, const Sync& sy, uint32_t sb, uint32_t tmem) {
+  uint32_t c_tile = 0, c_unit = 0;
   const int64_t units = p.T * p.Hkv;
   bool ok = true;
-  const uint32_t t_s = tmem;          // S buffers: columns 0-15, 16-31
-  const uint32_t t_o = tmem + 32;     // O halves: columns 32-47, 48-63
-
-  // PV for tile index `c` (ring slots start at c_slot0), first = first tile of the unit.
-  auto pv = [&](uint32_t c, uint32_t slot0, bool first, uint32_t unit_idx) -> bool {
-    const uint32_t pb = c & 1u;
-    if (!sy.wait(B_PFULL + pb, (c >> 1) & 1u)) return false;
-    if (first && !sy.wait(B_OEMPTY, (unit_idx & 1u) ^ 1u)) return false;
-#pragma unroll 1
-    for (int mh = 0; mh < 2; ++mh) {
-      const uint32_t cv = slot0 + 2 + mh;
-      const uint32_t slot = cv % kSlots;
-      if (!sy.wait(B_FULL + slot, (cv / kSlots) & 1u)) return false;
-      tc_fence_after();
-#pragma unroll
-      for (int kk = 0; kk < 8; ++kk) {
-        // A = V^T: MN-major, 128-byte swizzle; the two 64-dim blocks of the
-        // half are 16 KB apart (LBO), groups of 8 keys 1 KB apart (SBO).
-        const uint64_t a = smem_desc(sb + OFF_RING + slot * kSlotBytes + kk * 2048, kBlockBytes, 1024, 2);
-        // B = P^T: MN-major, no swizzle; 8x8 core matrices, keys groups 128 B
-        // apart (LBO), head groups 2 KB apart (SBO).
-        const uint64_t b = smem_desc(sb + OFF_P + pb * kPBytes + kk * 256, 128, 2048, 0);
-        umma_f16_ss(t_o + mh * 16, a, b, kIdescPV, (first && kk == 0) ? 0u : 1u);
-      }
-      umma_commit(sy.bar(B_EMPTY + slot));
-    }
-    umma_commit(sy.bar(B_PEMPTY + pb));
-    return true;
-  };
-
   for (int64_t u = blockIdx.x; u < units && ok; u += gridDim.x) {
     const Unit un = decode_unit(p, u);
     const uint32_t qb = c_unit & 1u;
     ok = sy.wait(B_QFULL + qb, (c_unit >> 1) & 1u);
     if (!ok) break;
+    ++c_unit;
     if (un.n_tiles == 0) {
       mbar_arrive(sy.bar(B_QEMPTY + qb));
-      ok = sy.wait(B_OEMPTY, (c_unit & 1u) ^ 1u);
-      if (ok) mbar_arrive(sy.bar(B_OFULL));
-      ++c_unit;
       continue;
     }
     const uint32_t qaddr = sb + OFF_Q + qb * kQBytes;
-    for (int i = 0; i < un.n_tiles && ok; ++i) {
-      const uint32_t c = c_tile + i;
+    for (int i = 0; i < un.n_tiles && ok; ++i, ++c_tile) {
+      const uint32_t c = c_tile;
       const uint32_t sbuf = c & 1u;
-      const uint32_t slot0 = c_slot + 4u * i;
       ok = sy.wait(B_SFREE + sbuf, ((c >> 1) & 1u) ^ 1u);
       for (int h = 0; h < 2 && ok; ++h) {
-        const uint32_t ck = slot0 + h;
+        const uint32_t ck = 4u * c + h;
         const uint32_t slot = ck % kSlots;
         ok = sy.wait(B_FULL + slot, (ck / kSlots) & 1u);
         if (!ok) break;
@@ -328,24 +305,65 @@ __device__ void mma_role(const TcParams& p, const Sync& sy, uint32_t sb, uint32_
           const uint64_t a = smem_desc(
               sb + OFF_RING + slot * kSlotBytes + (kk >> 2) * kBlockBytes + (kk & 3) * 32, 16, 1024, 2);
           const uint64_t b = smem_desc(qaddr + (ks >> 2) * (kQBytes / 4) + (ks & 3) * 32, 16, 1024, 2);
-          umma_f16_ss(t_s + sbuf * 16, a, b, kIdescQK, ks > 0 ? 1u : 0u);
+          umma_f16_ss(tmem + sbuf * 16, a, b, kIdescQK, ks > 0 ? 1u : 0u);
         }
         umma_commit(sy.bar(B_EMPTY + slot));
       }
       if (!ok) break;
       umma_commit(sy.bar(B_SFULL + sbuf));
       if (i == un.n_tiles - 1) umma_commit(sy.bar(B_QEMPTY + qb));
-      if (i > 0) ok = pv(c - 1, slot0 - 4, i == 1, c_unit);
     }
-    if (ok) ok = pv(c_tile + un.n_tiles - 1, c_slot + 4u * (un.n_tiles - 1), un.n_tiles == 1, c_unit);
-    if (ok) umma_commit(sy.bar(B_OFULL));
-    c_tile += un.n_tiles;
-    c_slot += 4u * un.n_tiles;
-    ++c_unit;
   }
-  // no tensor-core operation may still be running when the CTA releases TMEM
+  // no tensor-core operation of this thread may still run when TMEM is released
   umma_commit(sy.bar(B_DONE));
   sy.drain(B_DONE, 0);
+}
+
+// PV: O^T (two M=128 halves) += V_tile(c)^T . P^T(c) for every tile c.
+__device__ void pv_role(const TcParams& p, const Sync& sy, uint32_t sb, uint32_t tmem) {
+  uint32_t c_tile = 0, c_unit = 0;
+  const int64_t units = p.T * p.Hkv;
+  const uint32_t t_o = tmem + 32;  // O halves: columns 32-47 and 48-63
+  bool ok = true;
+  for (int64_t u = blockIdx.x; u < units && ok; u += gridDim.x) {
+    const Unit un = decode_unit(p, u);
+    const uint32_t ue = c_unit++;
+    // the previous unit's epilogue has read O
+    ok = sy.wait(B_OEMPTY, (ue & 1u) ^ 1u);
+    if (!ok) break;
+    if (un.n_tiles == 0) {
+      mbar_arrive(sy.bar(B_OFULL));
+      continue;
+    }
+    for (int i = 0; i < un.n_tiles && ok; ++i, ++c_tile) {
+      const uint32_t c = c_tile;
+      const uint32_t pb = c & 1u;
+      ok = sy.wait(B_PFULL + pb, (c >> 1) & 1u);
+      for (int mh = 0; mh < 2 && ok; ++mh) {
+        const uint32_t cv = 4u * c + 2 + mh;
+        const uint32_t slot = cv % kSlots;
+        ok = sy.wait(B_FULL + slot, (cv / kSlots) & 1u);
+        if (!ok) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          // A = V^T: MN-major, 128-byte swizzle; the two 64-dim blocks of the
+          // half are 16 KB apart (LBO), groups of 8 keys 1 KB apart (SBO).
+          const uint64_t a = smem_desc(sb + OFF_RING + slot * kSlotBytes + kk * 2048, kBlockBytes, 1024, 2);
+          // B = P^T: MN-major, no swizzle; 8x8 core matrices, key groups 128 B
+          // apart (LBO), head groups 2 KB apart (SBO).
+          const uint64_t b = smem_desc(sb + OFF_P + pb * kPBytes + kk * 256, 128, 2048, 0);
+          umma_f16_ss(t_o + mh * 16, a, b, kIdescPV, (i == 0 && kk == 0) ? 0u : 1u);
+        }
+        umma_commit(sy.bar(B_EMPTY + slot));
+      }
+      if (!ok) break;
+      umma_commit(sy.bar(B_PEMPTY + pb));
+    }
+    if (ok) umma_commit(sy.bar(B_OFULL));
+  }
+  umma_commit(sy.bar(B_DONE + 1));
+  sy.drain(B_DONE + 1, 0);
 }
 
 // ------------------------------------------------------------------ softmax
@@ -370,11 +388,14 @@ __device__ void softmax_role(const TcParams& p, const Sync& sy, uint32_t sb, uin
       m_run[h] = -INFINITY;
       l_part[h] = 0.f;
     }
+    // list entry of this thread's key, read one tile ahead
+    int32_t id_next = (un.n_tiles > 0 && key < un.n_eff) ? __ldg(list + key) : -1;
     for (int i = 0; i < un.n_tiles; ++i) {
       const uint32_t c = c_tile + i;
       const uint32_t buf = c & 1u;
-      const int j = i * kKeys + key;
-      const int32_t id = j < un.n_eff ? __ldg(list + j) : -1;
+      const int32_t id = id_next;
+      const int jn = (i + 1) * kKeys + key;
+      id_next = (i + 1 < un.n_tiles && jn < un.n_eff) ? __ldg(list + jn) : -1;
       const bool valid = id >= 0 && id < p.S;
       ok = sy.wait(B_SFULL + buf, (c >> 1) & 1u);
       if (!ok) break;
@@ -527,7 +548,7 @@ __global__ void __launch_bounds__(kThreads, 1) qsa_prefill_tc_kernel(const __gri
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kSlots; ++s) {
-      mbar_init(sy.bar(B_FULL + s), 1);
+      mbar_init(sy.bar(B_FULL + s), 32 * kProducerWarps);
       mbar_init(sy.bar(B_EMPTY + s), 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -545,13 +566,12 @@ __global__ void __launch_bounds__(kThreads, 1) qsa_prefill_tc_kernel(const __gri
     mbar_init(sy.bar(B_OFULL), 1);
     mbar_init(sy.bar(B_OEMPTY), 4);
     mbar_init(sy.bar(B_DONE), 1);
+    mbar_init(sy.bar(B_DONE + 1), 1);
     *sy.abort_flag = 0u;
     mbar_fence_init();
   }
-  if (warp == 0 && lane == 0) {
-    prefetch_tensormap(&p.tm_q);
-  }
-  if (warp == 1) {
+  if (warp == 0 && lane == 0) prefetch_tensormap(&p.tm_q);
+  if (warp == kWarpQK) {
     tmem_alloc(sb + OFF_MISC, kTmemCols);
     tmem_relinquish();
   }
@@ -560,10 +580,13 @@ __global__ void __launch_bounds__(kThreads, 1) qsa_prefill_tc_kernel(const __gri
   tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(sp + OFF_MISC);
 
-  if (warp == 0) {
-    producer_role<kDump>(p, sy, sb, lane);
-  } else if (warp == 1) {
-    if (lane == 0) mma_role(p, sy, sb, tmem);
+  if (warp < kProducerWarps) {
+    producer_role<kDump>(p, sy, sb, warp, lane);
+  } else if (warp == kWarpQK) {
+    if (lane == 0) qk_role(p, sy, sb, tmem);
+    __syncwarp();
+  } else if (warp == kWarpPV) {
+    if (lane == 0) pv_role(p, sy, sb, tmem);
     __syncwarp();
   } else {
     softmax_role(p, sy, sb, sp, tmem, warp, lane);
@@ -572,7 +595,7 @@ __global__ void __launch_bounds__(kThreads, 1) qsa_prefill_tc_kernel(const __gri
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 1) tmem_dealloc(tmem, kTmemCols);
+  if (warp == kWarpQK) tmem_dealloc(tmem, kTmemCols);
 }
 
 }  // namespace tc

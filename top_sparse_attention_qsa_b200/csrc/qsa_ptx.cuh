@@ -37,6 +37,12 @@ __device__ __forceinline__ uint64_t policy_evict_first() {
   return p;
 }
 
+// Arrive on an mbarrier once every cp.async this thread issued so far has
+// landed (the arrival is counted in the barrier's expected count).
+__device__ __forceinline__ void cp_async_mbar_arrive(uint32_t bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];\n" ::"r"(bar) : "memory");
+}
+
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
 
 template <int N>
