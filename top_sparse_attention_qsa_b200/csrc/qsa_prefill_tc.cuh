@@ -56,7 +56,12 @@ constexpr int kSlots = 6;
 constexpr int kBlockBytes = 16384;         // 128 rows x 64 dims (one 128-byte swizzle column block)
 constexpr int kQBytes = kGp * 512;         // 16 rows x 256 dims x 2 B
 constexpr int kPBytes = kKeys * kGp * 2;   // 128 keys x 16 heads x 2 B
-constexpr int kProducerWarps = 4;
+#ifndef QSA_TC_PRODUCER_WARPS
+#define QSA_TC_PRODUCER_WARPS 4
+#endif
+constexpr int kProducerWarps = QSA_TC_PRODUCER_WARPS;  // must divide 128 rows into 2-row steps
+static_assert(kKeys % (2 * kProducerWarps) == 0 && kKeys / kProducerWarps <= 32,
+              "each producer lane holds at most one row id; rows per warp must be even");
 constexpr int kWarpQK = kProducerWarps, kWarpPV = kProducerWarps + 1, kWarpSoftmax0 = kProducerWarps + 2;
 constexpr int kThreads = 32 * (kProducerWarps + 6);
 constexpr int kTmemCols = 64;              // S double buffer (2 x 16) + O (2 halves x 16)
@@ -194,8 +199,9 @@ __device__ __forceinline__ float xreduce16(const float (&v)[16], int lane) {
 
 // kProducerWarps warps gather the K and V rows of each tile with 16-byte
 // cp.async copies written straight into the 128-byte-swizzled K-major layout
-// the tensor core reads.  Warp w owns rows 32w .. 32w+31 of every tile; one
-// warp instruction moves the 256-byte half rows of two keys (16 lanes each).
+// the tensor core reads.  Warp w owns rows_w = 128 / kProducerWarps rows of
+// every tile; one warp instruction moves the 256-byte half rows of two keys
+// (16 lanes each).
 // Masked entries are zero-filled without a global read.  Every lane signals
 // the slot's full barrier when its own copies land (cp.async.mbarrier.arrive).
 template <bool kDump>
@@ -228,19 +234,21 @@ __device__ void producer_role(const TcParams& p, const Sync& sy, uint32_t sb, in
     const char* kbase = reinterpret_cast<const char*>(p.kraw) + static_cast<int64_t>(un.g) * p.kv_sh * 2 + cc * 16;
     const char* vbase = reinterpret_cast<const char*>(p.vraw) + static_cast<int64_t>(un.g) * p.kv_sh * 2 + cc * 16;
     const int64_t row_bytes = p.kv_ss * 2;
-    // list entry of row 32*pw + lane, one tile ahead
-    const int jr = 32 * pw + lane;
-    int32_t id_next = (un.n_tiles > 0 && jr < un.n_eff) ? __ldg(list + jr) : -1;
+    // list entry of this lane's row (rows_w rows per warp; lanes >= rows_w idle), one tile ahead
+    constexpr int rows_w = kKeys / kProducerWarps;
+    const int jr = rows_w * pw + lane;
+    const bool own = lane < rows_w;
+    int32_t id_next = (own && un.n_tiles > 0 && jr < un.n_eff) ? __ldg(list + jr) : -1;
     for (int i = 0; i < un.n_tiles && ok; ++i) {
       int32_t id = id_next;
       const int jn = (i + 1) * kKeys + jr;
-      id_next = (i + 1 < un.n_tiles && jn < un.n_eff) ? __ldg(list + jn) : -1;
+      id_next = (own && i + 1 < un.n_tiles && jn < un.n_eff) ? __ldg(list + jn) : -1;
       const bool bad = id >= p.S;
       if (bad) {
         id = -1;
         if (p.status != nullptr) atomicOr(p.status, static_cast<int32_t>(kStatusOob));
       }
-      if (kDump) {
+      if (kDump && own) {
         const int j = i * kKeys + jr;
         if (j < p.K) p.gathered[(un.t * p.Hkv + un.g) * static_cast<int64_t>(p.K) + j] = id < 0 ? -1 : id;
       }
@@ -253,8 +261,8 @@ __device__ void producer_role(const TcParams& p, const Sync& sy, uint32_t sb, in
         const char* src0 = (h < 2 ? kbase : vbase) + (h & 1) * 256;
         const uint32_t dst0 = sb + OFF_RING + slot * kSlotBytes + dchunk;
 #pragma unroll
-        for (int k = 0; k < 16; ++k) {
-          const int r = 32 * pw + 2 * k + rsel;                   // row of the tile
+        for (int k = 0; k < rows_w / 2; ++k) {
+          const int r = rows_w * pw + 2 * k + rsel;               // row of the tile
           const int32_t rid = __shfl_sync(0xffffffffu, id, 2 * k + rsel);
           const bool live = rid >= 0;
           const char* src = live ? src0 + static_cast<int64_t>(rid) * row_bytes : src0;
