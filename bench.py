@@ -61,6 +61,8 @@ def parse_args():
     ap.add_argument("--kernel", default="auto", choices=["auto", "tcgen05", "warp_mma"])
     ap.add_argument("--compare", default="warp_mma",
                     help="second kernel timed on the same workload ('' to skip)")
+    ap.add_argument("--decode", default="decode",
+                    help="decode workload timed under 'decode' ('' to skip)")
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -411,6 +413,8 @@ def run_cuda(args):
     if args.secondary and not args.profile and args.secondary != args.workload:
         line["secondary"] = run_secondary(args.secondary, dev, barrier, max_over_ranks, world, hbm,
                                           bf16, args.kernel)
+    if args.decode and not args.profile:
+        line["decode"] = run_decode_bench(args.decode, dev, barrier, max_over_ranks, world, hbm)
     if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.profile:
         line["cpu_baseline"] = time_oracle(w, args.cpu_budget)
     elif not args.profile:
@@ -474,6 +478,34 @@ def run_secondary(name, dev, barrier, max_over_ranks, world, hbm, bf16, kernel="
             "effective_tflops": acct["flops"] / (ms / 1e3) / 1e12,
             "algo_gbs": acct["algo_bytes"] / (ms / 1e3) / 1e9,
             "frac_of_roofline_time": roof_ms / ms, "steps": steps}
+
+
+def run_decode_bench(name, dev, barrier, max_over_ranks, world, hbm):
+    """Split-K decode (one query token per sequence): two launches per step
+    (chunk kernel + merge), workspace allocated once outside the timed loop."""
+    from top_sparse_attention_qsa_b200 import _capi
+    w = make_workload(name, dev)
+    acct = workload_accounting(w)
+    out = torch.empty_like(w.q)
+    lse = torch.empty(w.q.shape[:2], dtype=torch.float32, device=dev)
+    splits = _capi.decode_num_splits(w.q, w.k_cache, w.topk_idx, 0)
+    need = _capi.decode_workspace_bytes(w.q, w.k_cache, w.topk_idx, 0, out, lse)
+    ws = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+
+    def step():
+        _capi.sparse_decode_fwd(w.q, w.k_cache, w.v_cache, w.topk_idx, w.n_valid, w.scale,
+                                num_splits=0, workspace=ws, out=out, lse=lse)
+
+    steps = 50
+    total_ms, per_ms, _ = time_launches(step, steps, 5, barrier, "decode")
+    total_ms = max_over_ranks(total_ms)
+    ms = statistics.mean(per_ms)
+    algo = acct["algo_bytes"] + need  # partial results are written once and read once by the merge
+    return {"workload": w.name, "desc": w.description, "splits": splits,
+            "workspace_bytes": need, "tokens_per_s": w.shape["T"] * steps * world / (total_ms / 1e3),
+            "mean_step_ms": ms, "gathered_kv_gbs": acct["gathered_bytes"] / (ms / 1e3) / 1e9,
+            "algo_gbs": algo / (ms / 1e3) / 1e9, "frac_of_hbm": algo / (ms / 1e3) / 1e9 / hbm,
+            "launches_per_step": 2 if need > 0 else 1, "steps": steps}
 
 
 def main():

@@ -40,6 +40,7 @@
 #ifndef QSA_H
 #define QSA_H
 
+#include <stddef.h>
 #include <stdint.h>
 
 #ifdef __cplusplus
@@ -135,6 +136,45 @@ qsa_status_t qsa_sparse_prefill_debug_gather(
     const void* v_cache, const int32_t* topk_idx, const int32_t* n_valid,
     float scale, void* out, float* lse, int32_t* status,
     int32_t* gathered_ids, void* stream);
+
+/*
+ * Split-K sparse attention for decode-shaped calls: few query tokens per KV
+ * head (one per sequence in decode) with long lists.  Each list is cut into
+ * chunks of a multiple of 128 entries; every (token, KV head, chunk) runs on
+ * its own CTA of the tcgen05 kernel and writes a normalised partial output and
+ * its log-sum-exp to `workspace`; a merge launch then combines the chunks
+ *   lse = log sum_c exp(lse_c),  out = sum_c exp(lse_c - lse) out_c,
+ * which is the same attention (the combine step of decode context
+ * parallelism, page "Qwen4-Exp QSA llega al Ascend de Huawei", section "Dónde
+ * encaja esto en el despliegue del servicio de Qwen4Exp", vLLM #59279).
+ * Same operation, arguments and conventions as qsa_sparse_prefill_fwd, plus:
+ *   num_splits      : chunks per list; <= 0 picks enough for two units per SM
+ *                     (never chunks shorter than 128 entries).
+ *   workspace       : caller-owned device scratch, 256-byte aligned, of at
+ *                     least qsa_sparse_decode_workspace_bytes(shape,
+ *                     num_splits) bytes (FP32 partial outputs and lse).  It
+ *                     may be NULL when that size is 0 (a single chunk: the
+ *                     call then runs the prefill kernel directly).
+ * QSA_ERR_SHAPE when workspace_bytes is too small.  Two launches (split
+ * kernel, merge kernel) on `stream`; no allocation, no sync.
+ */
+qsa_status_t qsa_sparse_decode_fwd(const qsa_shape_t* shape, const void* q,
+                                   const void* k_cache, const void* v_cache,
+                                   const int32_t* topk_idx,
+                                   const int32_t* n_valid, float scale,
+                                   void* out, float* lse, int32_t* status,
+                                   int32_t num_splits, void* workspace,
+                                   size_t workspace_bytes, void* stream);
+
+/* Workspace bytes qsa_sparse_decode_fwd needs for this shape and num_splits
+ * (0: no workspace needed, or an invalid shape).  With num_splits <= 0 the
+ * answer depends on the current device's SM count. */
+size_t qsa_sparse_decode_workspace_bytes(const qsa_shape_t* shape,
+                                         int32_t num_splits);
+
+/* Chunk count qsa_sparse_decode_fwd will use (0 for an invalid shape). */
+int32_t qsa_sparse_decode_num_splits(const qsa_shape_t* shape,
+                                     int32_t num_splits);
 
 /* Device staging buffers for the host-buffer entry point (caller-owned,
  * sized for the layouts of `shape`; n_valid / lse / status may be NULL when

@@ -21,6 +21,8 @@ Pins (what the pages and the mathematics fix):
   twice; out-of-range slots are reported and ignored.
 * brute_force   -- an independent numpy evaluation without the max trick.
 * worked_example -- the hand-derived fixture in tests/golden.
+* split_merge   -- attention over a list equals the log-sum-exp merge of
+  attention over any split of it (the combine step of split-K decode).
 """
 from __future__ import annotations
 
@@ -237,5 +239,28 @@ def check_worked_example(orc):
     np.testing.assert_allclose(lse[0, 0], float(ex["expected_lse"]), rtol=1e-14)
 
 
+def check_split_merge(orc):
+    """Attention over a list equals the lse-weighted mix of attention over any
+    split of the list into chunks (the combine step of split-K / decode
+    context parallelism): lse = log sum_c exp(lse_c), out = sum_c
+    exp(lse_c - lse) out_c; an empty chunk has lse_c = -inf and weight 0."""
+    w = W.generic_case(T=5, S=900, Hq=24, Hkv=2, K=300, seed=41)
+    full, lse_full, _ = orc.sparse_prefill(w.q, w.k_cache, w.v_cache, w.topk_idx)
+    for bounds in ((0, 128, 256, 300), (0, 7, 8, 300), (0, 300, 300)):
+        outs, lses = [], []
+        for a, b in zip(bounds[:-1], bounds[1:]):
+            o, l, _ = orc.sparse_prefill(w.q, w.k_cache, w.v_cache, w.topk_idx[:, :, a:b].contiguous())
+            outs.append(o)
+            lses.append(l)
+        L = np.stack(lses)                                  # [chunks, T, Hq]
+        m = L.max(axis=0)
+        wts = np.where(np.isneginf(L), 0.0, np.exp(L - m))
+        lse = m + np.log(wts.sum(axis=0))
+        out = (wts[..., None] * np.stack(outs)).sum(axis=0) / wts.sum(axis=0)[..., None]
+        np.testing.assert_allclose(out, full, **TOL)
+        np.testing.assert_allclose(lse, lse_full, **TOL)
+
+
 ALL_CHECKS = [check_bf16_widening, check_dense_causal, check_packing, check_permutation,
-              check_head_padding, check_closed_forms, check_brute_force, check_worked_example]
+              check_head_padding, check_closed_forms, check_brute_force, check_worked_example,
+              check_split_merge]

@@ -8,6 +8,7 @@ libqsa.so raises ImportError (there is no fallback).
 """
 
 _API = ("sparse_prefill_fwd", "sparse_prefill_debug_gather", "sparse_prefill_fwd_host",
+        "sparse_decode_fwd", "decode_workspace_bytes", "decode_num_splits",
         "status_string", "abi_version", "QSAError", "STATUS_OOB_SLOT")
 
 

@@ -31,7 +31,8 @@ HEAD_DIM = 256
 
 # Every symbol include/qsa.h declares.
 EXPORTS = ("qsa_sparse_prefill_fwd", "qsa_sparse_prefill_fwd_with", "qsa_sparse_prefill_debug_gather",
-           "qsa_sparse_prefill_fwd_host", "qsa_status_string", "qsa_abi_version")
+           "qsa_sparse_prefill_fwd_host", "qsa_sparse_decode_fwd", "qsa_sparse_decode_workspace_bytes",
+           "qsa_sparse_decode_num_splits", "qsa_status_string", "qsa_abi_version")
 
 
 class Shape(ctypes.Structure):
@@ -73,6 +74,13 @@ _lib.qsa_sparse_prefill_fwd_host.restype = ctypes.c_int
 _lib.qsa_sparse_prefill_fwd_host.argtypes = [ctypes.POINTER(Shape), _vp, _vp, _vp, _vp, _vp,
                                              ctypes.c_float, _vp, _vp,
                                              ctypes.POINTER(DeviceBuffers), _vp]
+_lib.qsa_sparse_decode_fwd.restype = ctypes.c_int
+_lib.qsa_sparse_decode_fwd.argtypes = [ctypes.POINTER(Shape), _vp, _vp, _vp, _vp, _vp, ctypes.c_float,
+                                       _vp, _vp, _vp, ctypes.c_int32, _vp, ctypes.c_size_t, _vp]
+_lib.qsa_sparse_decode_workspace_bytes.restype = ctypes.c_size_t
+_lib.qsa_sparse_decode_workspace_bytes.argtypes = [ctypes.POINTER(Shape), ctypes.c_int32]
+_lib.qsa_sparse_decode_num_splits.restype = ctypes.c_int32
+_lib.qsa_sparse_decode_num_splits.argtypes = [ctypes.POINTER(Shape), ctypes.c_int32]
 _lib.qsa_status_string.restype = ctypes.c_char_p
 _lib.qsa_status_string.argtypes = [ctypes.c_int]
 _lib.qsa_abi_version.restype = ctypes.c_int32
@@ -235,5 +243,60 @@ def sparse_prefill_fwd_host(q, k_cache, v_cache, topk_idx, n_valid, scale, out, 
                                           _ptr(v_cache), _ptr(topk_idx), _ptr(n_valid),
                                           float(scale), _ptr(out), _ptr(lse), ctypes.byref(db),
                                           stream)
+    _raise(rc)
+    return out, lse
+
+
+def decode_workspace_bytes(q, k_cache, topk_idx, num_splits: int = 0, out=None, lse=None) -> int:
+    """Scratch bytes sparse_decode_fwd needs (0 when a single chunk runs)."""
+    if out is None:
+        out = q
+    shape = make_shape(q, k_cache, topk_idx, out, lse)
+    return int(_lib.qsa_sparse_decode_workspace_bytes(ctypes.byref(shape), int(num_splits)))
+
+
+def decode_num_splits(q, k_cache, topk_idx, num_splits: int = 0) -> int:
+    shape = make_shape(q, k_cache, topk_idx, q)
+    return int(_lib.qsa_sparse_decode_num_splits(ctypes.byref(shape), int(num_splits)))
+
+
+def sparse_decode_fwd(q, k_cache, v_cache, topk_idx, n_valid=None, scale: float = 0.0,
+                      num_splits: int = 0, workspace=None, out=None, lse=None, status=None,
+                      stream=None, want_lse: bool = True):
+    """Split-K sparse attention (decode-shaped calls).  `workspace` is a CUDA
+    tensor of at least decode_workspace_bytes(...) bytes (allocated here with
+    torch when None).  Returns (out, lse)."""
+    dev = q.device
+    _need(q, "q", torch.bfloat16, dev)
+    _need(k_cache, "k_cache", torch.bfloat16, dev)
+    _need(v_cache, "v_cache", torch.bfloat16, dev)
+    _need(topk_idx, "topk_idx", torch.int32, dev)
+    _check_kv(k_cache, v_cache)
+    if n_valid is not None:
+        _need(n_valid, "n_valid", torch.int32, dev)
+        if not n_valid.is_contiguous() or tuple(n_valid.shape) != tuple(topk_idx.shape[:2]):
+            raise ValueError("n_valid must be a contiguous [T, Hkv] tensor")
+    if out is None:
+        out = torch.empty(q.shape, dtype=torch.bfloat16, device=dev)
+    _need(out, "out", torch.bfloat16, dev)
+    if lse is None and want_lse:
+        lse = torch.empty(q.shape[:2], dtype=torch.float32, device=dev)
+    if lse is not None:
+        _need(lse, "lse", torch.float32, dev)
+    if status is not None:
+        _need(status, "status", torch.int32, dev)
+    shape = make_shape(q, k_cache, topk_idx, out, lse)
+    need = int(_lib.qsa_sparse_decode_workspace_bytes(ctypes.byref(shape), int(num_splits)))
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    ws_bytes = 0
+    if workspace is not None:
+        _need(workspace, "workspace", workspace.dtype, dev)
+        ws_bytes = workspace.numel() * workspace.element_size()
+    if stream is None:
+        stream = torch.cuda.current_stream(dev).cuda_stream
+    rc = _lib.qsa_sparse_decode_fwd(ctypes.byref(shape), _ptr(q), _ptr(k_cache), _ptr(v_cache),
+                                    _ptr(topk_idx), _ptr(n_valid), float(scale), _ptr(out), _ptr(lse),
+                                    _ptr(status), int(num_splits), _ptr(workspace), ws_bytes, stream)
     _raise(rc)
     return out, lse

@@ -11,6 +11,7 @@
 #include <mutex>
 
 #include "qsa.h"
+#include "qsa_merge.cuh"
 #include "qsa_prefill_mma.cuh"
 #include "qsa_prefill_tc.cuh"
 
@@ -220,12 +221,121 @@ qsa_status_t run_forward(const qsa_shape_t* s, const void* q, const void* k, con
     tp.K = p.K;
     tp.S = static_cast<int32_t>(p.S);
     tp.scale_log2 = p.scale_log2;
+    tp.splits = 1;
+    tp.chunk = p.K;
+    tp.part_o = nullptr;
+    tp.part_lse = nullptr;
     e = dump ? launch_tc<true>(tp, st) : launch_tc<false>(tp, st);
   } else if (p.G <= 8)
     e = dump ? launch_mma<1, true>(p, st) : launch_mma<1, false>(p, st);
   else
     e = dump ? launch_mma<2, true>(p, st) : launch_mma<2, false>(p, st);
   return e == cudaSuccess ? QSA_OK : QSA_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------- split-K decode
+
+struct SplitPlan {
+  int32_t splits;
+  int32_t chunk;
+  size_t part_o_bytes;   // [T*Hq][splits][256] FP32
+  size_t lse_offset;     // 256-byte aligned
+  size_t total_bytes;
+};
+
+// Chunk count for a decode-shaped call: enough (token, KV head, chunk) units
+// for two per SM when num_splits <= 0, never chunks shorter than one 128-entry
+// tile.  Deterministic for a given shape and device.
+bool plan_splits(const qsa_shape_t* s, int32_t num_splits, SplitPlan* pl) {
+  const int64_t K = s->topk;
+  const int64_t max_splits = K > 0 ? (K + qsa::tc::kKeys - 1) / qsa::tc::kKeys : 1;
+  int64_t splits = num_splits;
+  if (num_splits <= 0) {
+    const int nsm = sm_count();
+    if (nsm <= 0) return false;
+    const int64_t units = s->num_tokens * s->num_kv_heads;
+    splits = units > 0 ? (2 * static_cast<int64_t>(nsm) + units - 1) / units : 1;
+  }
+  splits = splits < 1 ? 1 : (splits > max_splits ? max_splits : splits);
+  int64_t chunk = K > 0 ? (K + splits - 1) / splits : 0;
+  chunk = (chunk + qsa::tc::kKeys - 1) / qsa::tc::kKeys * qsa::tc::kKeys;
+  if (chunk > 0) splits = (K + chunk - 1) / chunk;
+  pl->splits = static_cast<int32_t>(splits);
+  pl->chunk = static_cast<int32_t>(chunk);
+  const size_t rows = static_cast<size_t>(s->num_tokens) * s->num_q_heads;
+  pl->part_o_bytes = rows * pl->splits * 256 * sizeof(float);
+  pl->lse_offset = (pl->part_o_bytes + 255) / 256 * 256;
+  pl->total_bytes = pl->lse_offset + rows * pl->splits * sizeof(float);
+  return true;
+}
+
+cudaError_t launch_merge(const qsa_shape_t* s, const float* part_o, const float* part_lse,
+                         int32_t splits, void* out, float* lse, cudaStream_t stream) {
+  qsa::MergeParams mp;
+  mp.part_o = part_o;
+  mp.part_lse = part_lse;
+  mp.out = static_cast<__nv_bfloat16*>(out);
+  mp.lse = lse;
+  mp.rows = s->num_tokens * s->num_q_heads;
+  mp.Hq = s->num_q_heads;
+  mp.splits = splits;
+  mp.o_st = s->o_stride_tok;
+  mp.o_sh = s->o_stride_head;
+  mp.lse_st = s->lse_stride_tok;
+  if (mp.rows > 0x7fffffffLL) return cudaErrorInvalidValue;
+  qsa::qsa_merge_splits_kernel<<<static_cast<unsigned>(mp.rows), 64, 0, stream>>>(mp);
+  return cudaGetLastError();
+}
+
+// Split-K forward: partial results of every chunk go to `workspace` (laid
+// out by plan_splits), then one merge launch writes out/lse.
+qsa_status_t run_decode(const qsa_shape_t* s, const void* q, const void* k, const void* v,
+                        const int32_t* idx, const int32_t* n_valid, float scale, void* out,
+                        float* lse, int32_t* status, int32_t num_splits, void* workspace,
+                        size_t workspace_bytes, void* stream) {
+  qsa_status_t rc = validate(s, q, k, v, idx, out);
+  if (rc != QSA_OK) return rc;
+  if (s->num_tokens == 0) return QSA_OK;
+  SplitPlan pl;
+  if (!plan_splits(s, num_splits, &pl)) return QSA_ERR_CUDA;
+  static thread_local qsa::tc::TcParams tp;
+  if (pl.splits <= 1 || !make_tc_params(s, q, &tp))
+    return run_forward(s, q, k, v, idx, n_valid, scale, out, lse, status, nullptr, stream);
+  if (workspace == nullptr) return QSA_ERR_NULL;
+  if (workspace_bytes < pl.total_bytes) return QSA_ERR_SHAPE;
+  if (reinterpret_cast<uintptr_t>(workspace) & 255u) return QSA_ERR_ALIGN;
+  float* part_o = static_cast<float*>(workspace);
+  float* part_lse = reinterpret_cast<float*>(static_cast<char*>(workspace) + pl.lse_offset);
+  const float sc = scale > 0.f ? scale : 0.0625f;
+  tp.idx = idx;
+  tp.n_valid = n_valid;
+  tp.kraw = k;
+  tp.vraw = v;
+  tp.out = static_cast<__nv_bfloat16*>(out);
+  tp.lse = lse;
+  tp.status = status;
+  tp.gathered = nullptr;
+  tp.T = s->num_tokens;
+  tp.idx_st = s->idx_stride_tok;
+  tp.idx_sh = s->idx_stride_head;
+  tp.o_st = s->o_stride_tok;
+  tp.o_sh = s->o_stride_head;
+  tp.lse_st = s->lse_stride_tok;
+  tp.kv_ss = s->kv_stride_slot;
+  tp.kv_sh = s->kv_stride_head;
+  tp.Hkv = s->num_kv_heads;
+  tp.G = s->num_q_heads / s->num_kv_heads;
+  tp.K = s->topk;
+  tp.S = static_cast<int32_t>(s->num_slots);
+  tp.scale_log2 = sc * 1.4426950408889634f;
+  tp.splits = pl.splits;
+  tp.chunk = pl.chunk;
+  tp.part_o = part_o;
+  tp.part_lse = part_lse;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (launch_tc<false>(tp, st) != cudaSuccess) return QSA_ERR_CUDA;
+  if (launch_merge(s, part_o, part_lse, pl.splits, out, lse, st) != cudaSuccess) return QSA_ERR_CUDA;
+  return QSA_OK;
 }
 
 // Bytes spanned by a strided [n0, n1, inner] layout (first to last element).
@@ -306,6 +416,32 @@ qsa_status_t qsa_sparse_prefill_fwd_host(const qsa_shape_t* s, const void* q_hos
   if (lse_host != nullptr)
     ok = ok && d2h(lse_host, dev->lse, span_bytes(T, s->lse_stride_tok, 1, 0, Hq, 4));
   return ok ? QSA_OK : QSA_ERR_CUDA;
+}
+
+size_t qsa_sparse_decode_workspace_bytes(const qsa_shape_t* shape, int32_t num_splits) {
+  if (shape == nullptr || shape->num_tokens < 0 || shape->topk < 0 || shape->num_q_heads <= 0 ||
+      shape->num_kv_heads <= 0)
+    return 0;
+  SplitPlan pl;
+  if (!plan_splits(shape, num_splits, &pl) || pl.splits <= 1) return 0;
+  return pl.total_bytes;
+}
+
+int32_t qsa_sparse_decode_num_splits(const qsa_shape_t* shape, int32_t num_splits) {
+  if (shape == nullptr || shape->topk < 0 || shape->num_tokens < 0 || shape->num_kv_heads <= 0)
+    return 0;
+  SplitPlan pl;
+  if (!plan_splits(shape, num_splits, &pl)) return 0;
+  return pl.splits;
+}
+
+qsa_status_t qsa_sparse_decode_fwd(const qsa_shape_t* shape, const void* q, const void* k_cache,
+                                   const void* v_cache, const int32_t* topk_idx,
+                                   const int32_t* n_valid, float scale, void* out, float* lse,
+                                   int32_t* status, int32_t num_splits, void* workspace,
+                                   size_t workspace_bytes, void* stream) {
+  return run_decode(shape, q, k_cache, v_cache, topk_idx, n_valid, scale, out, lse, status,
+                    num_splits, workspace, workspace_bytes, stream);
 }
 
 const char* qsa_status_string(qsa_status_t status) {

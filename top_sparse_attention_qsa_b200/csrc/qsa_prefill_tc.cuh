@@ -7,25 +7,23 @@
 // heads of the group attend to the cache rows named by the token's list,
 // softmax(scale q K_sel^T) V_sel, -1 / n_valid masking, zeros for empty rows.
 //
-// Persistent CTAs (one per SM) walk the units in KV-head-major order.  Seven
+// Persistent CTAs (one per SM) walk the units in KV-head-major order.  Ten
 // warps with fixed roles, synchronised only through mbarriers:
-//   warp 0      producer: reads the 128 list entries of a tile two tiles
-//               ahead of its loads and asks L2 for those K and V rows (bulk
-//               prefetch), so the loads into shared memory meet L2 latency;
-//               then issues TMA tile::gather4 loads (4 rows x 128 B per
-//               instruction, 128-byte swizzle) of the K and V rows into a ring
-//               of six 32 KB slots (K dims 0-127, K dims 128-255, V dims 0-127,
-//               V dims 128-255); masked entries use an out-of-range row so the
-//               TMA zero-fills them without reading memory.  Also loads the 16
-//               Q rows of the unit (TMA, double-buffered).
-//   warp 1      one thread issues the score MMAs (tcgen05.mma, kind::f16):
+//   warps 0-3   producers: read each tile's 128 list entries one tile ahead
+//               and gather the K and V rows with 16-byte cp.async copies
+//               written straight into the 128-byte-swizzled layout the
+//               tensor core reads, into a ring of six 32 KB slots (K dims
+//               0-127, K dims 128-255, V dims 0-127, V dims 128-255); masked
+//               entries are zero-filled without a global read.  Warp 0 also
+//               loads the 16 Q rows of the unit (tiled TMA, double-buffered).
+//   warp 4      one thread issues the score MMAs (tcgen05.mma, kind::f16):
 //               S^T[128 keys x 16 heads] = K_tile . Q^T (M=128, N=16, K-major
 //               operands) into a TMEM double buffer.
-//   warp 6      one thread issues the PV MMAs: O^T[256 x 16] += V_tile^T . P^T
+//   warp 5      one thread issues the PV MMAs: O^T[256 x 16] += V_tile^T . P^T
 //               (two M=128 halves, V read MN-major from the same slots) into
 //               TMEM.  Two issuers keep PV of tile i from queueing behind the
 //               scores of tile i+1.
-//   warps 2-5   softmax: thread k owns TMEM lane k = key k of the tile; tile
+//   warps 6-9   softmax: thread k owns TMEM lane k = key k of the tile; tile
 //               max per head by a transposing shuffle reduction and a 4-warp
 //               exchange; exponentials in base 2; P^T written MN-major to
 //               shared memory; the running max is only raised (with an O
@@ -95,6 +93,13 @@ struct TcParams {
   int64_t idx_st, idx_sh, o_st, o_sh, lse_st, kv_ss, kv_sh;
   int32_t Hkv, G, K, S;
   float scale_log2;
+  // split-K: each list is cut into `splits` chunks of `chunk` entries (a
+  // multiple of 128); with part_o set, every (token, KV head, chunk) unit
+  // writes its normalised partial O (FP32 [T*Hq][splits][256]) and partial
+  // lse ([T*Hq][splits]) there instead of out/lse, for a merge pass.
+  int32_t splits, chunk;
+  float* part_o;
+  float* part_lse;
 };
 
 // Instruction descriptors (kind::f16): FP32 accumulator, BF16 A and B,
@@ -146,18 +151,28 @@ struct Sync {
 struct Unit {
   int64_t t;
   int g;
-  int n_eff;
+  int s;       // chunk of the list (split-K), 0 without splitting
+  int j0;      // first list entry of the chunk
+  int n_eff;   // live-range length inside the chunk
   int n_tiles;
 };
 
+__device__ __forceinline__ int64_t num_units(const TcParams& p) { return p.T * p.Hkv * p.splits; }
+
+// Unit u -> (KV head, token, chunk), KV head outermost so that concurrent
+// CTAs share one head's cache rows.
 __device__ __forceinline__ Unit decode_unit(const TcParams& p, int64_t u) {
   Unit r;
-  r.g = static_cast<int>(u / p.T);
-  r.t = u - static_cast<int64_t>(r.g) * p.T;
+  const int64_t per_head = p.T * p.splits;
+  r.g = static_cast<int>(u / per_head);
+  const int64_t rem = u - static_cast<int64_t>(r.g) * per_head;
+  r.t = rem / p.splits;
+  r.s = static_cast<int>(rem - r.t * p.splits);
   int n = p.K;
   if (p.n_valid != nullptr) n = min(n, max(__ldg(p.n_valid + r.t * p.Hkv + r.g), 0));
-  r.n_eff = n;
-  r.n_tiles = (n + kKeys - 1) / kKeys;
+  r.j0 = r.s * p.chunk;
+  r.n_eff = max(0, min(n - r.j0, p.chunk));
+  r.n_tiles = (r.n_eff + kKeys - 1) / kKeys;
   return r;
 }
 
@@ -207,7 +222,7 @@ __device__ __forceinline__ float xreduce16(const float (&v)[16], int lane) {
 template <bool kDump>
 __device__ void producer_role(const TcParams& p, const Sync& sy, uint32_t sb, int pw, int lane) {
   uint32_t c_slot = 0, c_unit = 0;
-  const int64_t units = p.T * p.Hkv;
+  const int64_t units = num_units(p);
   const int cc = lane & 15;                          // 16-byte chunk of the half row
   const int rsel = lane >> 4;                        // which of the two rows of an instruction
   const uint32_t dchunk = static_cast<uint32_t>((cc >> 3) * kBlockBytes);
@@ -230,7 +245,7 @@ __device__ void producer_role(const TcParams& p, const Sync& sy, uint32_t sb, in
     }
     ++c_unit;
     if (!ok) break;
-    const int32_t* list = p.idx + un.t * p.idx_st + static_cast<int64_t>(un.g) * p.idx_sh;
+    const int32_t* list = p.idx + un.t * p.idx_st + static_cast<int64_t>(un.g) * p.idx_sh + un.j0;
     const char* kbase = reinterpret_cast<const char*>(p.kraw) + static_cast<int64_t>(un.g) * p.kv_sh * 2 + cc * 16;
     const char* vbase = reinterpret_cast<const char*>(p.vraw) + static_cast<int64_t>(un.g) * p.kv_sh * 2 + cc * 16;
     const int64_t row_bytes = p.kv_ss * 2;
@@ -249,7 +264,7 @@ __device__ void producer_role(const TcParams& p, const Sync& sy, uint32_t sb, in
         if (p.status != nullptr) atomicOr(p.status, static_cast<int32_t>(kStatusOob));
       }
       if (kDump && own) {
-        const int j = i * kKeys + jr;
+        const int j = un.j0 + i * kKeys + jr;
         if (j < p.K) p.gathered[(un.t * p.Hkv + un.g) * static_cast<int64_t>(p.K) + j] = id < 0 ? -1 : id;
       }
 #pragma unroll 1
@@ -282,7 +297,7 @@ __device__ void producer_role(const TcParams& p, const Sync& sy, uint32_t sb, in
 // Scores: S^T[c & 1] = K_tile(c) . Q^T for every tile c of the CTA.
 __device__ void qk_role(const TcParams& p, const Sync& sy, uint32_t sb, uint32_t tmem) {
   uint32_t c_tile = 0, c_unit = 0;
-  const int64_t units = p.T * p.Hkv;
+  const int64_t units = num_units(p);
   bool ok = true;
   for (int64_t u = blockIdx.x; u < units && ok; u += gridDim.x) {
     const Unit un = decode_unit(p, u);
@@ -330,7 +345,7 @@ __device__ void qk_role(const TcParams& p, const Sync& sy, uint32_t sb, uint32_t
 // PV: O^T (two M=128 halves) += V_tile(c)^T . P^T(c) for every tile c.
 __device__ void pv_role(const TcParams& p, const Sync& sy, uint32_t sb, uint32_t tmem) {
   uint32_t c_tile = 0, c_unit = 0;
-  const int64_t units = p.T * p.Hkv;
+  const int64_t units = num_units(p);
   const uint32_t t_o = tmem + 32;  // O halves: columns 32-47 and 48-63
   bool ok = true;
   for (int64_t u = blockIdx.x; u < units && ok; u += gridDim.x) {
@@ -384,12 +399,12 @@ __device__ void softmax_role(const TcParams& p, const Sync& sy, uint32_t sb, uin
   float* red_max = reinterpret_cast<float*>(sp + OFF_RED);        // [2][4][16]
   float* red_sum = red_max + 128;                                  // [2][4][16]
   uint32_t c_tile = 0, c_unit = 0;
-  const int64_t units = p.T * p.Hkv;
+  const int64_t units = num_units(p);
   const int G = p.G;
   bool ok = true;
   for (int64_t u = blockIdx.x; u < units && ok; u += gridDim.x) {
     const Unit un = decode_unit(p, u);
-    const int32_t* list = p.idx + un.t * p.idx_st + static_cast<int64_t>(un.g) * p.idx_sh;
+    const int32_t* list = p.idx + un.t * p.idx_st + static_cast<int64_t>(un.g) * p.idx_sh + un.j0;
     float m_run[kGp], l_part[kGp];
 #pragma unroll
     for (int h = 0; h < kGp; ++h) {
@@ -512,6 +527,7 @@ __device__ void softmax_role(const TcParams& p, const Sync& sy, uint32_t sb, uin
     tc_fence_before();
     __syncwarp();
     if (lane == 0) mbar_arrive(sy.bar(B_OEMPTY));
+    const int64_t row0 = un.t * static_cast<int64_t>(p.Hkv) * G + static_cast<int64_t>(un.g) * G;
     __nv_bfloat16* orow = p.out + un.t * p.o_st + static_cast<int64_t>(un.g) * G * p.o_sh;
 #pragma unroll
     for (int h = 0; h < kGp; ++h) {
@@ -520,11 +536,17 @@ __device__ void softmax_role(const TcParams& p, const Sync& sy, uint32_t sb, uin
         const float inv = live ? 1.f / l_tot[h] : 0.f;
         const float v0 = live ? __uint_as_float(o0[h]) * inv : 0.f;
         const float v1 = live ? __uint_as_float(o1[h]) * inv : 0.f;
-        orow[h * p.o_sh + key] = __float2bfloat16_rn(v0);
-        orow[h * p.o_sh + 128 + key] = __float2bfloat16_rn(v1);
+        if (p.part_o != nullptr) {
+          float* po = p.part_o + ((row0 + h) * p.splits + un.s) * 256;
+          po[key] = v0;
+          po[128 + key] = v1;
+        } else {
+          orow[h * p.o_sh + key] = __float2bfloat16_rn(v0);
+          orow[h * p.o_sh + 128 + key] = __float2bfloat16_rn(v1);
+        }
       }
     }
-    if (p.lse != nullptr && key < G) {
+    if (key < G && (p.lse != nullptr || p.part_lse != nullptr)) {
       float mk = 0.f, lk = 0.f;
 #pragma unroll
       for (int h = 0; h < kGp; ++h)
@@ -532,8 +554,11 @@ __device__ void softmax_role(const TcParams& p, const Sync& sy, uint32_t sb, uin
           mk = m_run[h];
           lk = l_tot[h];
         }
-      p.lse[un.t * p.lse_st + static_cast<int64_t>(un.g) * G + key] =
-          lk > 0.f ? (mk + lg2(lk)) * 0.69314718055994531f : -INFINITY;
+      const float lv = lk > 0.f ? (mk + lg2(lk)) * 0.69314718055994531f : -INFINITY;
+      if (p.part_lse != nullptr)
+        p.part_lse[(row0 + key) * p.splits + un.s] = lv;
+      else
+        p.lse[un.t * p.lse_st + static_cast<int64_t>(un.g) * G + key] = lv;
     }
     c_tile += un.n_tiles;
     ++c_unit;

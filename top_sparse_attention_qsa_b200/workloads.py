@@ -239,12 +239,32 @@ def config_pages_long(device="cpu", seed=CONFIG_SEED_BASE + 6, heads=(24, 2)) ->
                     "T=7810 S=65536 (24,2) K=2051 (3-token tail + random), unsorted")
 
 
+def config_decode(device="cpu", seed=CONFIG_SEED_BASE + 7, B=64, ctx=32768, heads=(24, 2),
+                  topk=2048, local=256) -> Workload:
+    """Decode step: B sequences of `ctx` cached tokens each (sequence b owns
+    slots [b*ctx, (b+1)*ctx)), one new query token per sequence at its last
+    slot; per KV head `local` most recent slots + random earlier slots of the
+    same sequence, unsorted."""
+    gen = _gen(seed, device)
+    Hq, Hkv = heads
+    S = B * ctx
+    q = normal_bf16((B, Hq, HEAD_DIM), gen, device)
+    k = normal_bf16((S, Hkv, HEAD_DIM), gen, device)
+    v = normal_bf16((S, Hkv, HEAD_DIM), gen, device)
+    s0 = torch.arange(B, device=device) * ctx
+    pos = s0 + ctx - 1
+    idx, nv = causal_lists(pos, s0, topk, local, Hkv, gen, device, ordered=False)
+    return Workload(f"decode_b{B}_ctx{ctx}_g{Hq}x{Hkv}_k{topk}", q, k, v, idx, nv, 1.0 / 16, pos, s0,
+                    f"decode B={B} ctx={ctx} S={S} ({Hq},{Hkv}) K={topk} local{local}+random unsorted")
+
+
 CONFIGS = {
     "tiny": config_tiny,
     "c2": config_c2,
     "c3": config_c3,
     "c4": config_c4,
     "c5": config_c5,
+    "decode": config_decode,
 }
 
 
