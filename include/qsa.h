@@ -55,7 +55,9 @@ typedef enum {
   QSA_ERR_SHAPE = 2,       /* inconsistent sizes or strides */
   QSA_ERR_UNSUPPORTED = 3, /* head_dim != 256, G > 16, ... */
   QSA_ERR_ALIGN = 4,       /* a row is not 16-byte aligned */
-  QSA_ERR_CUDA = 5         /* a CUDA runtime call failed */
+  QSA_ERR_CUDA = 5,        /* a CUDA runtime call failed */
+  QSA_ERR_SCRATCH = 6      /* the call needs more scratch than the library's
+                              built-in array holds (allocation-free entry point) */
 } qsa_status_t;
 
 /* Bits of the device status word. */
@@ -175,6 +177,44 @@ size_t qsa_sparse_decode_workspace_bytes(const qsa_shape_t* shape,
 /* Chunk count qsa_sparse_decode_fwd will use (0 for an invalid shape). */
 int32_t qsa_sparse_decode_num_splits(const qsa_shape_t* shape,
                                      int32_t num_splits);
+
+/*
+ * Allocation-free decode.  The pages have no counterpart to this entry
+ * point; it exists for callers that cannot call cudaMalloc: code that runs
+ * where allocation is forbidden or unsafe (inside a caching allocator's own
+ * hooks, a real-time loop that must never block on the driver, an embedding
+ * runtime that owns every device allocation), and callers with no allocator
+ * at all.  It computes exactly what qsa_sparse_decode_fwd computes, but its
+ * scratch space (the partial outputs of the chunks) is a fixed array of
+ * QSA_NOALLOC_SCRATCH_BYTES compiled into the library, so the caller passes
+ * only inputs and outputs.
+ *
+ * Cost and limits:
+ *  - Every GPU on which the library's device code is loaded holds the
+ *    array (16 MiB) until the process exits.
+ *  - Calls whose chunks need more than the array holds (see
+ *    qsa_sparse_decode_workspace_bytes with the same shape and num_splits)
+ *    return QSA_ERR_SCRATCH before anything is enqueued.
+ *  - The first call on each device looks up the array's device address (no
+ *    allocation); make that first call before any stream capture on that
+ *    device.
+ *  - All calls in the process share the one array per device: two calls
+ *    whose work overlaps on the GPU (different streams, or host threads that
+ *    do not order their streams) race on it.  Serialise them.  Nothing in the
+ *    array needs to start at zero: every call overwrites each entry before
+ *    reading it, and the previous call's contents are simply left behind.
+ * Arguments as for qsa_sparse_decode_fwd, without workspace.
+ */
+#define QSA_NOALLOC_SCRATCH_BYTES (16u << 20)
+
+qsa_status_t qsa_sparse_decode_fwd_noalloc(const qsa_shape_t* shape,
+                                           const void* q, const void* k_cache,
+                                           const void* v_cache,
+                                           const int32_t* topk_idx,
+                                           const int32_t* n_valid, float scale,
+                                           void* out, float* lse,
+                                           int32_t* status, int32_t num_splits,
+                                           void* stream);
 
 /* Device staging buffers for the host-buffer entry point (caller-owned,
  * sized for the layouts of `shape`; n_valid / lse / status may be NULL when

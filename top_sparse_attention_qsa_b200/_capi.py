@@ -22,7 +22,8 @@ if not os.path.exists(LIB_PATH):
 
 _lib = ctypes.CDLL(LIB_PATH)
 
-QSA_OK, QSA_ERR_NULL, QSA_ERR_SHAPE, QSA_ERR_UNSUPPORTED, QSA_ERR_ALIGN, QSA_ERR_CUDA = range(6)
+QSA_OK, QSA_ERR_NULL, QSA_ERR_SHAPE, QSA_ERR_UNSUPPORTED, QSA_ERR_ALIGN, QSA_ERR_CUDA, QSA_ERR_SCRATCH = range(7)
+NOALLOC_SCRATCH_BYTES = 16 << 20
 STATUS_OOB_SLOT = 1
 STATUS_TIMEOUT = 2
 KERNEL_AUTO, KERNEL_TCGEN05, KERNEL_WARP_MMA = 0, 1, 2
@@ -32,7 +33,8 @@ HEAD_DIM = 256
 # Every symbol include/qsa.h declares.
 EXPORTS = ("qsa_sparse_prefill_fwd", "qsa_sparse_prefill_fwd_with", "qsa_sparse_prefill_debug_gather",
            "qsa_sparse_prefill_fwd_host", "qsa_sparse_decode_fwd", "qsa_sparse_decode_workspace_bytes",
-           "qsa_sparse_decode_num_splits", "qsa_status_string", "qsa_abi_version")
+           "qsa_sparse_decode_num_splits", "qsa_sparse_decode_fwd_noalloc", "qsa_status_string",
+           "qsa_abi_version")
 
 
 class Shape(ctypes.Structure):
@@ -81,6 +83,9 @@ _lib.qsa_sparse_decode_workspace_bytes.restype = ctypes.c_size_t
 _lib.qsa_sparse_decode_workspace_bytes.argtypes = [ctypes.POINTER(Shape), ctypes.c_int32]
 _lib.qsa_sparse_decode_num_splits.restype = ctypes.c_int32
 _lib.qsa_sparse_decode_num_splits.argtypes = [ctypes.POINTER(Shape), ctypes.c_int32]
+_lib.qsa_sparse_decode_fwd_noalloc.restype = ctypes.c_int
+_lib.qsa_sparse_decode_fwd_noalloc.argtypes = [ctypes.POINTER(Shape), _vp, _vp, _vp, _vp, _vp,
+                                               ctypes.c_float, _vp, _vp, _vp, ctypes.c_int32, _vp]
 _lib.qsa_status_string.restype = ctypes.c_char_p
 _lib.qsa_status_string.argtypes = [ctypes.c_int]
 _lib.qsa_abi_version.restype = ctypes.c_int32
@@ -298,5 +303,42 @@ def sparse_decode_fwd(q, k_cache, v_cache, topk_idx, n_valid=None, scale: float 
     rc = _lib.qsa_sparse_decode_fwd(ctypes.byref(shape), _ptr(q), _ptr(k_cache), _ptr(v_cache),
                                     _ptr(topk_idx), _ptr(n_valid), float(scale), _ptr(out), _ptr(lse),
                                     _ptr(status), int(num_splits), _ptr(workspace), ws_bytes, stream)
+    _raise(rc)
+    return out, lse
+
+
+def sparse_decode_fwd_noalloc(q, k_cache, v_cache, topk_idx, out, lse=None, n_valid=None,
+                              scale: float = 0.0, num_splits: int = 0, status=None, stream=None):
+    """Allocation-free decode for callers that cannot allocate device memory.
+
+    Same result as sparse_decode_fwd, but the library keeps the chunk
+    scratch in its own fixed device array (NOALLOC_SCRATCH_BYTES), and the
+    caller provides every output buffer (`out`, optional `lse`), so neither
+    this call nor the library allocates.  Concurrent calls on the same device
+    must be serialised (they share the array); the first call on a device
+    should precede any stream capture.  Raises QSAError(QSA_ERR_SCRATCH) when
+    the chunks would not fit."""
+    dev = q.device
+    _need(q, "q", torch.bfloat16, dev)
+    _need(k_cache, "k_cache", torch.bfloat16, dev)
+    _need(v_cache, "v_cache", torch.bfloat16, dev)
+    _need(topk_idx, "topk_idx", torch.int32, dev)
+    _check_kv(k_cache, v_cache)
+    _need(out, "out", torch.bfloat16, dev)
+    if lse is not None:
+        _need(lse, "lse", torch.float32, dev)
+    if n_valid is not None:
+        _need(n_valid, "n_valid", torch.int32, dev)
+        if not n_valid.is_contiguous() or tuple(n_valid.shape) != tuple(topk_idx.shape[:2]):
+            raise ValueError("n_valid must be a contiguous [T, Hkv] tensor")
+    if status is not None:
+        _need(status, "status", torch.int32, dev)
+    shape = make_shape(q, k_cache, topk_idx, out, lse)
+    if stream is None:
+        stream = torch.cuda.current_stream(dev).cuda_stream
+    rc = _lib.qsa_sparse_decode_fwd_noalloc(ctypes.byref(shape), _ptr(q), _ptr(k_cache),
+                                            _ptr(v_cache), _ptr(topk_idx), _ptr(n_valid),
+                                            float(scale), _ptr(out), _ptr(lse), _ptr(status),
+                                            int(num_splits), stream)
     _raise(rc)
     return out, lse

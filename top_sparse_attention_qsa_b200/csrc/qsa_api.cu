@@ -344,6 +344,37 @@ size_t span_bytes(int64_t n0, int64_t s0, int64_t n1, int64_t s1, int64_t inner,
   return static_cast<size_t>((n0 - 1) * s0 + (n1 - 1) * s1 + inner) * elem;
 }
 
+// ---------------------------------------------------------------- allocation-free decode
+
+// Scratch for qsa_sparse_decode_fwd_noalloc: lives in the library's device
+// image, so it exists on every device the module is loaded on.  Host code
+// must not pass `g_noalloc_scratch` itself to a kernel (in host code it is
+// only a stand-in symbol); it passes the device address looked up below.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[QSA_NOALLOC_SCRATCH_BYTES];
+
+// Device address of g_noalloc_scratch on the current device, looked up once
+// per device (cudaGetSymbolAddress allocates nothing).
+cudaError_t noalloc_scratch_address(void** ptr) {
+  static std::atomic<void*> cache[kMaxDevices];
+  static std::mutex lock;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  void* p = cache[dev].load(std::memory_order_acquire);
+  if (p == nullptr) {
+    std::lock_guard<std::mutex> g(lock);
+    p = cache[dev].load(std::memory_order_acquire);
+    if (p == nullptr) {
+      e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+      if (e != cudaSuccess) return e;
+      cache[dev].store(p, std::memory_order_release);
+    }
+  }
+  *ptr = p;
+  return cudaSuccess;
+}
+
 }  // namespace
 
 extern "C" {
@@ -444,6 +475,24 @@ qsa_status_t qsa_sparse_decode_fwd(const qsa_shape_t* shape, const void* q, cons
                     num_splits, workspace, workspace_bytes, stream);
 }
 
+qsa_status_t qsa_sparse_decode_fwd_noalloc(const qsa_shape_t* shape, const void* q,
+                                           const void* k_cache, const void* v_cache,
+                                           const int32_t* topk_idx, const int32_t* n_valid,
+                                           float scale, void* out, float* lse, int32_t* status,
+                                           int32_t num_splits, void* stream) {
+  qsa_status_t rc = validate(shape, q, k_cache, v_cache, topk_idx, out);
+  if (rc != QSA_OK) return rc;
+  if (shape->num_tokens == 0) return QSA_OK;
+  SplitPlan pl;
+  if (!plan_splits(shape, num_splits, &pl)) return QSA_ERR_CUDA;
+  const size_t need = pl.splits > 1 ? pl.total_bytes : 0;
+  if (need > QSA_NOALLOC_SCRATCH_BYTES) return QSA_ERR_SCRATCH;
+  void* scratch = nullptr;
+  if (need > 0 && noalloc_scratch_address(&scratch) != cudaSuccess) return QSA_ERR_CUDA;
+  return run_decode(shape, q, k_cache, v_cache, topk_idx, n_valid, scale, out, lse, status,
+                    num_splits, scratch, need, stream);
+}
+
 const char* qsa_status_string(qsa_status_t status) {
   switch (status) {
     case QSA_OK: return "ok";
@@ -452,6 +501,7 @@ const char* qsa_status_string(qsa_status_t status) {
     case QSA_ERR_UNSUPPORTED: return "unsupported configuration (needs BF16, head_dim 256, G <= 16)";
     case QSA_ERR_ALIGN: return "rows must start on 16-byte boundaries";
     case QSA_ERR_CUDA: return "a CUDA runtime call failed";
+    case QSA_ERR_SCRATCH: return "the call needs more scratch than the built-in array holds (QSA_NOALLOC_SCRATCH_BYTES)";
   }
   return "unknown status";
 }
