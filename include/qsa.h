@@ -246,6 +246,24 @@ qsa_status_t qsa_sparse_prefill_fwd_host(
     const int32_t* n_valid_host, float scale, void* out_host,
     float* lse_host, const qsa_device_buffers_t* dev, void* stream);
 
+/*
+ * Failure-detection test hook (used by the test suite; not for production
+ * calls).  Runs the tcgen05 kernel of qsa_sparse_prefill_fwd_with on the given
+ * buffers with the producers' completion signal for the first shared-memory
+ * slot of every CTA withheld, so that no pipeline stage can ever complete.
+ * Every wait inside the kernel is bounded (2 s), so the kernel must end on
+ * its own, with QSA_STATUS_TIMEOUT set in *status (required here) and the
+ * CUDA context still usable; out/lse are left unspecified.  Same arguments
+ * as qsa_sparse_prefill_fwd; QSA_ERR_UNSUPPORTED when the tcgen05 kernel
+ * cannot take the layout.
+ */
+qsa_status_t qsa_test_stalled_pipeline(const qsa_shape_t* shape, const void* q,
+                                       const void* k_cache, const void* v_cache,
+                                       const int32_t* topk_idx,
+                                       const int32_t* n_valid, float scale,
+                                       void* out, float* lse, int32_t* status,
+                                       void* stream);
+
 /* Static description of a status code. */
 const char* qsa_status_string(qsa_status_t status);
 

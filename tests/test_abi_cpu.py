@@ -111,3 +111,9 @@ def test_binding_rejects_host_tensors(capi):
         capi.sparse_prefill_fwd(q, k, k, idx)
     with pytest.raises(TypeError):
         capi.sparse_prefill_fwd(q.float(), k, k, idx)
+
+
+def test_stall_hook_needs_a_status_word(capi):
+    s = _shape(capi)
+    assert capi.library().qsa_test_stalled_pipeline(ctypes.byref(s), P, P, P, P, None, 0.0, P, None,
+                                                    None, None) == 1

@@ -33,8 +33,8 @@ HEAD_DIM = 256
 # Every symbol include/qsa.h declares.
 EXPORTS = ("qsa_sparse_prefill_fwd", "qsa_sparse_prefill_fwd_with", "qsa_sparse_prefill_debug_gather",
            "qsa_sparse_prefill_fwd_host", "qsa_sparse_decode_fwd", "qsa_sparse_decode_workspace_bytes",
-           "qsa_sparse_decode_num_splits", "qsa_sparse_decode_fwd_noalloc", "qsa_status_string",
-           "qsa_abi_version")
+           "qsa_sparse_decode_num_splits", "qsa_sparse_decode_fwd_noalloc", "qsa_test_stalled_pipeline",
+           "qsa_status_string", "qsa_abi_version")
 
 
 class Shape(ctypes.Structure):
@@ -86,6 +86,9 @@ _lib.qsa_sparse_decode_num_splits.argtypes = [ctypes.POINTER(Shape), ctypes.c_in
 _lib.qsa_sparse_decode_fwd_noalloc.restype = ctypes.c_int
 _lib.qsa_sparse_decode_fwd_noalloc.argtypes = [ctypes.POINTER(Shape), _vp, _vp, _vp, _vp, _vp,
                                                ctypes.c_float, _vp, _vp, _vp, ctypes.c_int32, _vp]
+_lib.qsa_test_stalled_pipeline.restype = ctypes.c_int
+_lib.qsa_test_stalled_pipeline.argtypes = [ctypes.POINTER(Shape), _vp, _vp, _vp, _vp, _vp,
+                                           ctypes.c_float, _vp, _vp, _vp, _vp]
 _lib.qsa_status_string.restype = ctypes.c_char_p
 _lib.qsa_status_string.argtypes = [ctypes.c_int]
 _lib.qsa_abi_version.restype = ctypes.c_int32
@@ -342,3 +345,23 @@ def sparse_decode_fwd_noalloc(q, k_cache, v_cache, topk_idx, out, lse=None, n_va
                                             int(num_splits), stream)
     _raise(rc)
     return out, lse
+
+
+def run_stalled_pipeline_check(q, k_cache, v_cache, topk_idx, status, n_valid=None, scale: float = 0.0,
+                               stream=None):
+    """Failure-detection hook: runs the tcgen05 kernel with one pipeline signal
+    withheld; the kernel must stop on its own and set STATUS_TIMEOUT in `status`."""
+    dev = q.device
+    for name, x, dt in (("q", q, torch.bfloat16), ("k_cache", k_cache, torch.bfloat16),
+                        ("v_cache", v_cache, torch.bfloat16), ("topk_idx", topk_idx, torch.int32),
+                        ("status", status, torch.int32)):
+        _need(x, name, dt, dev)
+    _check_kv(k_cache, v_cache)
+    out = torch.empty(q.shape, dtype=torch.bfloat16, device=dev)
+    lse = torch.empty(q.shape[:2], dtype=torch.float32, device=dev)
+    shape = make_shape(q, k_cache, topk_idx, out, lse)
+    if stream is None:
+        stream = torch.cuda.current_stream(dev).cuda_stream
+    _raise(_lib.qsa_test_stalled_pipeline(ctypes.byref(shape), _ptr(q), _ptr(k_cache), _ptr(v_cache),
+                                          _ptr(topk_idx), _ptr(n_valid), float(scale), _ptr(out),
+                                          _ptr(lse), _ptr(status), stream))

@@ -155,7 +155,7 @@ cudaError_t launch_tc(const qsa::tc::TcParams& tp, cudaStream_t stream) {
 qsa_status_t run_forward(const qsa_shape_t* s, const void* q, const void* k, const void* v,
                          const int32_t* idx, const int32_t* n_valid, float scale, void* out,
                          float* lse, int32_t* status, int32_t* gathered, void* stream,
-                         qsa_kernel_t which = QSA_KERNEL_AUTO) {
+                         qsa_kernel_t which = QSA_KERNEL_AUTO, bool stall_test = false) {
   if (which != QSA_KERNEL_AUTO && which != QSA_KERNEL_TCGEN05 && which != QSA_KERNEL_WARP_MMA)
     return QSA_ERR_UNSUPPORTED;
   qsa_status_t rc = validate(s, q, k, v, idx, out);
@@ -225,6 +225,7 @@ qsa_status_t run_forward(const qsa_shape_t* s, const void* q, const void* k, con
     tp.chunk = p.K;
     tp.part_o = nullptr;
     tp.part_lse = nullptr;
+    tp.inject_stall = stall_test ? 1 : 0;
     e = dump ? launch_tc<true>(tp, st) : launch_tc<false>(tp, st);
   } else if (p.G <= 8)
     e = dump ? launch_mma<1, true>(p, st) : launch_mma<1, false>(p, st);
@@ -332,6 +333,7 @@ qsa_status_t run_decode(const qsa_shape_t* s, const void* q, const void* k, cons
   tp.chunk = pl.chunk;
   tp.part_o = part_o;
   tp.part_lse = part_lse;
+  tp.inject_stall = 0;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (launch_tc<false>(tp, st) != cudaSuccess) return QSA_ERR_CUDA;
   if (launch_merge(s, part_o, part_lse, pl.splits, out, lse, st) != cudaSuccess) return QSA_ERR_CUDA;
@@ -491,6 +493,16 @@ qsa_status_t qsa_sparse_decode_fwd_noalloc(const qsa_shape_t* shape, const void*
   if (need > 0 && noalloc_scratch_address(&scratch) != cudaSuccess) return QSA_ERR_CUDA;
   return run_decode(shape, q, k_cache, v_cache, topk_idx, n_valid, scale, out, lse, status,
                     num_splits, scratch, need, stream);
+}
+
+qsa_status_t qsa_test_stalled_pipeline(const qsa_shape_t* shape, const void* q,
+                                       const void* k_cache, const void* v_cache,
+                                       const int32_t* topk_idx, const int32_t* n_valid,
+                                       float scale, void* out, float* lse, int32_t* status,
+                                       void* stream) {
+  if (status == nullptr) return QSA_ERR_NULL;
+  return run_forward(shape, q, k_cache, v_cache, topk_idx, n_valid, scale, out, lse, status,
+                     nullptr, stream, QSA_KERNEL_TCGEN05, true);
 }
 
 const char* qsa_status_string(qsa_status_t status) {

@@ -100,6 +100,10 @@ struct TcParams {
   int32_t splits, chunk;
   float* part_o;
   float* part_lse;
+  // test hook: nonzero withholds the producers' signal for the first ring
+  // slot, so every wait must expire and the kernel must stop with
+  // kStatusTimeout (set only by the stall-test entry point)
+  int32_t inject_stall;
 };
 
 // Instruction descriptors (kind::f16): FP32 accumulator, BF16 A and B,
@@ -137,6 +141,17 @@ struct Sync {
         }
       }
     }
+  }
+
+  // Warp-collective bounded wait: lane 0 waits, every lane gets its verdict,
+  // so the lanes of a warp never split on an abort (which would strand the
+  // others at a later warp-synchronous instruction).  All 32 lanes must call it.
+  __device__ bool wait_warp(int i, uint32_t parity, int lane) const {
+    bool ok = true;
+    if (lane == 0) ok = wait(i, parity);
+    ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+    __syncwarp();  // orders lane 0's acquire before the other lanes' reads
+    return ok;
   }
 
   // Bounded wait that ignores the abort flag (used to drain in-flight copies).
@@ -223,6 +238,7 @@ template <bool kDump>
 __device__ void producer_role(const TcParams& p, const Sync& sy, uint32_t sb, int pw, int lane) {
   uint32_t c_slot = 0, c_unit = 0;
   const int64_t units = num_units(p);
+  uint32_t q_issued = 0, q_par = 0;                  // per Q buffer: load issued, its phase parity
   const int cc = lane & 15;                          // 16-byte chunk of the half row
   const int rsel = lane >> 4;                        // which of the two rows of an instruction
   const uint32_t dchunk = static_cast<uint32_t>((cc >> 3) * kBlockBytes);
@@ -239,6 +255,8 @@ __device__ void producer_role(const TcParams& p, const Sync& sy, uint32_t sb, in
           for (int b = 0; b < 4; ++b)
             tma_load_3d(sb + OFF_Q + qb * kQBytes + b * (kQBytes / 4), &p.tm_q, b * 64, un.g * p.G,
                         static_cast<int32_t>(un.t), sy.bar(B_QFULL + qb));
+          q_issued |= 1u << qb;
+          q_par = (q_par & ~(1u << qb)) | (((c_unit >> 1) & 1u) << qb);
         }
       }
       ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -271,7 +289,7 @@ __device__ void producer_role(const TcParams& p, const Sync& sy, uint32_t sb, in
       for (int h = 0; h < 4; ++h) {
         const uint32_t slot = c_slot % kSlots;
         const uint32_t round = c_slot / kSlots;
-        ok = sy.wait(B_EMPTY + slot, (round & 1u) ^ 1u);
+        ok = sy.wait_warp(B_EMPTY + slot, (round & 1u) ^ 1u, lane);
         if (!ok) break;
         const char* src0 = (h < 2 ? kbase : vbase) + (h & 1) * 256;
         const uint32_t dst0 = sb + OFF_RING + slot * kSlotBytes + dchunk;
@@ -283,13 +301,16 @@ __device__ void producer_role(const TcParams& p, const Sync& sy, uint32_t sb, in
           const char* src = live ? src0 + static_cast<int64_t>(rid) * row_bytes : src0;
           cp_async_16(dst0 + r * 128 + (((cc & 7) ^ (r & 7)) << 4), src, live ? 16 : 0);
         }
-        cp_async_mbar_arrive(sy.bar(B_FULL + slot));
+        if (!(p.inject_stall != 0 && c_slot == 0)) cp_async_mbar_arrive(sy.bar(B_FULL + slot));
         ++c_slot;
       }
     }
   }
   // every copy this lane issued has landed before the CTA can exit
   asm volatile("cp.async.wait_all;\n" ::: "memory");
+  if (pw == 0 && lane == 0)
+    for (int b = 0; b < 2; ++b)
+      if (q_issued & (1u << b)) sy.drain(B_QFULL + b, (q_par >> b) & 1u);
 }
 
 // ------------------------------------------------------------------ MMA issuers
@@ -420,7 +441,7 @@ __device__ void softmax_role(const TcParams& p, const Sync& sy, uint32_t sb, uin
       const int jn = (i + 1) * kKeys + key;
       id_next = (i + 1 < un.n_tiles && jn < un.n_eff) ? __ldg(list + jn) : -1;
       const bool valid = id >= 0 && id < p.S;
-      ok = sy.wait(B_SFULL + buf, (c >> 1) & 1u);
+      ok = sy.wait_warp(B_SFULL + buf, (c >> 1) & 1u, lane);
       if (!ok) break;
       tc_fence_after();
       uint32_t r[16];
@@ -439,7 +460,7 @@ __device__ void softmax_role(const TcParams& p, const Sync& sy, uint32_t sb, uin
       if ((lane & 1) == 0) rm[wq * 16 + ((lane >> 1) & 15)] = wmax;
       __syncwarp();
       if (lane == 0) mbar_arrive(sy.bar(B_RMAX + buf));
-      ok = sy.wait(B_RMAX + buf, (c >> 1) & 1u);  // all four warps' maxima are in
+      ok = sy.wait_warp(B_RMAX + buf, (c >> 1) & 1u, lane);  // all four warps' maxima are in
       if (!ok) break;
       float tmax[kGp];
 #pragma unroll
@@ -453,7 +474,7 @@ __device__ void softmax_role(const TcParams& p, const Sync& sy, uint32_t sb, uin
         // raise the running max: O (TMEM) and the partial sums scale by 2^(m_old - m_new)
         if (i > 0) {
           const uint32_t cp = c - 1;
-          ok = sy.wait(B_PEMPTY + (cp & 1u), (cp >> 1) & 1u);  // the previous PV has finished
+          ok = sy.wait_warp(B_PEMPTY + (cp & 1u), (cp >> 1) & 1u, lane);  // the previous PV has finished
           if (!ok) break;
         }
         tc_fence_after();
@@ -491,7 +512,7 @@ __device__ void softmax_role(const TcParams& p, const Sync& sy, uint32_t sb, uin
         l_part[h + 1] += p1;
         pk[h >> 1] = pack_bf16x2(p0, p1);
       }
-      ok = sy.wait(B_PEMPTY + buf, ((c >> 1) & 1u) ^ 1u);
+      ok = sy.wait_warp(B_PEMPTY + buf, ((c >> 1) & 1u) ^ 1u, lane);
       if (!ok) break;
       // P^T row of this key: heads 0-7 in the first 8x8 core-matrix column,
       // heads 8-15 in the second (2 KB further)
@@ -510,12 +531,12 @@ __device__ void softmax_role(const TcParams& p, const Sync& sy, uint32_t sb, uin
     if ((lane & 1) == 0) rs[wq * 16 + ((lane >> 1) & 15)] = wsum;
     __syncwarp();
     if (lane == 0) mbar_arrive(sy.bar(B_RSUM + (c_unit & 1u)));
-    ok = sy.wait(B_RSUM + (c_unit & 1u), (c_unit >> 1) & 1u);
+    ok = sy.wait_warp(B_RSUM + (c_unit & 1u), (c_unit >> 1) & 1u, lane);
     if (!ok) break;
     float l_tot[kGp];
 #pragma unroll
     for (int h = 0; h < kGp; ++h) l_tot[h] = (rs[h] + rs[16 + h]) + (rs[32 + h] + rs[48 + h]);
-    ok = sy.wait(B_OFULL, c_unit & 1u);
+    ok = sy.wait_warp(B_OFULL, c_unit & 1u, lane);
     if (!ok) break;
     tc_fence_after();
     uint32_t o0[16] = {}, o1[16] = {};
