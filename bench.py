@@ -59,6 +59,8 @@ def parse_args():
     ap.add_argument("--secondary", default="c4",
                     help="second workload reported under 'secondary' ('' to skip)")
     ap.add_argument("--kernel", default="auto", choices=["auto", "tcgen05", "warp_mma"])
+    ap.add_argument("--shard", default="replicas", choices=["replicas", "tokens"],
+                    help="N>1: independent replicas (weak scaling) or one workload's tokens split (strong)")
     ap.add_argument("--compare", default="warp_mma",
                     help="second kernel timed on the same workload ('' to skip)")
     ap.add_argument("--decode", default="decode",
@@ -82,6 +84,32 @@ def dist_env():
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     return world, rank, local
+
+
+def shard_range(n, world, rank):
+    """[start, end) of rank's share of n units (contiguous, sizes differ by at most 1)."""
+    base, rem = divmod(n, world)
+    start = rank * base + min(rank, rem)
+    return start, start + base + (1 if rank < rem else 0)
+
+
+def max_over_ranks(x, dist=None, device="cpu"):
+    """Max of a host float over all ranks (the identity without a process group)."""
+    if dist is None:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def shard_workload(w, world, rank):
+    """The rank's token slice of a workload (views into the same tensors)."""
+    t0, t1 = shard_range(w.shape["T"], world, rank)
+    import dataclasses
+    return dataclasses.replace(
+        w, q=w.q[t0:t1], topk_idx=w.topk_idx[t0:t1],
+        n_valid=None if w.n_valid is None else w.n_valid[t0:t1],
+        positions=w.positions[t0:t1], seq_start=w.seq_start[t0:t1])
 
 
 def measured_peaks():
@@ -333,28 +361,31 @@ def run_cuda(args):
     if world > 1:
         import torch.distributed as dist
         dist.init_process_group("nccl", device_id=dev, timeout=datetime.timedelta(seconds=120))
+        # the path has no exchange step: NCCL carries only the barrier and the
+        # max-over-ranks timing reduction
         pg = dist
 
     def barrier():
         if pg is not None:
             pg.barrier()
 
-    def max_over_ranks(x):
-        if pg is None:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        return float(t.item())
+    def max_ranks(x):
+        return max_over_ranks(x, pg, dev)
 
     from top_sparse_attention_qsa_b200 import _capi
     from top_sparse_attention_qsa_b200 import workloads as W
 
-    seed_off = 1000 * rank
+    # weak scaling (default): every rank runs its own replica (own seed);
+    # strong scaling (--shard tokens): the ranks split one workload's tokens
+    seed_off = 1000 * rank if args.shard == "replicas" else 0
     kw = {"seed": W.CONFIG_SEED_BASE + {"tiny": 1, "c2": 2, "c3": 3, "c4": 4, "c5": 5,
                                         "pages_long": 6}[args.workload] + seed_off}
     if args.tokens and args.workload in ("c4", "c5"):
         kw["T"] = args.tokens
     w = W.make(args.workload, device=dev, **kw)
+    T_job = w.shape["T"] * (world if args.shard == "replicas" else 1)
+    if args.shard == "tokens":
+        w = shard_workload(w, world, rank)
     acct = workload_accounting(w)
     out = torch.empty_like(w.q)
     lse = torch.empty(w.q.shape[:2], dtype=torch.float32, device=dev)
@@ -371,9 +402,9 @@ def run_cuda(args):
         time.sleep(0.3)
     total_ms, per_ms, (t0, t1) = time_launches(step, args.steps, args.warmup, barrier)
     clocks = sampler.stop(t0, t1) if sampler is not None else None
-    total_ms = max_over_ranks(total_ms)
+    total_ms = max_ranks(total_ms)
     T = w.shape["T"]
-    value = T * args.steps * world / (total_ms / 1e3)
+    value = T_job * args.steps / (total_ms / 1e3)
     mean_launch_ms = statistics.mean(per_ms)
     hbm, bf16, peak_src = measured_peaks()
     achieved = acct["algo_bytes"] / (mean_launch_ms / 1e3) / 1e9
@@ -389,8 +420,9 @@ def run_cuda(args):
     roof_time_ms = 1e3 * max(acct["gathered_bytes"] / (hbm * 1e9), acct["flops"] / (bf16 * 1e12))
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": config_of(w, acct), "gpu_launches": args.steps,
+            "scaling": "weak" if args.shard == "replicas" else "strong", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic", "config": config_of(w, acct),
+            "gpu_launches": args.steps,
             "gathered_kv_gbs": gathered_gbs, "effective_tflops": tflops,
             "roofline_time_ms": roof_time_ms, "frac_of_roofline_time": roof_time_ms / mean_launch_ms,
             "roofline": roof, "clocks": clocks}
@@ -402,19 +434,19 @@ def run_cuda(args):
             _capi.sparse_prefill_fwd(w.q, w.k_cache, w.v_cache, w.topk_idx, w.n_valid, w.scale,
                                      out=out, lse=lse, kernel=args.compare)
         cmp_ms, cmp_per, _ = time_launches(step_cmp, min(args.steps, 20), 3, barrier, "compare")
-        cmp_ms = max_over_ranks(cmp_ms)
+        cmp_ms = max_ranks(cmp_ms)
         n_cmp = min(args.steps, 20)
         line["compare"] = {"kernel": KERNEL_NAMES[args.compare],
                            "tokens_per_s": T * n_cmp * world / (cmp_ms / 1e3),
                            "mean_launch_ms": statistics.mean(cmp_per),
                            "algo_gbs": acct["algo_bytes"] / (statistics.mean(cmp_per) / 1e3) / 1e9}
     if not args.no_e2e and not args.profile:
-        line["e2e"] = run_e2e(w, args, barrier, max_over_ranks, world, dev)
+        line["e2e"] = run_e2e(w, args, barrier, max_ranks, T_job, dev)
     if args.secondary and not args.profile and args.secondary != args.workload:
-        line["secondary"] = run_secondary(args.secondary, dev, barrier, max_over_ranks, world, hbm,
+        line["secondary"] = run_secondary(args.secondary, dev, barrier, max_ranks, world, hbm,
                                           bf16, args.kernel)
     if args.decode and not args.profile:
-        line["decode"] = run_decode_bench(args.decode, dev, barrier, max_over_ranks, world, hbm)
+        line["decode"] = run_decode_bench(args.decode, dev, barrier, max_ranks, world, hbm)
     if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.profile:
         line["cpu_baseline"] = time_oracle(w, args.cpu_budget)
     elif not args.profile:
@@ -427,7 +459,7 @@ def run_cuda(args):
     return 0
 
 
-def run_e2e(w, args, barrier, max_over_ranks, world, dev):
+def run_e2e(w, args, barrier, reduce_max, T_job, dev):
     from top_sparse_attention_qsa_b200 import _capi
     hq = w.q.cpu().pin_memory()
     hk = w.k_cache.cpu().pin_memory()
@@ -447,17 +479,16 @@ def run_e2e(w, args, barrier, max_over_ranks, world, dev):
 
     steps = max(1, args.e2e_steps)
     total_ms, _, _ = time_launches(step, steps, 2, barrier, "e2e")
-    total_ms = max_over_ranks(total_ms)
+    total_ms = reduce_max(total_ms)
     h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv, hi) + ((hn,) if hn is not None else ()))
     d2h = ho.numel() * 2 + hl.numel() * 4
-    T = w.shape["T"]
-    return {"value": T * steps * world / (total_ms / 1e3), "unit": UNIT,
+    return {"value": T_job * steps / (total_ms / 1e3), "unit": UNIT,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
             "ms_per_step": total_ms / steps, "steps": steps,
             "api": "qsa_sparse_prefill_fwd_host (pinned host buffers)"}
 
 
-def run_secondary(name, dev, barrier, max_over_ranks, world, hbm, bf16, kernel="auto"):
+def run_secondary(name, dev, barrier, reduce_max, world, hbm, bf16, kernel="auto"):
     from top_sparse_attention_qsa_b200 import _capi
     w = make_workload(name, dev)
     acct = workload_accounting(w)
@@ -470,7 +501,7 @@ def run_secondary(name, dev, barrier, max_over_ranks, world, hbm, bf16, kernel="
 
     steps = 20
     total_ms, per_ms, _ = time_launches(step, steps, 3, barrier, "secondary")
-    total_ms = max_over_ranks(total_ms)
+    total_ms = reduce_max(total_ms)
     ms = statistics.mean(per_ms)
     roof_ms = 1e3 * max(acct["gathered_bytes"] / (hbm * 1e9), acct["flops"] / (bf16 * 1e12))
     return {"workload": w.name, "tokens_per_s": w.shape["T"] * steps * world / (total_ms / 1e3),
@@ -480,7 +511,7 @@ def run_secondary(name, dev, barrier, max_over_ranks, world, hbm, bf16, kernel="
             "frac_of_roofline_time": roof_ms / ms, "steps": steps}
 
 
-def run_decode_bench(name, dev, barrier, max_over_ranks, world, hbm):
+def run_decode_bench(name, dev, barrier, reduce_max, world, hbm):
     """Split-K decode (one query token per sequence): two launches per step
     (chunk kernel + merge), workspace allocated once outside the timed loop."""
     from top_sparse_attention_qsa_b200 import _capi
@@ -498,7 +529,7 @@ def run_decode_bench(name, dev, barrier, max_over_ranks, world, hbm):
 
     steps = 50
     total_ms, per_ms, _ = time_launches(step, steps, 5, barrier, "decode")
-    total_ms = max_over_ranks(total_ms)
+    total_ms = reduce_max(total_ms)
     ms = statistics.mean(per_ms)
     algo = acct["algo_bytes"] + need  # partial results are written once and read once by the merge
     return {"workload": w.name, "desc": w.description, "splits": splits,
