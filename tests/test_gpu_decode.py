@@ -42,8 +42,16 @@ def test_decode_config_full():
     """64 sequences x 32768 cached tokens, heads (24,2), K=2048, auto chunks."""
     from top_sparse_attention_qsa_b200 import _capi as C
     w = W.make("decode", device=DEV)
-    assert C.decode_num_splits(w.q, w.k_cache, w.topk_idx) > 1
     print(check(C, w, "decode"))
+    print(check(C, w, "decode_4_chunks", num_splits=4))
+
+
+def test_decode_few_units_auto_splits():
+    """Two sequences, one KV head: units are scarce, so the automatic choice splits."""
+    from top_sparse_attention_qsa_b200 import _capi as C
+    w = W.config_decode(device=DEV, B=2, ctx=20000, heads=(12, 1), topk=4096, local=128)
+    assert C.decode_num_splits(w.q, w.k_cache, w.topk_idx) > 1
+    check(C, w, "decode_auto")
 
 
 @pytest.mark.parametrize("splits", [0, 1, 2, 3, 7, 16, 100])

@@ -244,9 +244,13 @@ struct SplitPlan {
   size_t total_bytes;
 };
 
-// Chunk count for a decode-shaped call: enough (token, KV head, chunk) units
-// for two per SM when num_splits <= 0, never chunks shorter than one 128-entry
-// tile.  Deterministic for a given shape and device.
+// Chunk count for a decode-shaped call, never chunks shorter than one
+// 128-entry tile.  With num_splits <= 0: one chunk unless the (token, KV head)
+// units would leave most SMs idle (fewer than SMs / 8), then enough chunks of
+// at least 256 entries for about one unit per SM.  (Each unit carries a few
+// microseconds of serial start and epilogue latency, so short chunks cost
+// more than idle SMs until the units are that scarce.)  Deterministic for a
+// given shape and device.
 bool plan_splits(const qsa_shape_t* s, int32_t num_splits, SplitPlan* pl) {
   const int64_t K = s->topk;
   const int64_t max_splits = K > 0 ? (K + qsa::tc::kKeys - 1) / qsa::tc::kKeys : 1;
@@ -255,7 +259,12 @@ bool plan_splits(const qsa_shape_t* s, int32_t num_splits, SplitPlan* pl) {
     const int nsm = sm_count();
     if (nsm <= 0) return false;
     const int64_t units = s->num_tokens * s->num_kv_heads;
-    splits = units > 0 ? (2 * static_cast<int64_t>(nsm) + units - 1) / units : 1;
+    splits = 1;
+    if (units > 0 && units * 8 < nsm) {
+      splits = (nsm + units - 1) / units;
+      const int64_t by_len = K / 256;
+      if (splits > by_len) splits = by_len < 1 ? 1 : by_len;
+    }
   }
   splits = splits < 1 ? 1 : (splits > max_splits ? max_splits : splits);
   int64_t chunk = K > 0 ? (K + splits - 1) / splits : 0;
