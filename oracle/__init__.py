@@ -63,6 +63,8 @@ class _Args(ctypes.Structure):
         ("idx", ctypes.c_void_p),
         ("n_valid", ctypes.c_void_p),
         ("scale", ctypes.c_double),
+        ("block_size", ctypes.c_int64),
+        ("last_slot", ctypes.c_void_p),
     ]
 
 
@@ -84,9 +86,9 @@ class Oracle:
         return self.lib.qsa_oracle_bf16_to_double(ctypes.c_uint16(bits))
 
     def sparse_prefill(self, q, k_cache, v_cache, topk_idx, n_valid=None, scale=0.0,
-                       tokens=None, n_threads=None):
+                       tokens=None, n_threads=None, block_size=1, last_slot=None):
         return _sparse_prefill(self.lib, q, k_cache, v_cache, topk_idx, n_valid, scale,
-                               tokens, n_threads)
+                               tokens, n_threads, block_size, last_slot)
 
 
 _default = None
@@ -140,14 +142,19 @@ def bf16_to_double(bits: int) -> float:
 
 
 def sparse_prefill(q, k_cache, v_cache, topk_idx, n_valid=None, scale=0.0,
-                   tokens=None, n_threads=None):
+                   tokens=None, n_threads=None, block_size=1, last_slot=None):
     return default().sparse_prefill(q, k_cache, v_cache, topk_idx, n_valid, scale,
-                                    tokens, n_threads)
+                                    tokens, n_threads, block_size, last_slot)
 
 
-def _sparse_prefill(lib, q, k_cache, v_cache, topk_idx, n_valid, scale, tokens, n_threads):
+def _sparse_prefill(lib, q, k_cache, v_cache, topk_idx, n_valid, scale, tokens, n_threads,
+                    block_size=1, last_slot=None):
     """FP64 oracle.  q [T,Hq,D], k_cache/v_cache [S,Hkv,D] (BF16, host),
     topk_idx [T,Hkv,K] int32, n_valid [T,Hkv] int32 or None.
+
+    block_size > 1: list entries name microblocks of that many consecutive
+    slots (n_valid counts entries); last_slot [T] int32 bounds the slots each
+    token sees (None: no bound).
 
     Returns (out [n,Hq,D] float64, lse [n,Hq] float64, n_out_of_range) for the
     tokens listed in ``tokens`` (all tokens when None).
@@ -179,9 +186,15 @@ def _sparse_prefill(lib, q, k_cache, v_cache, topk_idx, n_valid, scale, tokens, 
     n = tokens.shape[0]
     out = np.zeros((n, Hq, D), dtype=np.float64)
     lse = np.zeros((n, Hq), dtype=np.float64)
+    ls = _as_i32(last_slot)
+    if ls is not None:
+        if ls.shape != (T,):
+            raise ValueError("last_slot must be [T]")
+        ls = np.ascontiguousarray(ls)
     a = _Args(T, Hq, Hkv, D, K, S, qs[0], qs[1], ks[0], ks[1], ist[0], ist[1],
               q.ctypes.data, k.ctypes.data, v.ctypes.data, idx.ctypes.data,
-              nv.ctypes.data if nv is not None else None, float(scale))
+              nv.ctypes.data if nv is not None else None, float(scale), int(block_size),
+              ls.ctypes.data if ls is not None else None)
     if n_threads is None:
         n_threads = os.cpu_count() or 1
     rc = lib.qsa_oracle_fwd(ctypes.byref(a), tokens.ctypes.data, n, int(n_threads),

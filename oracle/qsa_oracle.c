@@ -12,6 +12,7 @@
 
 #include <math.h>
 #include <pthread.h>
+#include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
 
@@ -52,15 +53,24 @@ static int64_t one_row(const qsa_oracle_args* a, int64_t t, int64_t h,
     if (n_list < 0) n_list = 0;
   }
   const int32_t* list = a->idx + t * a->idx_stride_tok + g * a->idx_stride_head;
+  /* Microblock lists: entry j covers block_size consecutive slots, each a key
+   * (page "Qwen4-Exp QSA llega al Ascend de Huawei", section "Por qué QSA es
+   * la parte incómoda, en cifras": QSA selects at microblock granularity). */
+  const int64_t bs = a->block_size > 1 ? a->block_size : 1;
+  const int64_t limit = a->last_slot ? a->last_slot[t] : INT64_MAX;
   int64_t n = 0;
   for (int64_t j = 0; j < n_list; ++j) {
-    int64_t slot = list[j];
-    if (slot < 0) continue;
-    if (slot >= a->num_slots) {
+    int64_t id = list[j];
+    if (id < 0) continue;
+    if (id * bs >= a->num_slots) {
       if (h % G == 0) ++oob; /* count each list entry once, not per head */
       continue;
     }
-    sel[n++] = slot;
+    for (int64_t r = 0; r < bs; ++r) {
+      const int64_t slot = id * bs + r;
+      if (slot >= a->num_slots || slot > limit) continue;
+      sel[n++] = slot;
+    }
   }
 
   /* Empty selection: zero output, lse = -inf. */
@@ -102,7 +112,7 @@ static void* worker(void* arg) {
   job_t* job = (job_t*)arg;
   const qsa_oracle_args* a = job->a;
   const int64_t Hq = a->num_q_heads, D = a->head_dim;
-  const int64_t cap = a->topk > 0 ? a->topk : 1;
+  const int64_t cap = (a->topk > 0 ? a->topk : 1) * (a->block_size > 1 ? a->block_size : 1);
   int64_t* sel = (int64_t*)malloc((size_t)cap * sizeof(int64_t));
   double* s = (double*)malloc((size_t)cap * sizeof(double));
   if (!sel || !s) {

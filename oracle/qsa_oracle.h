@@ -45,6 +45,11 @@ typedef struct {
   const int32_t* idx;       /* -1 (or any negative) = empty entry */
   const int32_t* n_valid;   /* [T, Hkv] contiguous, or NULL meaning K */
   double scale;             /* <= 0 selects 1/sqrt(D) */
+  /* Microblock lists (0 or 1 = token lists): entry j names block idx[j], the
+   * slots idx[j]*block_size + r, r < block_size; n_valid counts entries. */
+  int64_t block_size;
+  /* [T] largest visible slot per token (slots above it are empty), or NULL. */
+  const int32_t* last_slot;
 } qsa_oracle_args;
 
 /*

@@ -23,6 +23,8 @@ Pins (what the pages and the mathematics fix):
 * worked_example -- the hand-derived fixture in tests/golden.
 * split_merge   -- attention over a list equals the log-sum-exp merge of
   attention over any split of it (the combine step of split-K decode).
+* block_lists   -- a microblock list equals the token list naming each of its
+  slots (with the cache end and the token's last visible slot applied).
 """
 from __future__ import annotations
 
@@ -261,6 +263,39 @@ def check_split_merge(orc):
         np.testing.assert_allclose(lse, lse_full, **TOL)
 
 
+def check_block_lists(orc):
+    """A microblock list equals the token list that names each of its slots
+    (entry b -> slots b*bs .. b*bs+bs-1), with slots beyond the cache or the
+    token's last visible slot dropped; block size 1 is the token list."""
+    gen = torch.Generator().manual_seed(61)
+    T, S, Hq, Hkv, E = 6, 203, 16, 2, 9
+    q = W.normal_bf16((T, Hq, 256), gen, "cpu")
+    k = W.normal_bf16((S, Hkv, 256), gen, "cpu")
+    v = W.normal_bf16((S, Hkv, 256), gen, "cpu")
+    for bs in (1, 2, 4):
+        nb = (S + bs - 1) // bs
+        blocks = torch.stack([torch.randperm(nb, generator=gen)[:E] for _ in range(T * Hkv)]).view(T, Hkv, E)
+        blocks[0, 0, 3] = -1
+        blocks = blocks.to(torch.int32)
+        last = torch.randint(S // 2, S, (T,), generator=gen, dtype=torch.int32)
+        nv = torch.randint(0, E + 1, (T, Hkv), generator=gen, dtype=torch.int32)
+        got = orc.sparse_prefill(q, k, v, blocks, nv, 0.0, block_size=bs, last_slot=last)
+        tok = torch.full((T, Hkv, E * bs), -1, dtype=torch.int32)
+        for t in range(T):
+            for g in range(Hkv):
+                for j in range(int(nv[t, g])):
+                    b = int(blocks[t, g, j])
+                    if b < 0:
+                        continue
+                    for r in range(bs):
+                        s_ = b * bs + r
+                        if s_ < S and s_ <= int(last[t]):
+                            tok[t, g, j * bs + r] = s_
+        want = orc.sparse_prefill(q, k, v, tok, None, 0.0)
+        np.testing.assert_allclose(got[0], want[0], **TOL)
+        np.testing.assert_allclose(got[1], want[1], **TOL)
+
+
 ALL_CHECKS = [check_bf16_widening, check_dense_causal, check_packing, check_permutation,
               check_head_padding, check_closed_forms, check_brute_force, check_worked_example,
-              check_split_merge]
+              check_split_merge, check_block_lists]

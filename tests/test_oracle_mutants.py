@@ -28,6 +28,8 @@ MUTANTS = {
     "widening_shift": ("((uint32_t)bits) << 16", "((uint32_t)bits) << 15"),
     "idx_head_stride_dropped": ("g * a->idx_stride_head", "0 * a->idx_stride_head"),
     "sum_before_exp": ("{ s[j] = exp(s[j] - m); l += s[j]; }", "{ l += s[j]; s[j] = exp(s[j] - m); }"),
+    "block_offset_dropped": ("const int64_t slot = id * bs + r;", "const int64_t slot = id * bs;"),
+    "last_slot_ignored": ("if (slot >= a->num_slots || slot > limit) continue;", "if (slot >= a->num_slots) continue;"),
     "v_head_stride_dropped": ("const uint16_t* vr = a->v + sel[j] * a->kv_stride_slot + g * a->kv_stride_head;",
                               "const uint16_t* vr = a->v + sel[j] * a->kv_stride_slot;"),
 }
