@@ -65,6 +65,8 @@ def parse_args():
                     help="second kernel timed on the same workload ('' to skip)")
     ap.add_argument("--decode", default="decode",
                     help="decode workload timed under 'decode' ('' to skip)")
+    ap.add_argument("--blocks", default="c5_block4",
+                    help="microblock-list workload timed under 'blocks' ('' to skip)")
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -447,6 +449,8 @@ def run_cuda(args):
                                           bf16, args.kernel)
     if args.decode and not args.profile:
         line["decode"] = run_decode_bench(args.decode, dev, barrier, max_ranks, world, hbm)
+    if args.blocks and not args.profile:
+        line["blocks"] = run_blocks_bench(args.blocks, dev, barrier, max_ranks, world, hbm)
     if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.profile:
         line["cpu_baseline"] = time_oracle(w, args.cpu_budget)
     elif not args.profile:
@@ -537,6 +541,38 @@ def run_decode_bench(name, dev, barrier, reduce_max, world, hbm):
             "mean_step_ms": ms, "gathered_kv_gbs": acct["gathered_bytes"] / (ms / 1e3) / 1e9,
             "algo_gbs": algo / (ms / 1e3) / 1e9, "frac_of_hbm": algo / (ms / 1e3) / 1e9 / hbm,
             "launches_per_step": 2 if need > 0 else 1, "steps": steps}
+
+
+def run_blocks_bench(name, dev, barrier, reduce_max, world, hbm):
+    """Microblock lists on the c5 shape: the same 2048 keys per (token, KV
+    head) as c5, named by 512 blocks of 4 slots."""
+    from top_sparse_attention_qsa_b200 import _capi
+    w = make_workload(name, dev)
+    out = torch.empty_like(w.q)
+    lse = torch.empty(w.q.shape[:2], dtype=torch.float32, device=dev)
+    bs = w.block_size
+    # live keys: expand each live entry to its visible slots
+    idx = w.topk_idx.to(torch.int64)
+    E = idx.shape[2]
+    live_e = (idx >= 0) & (torch.arange(E, device=dev)[None, None, :] < w.n_valid[:, :, None])
+    slots = idx[..., None] * bs + torch.arange(bs, device=dev)
+    vis = live_e[..., None] & (slots < w.shape["S"]) & (slots <= w.last_slot.to(torch.int64)[:, None, None, None])
+    keys = int(vis.sum().item())
+    s = w.shape
+    algo = keys * 1024 + int(live_e.sum().item()) * 4 + s["T"] * s["Hq"] * s["D"] * 4 + s["T"] * s["Hq"] * 4
+
+    def step():
+        _capi.sparse_prefill_block_fwd(w.q, w.k_cache, w.v_cache, w.topk_idx, bs, w.last_slot,
+                                       w.n_valid, w.scale, out=out, lse=lse)
+
+    steps = 20
+    total_ms, per_ms, _ = time_launches(step, steps, 3, barrier, "blocks")
+    total_ms = reduce_max(total_ms)
+    ms = statistics.mean(per_ms)
+    return {"workload": w.name, "desc": w.description, "tokens_per_s": s["T"] * steps * world / (total_ms / 1e3),
+            "mean_launch_ms": ms, "live_keys": keys, "gathered_kv_gbs": keys * 1024 / (ms / 1e3) / 1e9,
+            "algo_gbs": algo / (ms / 1e3) / 1e9, "frac_of_hbm": algo / (ms / 1e3) / 1e9 / hbm,
+            "steps": steps}
 
 
 def main():

@@ -140,6 +140,31 @@ qsa_status_t qsa_sparse_prefill_debug_gather(
     int32_t* gathered_ids, void* stream);
 
 /*
+ * Microblock lists (page "Qwen4-Exp QSA llega al Ascend de Huawei", section
+ * "Por qué QSA es la parte incómoda, en cifras": QSA selects microblocks,
+ * 2048 per query at compression ratio 4).  Entry j of a list names block
+ * idx[t,g,j]; the block's block_size consecutive slots idx*block_size + r,
+ * r < block_size, are each one key of the attention.  K = shape->topk and
+ * n_valid count entries; an entry whose block starts at or beyond S is
+ * empty and sets status bit 0; slots of a live block at or beyond S are
+ * empty.  last_slot (int32 device [T], or NULL) is the largest slot each
+ * token may see: slots above it are empty, which masks the part of the
+ * newest block past the query's own position (the causal tail).  block_size
+ * is 1, 2, 4, 8 or 16; K * block_size < 2^31.  Runs the tcgen05 kernel only
+ * (QSA_ERR_UNSUPPORTED when the Q layout does not fit a TMA descriptor).
+ * Other arguments and conventions as qsa_sparse_prefill_fwd.
+ */
+qsa_status_t qsa_sparse_prefill_block_fwd(const qsa_shape_t* shape,
+                                          int32_t block_size,
+                                          const int32_t* last_slot,
+                                          const void* q, const void* k_cache,
+                                          const void* v_cache,
+                                          const int32_t* topk_idx,
+                                          const int32_t* n_valid, float scale,
+                                          void* out, float* lse,
+                                          int32_t* status, void* stream);
+
+/*
  * Split-K sparse attention for decode-shaped calls: few query tokens per KV
  * head (one per sequence in decode) with long lists.  Each list is cut into
  * chunks of a multiple of 128 entries; every (token, KV head, chunk) runs on

@@ -32,6 +32,7 @@ HEAD_DIM = 256
 
 # Every symbol include/qsa.h declares.
 EXPORTS = ("qsa_sparse_prefill_fwd", "qsa_sparse_prefill_fwd_with", "qsa_sparse_prefill_debug_gather",
+           "qsa_sparse_prefill_block_fwd",
            "qsa_sparse_prefill_fwd_host", "qsa_sparse_decode_fwd", "qsa_sparse_decode_workspace_bytes",
            "qsa_sparse_decode_num_splits", "qsa_sparse_decode_fwd_noalloc", "qsa_test_stalled_pipeline",
            "qsa_status_string", "qsa_abi_version")
@@ -89,6 +90,9 @@ _lib.qsa_sparse_decode_fwd_noalloc.argtypes = [ctypes.POINTER(Shape), _vp, _vp, 
 _lib.qsa_test_stalled_pipeline.restype = ctypes.c_int
 _lib.qsa_test_stalled_pipeline.argtypes = [ctypes.POINTER(Shape), _vp, _vp, _vp, _vp, _vp,
                                            ctypes.c_float, _vp, _vp, _vp, _vp]
+_lib.qsa_sparse_prefill_block_fwd.restype = ctypes.c_int
+_lib.qsa_sparse_prefill_block_fwd.argtypes = [ctypes.POINTER(Shape), ctypes.c_int32, _vp, _vp, _vp, _vp,
+                                              _vp, _vp, ctypes.c_float, _vp, _vp, _vp, _vp]
 _lib.qsa_status_string.restype = ctypes.c_char_p
 _lib.qsa_status_string.argtypes = [ctypes.c_int]
 _lib.qsa_abi_version.restype = ctypes.c_int32
@@ -365,3 +369,41 @@ def run_stalled_pipeline_check(q, k_cache, v_cache, topk_idx, status, n_valid=No
     _raise(_lib.qsa_test_stalled_pipeline(ctypes.byref(shape), _ptr(q), _ptr(k_cache), _ptr(v_cache),
                                           _ptr(topk_idx), _ptr(n_valid), float(scale), _ptr(out),
                                           _ptr(lse), _ptr(status), stream))
+
+
+def sparse_prefill_block_fwd(q, k_cache, v_cache, block_idx, block_size: int, last_slot=None,
+                             n_valid=None, scale: float = 0.0, out=None, lse=None, status=None,
+                             stream=None, want_lse: bool = True):
+    """Microblock lists: block_idx [T, Hkv, E] names blocks of `block_size`
+    consecutive slots; last_slot [T] int32 bounds the slots each token sees."""
+    dev = q.device
+    _need(q, "q", torch.bfloat16, dev)
+    _need(k_cache, "k_cache", torch.bfloat16, dev)
+    _need(v_cache, "v_cache", torch.bfloat16, dev)
+    _need(block_idx, "block_idx", torch.int32, dev)
+    _check_kv(k_cache, v_cache)
+    if last_slot is not None:
+        _need(last_slot, "last_slot", torch.int32, dev)
+        if not last_slot.is_contiguous() or tuple(last_slot.shape) != (q.shape[0],):
+            raise ValueError("last_slot must be a contiguous [T] tensor")
+    if n_valid is not None:
+        _need(n_valid, "n_valid", torch.int32, dev)
+        if not n_valid.is_contiguous() or tuple(n_valid.shape) != tuple(block_idx.shape[:2]):
+            raise ValueError("n_valid must be a contiguous [T, Hkv] tensor")
+    if out is None:
+        out = torch.empty(q.shape, dtype=torch.bfloat16, device=dev)
+    _need(out, "out", torch.bfloat16, dev)
+    if lse is None and want_lse:
+        lse = torch.empty(q.shape[:2], dtype=torch.float32, device=dev)
+    if lse is not None:
+        _need(lse, "lse", torch.float32, dev)
+    if status is not None:
+        _need(status, "status", torch.int32, dev)
+    shape = make_shape(q, k_cache, block_idx, out, lse)
+    if stream is None:
+        stream = torch.cuda.current_stream(dev).cuda_stream
+    _raise(_lib.qsa_sparse_prefill_block_fwd(ctypes.byref(shape), int(block_size), _ptr(last_slot),
+                                             _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_idx),
+                                             _ptr(n_valid), float(scale), _ptr(out), _ptr(lse),
+                                             _ptr(status), stream))
+    return out, lse

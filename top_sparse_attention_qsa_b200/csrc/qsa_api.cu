@@ -138,10 +138,10 @@ bool make_tc_params(const qsa_shape_t* s, const void* q, qsa::tc::TcParams* tp) 
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <bool kDump>
+template <bool kDump, bool kStall = false, bool kBlocks = false>
 cudaError_t launch_tc(const qsa::tc::TcParams& tp, cudaStream_t stream) {
   static std::atomic<int> done[kMaxDevices];
-  auto kernel = qsa::tc::qsa_prefill_tc_kernel<kDump>;
+  auto kernel = qsa::tc::qsa_prefill_tc_kernel<kDump, kStall, kBlocks>;
   cudaError_t e = set_smem_once(kernel, qsa::tc::SMEM_BYTES, done);
   if (e != cudaSuccess) return e;
   const int64_t units = tp.T * tp.Hkv;
@@ -225,8 +225,10 @@ qsa_status_t run_forward(const qsa_shape_t* s, const void* q, const void* k, con
     tp.chunk = p.K;
     tp.part_o = nullptr;
     tp.part_lse = nullptr;
-    tp.inject_stall = stall_test ? 1 : 0;
-    e = dump ? launch_tc<true>(tp, st) : launch_tc<false>(tp, st);
+    tp.block_shift = 0;
+    tp.last_slot = nullptr;
+    e = stall_test ? launch_tc<false, true>(tp, st)
+                   : (dump ? launch_tc<true>(tp, st) : launch_tc<false>(tp, st));
   } else if (p.G <= 8)
     e = dump ? launch_mma<1, true>(p, st) : launch_mma<1, false>(p, st);
   else
@@ -342,7 +344,8 @@ qsa_status_t run_decode(const qsa_shape_t* s, const void* q, const void* k, cons
   tp.chunk = pl.chunk;
   tp.part_o = part_o;
   tp.part_lse = part_lse;
-  tp.inject_stall = 0;
+  tp.block_shift = 0;
+  tp.last_slot = nullptr;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (launch_tc<false>(tp, st) != cudaSuccess) return QSA_ERR_CUDA;
   if (launch_merge(s, part_o, part_lse, pl.splits, out, lse, st) != cudaSuccess) return QSA_ERR_CUDA;
@@ -502,6 +505,56 @@ qsa_status_t qsa_sparse_decode_fwd_noalloc(const qsa_shape_t* shape, const void*
   if (need > 0 && noalloc_scratch_address(&scratch) != cudaSuccess) return QSA_ERR_CUDA;
   return run_decode(shape, q, k_cache, v_cache, topk_idx, n_valid, scale, out, lse, status,
                     num_splits, scratch, need, stream);
+}
+
+qsa_status_t qsa_sparse_prefill_block_fwd(const qsa_shape_t* shape, int32_t block_size,
+                                          const int32_t* last_slot, const void* q,
+                                          const void* k_cache, const void* v_cache,
+                                          const int32_t* topk_idx, const int32_t* n_valid,
+                                          float scale, void* out, float* lse, int32_t* status,
+                                          void* stream) {
+  qsa_status_t rc = validate(shape, q, k_cache, v_cache, topk_idx, out);
+  if (rc != QSA_OK) return rc;
+  int shift = -1;
+  for (int b = 0; b <= 4; ++b)
+    if (block_size == (1 << b)) shift = b;
+  if (shift < 0) return QSA_ERR_UNSUPPORTED;
+  if ((static_cast<int64_t>(shape->topk) << shift) > 0x7fffffffLL) return QSA_ERR_UNSUPPORTED;
+  if (shape->num_tokens == 0) return QSA_OK;
+  static thread_local qsa::tc::TcParams tp;
+  if (!make_tc_params(shape, q, &tp)) return QSA_ERR_UNSUPPORTED;
+  const float sc = scale > 0.f ? scale : 0.0625f;
+  tp.idx = topk_idx;
+  tp.n_valid = n_valid;
+  tp.kraw = k_cache;
+  tp.vraw = v_cache;
+  tp.out = static_cast<__nv_bfloat16*>(out);
+  tp.lse = lse;
+  tp.status = status;
+  tp.gathered = nullptr;
+  tp.T = shape->num_tokens;
+  tp.idx_st = shape->idx_stride_tok;
+  tp.idx_sh = shape->idx_stride_head;
+  tp.o_st = shape->o_stride_tok;
+  tp.o_sh = shape->o_stride_head;
+  tp.lse_st = shape->lse_stride_tok;
+  tp.kv_ss = shape->kv_stride_slot;
+  tp.kv_sh = shape->kv_stride_head;
+  tp.Hkv = shape->num_kv_heads;
+  tp.G = shape->num_q_heads / shape->num_kv_heads;
+  tp.K = shape->topk;
+  tp.S = static_cast<int32_t>(shape->num_slots);
+  tp.scale_log2 = sc * 1.4426950408889634f;
+  tp.splits = 1;
+  tp.chunk = shape->topk << shift;
+  tp.part_o = nullptr;
+  tp.part_lse = nullptr;
+  tp.block_shift = shift;
+  tp.last_slot = last_slot;
+  const cudaError_t e = shift == 0 && last_slot == nullptr
+                            ? launch_tc<false>(tp, static_cast<cudaStream_t>(stream))
+                            : launch_tc<false, false, true>(tp, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? QSA_OK : QSA_ERR_CUDA;
 }
 
 qsa_status_t qsa_test_stalled_pipeline(const qsa_shape_t* shape, const void* q,

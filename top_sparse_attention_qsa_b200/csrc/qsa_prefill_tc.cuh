@@ -100,10 +100,12 @@ struct TcParams {
   int32_t splits, chunk;
   float* part_o;
   float* part_lse;
-  // test hook: nonzero withholds the producers' signal for the first ring
-  // slot, so every wait must expire and the kernel must stop with
-  // kStatusTimeout (set only by the stall-test entry point)
-  int32_t inject_stall;
+  // microblock lists: entry e names slots (idx[e] << block_shift) + r, r <
+  // 2^block_shift, each one key (0: token lists); last_slot [T] bounds the
+  // slots a token sees (nullptr: no bound).  K and n_valid count entries;
+  // chunk counts keys.
+  int32_t block_shift;
+  const int32_t* last_slot;
 };
 
 // Instruction descriptors (kind::f16): FP32 accumulator, BF16 A and B,
@@ -143,16 +145,12 @@ struct Sync {
     }
   }
 
-  // Warp-collective bounded wait: lane 0 waits, every lane gets its verdict,
-  // so the lanes of a warp never split on an abort (which would strand the
-  // others at a later warp-synchronous instruction).  All 32 lanes must call it.
-  __device__ bool wait_warp(int i, uint32_t parity, int lane) const {
-    bool ok = true;
-    if (lane == 0) ok = wait(i, parity);
-    ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-    __syncwarp();  // orders lane 0's acquire before the other lanes' reads
-    return ok;
-  }
+  // Bounded wait called by all 32 lanes of a warp in convergent code.  The
+  // lanes poll the same barrier word and read the same abort flag and timer
+  // in the same instructions, so they leave the loop together with the same
+  // verdict; an explicit vote after every wait measured 5-6 % slower on the
+  // full workloads.
+  __device__ bool wait_warp(int i, uint32_t parity) const { return wait(i, parity); }
 
   // Bounded wait that ignores the abort flag (used to drain in-flight copies).
   __device__ void drain(int i, uint32_t parity) const {
@@ -185,10 +183,41 @@ __device__ __forceinline__ Unit decode_unit(const TcParams& p, int64_t u) {
   r.s = static_cast<int>(rem - r.t * p.splits);
   int n = p.K;
   if (p.n_valid != nullptr) n = min(n, max(__ldg(p.n_valid + r.t * p.Hkv + r.g), 0));
+  const int n_keys = n << p.block_shift;
   r.j0 = r.s * p.chunk;
-  r.n_eff = max(0, min(n - r.j0, p.chunk));
+  r.n_eff = max(0, min(n_keys - r.j0, p.chunk));
   r.n_tiles = (r.n_eff + kKeys - 1) / kKeys;
   return r;
+}
+
+// List entry behind key `local` (counted from the unit's first key), or -1
+// past the unit's live range.  A plain load with no use of its value, so it
+// can be issued a tile ahead and resolved (key_slot) when needed.
+template <bool kBlocks>
+__device__ __forceinline__ int32_t key_entry(const TcParams& p, const int32_t* list, const Unit& un,
+                                             int local) {
+  const int key = un.j0 + local;
+  return local < un.n_eff ? __ldg(list + (kBlocks ? key >> p.block_shift : key)) : -1;
+}
+
+// Cache slot of key `local` given its list entry: -1 when the key is masked
+// (negative entry, past the cache end or the token's last visible slot), -2
+// when the entry names a block that starts beyond the cache (reported
+// through the status word).
+template <bool kBlocks>
+__device__ __forceinline__ int32_t key_slot(const TcParams& p, const Unit& un, int local,
+                                            int32_t entry, int32_t last) {
+  if (entry < 0) return -1;
+  if (!kBlocks) return entry >= p.S ? -2 : entry;
+  const int64_t start = static_cast<int64_t>(entry) << p.block_shift;
+  if (start >= p.S) return -2;
+  const int64_t slot = start + ((un.j0 + local) & ((1 << p.block_shift) - 1));
+  if (slot >= p.S || slot > last) return -1;
+  return static_cast<int32_t>(slot);
+}
+
+__device__ __forceinline__ int32_t last_visible(const TcParams& p, int64_t t) {
+  return p.last_slot != nullptr ? __ldg(p.last_slot + t) : 0x7fffffff;
 }
 
 // Reduce 16 per-lane values across the 32 lanes of a warp by exchanging
@@ -234,7 +263,9 @@ __device__ __forceinline__ float xreduce16(const float (&v)[16], int lane) {
 // (16 lanes each).
 // Masked entries are zero-filled without a global read.  Every lane signals
 // the slot's full barrier when its own copies land (cp.async.mbarrier.arrive).
-template <bool kDump>
+// kStall (test hook): withhold the completion signal of the first ring slot,
+// so that every wait must expire and the kernel must stop with kStatusTimeout.
+template <bool kDump, bool kStall, bool kBlocks>
 __device__ void producer_role(const TcParams& p, const Sync& sy, uint32_t sb, int pw, int lane) {
   uint32_t c_slot = 0, c_unit = 0;
   const int64_t units = num_units(p);
@@ -263,7 +294,8 @@ __device__ void producer_role(const TcParams& p, const Sync& sy, uint32_t sb, in
     }
     ++c_unit;
     if (!ok) break;
-    const int32_t* list = p.idx + un.t * p.idx_st + static_cast<int64_t>(un.g) * p.idx_sh + un.j0;
+    const int32_t* list = p.idx + un.t * p.idx_st + static_cast<int64_t>(un.g) * p.idx_sh;
+    const int32_t last = kBlocks ? last_visible(p, un.t) : 0x7fffffff;
     const char* kbase = reinterpret_cast<const char*>(p.kraw) + static_cast<int64_t>(un.g) * p.kv_sh * 2 + cc * 16;
     const char* vbase = reinterpret_cast<const char*>(p.vraw) + static_cast<int64_t>(un.g) * p.kv_sh * 2 + cc * 16;
     const int64_t row_bytes = p.kv_ss * 2;
@@ -271,13 +303,11 @@ __device__ void producer_role(const TcParams& p, const Sync& sy, uint32_t sb, in
     constexpr int rows_w = kKeys / kProducerWarps;
     const int jr = rows_w * pw + lane;
     const bool own = lane < rows_w;
-    int32_t id_next = (own && un.n_tiles > 0 && jr < un.n_eff) ? __ldg(list + jr) : -1;
+    int32_t entry_next = own ? key_entry<kBlocks>(p, list, un, jr) : -1;
     for (int i = 0; i < un.n_tiles && ok; ++i) {
-      int32_t id = id_next;
-      const int jn = (i + 1) * kKeys + jr;
-      id_next = (own && i + 1 < un.n_tiles && jn < un.n_eff) ? __ldg(list + jn) : -1;
-      const bool bad = id >= p.S;
-      if (bad) {
+      int32_t id = key_slot<kBlocks>(p, un, i * kKeys + jr, entry_next, last);
+      entry_next = (own && i + 1 < un.n_tiles) ? key_entry<kBlocks>(p, list, un, (i + 1) * kKeys + jr) : -1;
+      if (id == -2) {
         id = -1;
         if (p.status != nullptr) atomicOr(p.status, static_cast<int32_t>(kStatusOob));
       }
@@ -289,7 +319,7 @@ __device__ void producer_role(const TcParams& p, const Sync& sy, uint32_t sb, in
       for (int h = 0; h < 4; ++h) {
         const uint32_t slot = c_slot % kSlots;
         const uint32_t round = c_slot / kSlots;
-        ok = sy.wait_warp(B_EMPTY + slot, (round & 1u) ^ 1u, lane);
+        ok = sy.wait_warp(B_EMPTY + slot, (round & 1u) ^ 1u);
         if (!ok) break;
         const char* src0 = (h < 2 ? kbase : vbase) + (h & 1) * 256;
         const uint32_t dst0 = sb + OFF_RING + slot * kSlotBytes + dchunk;
@@ -301,7 +331,7 @@ __device__ void producer_role(const TcParams& p, const Sync& sy, uint32_t sb, in
           const char* src = live ? src0 + static_cast<int64_t>(rid) * row_bytes : src0;
           cp_async_16(dst0 + r * 128 + (((cc & 7) ^ (r & 7)) << 4), src, live ? 16 : 0);
         }
-        if (!(p.inject_stall != 0 && c_slot == 0)) cp_async_mbar_arrive(sy.bar(B_FULL + slot));
+        if (!(kStall && c_slot == 0)) cp_async_mbar_arrive(sy.bar(B_FULL + slot));
         ++c_slot;
       }
     }
@@ -412,6 +442,7 @@ __device__ void pv_role(const TcParams& p, const Sync& sy, uint32_t sb, uint32_t
 
 // ------------------------------------------------------------------ softmax
 
+template <bool kBlocks>
 __device__ void softmax_role(const TcParams& p, const Sync& sy, uint32_t sb, uint8_t* sp,
                              uint32_t tmem, int warp, int lane) {
   const int wq = warp & 3;                       // TMEM lane quadrant of this warp
@@ -425,7 +456,8 @@ __device__ void softmax_role(const TcParams& p, const Sync& sy, uint32_t sb, uin
   bool ok = true;
   for (int64_t u = blockIdx.x; u < units && ok; u += gridDim.x) {
     const Unit un = decode_unit(p, u);
-    const int32_t* list = p.idx + un.t * p.idx_st + static_cast<int64_t>(un.g) * p.idx_sh + un.j0;
+    const int32_t* list = p.idx + un.t * p.idx_st + static_cast<int64_t>(un.g) * p.idx_sh;
+    const int32_t last = kBlocks ? last_visible(p, un.t) : 0x7fffffff;
     float m_run[kGp], l_part[kGp];
 #pragma unroll
     for (int h = 0; h < kGp; ++h) {
@@ -433,15 +465,14 @@ __device__ void softmax_role(const TcParams& p, const Sync& sy, uint32_t sb, uin
       l_part[h] = 0.f;
     }
     // list entry of this thread's key, read one tile ahead
-    int32_t id_next = (un.n_tiles > 0 && key < un.n_eff) ? __ldg(list + key) : -1;
+    int32_t entry_next = un.n_tiles > 0 ? key_entry<kBlocks>(p, list, un, key) : -1;
     for (int i = 0; i < un.n_tiles; ++i) {
       const uint32_t c = c_tile + i;
       const uint32_t buf = c & 1u;
-      const int32_t id = id_next;
-      const int jn = (i + 1) * kKeys + key;
-      id_next = (i + 1 < un.n_tiles && jn < un.n_eff) ? __ldg(list + jn) : -1;
-      const bool valid = id >= 0 && id < p.S;
-      ok = sy.wait_warp(B_SFULL + buf, (c >> 1) & 1u, lane);
+      // this tile's entry was loaded a tile ago: resolve it before waiting for S
+      const bool valid = key_slot<kBlocks>(p, un, i * kKeys + key, entry_next, last) >= 0;
+      entry_next = i + 1 < un.n_tiles ? key_entry<kBlocks>(p, list, un, (i + 1) * kKeys + key) : -1;
+      ok = sy.wait_warp(B_SFULL + buf, (c >> 1) & 1u);
       if (!ok) break;
       tc_fence_after();
       uint32_t r[16];
@@ -460,7 +491,7 @@ __device__ void softmax_role(const TcParams& p, const Sync& sy, uint32_t sb, uin
       if ((lane & 1) == 0) rm[wq * 16 + ((lane >> 1) & 15)] = wmax;
       __syncwarp();
       if (lane == 0) mbar_arrive(sy.bar(B_RMAX + buf));
-      ok = sy.wait_warp(B_RMAX + buf, (c >> 1) & 1u, lane);  // all four warps' maxima are in
+      ok = sy.wait_warp(B_RMAX + buf, (c >> 1) & 1u);  // all four warps' maxima are in
       if (!ok) break;
       float tmax[kGp];
 #pragma unroll
@@ -474,7 +505,7 @@ __device__ void softmax_role(const TcParams& p, const Sync& sy, uint32_t sb, uin
         // raise the running max: O (TMEM) and the partial sums scale by 2^(m_old - m_new)
         if (i > 0) {
           const uint32_t cp = c - 1;
-          ok = sy.wait_warp(B_PEMPTY + (cp & 1u), (cp >> 1) & 1u, lane);  // the previous PV has finished
+          ok = sy.wait_warp(B_PEMPTY + (cp & 1u), (cp >> 1) & 1u);  // the previous PV has finished
           if (!ok) break;
         }
         tc_fence_after();
@@ -512,7 +543,7 @@ __device__ void softmax_role(const TcParams& p, const Sync& sy, uint32_t sb, uin
         l_part[h + 1] += p1;
         pk[h >> 1] = pack_bf16x2(p0, p1);
       }
-      ok = sy.wait_warp(B_PEMPTY + buf, ((c >> 1) & 1u) ^ 1u, lane);
+      ok = sy.wait_warp(B_PEMPTY + buf, ((c >> 1) & 1u) ^ 1u);
       if (!ok) break;
       // P^T row of this key: heads 0-7 in the first 8x8 core-matrix column,
       // heads 8-15 in the second (2 KB further)
@@ -531,12 +562,12 @@ __device__ void softmax_role(const TcParams& p, const Sync& sy, uint32_t sb, uin
     if ((lane & 1) == 0) rs[wq * 16 + ((lane >> 1) & 15)] = wsum;
     __syncwarp();
     if (lane == 0) mbar_arrive(sy.bar(B_RSUM + (c_unit & 1u)));
-    ok = sy.wait_warp(B_RSUM + (c_unit & 1u), (c_unit >> 1) & 1u, lane);
+    ok = sy.wait_warp(B_RSUM + (c_unit & 1u), (c_unit >> 1) & 1u);
     if (!ok) break;
     float l_tot[kGp];
 #pragma unroll
     for (int h = 0; h < kGp; ++h) l_tot[h] = (rs[h] + rs[16 + h]) + (rs[32 + h] + rs[48 + h]);
-    ok = sy.wait_warp(B_OFULL, c_unit & 1u, lane);
+    ok = sy.wait_warp(B_OFULL, c_unit & 1u);
     if (!ok) break;
     tc_fence_after();
     uint32_t o0[16] = {}, o1[16] = {};
@@ -588,7 +619,7 @@ __device__ void softmax_role(const TcParams& p, const Sync& sy, uint32_t sb, uin
 
 // ------------------------------------------------------------------ kernel
 
-template <bool kDump>
+template <bool kDump, bool kStall = false, bool kBlocks = false>
 __global__ void __launch_bounds__(kThreads, 1) qsa_prefill_tc_kernel(const __grid_constant__ TcParams p) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -635,7 +666,7 @@ __global__ void __launch_bounds__(kThreads, 1) qsa_prefill_tc_kernel(const __gri
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(sp + OFF_MISC);
 
   if (warp < kProducerWarps) {
-    producer_role<kDump>(p, sy, sb, warp, lane);
+    producer_role<kDump, kStall, kBlocks>(p, sy, sb, warp, lane);
   } else if (warp == kWarpQK) {
     if (lane == 0) qk_role(p, sy, sb, tmem);
     __syncwarp();
@@ -643,7 +674,7 @@ __global__ void __launch_bounds__(kThreads, 1) qsa_prefill_tc_kernel(const __gri
     if (lane == 0) pv_role(p, sy, sb, tmem);
     __syncwarp();
   } else {
-    softmax_role(p, sy, sb, sp, tmem, warp, lane);
+    softmax_role<kBlocks>(p, sy, sb, sp, tmem, warp, lane);
   }
 
   tc_fence_before();

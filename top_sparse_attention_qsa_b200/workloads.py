@@ -258,6 +258,32 @@ def config_decode(device="cpu", seed=CONFIG_SEED_BASE + 7, B=64, ctx=32768, head
                     f"decode B={B} ctx={ctx} S={S} ({Hq},{Hkv}) K={topk} local{local}+random unsorted")
 
 
+def config_c5_block4(device="cpu", seed=CONFIG_SEED_BASE + 8, T=8192, S=131072, heads=(24, 2),
+                     blocks=512, local_blocks=64, block_size=4) -> Workload:
+    """c5 with microblock lists: 8192 new tokens at positions 122880..131071
+    over a 131072-slot cache, heads (24,2); per KV head `blocks` entries of
+    `block_size` slots (the `local_blocks` newest blocks + random earlier
+    blocks, unsorted).  The newest block reaches past the token's own slot;
+    last_slot (= the token's slot) masks that tail.  Lists are drawn like
+    token lists, in block units.  The returned Workload carries
+    block_size and last_slot as attributes."""
+    gen = _gen(seed, device)
+    Hq, Hkv = heads
+    q = normal_bf16((T, Hq, HEAD_DIM), gen, device)
+    k = normal_bf16((S, Hkv, HEAD_DIM), gen, device)
+    v = normal_bf16((S, Hkv, HEAD_DIM), gen, device)
+    pos = torch.arange(S - T, S, device=device)
+    s0 = torch.zeros(T, dtype=torch.int64, device=device)
+    idx, nv = causal_lists(pos // block_size, s0 // block_size, blocks, local_blocks, Hkv, gen,
+                           device, ordered=False)
+    w = Workload(f"c5_block{block_size}_{blocks}blk", q, k, v, idx, nv, 1.0 / 16, pos, s0,
+                 f"T={T} at {S - T}..{S - 1}, S={S} ({Hq},{Hkv}) {blocks} blocks of {block_size} "
+                 f"(local {local_blocks} + random), unsorted, causal tail masked")
+    w.block_size = block_size
+    w.last_slot = pos.to(torch.int32)
+    return w
+
+
 CONFIGS = {
     "tiny": config_tiny,
     "c2": config_c2,
@@ -265,6 +291,7 @@ CONFIGS = {
     "c4": config_c4,
     "c5": config_c5,
     "decode": config_decode,
+    "c5_block4": config_c5_block4,
 }
 
 
