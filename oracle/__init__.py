@@ -68,6 +68,23 @@ class _Args(ctypes.Structure):
     ]
 
 
+class _IndexerArgs(ctypes.Structure):
+    _fields_ = [
+        ("num_tokens", ctypes.c_int64),
+        ("num_heads", ctypes.c_int64),
+        ("head_dim", ctypes.c_int64),
+        ("num_blocks", ctypes.c_int64),
+        ("block_size", ctypes.c_int64),
+        ("q_stride_tok", ctypes.c_int64),
+        ("q_stride_head", ctypes.c_int64),
+        ("k_stride_block", ctypes.c_int64),
+        ("q", ctypes.c_void_p),
+        ("k", ctypes.c_void_p),
+        ("positions", ctypes.c_void_p),
+        ("seq_start", ctypes.c_void_p),
+    ]
+
+
 class Oracle:
     """ctypes handle on one build of qsa_oracle.c (the default build, or a
     copy with a planted mistake that the pin tests must reject)."""
@@ -79,6 +96,12 @@ class Oracle:
                                        ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p]
         lib.qsa_oracle_bf16_to_double.restype = ctypes.c_double
         lib.qsa_oracle_bf16_to_double.argtypes = [ctypes.c_uint16]
+        lib.qsa_oracle_indexer_scores.restype = ctypes.c_int
+        lib.qsa_oracle_indexer_scores.argtypes = [ctypes.POINTER(_IndexerArgs), ctypes.c_void_p,
+                                                  ctypes.c_int64, ctypes.c_int, ctypes.c_void_p]
+        lib.qsa_oracle_topk.restype = ctypes.c_int
+        lib.qsa_oracle_topk.argtypes = [ctypes.POINTER(_IndexerArgs), ctypes.c_void_p, ctypes.c_int64,
+                                        ctypes.c_int64, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p]
         self.lib = lib
         self.path = lib_path
 
@@ -89,6 +112,69 @@ class Oracle:
                        tokens=None, n_threads=None, block_size=1, last_slot=None):
         return _sparse_prefill(self.lib, q, k_cache, v_cache, topk_idx, n_valid, scale,
                                tokens, n_threads, block_size, last_slot)
+
+
+    def indexer_scores(self, q_idx, k_idx, positions, seq_start, block_size=4, tokens=None):
+        """FP64 indexer scores [n, NB]: sum over heads of <q_idx[t,h], k_idx[b]>,
+        -inf outside the token's complete causal microblocks."""
+        a, keep = _indexer_args(q_idx, k_idx, positions, seq_start, block_size)
+        T = a.num_tokens
+        if tokens is None:
+            tokens = np.arange(T, dtype=np.int64)
+        tokens = np.ascontiguousarray(np.asarray(tokens, dtype=np.int64))
+        out = np.zeros((tokens.shape[0], a.num_blocks), dtype=np.float64)
+        rc = self.lib.qsa_oracle_indexer_scores(ctypes.byref(a), tokens.ctypes.data, tokens.shape[0], 1,
+                                                out.ctypes.data)
+        if rc != 0:
+            raise ValueError("oracle rejected its arguments")
+        return out
+
+    def topk(self, scores, positions, seq_start, num_blocks, budget, block_size=4, append_tail=False):
+        """Selection over given FP32 scores [T, ld]: ascending block ids of the
+        `budget` highest candidates (ties to the smaller id), then with
+        `append_tail` the token's own incomplete block, -1 padded; and counts."""
+        sc = np.ascontiguousarray(_as_f32(scores))
+        T, ld = sc.shape
+        pos = np.ascontiguousarray(_as_i32(positions))
+        s0 = np.ascontiguousarray(_as_i32(seq_start))
+        a = _IndexerArgs(T, 0, 0, num_blocks, block_size, 0, 0, 0, None, None, pos.ctypes.data,
+                         s0.ctypes.data)
+        sel = np.zeros((T, budget + (1 if append_tail else 0)), dtype=np.int32)
+        cnt = np.zeros((T,), dtype=np.int32)
+        rc = self.lib.qsa_oracle_topk(ctypes.byref(a), sc.ctypes.data, ld, budget, int(bool(append_tail)),
+                                      sel.ctypes.data, cnt.ctypes.data)
+        if rc != 0:
+            raise ValueError("oracle rejected its arguments")
+        return sel, cnt
+
+
+def _as_f32(x):
+    if hasattr(x, "numpy") and not isinstance(x, np.ndarray):
+        x = x.detach().cpu().numpy()
+    x = np.asarray(x)
+    if x.dtype != np.float32:
+        raise TypeError(f"expected float32, got {x.dtype}")
+    return x
+
+
+def _indexer_args(q_idx, k_idx, positions, seq_start, block_size):
+    q = _as_u16(q_idx)
+    k = _as_u16(k_idx)
+    T, H, Dh = q.shape
+    NB, Dk = k.shape
+    if Dk != Dh:
+        raise ValueError("q_idx / k_idx head dims differ")
+    qs = _strides(q, 3)
+    ks = _strides(k, 2)
+    if qs[2] != 1 or ks[1] != 1:
+        raise ValueError("head dim must be contiguous")
+    pos = np.ascontiguousarray(_as_i32(positions))
+    s0 = np.ascontiguousarray(_as_i32(seq_start))
+    if pos.shape != (T,) or s0.shape != (T,):
+        raise ValueError("positions / seq_start must be [T]")
+    a = _IndexerArgs(T, H, Dh, NB, block_size, qs[0], qs[1], ks[0], q.ctypes.data, k.ctypes.data,
+                     pos.ctypes.data, s0.ctypes.data)
+    return a, (q, k, pos, s0)
 
 
 _default = None

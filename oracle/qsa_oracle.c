@@ -166,3 +166,98 @@ int64_t qsa_oracle_fwd(const qsa_oracle_args* a, const int64_t* tokens,
   if (job.error) return -1;
   return job.oob;
 }
+
+/* ------------------------------------------------------------------------
+ * QSA indexer: candidate scores and top-budget selection.
+ * ---------------------------------------------------------------------- */
+
+void qsa_oracle_indexer_candidates(const qsa_oracle_indexer_args* a, int64_t t,
+                                   int64_t* b0, int64_t* b1) {
+  const int64_t bs = a->block_size > 0 ? a->block_size : 1;
+  int64_t lo = a->seq_start[t] / bs;
+  int64_t hi = ((int64_t)a->positions[t] + 1) / bs; /* complete blocks only */
+  if (hi > a->num_blocks) hi = a->num_blocks;
+  if (lo < 0) lo = 0;
+  if (hi < lo) hi = lo;
+  *b0 = lo;
+  *b1 = hi;
+}
+
+int qsa_oracle_indexer_scores(const qsa_oracle_indexer_args* a,
+                              const int64_t* tokens, int64_t n_tokens,
+                              int n_threads, double* scores) {
+  (void)n_threads;
+  if (!a || (n_tokens > 0 && (!tokens || !scores || !a->q || !a->k))) return -1;
+  const int64_t NB = a->num_blocks, Dh = a->head_dim;
+  for (int64_t i = 0; i < n_tokens; ++i) {
+    const int64_t t = tokens[i];
+    if (t < 0 || t >= a->num_tokens) return -1;
+    int64_t b0, b1;
+    qsa_oracle_indexer_candidates(a, t, &b0, &b1);
+    double* row = scores + i * NB;
+    for (int64_t b = 0; b < NB; ++b) row[b] = -INFINITY;
+    for (int64_t b = b0; b < b1; ++b) {
+      const uint16_t* kr = a->k + b * a->k_stride_block;
+      double sum = 0.0;
+      for (int64_t h = 0; h < a->num_heads; ++h) {
+        const uint16_t* qr = a->q + t * a->q_stride_tok + h * a->q_stride_head;
+        double dot = 0.0;
+        for (int64_t d = 0; d < Dh; ++d)
+          dot += qsa_oracle_bf16_to_double(qr[d]) * qsa_oracle_bf16_to_double(kr[d]);
+        sum += dot;
+      }
+      row[b] = sum;
+    }
+  }
+  return 0;
+}
+
+typedef struct {
+  float score;
+  int64_t block;
+} scored_t;
+
+/* Higher score first; equal scores: smaller block first. */
+static int by_score_then_index(const void* x, const void* y) {
+  const scored_t* a = (const scored_t*)x;
+  const scored_t* b = (const scored_t*)y;
+  if (a->score > b->score) return -1;
+  if (a->score < b->score) return 1;
+  return (a->block > b->block) - (a->block < b->block);
+}
+
+static int by_block(const void* x, const void* y) {
+  const int32_t a = *(const int32_t*)x, b = *(const int32_t*)y;
+  return (a > b) - (a < b);
+}
+
+int qsa_oracle_topk(const qsa_oracle_indexer_args* a, const float* scores,
+                    int64_t ld, int64_t budget, int append_tail, int32_t* sel,
+                    int32_t* count) {
+  if (!a || !scores || !sel || !count || budget < 0) return -1;
+  const int64_t bs = a->block_size > 0 ? a->block_size : 1;
+  const int64_t width = budget + (append_tail ? 1 : 0);
+  scored_t* buf = (scored_t*)malloc((size_t)(a->num_blocks > 0 ? a->num_blocks : 1) * sizeof(scored_t));
+  if (!buf) return -1;
+  for (int64_t t = 0; t < a->num_tokens; ++t) {
+    int64_t b0, b1;
+    qsa_oracle_indexer_candidates(a, t, &b0, &b1);
+    int64_t n = 0;
+    for (int64_t b = b0; b < b1; ++b) {
+      buf[n].score = scores[t * ld + b];
+      buf[n].block = b;
+      ++n;
+    }
+    qsort(buf, (size_t)n, sizeof(scored_t), by_score_then_index);
+    int64_t k = n < budget ? n : budget;
+    int32_t* out = sel + t * width;
+    for (int64_t j = 0; j < k; ++j) out[j] = (int32_t)buf[j].block;
+    qsort(out, (size_t)k, sizeof(int32_t), by_block);
+    if (append_tail && ((int64_t)a->positions[t] + 1) % bs != 0)
+      out[k++] = (int32_t)((int64_t)a->positions[t] / bs);
+    for (int64_t j = k; j < width; ++j) out[j] = -1;
+    count[t] = (int32_t)k;
+  }
+  free(buf);
+  return 0;
+}

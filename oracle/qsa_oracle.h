@@ -66,6 +66,56 @@ int64_t qsa_oracle_fwd(const qsa_oracle_args* a, const int64_t* tokens,
 /* Exact BF16 -> double widening of one bit pattern (exposed for tests). */
 double qsa_oracle_bf16_to_double(uint16_t bits);
 
+/* ------------------------------------------------------------------------
+ * QSA indexer (page "Qwen4-Exp QSA llega al Ascend de Huawei", section "Por
+ * qué QSA es la parte incómoda, en cifras": a multi-query indexer with 4
+ * query heads sharing one key head of dim 128, compression ratio 4, a budget
+ * of 2048 microblocks per query).  TEST INFRASTRUCTURE ONLY, like the rest of
+ * this library.
+ *
+ * Readings where the page is silent: the score of microblock b for token t
+ * is the plain sum over the query heads of <q_idx[t,i,:], k_idx[b,:]>; the
+ * candidates of token t are the complete causal microblocks of its sequence,
+ * b in [seq_start/bs, (pos+1)/bs); the selection is the `budget` highest
+ * scores, ties to the smaller block index.
+ * ---------------------------------------------------------------------- */
+
+typedef struct {
+  int64_t num_tokens;     /* T */
+  int64_t num_heads;      /* indexer query heads (4) */
+  int64_t head_dim;       /* 128 */
+  int64_t num_blocks;     /* NB: rows of k_idx */
+  int64_t block_size;     /* tokens per microblock (4) */
+  int64_t q_stride_tok, q_stride_head;   /* q_idx [T, H, Dh] BF16 */
+  int64_t k_stride_block;                /* k_idx [NB, Dh] BF16 */
+  const uint16_t* q;
+  const uint16_t* k;
+  const int32_t* positions;              /* [T] slot of the token */
+  const int32_t* seq_start;              /* [T] first slot of its sequence */
+} qsa_oracle_indexer_args;
+
+/* Candidate range of token t: [*b0, *b1). */
+void qsa_oracle_indexer_candidates(const qsa_oracle_indexer_args* a, int64_t t,
+                                   int64_t* b0, int64_t* b1);
+
+/* scores [n_tokens, NB] doubles (row of token tokens[i]); entries outside the
+ * token's candidate range are -inf.  Returns 0, or -1 on bad arguments. */
+int qsa_oracle_indexer_scores(const qsa_oracle_indexer_args* a,
+                              const int64_t* tokens, int64_t n_tokens,
+                              int n_threads, double* scores);
+
+/* Selection over given FP32 scores [T, ld] (the caller's scores; entries of
+ * token t at columns [b0, b1) are its candidates).  Row t of sel holds the
+ * chosen block ids in ascending order, then -1 padding; its width is budget,
+ * plus one when append_tail is set: then the token's own block pos/bs follows
+ * the chosen ones whenever it is incomplete ((pos+1) % bs != 0: a causal tail
+ * of 1..bs-1 slots, masked above pos by the attention's last visible slot).
+ * count[t] is the number of ids written.  Highest score first, ties to the
+ * smaller block index; -0.0 and +0.0 are equal.  Returns 0, or -1. */
+int qsa_oracle_topk(const qsa_oracle_indexer_args* a, const float* scores,
+                    int64_t ld, int64_t budget, int append_tail, int32_t* sel,
+                    int32_t* count);
+
 #ifdef __cplusplus
 }
 #endif

@@ -25,6 +25,17 @@ Pins (what the pages and the mathematics fix):
   attention over any split of it (the combine step of split-K decode).
 * block_lists   -- a microblock list equals the token list naming each of its
   slots (with the cache end and the token's last visible slot applied).
+* indexer_scores -- page "Qwen4-Exp QSA llega al Ascend de Huawei", section
+  "Por qué QSA es la parte incómoda, en cifras" (4 query heads sharing one
+  key head, dim 128, compression 4): with one head the scores are a plain
+  matrix product (numpy matmul); with four they are the sum of the one-head
+  scores; the candidate ranges of hand-picked positions (causal tails 0..3,
+  a later sequence start) are the complete causal blocks; strides do not
+  matter.
+* topk          -- the selection equals a lexicographic sort on (-score,
+  block) by numpy (library routine); every chosen score >= every unchosen
+  one; all-equal scores take the first blocks; -0.0 ties +0.0; the causal
+  tail is appended for remainders 1..3 only.
 """
 from __future__ import annotations
 
@@ -296,6 +307,91 @@ def check_block_lists(orc):
         np.testing.assert_allclose(got[1], want[1], **TOL)
 
 
+# Positions with causal tails 0..3 at ratio 4 and a second sequence starting
+# at slot 16, with their complete-block candidate ranges worked out by hand:
+# a token at position p sees blocks [start/4, (p+1)/4).
+IDX_POS = [3, 4, 5, 6, 7, 30, 43, 0]
+IDX_START = [0, 0, 0, 0, 0, 16, 16, 0]
+IDX_RANGES = [(0, 1), (0, 1), (0, 1), (0, 1), (0, 2), (4, 7), (4, 11), (0, 0)]
+
+
+def check_indexer_scores(orc):
+    gen = torch.Generator().manual_seed(71)
+    T, NB, Dh = len(IDX_POS), 11, 128
+    pos = torch.tensor(IDX_POS, dtype=torch.int32)
+    s0 = torch.tensor(IDX_START, dtype=torch.int32)
+    k = W.normal_bf16((NB, Dh), gen, "cpu")
+    q = W.normal_bf16((T, 4, Dh), gen, "cpu")
+    got = orc.indexer_scores(q, k, pos, s0, block_size=4)
+    # candidate ranges: finite exactly on [lo, hi)
+    for t, (lo, hi) in enumerate(IDX_RANGES):
+        fin = np.isfinite(got[t])
+        assert fin[lo:hi].all() and not fin[:lo].any() and not fin[hi:].any(), t
+    mask = np.isfinite(got)
+    kd = _np64(k)
+    # one head: a plain matrix product
+    for h in range(4):
+        one = orc.indexer_scores(q[:, h:h + 1].contiguous(), k, pos, s0, block_size=4)
+        want = _np64(q[:, h]) @ kd.T
+        np.testing.assert_allclose(one[mask], want[mask], rtol=1e-12, atol=1e-12)
+    # four heads: the sum of the one-head scores (matmul of the head sum)
+    want = _np64(q).sum(axis=1) @ kd.T
+    np.testing.assert_allclose(got[mask], want[mask], rtol=1e-12, atol=1e-12)
+    # padded strides and a token subset give the same values
+    qp = torch.zeros((T, 6, Dh + 64), dtype=torch.bfloat16)
+    qp[:, 1:5, :Dh] = q
+    kp = torch.zeros((NB, Dh + 32), dtype=torch.bfloat16)
+    kp[:, :Dh] = k
+    sub = orc.indexer_scores(qp[:, 1:5, :Dh], kp[:, :Dh], pos, s0, block_size=4, tokens=[6, 2])
+    np.testing.assert_array_equal(sub, got[[6, 2]])
+
+
+def _lexsort_select(scores, lo, hi, budget):
+    b = np.arange(lo, hi)
+    order = np.lexsort((b, -scores[lo:hi].astype(np.float64)))
+    return np.sort(b[order[:budget]])
+
+
+def check_topk(orc):
+    rng = np.random.default_rng(73)
+    T, NB = len(IDX_POS), 11
+    pos = np.array(IDX_POS, dtype=np.int32)
+    s0 = np.array(IDX_START, dtype=np.int32)
+    sc = rng.standard_normal((T, NB)).astype(np.float32)
+    sc[6, [5, 8, 9]] = sc[6, 6]                  # ties inside the longest row
+    for budget in (0, 1, 2, 3, 5, 20):
+        for tail in (False, True):
+            sel, cnt = orc.topk(sc, pos, s0, NB, budget, block_size=4, append_tail=tail)
+            assert sel.shape == (T, budget + int(tail))
+            for t, (lo, hi) in enumerate(IDX_RANGES):
+                want = list(_lexsort_select(sc[t], lo, hi, budget))
+                # every chosen score is >= every unchosen candidate score
+                rest = [b for b in range(lo, hi) if b not in want]
+                if want and rest:
+                    assert sc[t, want].min() >= sc[t, rest].max()
+                rem = (IDX_POS[t] + 1) % 4
+                if tail and rem:
+                    want.append(IDX_POS[t] // 4)
+                n = len(want)
+                assert cnt[t] == n, (budget, tail, t)
+                np.testing.assert_array_equal(sel[t, :n], want)
+                assert (sel[t, n:] == -1).all()
+    # all-equal scores take the first blocks of the range
+    eq = np.full((T, NB), 0.5, dtype=np.float32)
+    sel, cnt = orc.topk(eq, pos, s0, NB, 3, block_size=4)
+    np.testing.assert_array_equal(sel[6], [4, 5, 6])
+    # -0.0 ties +0.0: the smaller block index wins either way round
+    z = np.full((T, NB), -1.0, dtype=np.float32)
+    z[6, 5], z[6, 7] = -0.0, 0.0
+    assert orc.topk(z, pos, s0, NB, 1, block_size=4)[0][6, 0] == 5
+    z[6, 5], z[6, 7] = 0.0, -0.0
+    assert orc.topk(z, pos, s0, NB, 1, block_size=4)[0][6, 0] == 5
+    # the tail block follows the chosen ones for remainders 1..3 only
+    sel, cnt = orc.topk(sc, pos, s0, NB, 0, block_size=4, append_tail=True)
+    assert [int(c) for c in cnt] == [0, 1, 1, 1, 0, 1, 0, 1]
+    assert int(sel[5, 0]) == 7 and int(sel[1, 0]) == 1
+
+
 ALL_CHECKS = [check_bf16_widening, check_dense_causal, check_packing, check_permutation,
               check_head_padding, check_closed_forms, check_brute_force, check_worked_example,
-              check_split_merge, check_block_lists]
+              check_split_merge, check_block_lists, check_indexer_scores, check_topk]

@@ -32,6 +32,18 @@ MUTANTS = {
     "last_slot_ignored": ("if (slot >= a->num_slots || slot > limit) continue;", "if (slot >= a->num_slots) continue;"),
     "v_head_stride_dropped": ("const uint16_t* vr = a->v + sel[j] * a->kv_stride_slot + g * a->kv_stride_head;",
                               "const uint16_t* vr = a->v + sel[j] * a->kv_stride_slot;"),
+    "indexer_head_dropped": ("for (int64_t h = 0; h < a->num_heads; ++h) {",
+                             "for (int64_t h = 1; h < a->num_heads; ++h) {"),
+    "indexer_partial_block": ("int64_t hi = ((int64_t)a->positions[t] + 1) / bs;",
+                              "int64_t hi = ((int64_t)a->positions[t] + bs) / bs;"),
+    "indexer_sequence_start_ignored": ("int64_t lo = a->seq_start[t] / bs;", "int64_t lo = 0;"),
+    "indexer_key_row_of_token": ("const uint16_t* kr = a->k + b * a->k_stride_block;",
+                                 "const uint16_t* kr = a->k + t * a->k_stride_block;"),
+    "topk_keeps_lowest": ("if (a->score > b->score) return -1;\n  if (a->score < b->score) return 1;",
+                          "if (a->score < b->score) return -1;\n  if (a->score > b->score) return 1;"),
+    "topk_ties_to_larger_block": ("return (a->block > b->block) - (a->block < b->block);",
+                                  "return (a->block < b->block) - (a->block > b->block);"),
+    "topk_tail_always": ("if (append_tail && ((int64_t)a->positions[t] + 1) % bs != 0)", "if (append_tail)"),
 }
 
 
