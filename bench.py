@@ -26,7 +26,6 @@ from __future__ import annotations
 
 import argparse
 import datetime
-import glob
 import hashlib
 import json
 import os
@@ -67,6 +66,8 @@ def parse_args():
                     help="decode workload timed under 'decode' ('' to skip)")
     ap.add_argument("--blocks", default="c5_block4",
                     help="microblock-list workload timed under 'blocks' ('' to skip)")
+    ap.add_argument("--indexer", default="indexer",
+                    help="indexer + top-K workload timed under 'indexer' ('' to skip)")
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -140,10 +141,16 @@ def workload_accounting(w):
     return dict(entries=entries, gathered_bytes=gathered, algo_bytes=algo, flops=flops)
 
 
-def kernel_source_hash():
+# Sources the sparse-prefill kernels compile from (the launch code in
+# qsa_api.cu included); the indexer's file is not among them.
+PREFILL_SOURCES = ("qsa_api.cu", "qsa_host.cuh", "qsa_prefill_tc.cuh", "qsa_prefill_mma.cuh", "qsa_tc_ptx.cuh",
+                   "qsa_ptx.cuh", "qsa_merge.cuh")
+
+
+def kernel_source_hash(files=PREFILL_SOURCES):
     h = hashlib.sha256()
     pkg = os.path.join(ROOT, "top_sparse_attention_qsa_b200", "csrc")
-    for p in sorted(glob.glob(os.path.join(pkg, "*.cu")) + glob.glob(os.path.join(pkg, "*.cuh"))):
+    for p in sorted(os.path.join(pkg, f) for f in files):
         with open(p, "rb") as f:
             h.update(os.path.basename(p).encode())
             h.update(f.read())
@@ -451,6 +458,8 @@ def run_cuda(args):
         line["decode"] = run_decode_bench(args.decode, dev, barrier, max_ranks, world, hbm)
     if args.blocks and not args.profile:
         line["blocks"] = run_blocks_bench(args.blocks, dev, barrier, max_ranks, world, hbm)
+    if args.indexer and not args.profile:
+        line["indexer"] = run_indexer_bench(dev, barrier, max_ranks, world, hbm, bf16)
     if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.profile:
         line["cpu_baseline"] = time_oracle(w, args.cpu_budget)
     elif not args.profile:
@@ -573,6 +582,56 @@ def run_blocks_bench(name, dev, barrier, reduce_max, world, hbm):
             "mean_launch_ms": ms, "live_keys": keys, "gathered_kv_gbs": keys * 1024 / (ms / 1e3) / 1e9,
             "algo_gbs": algo / (ms / 1e3) / 1e9, "frac_of_hbm": algo / (ms / 1e3) / 1e9 / hbm,
             "steps": steps}
+
+
+def run_indexer_bench(dev, barrier, reduce_max, world, hbm, bf16, **kw):
+    """Indexer scores (tcgen05) then top-K selection on the c5 size: 8192
+    tokens, 32768 block keys, 4 heads x 128, budget 2048 + causal tail.  Each
+    kernel is timed on its own (events on the launching stream) and as the
+    pair; the scores buffer (1 GiB) is larger than L2."""
+    from top_sparse_attention_qsa_b200 import _capi
+    from top_sparse_attention_qsa_b200 import workloads as W
+    w = W.config_indexer(device=dev, **kw)
+    T, H, Dh = w.q_idx.shape
+    NB = w.k_idx.shape[0]
+    pos = w.positions.to(torch.int64)
+    n = ((pos + 1) // w.block_size).clamp(max=NB) - w.seq_start.to(torch.int64) // w.block_size
+    cand = int(n.clamp(min=0).sum().item())
+    width = w.budget + 1
+    scores = torch.empty((T, NB), dtype=torch.float32, device=dev)
+    lists = torch.empty((T, width), dtype=torch.int32, device=dev)
+    nv = torch.empty((T, 2), dtype=torch.int32, device=dev)
+
+    def s_step():
+        _capi.indexer_scores(w.q_idx, w.k_idx, w.positions, w.seq_start, w.block_size, scores=scores)
+
+    def k_step():
+        _capi.topk_select(scores, w.positions, w.seq_start, NB, w.budget, w.block_size, True,
+                          lists=lists, n_valid=nv, copies=2)
+
+    def pair():
+        s_step()
+        k_step()
+
+    steps = 20
+    _, s_per, _ = time_launches(s_step, steps, 3, barrier, "indexer_scores")
+    _, k_per, _ = time_launches(k_step, steps, 3, barrier, "topk_select")
+    total_ms, p_per, _ = time_launches(pair, steps, 3, barrier, "indexer_pair")
+    total_ms = reduce_max(total_ms)
+    s_ms, k_ms = statistics.mean(s_per), statistics.mean(k_per)
+    flops = cand * H * Dh * 2
+    s_bytes = w.q_idx.numel() * 2 + w.k_idx.numel() * 2 + cand * 4
+    k_bytes = cand * 4 + T * width * 4 + T * 2 * 4 + T * 8
+    s_roof = 1e3 * max(flops / (bf16 * 1e12), s_bytes / (hbm * 1e9))
+    return {"workload": w.name, "desc": w.description, "candidates": cand,
+            "tokens_per_s": T * steps * world / (total_ms / 1e3), "mean_pair_ms": statistics.mean(p_per),
+            "scores": {"mean_launch_ms": s_ms, "tflops": flops / (s_ms / 1e3) / 1e12,
+                       "algo_gbs": s_bytes / (s_ms / 1e3) / 1e9, "roofline_ms": s_roof,
+                       "frac_of_roofline_time": s_roof / s_ms,
+                       "bound": "tensor" if flops / (bf16 * 1e12) > s_bytes / (hbm * 1e9) else "hbm"},
+            "topk": {"mean_launch_ms": k_ms, "algo_gbs": k_bytes / (k_ms / 1e3) / 1e9,
+                     "frac_of_hbm": k_bytes / (k_ms / 1e3) / 1e9 / hbm},
+            "launches_per_step": 2, "steps": steps}
 
 
 def main():

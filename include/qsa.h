@@ -291,6 +291,78 @@ qsa_status_t qsa_test_stalled_pipeline(const qsa_shape_t* shape, const void* q,
                                        void* out, float* lse, int32_t* status,
                                        void* stream);
 
+/*
+ * QSA indexer and top-K microblock selection (page "Qwen4-Exp QSA llega al
+ * Ascend de Huawei", section "Por qué QSA es la parte incómoda, en cifras":
+ * a multi-query indexer, 4 query heads sharing one key head of dim 128, over
+ * keys compressed 4x, choosing 2048 microblocks per query).  The page gives
+ * the shapes only; this library computes, for query token t with slot
+ * position pos[t] in a sequence starting at slot seq_start[t],
+ *
+ *   candidates(t) = { b : seq_start[t]/bs <= b < (pos[t]+1)/bs, b < NB }
+ *                   (the complete causal microblocks; C division)
+ *   score(t, b)   = sum_h < q_idx[t,h,:], k_idx[b,:] >   (FP32 accumulate)
+ *
+ * and selects the `budget` candidates of highest score (ties to the smaller
+ * block; -0.0 equals +0.0), listed in ascending block order.  The token's
+ * own incomplete block ((pos+1) % bs != 0: a causal tail of 1..bs-1 slots)
+ * can follow them; qsa_sparse_prefill_block_fwd with last_slot = pos masks
+ * its slots past the token.  Sequences must start on block boundaries.
+ */
+typedef struct {
+  int64_t num_tokens;        /* T >= 0 */
+  int32_t num_heads;         /* H: indexer query heads, 1, 2, 4 or 8 */
+  int32_t head_dim;          /* must be 128 */
+  int64_t num_blocks;        /* NB: rows of k_idx, 1 <= NB < 2^31 */
+  int32_t block_size;        /* bs >= 1: slots per microblock (ratio 4) */
+  int32_t reserved;          /* 0 */
+  int64_t q_stride_tok, q_stride_head;  /* q_idx [T, H, 128] BF16, elements,
+                                           multiples of 8 */
+  int64_t k_stride_block;               /* k_idx [NB, 128] BF16, multiple of 8 */
+  int64_t score_stride_tok;             /* scores [T, ld] FP32, ld >= NB */
+} qsa_indexer_shape_t;
+
+/*
+ * Indexer scores.  q_idx, k_idx: BF16 device, 16-byte aligned.  positions,
+ * seq_start: int32 device [T].  scores: FP32 device [T, ld]; row t is written
+ * at the columns of candidates(t) only (all other entries are left as they
+ * were).  status: device int32 (bit 1 on an internal timeout) or NULL.  One
+ * launch of the persistent tcgen05 kernel on `stream`; no allocation.
+ * QSA_ERR_UNSUPPORTED: head_dim != 128, H not in {1,2,4,8}, or a layout a
+ * TMA descriptor cannot express.
+ */
+qsa_status_t qsa_indexer_scores(const qsa_indexer_shape_t* shape,
+                                const void* q_idx, const void* k_idx,
+                                const int32_t* positions,
+                                const int32_t* seq_start, float* scores,
+                                int32_t* status, void* stream);
+
+/*
+ * Top-K selection over scores laid out as qsa_indexer_scores writes them
+ * (only the candidate columns of each row are read).
+ *   budget      : blocks chosen per token, >= 0 (2048 in the model).
+ *   append_tail : nonzero appends the token's own incomplete block.
+ *   lists       : int32 device [T, list_stride_tok]; row t receives
+ *                 width = budget + (append_tail ? 1 : 0) entries: the chosen
+ *                 blocks ascending, the tail block, then -1.
+ *   n_valid     : int32 device [T, copies] or NULL: the entry count of row t
+ *                 written `copies` times (one per KV head of the attention
+ *                 that reads the list with head stride 0), copies in 1..32.
+ *   status      : device int32 (bit 1 when a row copy timed out) or NULL.
+ * scores must be 16-byte aligned with score_stride_tok a multiple of 4
+ * (QSA_ERR_ALIGN otherwise): each row's candidate span is copied to shared
+ * memory whole, widened to 16-byte boundaries inside the row.  Candidates
+ * per token are limited to 32768 (QSA_ERR_UNSUPPORTED when NB is larger).
+ * One launch of persistent CTAs; no allocation.  The device memory read is
+ * the candidate part of every score row.
+ */
+qsa_status_t qsa_topk_select(const qsa_indexer_shape_t* shape,
+                             const float* scores, const int32_t* positions,
+                             const int32_t* seq_start, int64_t budget,
+                             int32_t append_tail, int32_t* lists,
+                             int64_t list_stride_tok, int32_t* n_valid,
+                             int32_t copies, int32_t* status, void* stream);
+
 /* Static description of a status code. */
 const char* qsa_status_string(qsa_status_t status);
 

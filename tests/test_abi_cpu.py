@@ -117,3 +117,46 @@ def test_stall_hook_needs_a_status_word(capi):
     s = _shape(capi)
     assert capi.library().qsa_test_stalled_pipeline(ctypes.byref(s), P, P, P, P, None, 0.0, P, None,
                                                     None, None) == 1
+
+
+def _ishape(capi, **kw):
+    base = dict(num_tokens=4, num_heads=4, head_dim=128, num_blocks=64, block_size=4, reserved=0,
+                q_stride_tok=512, q_stride_head=128, k_stride_block=128, score_stride_tok=64)
+    base.update(kw)
+    return capi.IndexerShape(**base)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(head_dim=64), 3),
+    (dict(num_heads=3), 3),
+    (dict(num_heads=16), 3),
+    (dict(num_blocks=0), 2),
+    (dict(block_size=0), 2),
+    (dict(score_stride_tok=63), 2),
+    (dict(q_stride_head=132), 4),
+    (dict(k_stride_block=-128), 2),
+])
+def test_indexer_validation(capi, kw, code):
+    lib = capi.library()
+    assert lib.qsa_indexer_scores(ctypes.byref(_ishape(capi, **kw)), P, P, P, P, P, None, None) == code
+
+
+def test_indexer_nulls_and_topk_limits(capi):
+    lib = capi.library()
+    s = _ishape(capi)
+    assert lib.qsa_indexer_scores(None, P, P, P, P, P, None, None) == 1
+    assert lib.qsa_indexer_scores(ctypes.byref(s), None, P, P, P, P, None, None) == 1
+    assert lib.qsa_indexer_scores(ctypes.byref(s), P + 8, P, P, P, P, None, None) == 4
+    assert lib.qsa_indexer_scores(ctypes.byref(_ishape(capi, num_tokens=0)), None, None, None, None, None,
+                                  None, None) == 0
+    # selection: rows longer than 32768 candidates are refused, widths checked
+    big = _ishape(capi, num_blocks=32769, score_stride_tok=32772)
+    sel = lib.qsa_topk_select
+    assert sel(ctypes.byref(big), P, P, P, 8, 1, P, 9, P, 1, None, None) == 3
+    assert sel(ctypes.byref(s), P, P, P, 8, 1, P, 8, P, 1, None, None) == 2   # stride < width
+    assert sel(ctypes.byref(s), P, P, P, -1, 0, P, 8, P, 1, None, None) == 2
+    assert sel(ctypes.byref(s), P, P, P, 8, 0, P, 8, P, 33, None, None) == 2  # copies
+    assert sel(ctypes.byref(s), None, P, P, 8, 0, P, 8, P, 1, None, None) == 1
+    assert sel(ctypes.byref(s), P + 4, P, P, 8, 0, P, 8, P, 1, None, None) == 4  # scores not 16-byte aligned
+    odd = _ishape(capi, score_stride_tok=66)
+    assert sel(ctypes.byref(odd), P, P, P, 8, 0, P, 8, P, 1, None, None) == 4   # row stride not 4 floats

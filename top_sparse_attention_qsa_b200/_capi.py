@@ -35,7 +35,7 @@ EXPORTS = ("qsa_sparse_prefill_fwd", "qsa_sparse_prefill_fwd_with", "qsa_sparse_
            "qsa_sparse_prefill_block_fwd",
            "qsa_sparse_prefill_fwd_host", "qsa_sparse_decode_fwd", "qsa_sparse_decode_workspace_bytes",
            "qsa_sparse_decode_num_splits", "qsa_sparse_decode_fwd_noalloc", "qsa_test_stalled_pipeline",
-           "qsa_status_string", "qsa_abi_version")
+           "qsa_indexer_scores", "qsa_topk_select", "qsa_status_string", "qsa_abi_version")
 
 
 class Shape(ctypes.Structure):
@@ -55,6 +55,21 @@ class Shape(ctypes.Structure):
         ("o_stride_tok", ctypes.c_int64),
         ("o_stride_head", ctypes.c_int64),
         ("lse_stride_tok", ctypes.c_int64),
+    ]
+
+
+class IndexerShape(ctypes.Structure):
+    _fields_ = [
+        ("num_tokens", ctypes.c_int64),
+        ("num_heads", ctypes.c_int32),
+        ("head_dim", ctypes.c_int32),
+        ("num_blocks", ctypes.c_int64),
+        ("block_size", ctypes.c_int32),
+        ("reserved", ctypes.c_int32),
+        ("q_stride_tok", ctypes.c_int64),
+        ("q_stride_head", ctypes.c_int64),
+        ("k_stride_block", ctypes.c_int64),
+        ("score_stride_tok", ctypes.c_int64),
     ]
 
 
@@ -93,6 +108,9 @@ _lib.qsa_test_stalled_pipeline.argtypes = [ctypes.POINTER(Shape), _vp, _vp, _vp,
 _lib.qsa_sparse_prefill_block_fwd.restype = ctypes.c_int
 _lib.qsa_sparse_prefill_block_fwd.argtypes = [ctypes.POINTER(Shape), ctypes.c_int32, _vp, _vp, _vp, _vp,
                                               _vp, _vp, ctypes.c_float, _vp, _vp, _vp, _vp]
+_lib.qsa_indexer_scores.argtypes = [ctypes.POINTER(IndexerShape), _vp, _vp, _vp, _vp, _vp, _vp, _vp]
+_lib.qsa_topk_select.argtypes = [ctypes.POINTER(IndexerShape), _vp, _vp, _vp, ctypes.c_int64, ctypes.c_int32,
+                                 _vp, ctypes.c_int64, _vp, ctypes.c_int32, _vp, _vp]
 _lib.qsa_status_string.restype = ctypes.c_char_p
 _lib.qsa_status_string.argtypes = [ctypes.c_int]
 _lib.qsa_abi_version.restype = ctypes.c_int32
@@ -407,3 +425,107 @@ def sparse_prefill_block_fwd(q, k_cache, v_cache, block_idx, block_size: int, la
                                              _ptr(n_valid), float(scale), _ptr(out), _ptr(lse),
                                              _ptr(status), stream))
     return out, lse
+
+
+# ------------------------------------------------------------------ indexer
+
+INDEXER_HEAD_DIM = 128
+TOPK_MAX_CANDIDATES = 32768
+
+
+def make_indexer_shape(q_idx, k_idx, block_size: int, scores=None) -> IndexerShape:
+    """Shape/stride descriptor of an indexer call: q_idx [T, H, 128],
+    k_idx [NB, 128] (BF16), scores [T, ld] (FP32)."""
+    if q_idx.dim() != 3 or k_idx.dim() != 2:
+        raise ValueError("q_idx must be [T, H, Dh] and k_idx [NB, Dh]")
+    T, H, Dh = q_idx.shape
+    NB = k_idx.shape[0]
+    if k_idx.shape[1] != Dh:
+        raise ValueError("q_idx and k_idx head dims differ")
+    if q_idx.stride(2) != 1 or k_idx.stride(1) != 1:
+        raise ValueError("innermost dimensions must be contiguous")
+    ld = NB
+    if scores is not None:
+        if scores.dim() != 2 or scores.shape[0] != T or scores.shape[1] < NB or scores.stride(1) != 1:
+            raise ValueError("scores must be [T, >= NB] with unit column stride")
+        ld = scores.stride(0)
+    return IndexerShape(T, H, Dh, NB, int(block_size), 0, q_idx.stride(0), q_idx.stride(1),
+                        k_idx.stride(0), ld)
+
+
+def _need_tok(x, name, T, dev):
+    _need(x, name, torch.int32, dev)
+    if not x.is_contiguous() or tuple(x.shape) != (T,):
+        raise ValueError(f"{name} must be a contiguous [T] int32 tensor")
+
+
+def indexer_scores(q_idx, k_idx, positions, seq_start, block_size: int = 4, scores=None, status=None,
+                   stream=None):
+    """FP32 scores [T, NB]: sum over the H indexer heads of <q_idx[t,h], k_idx[b]>
+    at the complete causal microblocks of each token (other entries untouched;
+    a new buffer starts as -inf)."""
+    dev = q_idx.device
+    _need(q_idx, "q_idx", torch.bfloat16, dev)
+    _need(k_idx, "k_idx", torch.bfloat16, dev)
+    T = q_idx.shape[0]
+    _need_tok(positions, "positions", T, dev)
+    _need_tok(seq_start, "seq_start", T, dev)
+    if scores is None:
+        # rows padded to a multiple of 4 floats: the selection copies 16-byte spans
+        NB = k_idx.shape[0]
+        scores = torch.full((T, (NB + 3) // 4 * 4), float("-inf"), dtype=torch.float32, device=dev)[:, :NB]
+    _need(scores, "scores", torch.float32, dev)
+    if status is not None:
+        _need(status, "status", torch.int32, dev)
+    shape = make_indexer_shape(q_idx, k_idx, block_size, scores)
+    if stream is None:
+        stream = torch.cuda.current_stream(dev).cuda_stream
+    _raise(_lib.qsa_indexer_scores(ctypes.byref(shape), _ptr(q_idx), _ptr(k_idx), _ptr(positions),
+                                   _ptr(seq_start), _ptr(scores), _ptr(status), stream))
+    return scores
+
+
+def topk_select(scores, positions, seq_start, num_blocks: int, budget: int, block_size: int = 4,
+                append_tail: bool = False, lists=None, n_valid=None, copies: int = 1, status=None,
+                stream=None):
+    """Ascending block ids of the `budget` highest-scoring candidates of each
+    token (ties to the smaller block), then with `append_tail` the token's own
+    incomplete block, -1 padded: lists [T, budget (+1)] int32, and the entry
+    count per token written `copies` times: n_valid [T, copies] int32."""
+    dev = scores.device
+    _need(scores, "scores", torch.float32, dev)
+    T = scores.shape[0]
+    _need_tok(positions, "positions", T, dev)
+    _need_tok(seq_start, "seq_start", T, dev)
+    width = int(budget) + (1 if append_tail else 0)
+    if lists is None:
+        lists = torch.empty((T, width), dtype=torch.int32, device=dev)
+    _need(lists, "lists", torch.int32, dev)
+    if lists.dim() != 2 or lists.shape[0] != T or lists.shape[1] < width or (width > 1 and lists.stride(1) != 1):
+        raise ValueError("lists must be [T, >= width] with unit column stride")
+    if n_valid is None:
+        n_valid = torch.empty((T, copies), dtype=torch.int32, device=dev)
+    _need(n_valid, "n_valid", torch.int32, dev)
+    if not n_valid.is_contiguous() or tuple(n_valid.shape) != (T, copies):
+        raise ValueError("n_valid must be a contiguous [T, copies] tensor")
+    if scores.dim() != 2 or scores.shape[1] < num_blocks or (scores.shape[1] > 1 and scores.stride(1) != 1):
+        raise ValueError("scores must be [T, >= num_blocks] with unit column stride")
+    if status is not None:
+        _need(status, "status", torch.int32, dev)
+    shape = IndexerShape(T, 0, INDEXER_HEAD_DIM, int(num_blocks), int(block_size), 0, 0, 0, 0, scores.stride(0))
+    if stream is None:
+        stream = torch.cuda.current_stream(dev).cuda_stream
+    _raise(_lib.qsa_topk_select(ctypes.byref(shape), _ptr(scores), _ptr(positions), _ptr(seq_start),
+                                int(budget), 1 if append_tail else 0, _ptr(lists), lists.stride(0),
+                                _ptr(n_valid), int(copies), _ptr(status), stream))
+    return lists, n_valid
+
+
+def indexer_select(q_idx, k_idx, positions, seq_start, budget: int, block_size: int = 4,
+                   append_tail: bool = True, copies: int = 1, scores=None, stream=None):
+    """Indexer scores then top-K selection (two launches); returns
+    (lists, n_valid, scores)."""
+    scores = indexer_scores(q_idx, k_idx, positions, seq_start, block_size, scores=scores, stream=stream)
+    lists, nv = topk_select(scores, positions, seq_start, k_idx.shape[0], budget, block_size, append_tail,
+                            copies=copies, stream=stream)
+    return lists, nv, scores

@@ -11,15 +11,14 @@
 #include <mutex>
 
 #include "qsa.h"
+#include "qsa_host.cuh"
 #include "qsa_merge.cuh"
 #include "qsa_prefill_mma.cuh"
 #include "qsa_prefill_tc.cuh"
 
 namespace {
 
-constexpr int kMaxDevices = 64;
-
-bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+using namespace qsa::host;
 
 // Validates `s` and the pointers of a forward call.  Returns QSA_OK or the
 // first error found; never touches device memory.
@@ -54,18 +53,6 @@ qsa_status_t validate(const qsa_shape_t* s, const void* q, const void* k, const 
   return QSA_OK;
 }
 
-template <typename Kernel>
-cudaError_t set_smem_once(Kernel kernel, int bytes, std::atomic<int>* done) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-  if (done[dev].load(std::memory_order_acquire)) return cudaSuccess;
-  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-  if (e == cudaSuccess) done[dev].store(1, std::memory_order_release);
-  return e;
-}
-
 template <int NT, bool kDump>
 cudaError_t launch_mma(const qsa::PrefillParams& p, cudaStream_t stream) {
   using C = qsa::MmaCfg<NT>;
@@ -79,36 +66,6 @@ cudaError_t launch_mma(const qsa::PrefillParams& p, cudaStream_t stream) {
 }
 
 // ---------------------------------------------------------------- TMA path
-
-using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* f = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(f);
-  });
-  return fn;
-}
-
-int sm_count() {
-  static std::atomic<int> cache[kMaxDevices];
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 0;
-  int n = cache[dev].load(std::memory_order_relaxed);
-  if (n == 0) {
-    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
-    cache[dev].store(n, std::memory_order_relaxed);
-  }
-  return n;
-}
 
 // Fills the Q tensor map of the tcgen05 kernel.  Returns false when a TMA
 // descriptor cannot express the Q layout or there is nothing to gather (the
@@ -572,7 +529,7 @@ const char* qsa_status_string(qsa_status_t status) {
     case QSA_OK: return "ok";
     case QSA_ERR_NULL: return "a required pointer is NULL";
     case QSA_ERR_SHAPE: return "inconsistent sizes or strides";
-    case QSA_ERR_UNSUPPORTED: return "unsupported configuration (needs BF16, head_dim 256, G <= 16)";
+    case QSA_ERR_UNSUPPORTED: return "unsupported configuration (attention: BF16, head_dim 256, G <= 16; indexer: head_dim 128, 1/2/4/8 heads, <= 32768 candidates)";
     case QSA_ERR_ALIGN: return "rows must start on 16-byte boundaries";
     case QSA_ERR_CUDA: return "a CUDA runtime call failed";
     case QSA_ERR_SCRATCH: return "the call needs more scratch than the built-in array holds (QSA_NOALLOC_SCRATCH_BYTES)";

@@ -77,7 +77,6 @@ constexpr int B_FULL = 0, B_EMPTY = 6, B_SFULL = 12, B_SFREE = 14, B_PFULL = 16,
 constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;  // tmem base, abort flag
 constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + slack for 1024-byte alignment
 
-constexpr uint32_t kStatusOob = 1u, kStatusTimeout = 2u;
 
 struct TcParams {
   CUtensorMap tm_q;                 // Q as [T][Hq][256], box 16 heads x 64 dims
@@ -114,52 +113,6 @@ constexpr uint32_t kIdescQK = (1u << 4) | (1u << 7) | (1u << 10) | (2u << 17) | 
 // PV: both operands MN-major (bits 15 and 16).
 constexpr uint32_t kIdescPV = kIdescQK | (1u << 15) | (1u << 16);
 
-struct Sync {
-  uint32_t bars;
-  volatile uint32_t* abort_flag;
-  int32_t* status;
-
-  __device__ uint32_t bar(int i) const { return bars + 8u * i; }
-
-  __device__ bool aborted() const { return *abort_flag != 0; }
-
-  __device__ void raise_abort() const {
-    *abort_flag = 1u;
-    if (status != nullptr) atomicOr(status, static_cast<int32_t>(kStatusTimeout));
-  }
-
-  // Bounded wait for the phase of parity `parity` of barrier i.
-  __device__ bool wait(int i, uint32_t parity) const {
-    const uint32_t b = bar(i);
-    if (mbar_try_wait(b, parity)) return true;
-    const uint64_t t0 = globaltimer_ns();
-    for (uint32_t it = 1;; ++it) {
-      if (mbar_try_wait(b, parity)) return true;
-      if ((it & 63u) == 0u) {
-        if (aborted()) return false;
-        if (globaltimer_ns() - t0 > 2000000000ull) {
-          raise_abort();
-          return false;
-        }
-      }
-    }
-  }
-
-  // Bounded wait called by all 32 lanes of a warp in convergent code.  The
-  // lanes poll the same barrier word and read the same abort flag and timer
-  // in the same instructions, so they leave the loop together with the same
-  // verdict; an explicit vote after every wait measured 5-6 % slower on the
-  // full workloads.
-  __device__ bool wait_warp(int i, uint32_t parity) const { return wait(i, parity); }
-
-  // Bounded wait that ignores the abort flag (used to drain in-flight copies).
-  __device__ void drain(int i, uint32_t parity) const {
-    const uint32_t b = bar(i);
-    const uint64_t t0 = globaltimer_ns();
-    while (!mbar_try_wait(b, parity))
-      if (globaltimer_ns() - t0 > 2000000000ull) return;
-  }
-};
 
 struct Unit {
   int64_t t;

@@ -284,6 +284,41 @@ def config_c5_block4(device="cpu", seed=CONFIG_SEED_BASE + 8, T=8192, S=131072, 
     return w
 
 
+@dataclasses.dataclass
+class IndexerWorkload:
+    name: str
+    q_idx: torch.Tensor        # [T, H, 128] bf16
+    k_idx: torch.Tensor        # [NB, 128] bf16: one key per microblock
+    positions: torch.Tensor    # [T] int32
+    seq_start: torch.Tensor    # [T] int32
+    block_size: int
+    budget: int
+    description: str = ""
+
+
+def config_indexer(device="cpu", seed=CONFIG_SEED_BASE + 9, T=8192, S=131072, heads=4, head_dim=128,
+                   block_size=4, budget=2048, seq_starts=None) -> IndexerWorkload:
+    """The indexer of the published configuration at the c5 size: 8192 new
+    tokens at positions S-T..S-1 of one sequence, 4 heads x dim 128 sharing
+    one key per microblock of 4 slots (S/4 keys), budget 2048 blocks.  Values
+    are standard normal BF16 (synthetic weights: no checkpoint exists here).
+    `seq_starts` (optional list of slot offsets, multiples of block_size) cuts
+    the T tokens into sequences of equal length packed at the cache end."""
+    gen = _gen(seed, device)
+    NB = S // block_size
+    q = normal_bf16((T, heads, head_dim), gen, device)
+    k = normal_bf16((NB, head_dim), gen, device)
+    pos = torch.arange(S - T, S, device=device, dtype=torch.int32)
+    s0 = torch.zeros(T, dtype=torch.int32, device=device)
+    if seq_starts is not None:
+        per = T // len(seq_starts)
+        for i, st in enumerate(seq_starts):
+            s0[i * per:(i + 1) * per] = int(st)
+    return IndexerWorkload(f"indexer_T{T}_S{S}", q, k, pos, s0, block_size, budget,
+                           f"T={T} at {S - T}..{S - 1}, {NB} block keys, {heads}x{head_dim} heads, "
+                           f"ratio {block_size}, budget {budget}")
+
+
 CONFIGS = {
     "tiny": config_tiny,
     "c2": config_c2,
