@@ -98,6 +98,25 @@ __device__ __forceinline__ void candidates(const int32_t* positions, const int32
   hi = static_cast<int>(h);
 }
 
+// The same range from a token's position and sequence start.
+__device__ __forceinline__ void range_of(int32_t pos, int32_t s0, int32_t NB, int32_t bs, int& lo, int& hi) {
+  int64_t l = static_cast<int64_t>(s0) / bs;
+  int64_t h = (static_cast<int64_t>(pos) + 1) / bs;
+  if (l < 0) l = 0;
+  if (h > NB) h = NB;
+  if (h < l) h = l;
+  lo = static_cast<int>(l);
+  hi = static_cast<int>(h);
+}
+
+// Shared-memory add of 1 at `addr` when `pred` holds, without a branch.
+__device__ __forceinline__ void red_add_if(uint32_t addr, bool pred) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.u32 p, %1, 0;\n\t@p red.shared.add.u32 [%0], 1;\n\t}\n" ::"r"(addr),
+      "r"(static_cast<uint32_t>(pred))
+      : "memory");
+}
+
 struct IxUnit {
   int64_t tok0;
   int tile0;
@@ -418,9 +437,9 @@ constexpr int kTkThreads = 512;
 constexpr int kTkMax = 32768;                      // candidates per row
 constexpr int TK_OFF_ROW = 0;                      // row copy, 16-byte aligned span
 constexpr int TK_OFF_HIST = ((kTkMax + 4) * 4 + 127) / 128 * 128;
-constexpr int TK_OFF_GT = TK_OFF_HIST + 4096 * 4;  // bitmaps, one bit per candidate
+constexpr int TK_OFF_GT = TK_OFF_HIST + 2 * 4096 * 4;  // two histograms, then the bitmaps
 constexpr int TK_OFF_EQ = TK_OFF_GT + kTkMax / 8;
-constexpr int TK_OFF_MISC = TK_OFF_EQ + kTkMax / 8;  // wsum[17], sel_bin, sel_above, ok, mbarrier
+constexpr int TK_OFF_MISC = TK_OFF_EQ + kTkMax / 8;  // warp totals[16], results[4], mbarrier
 constexpr int TK_SMEM = TK_OFF_MISC + 256;
 
 // Persistent CTAs (one per SM) walk the rows t = blockIdx.x + i * gridDim.x.
@@ -428,16 +447,17 @@ constexpr int TK_SMEM = TK_OFF_MISC + 256;
 // one bulk copy (cp.async.bulk, completion on an mbarrier) while the CTA
 // works on the current row from registers: candidate e = j * 512 + tid
 // (j < kR) sits in a register of thread tid as its order-preserving key.
-// Radix select in three passes over key bits 31-20, 19-8 and 7-0 with one
+// Radix select in three passes over key bits 31-20, 19-8 and 7-0 with a
 // 4096-bin shared histogram (12 bits spread the few exponent values of real
 // scores over many bins, which keeps the shared atomics nearly
-// conflict-free); after each pass `prefix` and `mask` name the bin that
+// conflict-free; two histograms alternate so that clearing the next one
+// costs no barrier); after each pass `prefix` and `mask` name the bin that
 // holds the budget-th largest key and `need` how many keys of that bin are
 // still to take; a pass that finds the whole bin taken ends the search.
 // Keys above the bin are all taken, keys in it in block order until `need`
 // runs out: two bitmaps (above / in the bin; one warp ballot is one word)
 // and one packed scan of their word popcounts place every chosen block in
-// ascending order.
+// ascending order.  Every phase costs at most three CTA barriers.
 template <int kR>
 __global__ void __launch_bounds__(kTkThreads, 1) qsa_topk_kernel(const __grid_constant__ TopkParams p) {
   constexpr int kNT = kTkThreads, kW = kNT / 32;
@@ -450,8 +470,8 @@ __global__ void __launch_bounds__(kTkThreads, 1) qsa_topk_kernel(const __grid_co
   uint32_t* hist = reinterpret_cast<uint32_t*>(tk_smem + TK_OFF_HIST);
   uint32_t* gtw = reinterpret_cast<uint32_t*>(tk_smem + TK_OFF_GT);
   uint32_t* eqw = reinterpret_cast<uint32_t*>(tk_smem + TK_OFF_EQ);
-  uint32_t* wsum = reinterpret_cast<uint32_t*>(tk_smem + TK_OFF_MISC);
-  volatile uint32_t* shv = reinterpret_cast<volatile uint32_t*>(tk_smem + TK_OFF_MISC + 96);
+  uint32_t* wtot = reinterpret_cast<uint32_t*>(tk_smem + TK_OFF_MISC);
+  volatile uint32_t* shv = reinterpret_cast<volatile uint32_t*>(tk_smem + TK_OFF_MISC + 64);
   const uint32_t row_addr = smem_u32(tk_smem + TK_OFF_ROW);
   const uint32_t bar = smem_u32(tk_smem + TK_OFF_MISC + 128);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -462,11 +482,9 @@ __global__ void __launch_bounds__(kTkThreads, 1) qsa_topk_kernel(const __grid_co
   }
   __syncthreads();
 
-  // thread 0: start the copy of row t's candidate span (16-byte aligned
-  // around [lo, hi)), or complete the phase at once when nothing is read
-  auto issue = [&](int64_t t) {
-    int lo, hi;
-    candidates(p.positions, p.seq_start, p.NB, p.bs, t, lo, hi);
+  // thread 0: start the copy of row t's candidate span [lo, hi) widened to
+  // 16-byte boundaries, or complete the phase at once when nothing is read
+  auto issue = [&](int64_t t, int lo, int hi) {
     if (min(hi - lo, p.budget) <= 0) {
       mbar_arrive(bar);
       return;
@@ -480,11 +498,30 @@ __global__ void __launch_bounds__(kTkThreads, 1) qsa_topk_kernel(const __grid_co
 
   uint32_t it = 0;
   bool pending = false;
-  if (tid == 0 && blockIdx.x < p.T) {
-    issue(blockIdx.x);
-    pending = true;
+  // position and sequence start of the next row, loaded a row ahead so that
+  // their latency hides behind the current row
+  int32_t npos = 0, ns0 = 0;
+  if (blockIdx.x < p.T) {
+    npos = __ldg(p.positions + blockIdx.x);
+    ns0 = __ldg(p.seq_start + blockIdx.x);
+    if (tid == 0) {
+      int l0, h0;
+      range_of(npos, ns0, p.NB, p.bs, l0, h0);
+      issue(blockIdx.x, l0, h0);
+      pending = true;
+    }
   }
   for (int64_t t = blockIdx.x; t < p.T; t += gridDim.x, ++it) {
+    const int32_t pos_t = npos;
+    int lo, hi;
+    range_of(npos, ns0, p.NB, p.bs, lo, hi);
+    const int n = hi - lo;
+    const int k = min(n, p.budget);
+    const int64_t tn = t + gridDim.x;
+    if (tn < p.T) {
+      npos = __ldg(p.positions + tn);
+      ns0 = __ldg(p.seq_start + tn);
+    }
     if (tid == 0) {
       bool done = mbar_try_wait(bar, it & 1u);
       const uint64_t t0 = globaltimer_ns();
@@ -493,25 +530,30 @@ __global__ void __launch_bounds__(kTkThreads, 1) qsa_topk_kernel(const __grid_co
       else if (p.status != nullptr) atomicOr(p.status, 2);
       shv[2] = done ? 1u : 0u;
     }
+#pragma unroll
+    for (int i = 0; i < kBinsPer; ++i) hist[i * kNT + tid] = 0u;   // first pass's histogram
     __syncthreads();
     if (shv[2] == 0u) break;
-    int lo, hi;
-    candidates(p.positions, p.seq_start, p.NB, p.bs, t, lo, hi);
-    const int n = hi - lo;
-    const int k = min(n, p.budget);
     int32_t* out = p.lists + t * p.list_st;
     const int off = static_cast<int>((t * p.ld + lo) & 3);
     const int jn = n > tid ? (n - tid + kNT - 1) / kNT : 0;
     // key 0 marks "no candidate": a real score's key is at least 0x007fffff
     // (-inf), so 0 shares histogram bin 0 only with negative NaNs and never
     // reaches the selection threshold while n > k
+    // (reads past n stay inside the buffer, which holds kTkMax + 4 floats)
+    const int jv = k > 0 ? jn : 0;
     uint32_t key[kR];
 #pragma unroll
-    for (int j = 0; j < kR; ++j) key[j] = (k > 0 && j < jn) ? order_key(row_s[off + j * kNT + tid]) : 0u;
-    fence_proxy_async_smem();
+    for (int j = 0; j < kR; ++j) {
+      const uint32_t kk = order_key(row_s[off + j * kNT + tid]);
+      key[j] = j < jv ? kk : 0u;
+    }
     __syncthreads();                                   // the row buffer is free again
-    if (tid == 0 && t + gridDim.x < p.T) {
-      issue(t + gridDim.x);
+    if (tid == 0 && tn < p.T) {
+      int l1, h1;
+      range_of(npos, ns0, p.NB, p.bs, l1, h1);
+      fence_proxy_async_smem();
+      issue(tn, l1, h1);
       pending = true;
     }
 
@@ -527,28 +569,41 @@ __global__ void __launch_bounds__(kTkThreads, 1) qsa_topk_kernel(const __grid_co
         for (int pass = 0; pass < 3; ++pass) {
           const int shift = pass == 0 ? 20 : (pass == 1 ? 8 : 0);
           const uint32_t dmask = pass == 2 ? 0xffu : 0xfffu;
+          uint32_t* hb = hist + (pass & 1) * kBins;
+          if (pass < 2) {
+            uint32_t* hz = hist + ((pass + 1) & 1) * kBins;   // the next pass's
 #pragma unroll
-          for (int i = 0; i < kBinsPer; ++i) hist[i * kNT + tid] = 0u;
-          __syncthreads();
+            for (int i = 0; i < kBinsPer; ++i) hz[i * kNT + tid] = 0u;
+          }
           if (pass == 0) {
 #pragma unroll
-            for (int j = 0; j < kR; ++j) atomicAdd(&hist[key[j] >> 20], 1u);
+            for (int j = 0; j < kR; ++j) atomicAdd(&hb[key[j] >> 20], 1u);
           } else {
+            const uint32_t hbase = smem_u32(hb);
 #pragma unroll
             for (int j = 0; j < kR; ++j)
-              if ((key[j] & mask) == prefix) atomicAdd(&hist[(key[j] >> shift) & dmask], 1u);
+              red_add_if(hbase + 4u * ((key[j] >> shift) & dmask), (key[j] & mask) == prefix);
           }
           __syncthreads();
-          // thread i owns bins 4095 - i*kBinsPer .. (high to low)
+          // thread i owns bins 4095 - i*kBinsPer .. (high to low); warps in
+          // thread order cover the bins from the top
           uint32_t c[kBinsPer], own = 0u;
 #pragma unroll
           for (int i = 0; i < kBinsPer; ++i) {
-            c[i] = hist[kBins - 1 - tid * kBinsPer - i];
+            c[i] = hb[kBins - 1 - tid * kBinsPer - i];
             own += c[i];
           }
-          uint32_t total;
-          const uint32_t incl = block_scan<kNT>(own, wsum, warp, lane, total);
-          const uint32_t excl = incl - own;
+          uint32_t x = own;
+#pragma unroll
+          for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+            if (lane >= o) x += y;
+          }
+          if (lane == 31) wtot[warp] = x;
+          __syncthreads();
+          uint32_t before = 0u;
+          for (int w = 0; w < warp; ++w) before += wtot[w];
+          const uint32_t incl = before + x, excl = incl - own;
           if (excl < static_cast<uint32_t>(need) && static_cast<uint32_t>(need) <= incl) {
             uint32_t cum = excl;
 #pragma unroll
@@ -556,6 +611,7 @@ __global__ void __launch_bounds__(kTkThreads, 1) qsa_topk_kernel(const __grid_co
               if (cum + c[i] >= static_cast<uint32_t>(need)) {
                 shv[0] = kBins - 1u - tid * kBinsPer - i;
                 shv[1] = cum;
+                shv[3] = c[i];
                 break;
               }
               cum += c[i];
@@ -566,9 +622,7 @@ __global__ void __launch_bounds__(kTkThreads, 1) qsa_topk_kernel(const __grid_co
           need -= static_cast<int>(shv[1]);
           prefix |= d << shift;
           mask |= dmask << shift;
-          const bool whole = static_cast<uint32_t>(need) == hist[d];
-          __syncthreads();                               // hist and shv are rewritten next pass
-          if (whole) break;
+          if (static_cast<uint32_t>(need) == shv[3]) break;   // the whole bin is taken
         }
       }
       // bitmaps: word j*kW + warp, bit lane = candidate j*kNT + warp*32 + lane
@@ -592,8 +646,16 @@ __global__ void __launch_bounds__(kTkThreads, 1) qsa_topk_kernel(const __grid_co
         loc[i] = run;
         run += (static_cast<uint32_t>(__popc(gtw[w])) << 16) | __popc(eqw[w]);
       }
-      uint32_t total;
-      const uint32_t base = block_scan<kNT>(run, wsum, warp, lane, total) - run;
+      uint32_t x = run;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+      }
+      if (lane == 31) wtot[warp] = x;
+      __syncthreads();
+      uint32_t base = x - run;
+      for (int w = 0; w < warp; ++w) base += wtot[w];
 #pragma unroll
       for (int i = 0; i < kWPer; ++i) {
         const int w = tid * kWPer + i;
@@ -616,11 +678,10 @@ __global__ void __launch_bounds__(kTkThreads, 1) qsa_topk_kernel(const __grid_co
           sel &= sel - 1u;
         }
       }
-      __syncthreads();                                   // bitmaps are rewritten next row
     }
     // causal tail, padding, counts
     int cnt = k;
-    const int64_t pos = __ldg(p.positions + t);
+    const int64_t pos = pos_t;
     const bool tail = p.append_tail != 0 && (pos + 1) % p.bs != 0;
     if (tail) {
       if (tid == 0) out[k] = static_cast<int32_t>(pos / p.bs);
