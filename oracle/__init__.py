@@ -65,6 +65,11 @@ class _Args(ctypes.Structure):
         ("scale", ctypes.c_double),
         ("block_size", ctypes.c_int64),
         ("last_slot", ctypes.c_void_p),
+        ("kv_fp8", ctypes.c_int32),
+        ("k8", ctypes.c_void_p),
+        ("v8", ctypes.c_void_p),
+        ("k_scale", ctypes.c_double),
+        ("v_scale", ctypes.c_double),
     ]
 
 
@@ -96,6 +101,8 @@ class Oracle:
                                        ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p]
         lib.qsa_oracle_bf16_to_double.restype = ctypes.c_double
         lib.qsa_oracle_bf16_to_double.argtypes = [ctypes.c_uint16]
+        lib.qsa_oracle_e4m3_to_double.restype = ctypes.c_double
+        lib.qsa_oracle_e4m3_to_double.argtypes = [ctypes.c_uint8]
         lib.qsa_oracle_indexer_scores.restype = ctypes.c_int
         lib.qsa_oracle_indexer_scores.argtypes = [ctypes.POINTER(_IndexerArgs), ctypes.c_void_p,
                                                   ctypes.c_int64, ctypes.c_int, ctypes.c_void_p]
@@ -109,9 +116,16 @@ class Oracle:
         return self.lib.qsa_oracle_bf16_to_double(ctypes.c_uint16(bits))
 
     def sparse_prefill(self, q, k_cache, v_cache, topk_idx, n_valid=None, scale=0.0,
-                       tokens=None, n_threads=None, block_size=1, last_slot=None):
+                       tokens=None, n_threads=None, block_size=1, last_slot=None,
+                       k_scale=1.0, v_scale=1.0):
+        """k_cache / v_cache are BF16, or FP8 E4M3 (torch float8_e4m3fn, or
+        uint8 bytes) whose elements are the decoded byte times k_scale /
+        v_scale."""
         return _sparse_prefill(self.lib, q, k_cache, v_cache, topk_idx, n_valid, scale,
-                               tokens, n_threads, block_size, last_slot)
+                               tokens, n_threads, block_size, last_slot, k_scale, v_scale)
+
+    def e4m3_to_double(self, bits: int) -> float:
+        return self.lib.qsa_oracle_e4m3_to_double(int(bits))
 
 
     def indexer_scores(self, q_idx, k_idx, positions, seq_start, block_size=4, tokens=None):
@@ -228,13 +242,33 @@ def bf16_to_double(bits: int) -> float:
 
 
 def sparse_prefill(q, k_cache, v_cache, topk_idx, n_valid=None, scale=0.0,
-                   tokens=None, n_threads=None, block_size=1, last_slot=None):
+                   tokens=None, n_threads=None, block_size=1, last_slot=None,
+                   k_scale=1.0, v_scale=1.0):
     return default().sparse_prefill(q, k_cache, v_cache, topk_idx, n_valid, scale,
-                                    tokens, n_threads, block_size, last_slot)
+                                    tokens, n_threads, block_size, last_slot, k_scale, v_scale)
+
+
+def _as_u8(x):
+    """FP8 E4M3 data (torch float8_e4m3fn tensor or uint8 numpy bytes) -> uint8 ndarray view."""
+    if hasattr(x, "dtype") and str(x.dtype) == "torch.float8_e4m3fn":
+        x = x.detach()
+        if x.device.type != "cpu":
+            raise ValueError("oracle inputs must be on the host")
+        import torch
+        x = x.view(torch.uint8).numpy()
+    x = np.asarray(x)
+    if x.dtype != np.uint8:
+        raise TypeError(f"expected FP8 E4M3 bytes, got {x.dtype}")
+    return x
+
+
+def _is_fp8(x):
+    return (hasattr(x, "dtype") and str(x.dtype) == "torch.float8_e4m3fn") or \
+        (isinstance(x, np.ndarray) and x.dtype == np.uint8)
 
 
 def _sparse_prefill(lib, q, k_cache, v_cache, topk_idx, n_valid, scale, tokens, n_threads,
-                    block_size=1, last_slot=None):
+                    block_size=1, last_slot=None, k_scale=1.0, v_scale=1.0):
     """FP64 oracle.  q [T,Hq,D], k_cache/v_cache [S,Hkv,D] (BF16, host),
     topk_idx [T,Hkv,K] int32, n_valid [T,Hkv] int32 or None.
 
@@ -245,7 +279,12 @@ def _sparse_prefill(lib, q, k_cache, v_cache, topk_idx, n_valid, scale, tokens, 
     Returns (out [n,Hq,D] float64, lse [n,Hq] float64, n_out_of_range) for the
     tokens listed in ``tokens`` (all tokens when None).
     """
-    q = _as_u16(q); k = _as_u16(k_cache); v = _as_u16(v_cache)
+    fp8 = _is_fp8(k_cache)
+    q = _as_u16(q)
+    if fp8:
+        k = _as_u8(k_cache); v = _as_u8(v_cache)
+    else:
+        k = _as_u16(k_cache); v = _as_u16(v_cache)
     idx = _as_i32(topk_idx); nv = _as_i32(n_valid)
     T, Hq, D = q.shape
     S, Hkv, Dk = k.shape
@@ -278,9 +317,11 @@ def _sparse_prefill(lib, q, k_cache, v_cache, topk_idx, n_valid, scale, tokens, 
             raise ValueError("last_slot must be [T]")
         ls = np.ascontiguousarray(ls)
     a = _Args(T, Hq, Hkv, D, K, S, qs[0], qs[1], ks[0], ks[1], ist[0], ist[1],
-              q.ctypes.data, k.ctypes.data, v.ctypes.data, idx.ctypes.data,
-              nv.ctypes.data if nv is not None else None, float(scale), int(block_size),
-              ls.ctypes.data if ls is not None else None)
+              q.ctypes.data, None if fp8 else k.ctypes.data, None if fp8 else v.ctypes.data,
+              idx.ctypes.data, nv.ctypes.data if nv is not None else None, float(scale),
+              int(block_size), ls.ctypes.data if ls is not None else None,
+              1 if fp8 else 0, k.ctypes.data if fp8 else None, v.ctypes.data if fp8 else None,
+              float(k_scale), float(v_scale))
     if n_threads is None:
         n_threads = os.cpu_count() or 1
     rc = lib.qsa_oracle_fwd(ctypes.byref(a), tokens.ctypes.data, n, int(n_threads),

@@ -24,6 +24,13 @@ double qsa_oracle_bf16_to_double(uint16_t bits) {
   return (double)f;
 }
 
+double qsa_oracle_e4m3_to_double(uint8_t bits) {
+  const int sign = bits >> 7, e = (bits >> 3) & 15, m = bits & 7;
+  if (e == 15 && m == 7) return NAN;
+  const double mag = e == 0 ? ldexp((double)m, -9) : ldexp(1.0 + m / 8.0, e - 7);
+  return sign ? -mag : mag;
+}
+
 typedef struct {
   const qsa_oracle_args* a;
   const int64_t* tokens;
@@ -83,10 +90,16 @@ static int64_t one_row(const qsa_oracle_args* a, int64_t t, int64_t h,
   /* Step 2: scores s_j = scale * <q, k_j>. */
   const uint16_t* q = a->q + t * a->q_stride_tok + h * a->q_stride_head;
   for (int64_t j = 0; j < n; ++j) {
-    const uint16_t* kr = a->k + sel[j] * a->kv_stride_slot + g * a->kv_stride_head;
     double dot = 0.0;
-    for (int64_t d = 0; d < D; ++d)
-      dot += qsa_oracle_bf16_to_double(q[d]) * qsa_oracle_bf16_to_double(kr[d]);
+    if (a->kv_fp8) {
+      const uint8_t* kb = a->k8 + sel[j] * a->kv_stride_slot + g * a->kv_stride_head;
+      for (int64_t d = 0; d < D; ++d)
+        dot += qsa_oracle_bf16_to_double(q[d]) * (qsa_oracle_e4m3_to_double(kb[d]) * a->k_scale);
+    } else {
+      const uint16_t* kr = a->k + sel[j] * a->kv_stride_slot + g * a->kv_stride_head;
+      for (int64_t d = 0; d < D; ++d)
+        dot += qsa_oracle_bf16_to_double(q[d]) * qsa_oracle_bf16_to_double(kr[d]);
+    }
     s[j] = scale * dot;
   }
 
@@ -99,9 +112,14 @@ static int64_t one_row(const qsa_oracle_args* a, int64_t t, int64_t h,
   /* Step 4: weighted sum of the selected V rows, normalised by l. */
   for (int64_t d = 0; d < D; ++d) out_row[d] = 0.0;
   for (int64_t j = 0; j < n; ++j) {
-    const uint16_t* vr = a->v + sel[j] * a->kv_stride_slot + g * a->kv_stride_head;
     const double p = s[j];
-    for (int64_t d = 0; d < D; ++d) out_row[d] += p * qsa_oracle_bf16_to_double(vr[d]);
+    if (a->kv_fp8) {
+      const uint8_t* vb = a->v8 + sel[j] * a->kv_stride_slot + g * a->kv_stride_head;
+      for (int64_t d = 0; d < D; ++d) out_row[d] += p * (qsa_oracle_e4m3_to_double(vb[d]) * a->v_scale);
+    } else {
+      const uint16_t* vr = a->v + sel[j] * a->kv_stride_slot + g * a->kv_stride_head;
+      for (int64_t d = 0; d < D; ++d) out_row[d] += p * qsa_oracle_bf16_to_double(vr[d]);
+    }
   }
   for (int64_t d = 0; d < D; ++d) out_row[d] /= l;
   *lse_out = m + log(l);
@@ -140,7 +158,8 @@ int64_t qsa_oracle_fwd(const qsa_oracle_args* a, const int64_t* tokens,
   if (a->num_kv_heads <= 0 || a->num_q_heads <= 0 || a->head_dim <= 0 ||
       a->num_q_heads % a->num_kv_heads != 0 || a->topk < 0 || a->num_slots < 0)
     return -1;
-  if (n_tokens > 0 && (!a->q || (a->topk > 0 && (!a->idx || !a->k || !a->v)))) return -1;
+  const int has_kv = a->kv_fp8 ? (a->k8 && a->v8) : (a->k && a->v);
+  if (n_tokens > 0 && (!a->q || (a->topk > 0 && (!a->idx || !has_kv)))) return -1;
   for (int64_t i = 0; i < n_tokens; ++i)
     if (tokens[i] < 0 || tokens[i] >= a->num_tokens) return -1;
 

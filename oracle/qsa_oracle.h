@@ -50,6 +50,17 @@ typedef struct {
   int64_t block_size;
   /* [T] largest visible slot per token (slots above it are empty), or NULL. */
   const int32_t* last_slot;
+  /* FP8 KV cache (nonzero kv_fp8): k8 / v8 hold OCP FP8 E4M3 bytes with the
+   * strides above, k and v are unused; element value = decoded byte times
+   * k_scale (v_scale).  The pages name the cache format "fp8_e4m3" only
+   * (page "Qwen4-Exp QSA llega al Ascend de Huawei", second of the two
+   * observations on the NVIDIA side); the per-tensor scales are the plainest
+   * reading of a scaled FP8 cache. */
+  int32_t kv_fp8;
+  const uint8_t* k8;
+  const uint8_t* v8;
+  double k_scale;
+  double v_scale;
 } qsa_oracle_args;
 
 /*
@@ -65,6 +76,11 @@ int64_t qsa_oracle_fwd(const qsa_oracle_args* a, const int64_t* tokens,
 
 /* Exact BF16 -> double widening of one bit pattern (exposed for tests). */
 double qsa_oracle_bf16_to_double(uint16_t bits);
+
+/* Exact OCP FP8 E4M3 -> double decoding of one byte (exposed for tests):
+ * sign, 4 exponent bits with bias 7, 3 mantissa bits; exponent 0 holds the
+ * subnormals m * 2^-9; S.1111.111 is NaN; there are no infinities. */
+double qsa_oracle_e4m3_to_double(uint8_t bits);
 
 /* ------------------------------------------------------------------------
  * QSA indexer (page "Qwen4-Exp QSA llega al Ascend de Huawei", section "Por

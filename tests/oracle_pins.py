@@ -32,6 +32,12 @@ Pins (what the pages and the mathematics fix):
   scores; the candidate ranges of hand-picked positions (causal tails 0..3,
   a later sequence start) are the complete causal blocks; strides do not
   matter.
+* fp8_cache     -- page "Qwen4-Exp QSA llega al Ascend de Huawei" names an
+  fp8_e4m3 KV cache: the byte decoding equals torch's float8_e4m3fn over all
+  256 patterns; with power-of-two scales the FP8 attention equals the
+  (pinned) BF16 attention on the dequantized caches bit for bit; with other
+  scales it equals torch's scaled_dot_product_attention in float64 on the
+  dequantized values.
 * topk          -- the selection equals a lexicographic sort on (-score,
   block) by numpy (library routine); every chosen score >= every unchosen
   one; all-equal scores take the first blocks; -0.0 ties +0.0; the causal
@@ -392,6 +398,53 @@ def check_topk(orc):
     assert int(sel[5, 0]) == 7 and int(sel[1, 0]) == 1
 
 
+def check_fp8_cache(orc):
+    # byte decoding against torch's float8_e4m3fn (library routine)
+    allb = torch.arange(256, dtype=torch.uint8)
+    ref = allb.view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    got = np.array([orc.e4m3_to_double(b) for b in range(256)])
+    np.testing.assert_array_equal(np.isnan(got), np.isnan(ref))
+    fin = ~np.isnan(ref)
+    np.testing.assert_array_equal(got[fin], ref[fin])
+    gen = torch.Generator().manual_seed(83)
+    T, S, Hq, Hkv, K, D = 7, 60, 16, 2, 11, 256
+    q = W.normal_bf16((T, Hq, D), gen, "cpu")
+    k8 = W.normal_fp8((S, Hkv, D), gen, "cpu", std=3.0)
+    v8 = W.normal_fp8((S, Hkv, D), gen, "cpu")
+    k8[0, 0, :8] = torch.tensor([2 ** -9, -2 ** -8, 448.0, -448.0, 0.0, -0.0, 2 ** -6, 3 * 2 ** -9]).to(torch.float8_e4m3fn)
+    idx = torch.stack([torch.randperm(S, generator=gen)[:K] for _ in range(T * Hkv)]).view(T, Hkv, K).to(torch.int32)
+    idx[:, 0, 0] = 0                                   # every token sees the subnormal row
+    # power-of-two scales: the dequantized caches are exact in BF16
+    ks, vs = 0.5, 4.0
+    got = orc.sparse_prefill(q, k8, v8, idx, None, 0.0, k_scale=ks, v_scale=vs)
+    kb = (k8.to(torch.float64) * ks).to(torch.bfloat16)
+    vb = (v8.to(torch.float64) * vs).to(torch.bfloat16)
+    assert torch.equal(kb.to(torch.float64), k8.to(torch.float64) * ks)
+    want = orc.sparse_prefill(q, kb, vb, idx, None, 0.0)
+    np.testing.assert_array_equal(got[0], want[0])
+    np.testing.assert_array_equal(got[1], want[1])
+    # other scales: dense causal attention (every causal slot listed) against
+    # torch's SDPA on the dequantized values in float64
+    T2 = 12
+    q2 = W.normal_bf16((T2, 6, D), gen, "cpu")
+    k2 = W.normal_fp8((T2, 1, D), gen, "cpu", std=2.0)
+    v2 = W.normal_fp8((T2, 1, D), gen, "cpu")
+    idx2 = torch.full((T2, 1, T2), -1, dtype=torch.int32)
+    for t in range(T2):
+        idx2[t, 0, : t + 1] = torch.randperm(t + 1, generator=gen).to(torch.int32)
+    ks, vs = 0.37, 1.9
+    out, lse, _ = orc.sparse_prefill(q2, k2, v2, idx2, None, 0.0, k_scale=ks, v_scale=vs)
+    qd = q2.to(torch.float64).permute(1, 0, 2)[None]
+    kd = (k2.to(torch.float64) * ks).permute(1, 0, 2).repeat_interleave(6, dim=0)[None]
+    vd = (v2.to(torch.float64) * vs).permute(1, 0, 2).repeat_interleave(6, dim=0)[None]
+    ref = torch.nn.functional.scaled_dot_product_attention(qd, kd, vd, is_causal=True, scale=1 / 16)
+    np.testing.assert_allclose(out, ref[0].permute(1, 0, 2).numpy(), **TOL)
+    sc = (qd @ kd.transpose(-1, -2)) / 16
+    sc = sc.masked_fill(~torch.ones(T2, T2, dtype=torch.bool).tril(), float("-inf"))
+    np.testing.assert_allclose(lse, torch.logsumexp(sc, dim=-1)[0].permute(1, 0).numpy(), **TOL)
+
+
 ALL_CHECKS = [check_bf16_widening, check_dense_causal, check_packing, check_permutation,
               check_head_padding, check_closed_forms, check_brute_force, check_worked_example,
-              check_split_merge, check_block_lists, check_indexer_scores, check_topk]
+              check_split_merge, check_block_lists, check_indexer_scores, check_topk,
+              check_fp8_cache]

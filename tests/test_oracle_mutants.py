@@ -43,6 +43,11 @@ MUTANTS = {
                           "if (a->score < b->score) return -1;\n  if (a->score > b->score) return 1;"),
     "topk_ties_to_larger_block": ("return (a->block > b->block) - (a->block < b->block);",
                                   "return (a->block < b->block) - (a->block > b->block);"),
+    "e4m3_exponent_bias": ("ldexp(1.0 + m / 8.0, e - 7)", "ldexp(1.0 + m / 8.0, e - 8)"),
+    "e4m3_subnormal_as_normal": ("e == 0 ? ldexp((double)m, -9)", "e == 0 ? ldexp(1.0 + m / 8.0, -7)"),
+    "fp8_k_scale_dropped": ("(qsa_oracle_e4m3_to_double(kb[d]) * a->k_scale)", "qsa_oracle_e4m3_to_double(kb[d])"),
+    "fp8_v_scaled_by_k_scale": ("(qsa_oracle_e4m3_to_double(vb[d]) * a->v_scale)",
+                                "(qsa_oracle_e4m3_to_double(vb[d]) * a->k_scale)"),
     "topk_tail_always": ("if (append_tail && ((int64_t)a->positions[t] + 1) % bs != 0)", "if (append_tail)"),
 }
 

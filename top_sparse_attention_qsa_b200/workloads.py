@@ -73,6 +73,15 @@ def normal_bf16(shape, gen, device, std: float = 1.0) -> torch.Tensor:
     return x.to(torch.bfloat16)
 
 
+def normal_fp8(shape, gen, device, std: float = 1.0) -> torch.Tensor:
+    """N(0, std^2) values stored as OCP FP8 E4M3 (torch float8_e4m3fn,
+    round to nearest): a synthetic FP8 KV cache."""
+    x = torch.randn(shape, generator=gen, device=device, dtype=torch.float32)
+    if std != 1.0:
+        x.mul_(std)
+    return x.to(torch.float8_e4m3fn)
+
+
 def random_subset_rows(lo: torch.Tensor, width: torch.Tensor, count: int, gen,
                        device, max_chunk_elems: int = 1 << 27) -> torch.Tensor:
     """For each row r, `count` distinct integers drawn uniformly from
