@@ -66,6 +66,8 @@ def parse_args():
                     help="decode workload timed under 'decode' ('' to skip)")
     ap.add_argument("--blocks", default="c5_block4",
                     help="microblock-list workload timed under 'blocks' ('' to skip)")
+    ap.add_argument("--fp8", default="c5",
+                    help="workload timed with an FP8 E4M3 KV cache under 'fp8' ('' to skip)")
     ap.add_argument("--indexer", default="indexer",
                     help="indexer + top-K workload timed under 'indexer' ('' to skip)")
     ap.add_argument("--e2e-steps", type=int, default=10)
@@ -458,6 +460,8 @@ def run_cuda(args):
         line["decode"] = run_decode_bench(args.decode, dev, barrier, max_ranks, world, hbm)
     if args.blocks and not args.profile:
         line["blocks"] = run_blocks_bench(args.blocks, dev, barrier, max_ranks, world, hbm)
+    if args.fp8 and not args.profile:
+        line["fp8"] = run_fp8_bench(args.fp8, dev, barrier, max_ranks, world, hbm)
     if args.indexer and not args.profile:
         line["indexer"] = run_indexer_bench(dev, barrier, max_ranks, world, hbm, bf16)
     if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.profile:
@@ -580,6 +584,38 @@ def run_blocks_bench(name, dev, barrier, reduce_max, world, hbm):
     ms = statistics.mean(per_ms)
     return {"workload": w.name, "desc": w.description, "tokens_per_s": s["T"] * steps * world / (total_ms / 1e3),
             "mean_launch_ms": ms, "live_keys": keys, "gathered_kv_gbs": keys * 1024 / (ms / 1e3) / 1e9,
+            "algo_gbs": algo / (ms / 1e3) / 1e9, "frac_of_hbm": algo / (ms / 1e3) / 1e9 / hbm,
+            "steps": steps}
+
+
+def run_fp8_bench(name, dev, barrier, reduce_max, world, hbm):
+    """The same lists and Q as `name`, with the K and V caches stored as FP8
+    E4M3 (k_scale 0.5, v_scale 2): half the gathered bytes per key."""
+    from top_sparse_attention_qsa_b200 import _capi
+    from top_sparse_attention_qsa_b200 import workloads as W
+    w = make_workload(name, dev)
+    entries = workload_accounting(w)["entries"]
+    gen = torch.Generator(device=dev).manual_seed(77)
+    k8 = W.normal_fp8(tuple(w.k_cache.shape), gen, dev)
+    v8 = W.normal_fp8(tuple(w.v_cache.shape), gen, dev)
+    w.k_cache = w.v_cache = None                   # free the BF16 caches
+    T, Hq, D = w.q.shape
+    out = torch.empty_like(w.q)
+    lse = torch.empty((T, Hq), dtype=torch.float32, device=dev)
+    gathered = entries * 2 * D
+    algo = gathered + entries * 4 + T * Hq * D * 2 * 2 + T * Hq * 4
+
+    def step():
+        _capi.sparse_prefill_fp8_fwd(w.q, k8, v8, w.topk_idx, 0.5, 2.0, n_valid=w.n_valid, scale=w.scale,
+                                     out=out, lse=lse)
+
+    steps = 20
+    total_ms, per_ms, _ = time_launches(step, steps, 3, barrier, "fp8")
+    total_ms = reduce_max(total_ms)
+    ms = statistics.mean(per_ms)
+    return {"workload": w.name + "_fp8e4m3", "tokens_per_s": T * steps * world / (total_ms / 1e3),
+            "mean_launch_ms": ms, "live_entries": entries, "algo_bytes": algo,
+            "gathered_kv_gbs": gathered / (ms / 1e3) / 1e9,
             "algo_gbs": algo / (ms / 1e3) / 1e9, "frac_of_hbm": algo / (ms / 1e3) / 1e9 / hbm,
             "steps": steps}
 

@@ -65,6 +65,9 @@ typedef enum {
 #define QSA_STATUS_TIMEOUT 2  /* a pipeline wait inside the kernel exceeded its
                                  2 s bound; the kernel stopped early and its
                                  outputs are not valid */
+#define QSA_STATUS_Q_RANGE 4  /* FP8-cache path: a query element lies outside
+                                 the FP16 range (|q| > 65504); that unit's
+                                 outputs are not valid */
 
 typedef struct {
   int64_t num_tokens;     /* T >= 0: query tokens, packed over all sequences
@@ -163,6 +166,39 @@ qsa_status_t qsa_sparse_prefill_block_fwd(const qsa_shape_t* shape,
                                           const int32_t* n_valid, float scale,
                                           void* out, float* lse,
                                           int32_t* status, void* stream);
+
+/*
+ * FP8 KV cache (page "Qwen4-Exp QSA llega al Ascend de Huawei", the
+ * observations on the NVIDIA side: a KV cache in fp8_e4m3).  k_cache and
+ * v_cache hold OCP FP8 E4M3 bytes (finite-only "e4m3fn"; the NaN bytes 0x7f /
+ * 0xff give unspecified results) in the layout of qsa_shape_t, strides in
+ * elements = bytes; element value = decoded byte * k_scale (v_scale), one
+ * scale per tensor.  Q stays BF16; out is BF16; lse is natural-log FP32 of
+ * the scaled scores, as for the BF16 cache.  Lists are token lists
+ * (block_size 1, last_slot NULL) or microblock lists as in
+ * qsa_sparse_prefill_block_fwd.
+ *
+ * The kernel is the tcgen05 kernel with the cache rows converted to FP16 in
+ * shared memory (exact: every E4M3 value is an FP16 value); Q is converted to
+ * FP16 too (exact for 2^-14 <= |q| <= 65504, rounded to a multiple of 2^-24
+ * below that; beyond it QSA_STATUS_Q_RANGE is set) and the probabilities
+ * enter the PV product as FP16.  k_scale multiplies the softmax scale and
+ * v_scale the normalised output, both in FP32.
+ *
+ * Cache strides (slot and head) must be multiples of 16 elements and the
+ * cache bases 16-byte aligned (QSA_ERR_ALIGN otherwise).  Other arguments
+ * and conventions as qsa_sparse_prefill_block_fwd.
+ */
+qsa_status_t qsa_sparse_prefill_fp8_fwd(const qsa_shape_t* shape,
+                                        int32_t block_size,
+                                        const int32_t* last_slot,
+                                        const void* q, const void* k_cache,
+                                        const void* v_cache,
+                                        const int32_t* topk_idx,
+                                        const int32_t* n_valid, float scale,
+                                        float k_scale, float v_scale,
+                                        void* out, float* lse,
+                                        int32_t* status, void* stream);
 
 /*
  * Split-K sparse attention for decode-shaped calls: few query tokens per KV

@@ -160,3 +160,16 @@ def test_indexer_nulls_and_topk_limits(capi):
     assert sel(ctypes.byref(s), P + 4, P, P, 8, 0, P, 8, P, 1, None, None) == 4  # scores not 16-byte aligned
     odd = _ishape(capi, score_stride_tok=66)
     assert sel(ctypes.byref(odd), P, P, P, 8, 0, P, 8, P, 1, None, None) == 4   # row stride not 4 floats
+
+
+def test_fp8_entry_validation(capi):
+    lib = capi.library()
+    s = _shape(capi)
+    fp8 = lib.qsa_sparse_prefill_fp8_fwd
+    # kv strides must be multiples of 16 elements (bytes) for 16-byte copies
+    odd = _shape(capi, kv_stride_slot=264, kv_stride_head=264)
+    assert fp8(ctypes.byref(odd), 1, None, P, P, P, P, None, 0.0, 1.0, 1.0, P, None, None, None) == 4
+    assert fp8(ctypes.byref(s), 3, None, P, P, P, P, None, 0.0, 1.0, 1.0, P, None, None, None) == 3
+    assert fp8(ctypes.byref(s), 1, None, None, P, P, P, None, 0.0, 1.0, 1.0, P, None, None, None) == 1
+    assert fp8(ctypes.byref(_shape(capi, head_dim=128)), 1, None, P, P, P, P, None, 0.0, 1.0, 1.0, P,
+               None, None, None) == 3

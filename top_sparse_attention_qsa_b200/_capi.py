@@ -26,6 +26,7 @@ QSA_OK, QSA_ERR_NULL, QSA_ERR_SHAPE, QSA_ERR_UNSUPPORTED, QSA_ERR_ALIGN, QSA_ERR
 NOALLOC_SCRATCH_BYTES = 16 << 20
 STATUS_OOB_SLOT = 1
 STATUS_TIMEOUT = 2
+STATUS_Q_RANGE = 4
 KERNEL_AUTO, KERNEL_TCGEN05, KERNEL_WARP_MMA = 0, 1, 2
 KERNELS = {"auto": KERNEL_AUTO, "tcgen05": KERNEL_TCGEN05, "warp_mma": KERNEL_WARP_MMA}
 HEAD_DIM = 256
@@ -35,7 +36,8 @@ EXPORTS = ("qsa_sparse_prefill_fwd", "qsa_sparse_prefill_fwd_with", "qsa_sparse_
            "qsa_sparse_prefill_block_fwd",
            "qsa_sparse_prefill_fwd_host", "qsa_sparse_decode_fwd", "qsa_sparse_decode_workspace_bytes",
            "qsa_sparse_decode_num_splits", "qsa_sparse_decode_fwd_noalloc", "qsa_test_stalled_pipeline",
-           "qsa_indexer_scores", "qsa_topk_select", "qsa_status_string", "qsa_abi_version")
+           "qsa_sparse_prefill_fp8_fwd", "qsa_indexer_scores", "qsa_topk_select", "qsa_status_string",
+           "qsa_abi_version")
 
 
 class Shape(ctypes.Structure):
@@ -108,6 +110,9 @@ _lib.qsa_test_stalled_pipeline.argtypes = [ctypes.POINTER(Shape), _vp, _vp, _vp,
 _lib.qsa_sparse_prefill_block_fwd.restype = ctypes.c_int
 _lib.qsa_sparse_prefill_block_fwd.argtypes = [ctypes.POINTER(Shape), ctypes.c_int32, _vp, _vp, _vp, _vp,
                                               _vp, _vp, ctypes.c_float, _vp, _vp, _vp, _vp]
+_lib.qsa_sparse_prefill_fp8_fwd.argtypes = [ctypes.POINTER(Shape), ctypes.c_int32, _vp, _vp, _vp, _vp, _vp,
+                                            _vp, ctypes.c_float, ctypes.c_float, ctypes.c_float, _vp, _vp,
+                                            _vp, _vp]
 _lib.qsa_indexer_scores.argtypes = [ctypes.POINTER(IndexerShape), _vp, _vp, _vp, _vp, _vp, _vp, _vp]
 _lib.qsa_topk_select.argtypes = [ctypes.POINTER(IndexerShape), _vp, _vp, _vp, ctypes.c_int64, ctypes.c_int32,
                                  _vp, ctypes.c_int64, _vp, ctypes.c_int32, _vp, _vp]
@@ -424,6 +429,45 @@ def sparse_prefill_block_fwd(q, k_cache, v_cache, block_idx, block_size: int, la
                                              _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_idx),
                                              _ptr(n_valid), float(scale), _ptr(out), _ptr(lse),
                                              _ptr(status), stream))
+    return out, lse
+
+
+def sparse_prefill_fp8_fwd(q, k_cache, v_cache, topk_idx, k_scale: float = 1.0, v_scale: float = 1.0,
+                           n_valid=None, scale: float = 0.0, block_size: int = 1, last_slot=None,
+                           out=None, lse=None, status=None, stream=None, want_lse: bool = True):
+    """FP8 E4M3 KV cache (torch.float8_e4m3fn [S, Hkv, 256]); element value =
+    stored value * k_scale (v_scale).  Token lists (block_size 1) or
+    microblock lists with an optional last_slot [T] int32."""
+    dev = q.device
+    _need(q, "q", torch.bfloat16, dev)
+    _need(k_cache, "k_cache", torch.float8_e4m3fn, dev)
+    _need(v_cache, "v_cache", torch.float8_e4m3fn, dev)
+    _need(topk_idx, "topk_idx", torch.int32, dev)
+    _check_kv(k_cache, v_cache)
+    if last_slot is not None:
+        _need(last_slot, "last_slot", torch.int32, dev)
+        if not last_slot.is_contiguous() or tuple(last_slot.shape) != (q.shape[0],):
+            raise ValueError("last_slot must be a contiguous [T] tensor")
+    if n_valid is not None:
+        _need(n_valid, "n_valid", torch.int32, dev)
+        if not n_valid.is_contiguous() or tuple(n_valid.shape) != tuple(topk_idx.shape[:2]):
+            raise ValueError("n_valid must be a contiguous [T, Hkv] tensor")
+    if out is None:
+        out = torch.empty(q.shape, dtype=torch.bfloat16, device=dev)
+    _need(out, "out", torch.bfloat16, dev)
+    if lse is None and want_lse:
+        lse = torch.empty(q.shape[:2], dtype=torch.float32, device=dev)
+    if lse is not None:
+        _need(lse, "lse", torch.float32, dev)
+    if status is not None:
+        _need(status, "status", torch.int32, dev)
+    shape = make_shape(q, k_cache, topk_idx, out, lse)
+    if stream is None:
+        stream = torch.cuda.current_stream(dev).cuda_stream
+    _raise(_lib.qsa_sparse_prefill_fp8_fwd(ctypes.byref(shape), int(block_size), _ptr(last_slot), _ptr(q),
+                                           _ptr(k_cache), _ptr(v_cache), _ptr(topk_idx), _ptr(n_valid),
+                                           float(scale), float(k_scale), float(v_scale), _ptr(out),
+                                           _ptr(lse), _ptr(status), stream))
     return out, lse
 
 

@@ -95,10 +95,10 @@ bool make_tc_params(const qsa_shape_t* s, const void* q, qsa::tc::TcParams* tp) 
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <bool kDump, bool kStall = false, bool kBlocks = false>
+template <bool kDump, bool kStall = false, bool kBlocks = false, bool kFp8 = false>
 cudaError_t launch_tc(const qsa::tc::TcParams& tp, cudaStream_t stream) {
   static std::atomic<int> done[kMaxDevices];
-  auto kernel = qsa::tc::qsa_prefill_tc_kernel<kDump, kStall, kBlocks>;
+  auto kernel = qsa::tc::qsa_prefill_tc_kernel<kDump, kStall, kBlocks, kFp8>;
   cudaError_t e = set_smem_once(kernel, qsa::tc::SMEM_BYTES, done);
   if (e != cudaSuccess) return e;
   const int64_t units = tp.T * tp.Hkv;
@@ -184,6 +184,7 @@ qsa_status_t run_forward(const qsa_shape_t* s, const void* q, const void* k, con
     tp.part_lse = nullptr;
     tp.block_shift = 0;
     tp.last_slot = nullptr;
+    tp.o_scale = 1.f;
     e = stall_test ? launch_tc<false, true>(tp, st)
                    : (dump ? launch_tc<true>(tp, st) : launch_tc<false>(tp, st));
   } else if (p.G <= 8)
@@ -303,6 +304,7 @@ qsa_status_t run_decode(const qsa_shape_t* s, const void* q, const void* k, cons
   tp.part_lse = part_lse;
   tp.block_shift = 0;
   tp.last_slot = nullptr;
+  tp.o_scale = 1.f;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (launch_tc<false>(tp, st) != cudaSuccess) return QSA_ERR_CUDA;
   if (launch_merge(s, part_o, part_lse, pl.splits, out, lse, st) != cudaSuccess) return QSA_ERR_CUDA;
@@ -344,6 +346,64 @@ cudaError_t noalloc_scratch_address(void** ptr) {
   }
   *ptr = p;
   return cudaSuccess;
+}
+
+// Microblock (or token) lists on the tcgen05 kernel, BF16 or FP8 E4M3 cache.
+qsa_status_t run_lists(const qsa_shape_t* shape, int32_t block_size, const int32_t* last_slot,
+                       const void* q, const void* k_cache, const void* v_cache,
+                       const int32_t* topk_idx, const int32_t* n_valid, float scale,
+                       float k_scale, float v_scale, bool fp8, void* out, float* lse,
+                       int32_t* status, void* stream) {
+  qsa_status_t rc = validate(shape, q, k_cache, v_cache, topk_idx, out);
+  if (rc != QSA_OK) return rc;
+  if (fp8 && shape->topk > 0 && (shape->kv_stride_slot % 16 != 0 || shape->kv_stride_head % 16 != 0))
+    return QSA_ERR_ALIGN;   // FP8 rows move in 16-byte pieces of 16 elements
+  int shift = -1;
+  for (int b = 0; b <= 4; ++b)
+    if (block_size == (1 << b)) shift = b;
+  if (shift < 0) return QSA_ERR_UNSUPPORTED;
+  if ((static_cast<int64_t>(shape->topk) << shift) > 0x7fffffffLL) return QSA_ERR_UNSUPPORTED;
+  if (shape->num_tokens == 0) return QSA_OK;
+  static thread_local qsa::tc::TcParams tp;
+  if (!make_tc_params(shape, q, &tp)) return QSA_ERR_UNSUPPORTED;
+  const float sc = scale > 0.f ? scale : 0.0625f;
+  tp.idx = topk_idx;
+  tp.n_valid = n_valid;
+  tp.kraw = k_cache;
+  tp.vraw = v_cache;
+  tp.out = static_cast<__nv_bfloat16*>(out);
+  tp.lse = lse;
+  tp.status = status;
+  tp.gathered = nullptr;
+  tp.T = shape->num_tokens;
+  tp.idx_st = shape->idx_stride_tok;
+  tp.idx_sh = shape->idx_stride_head;
+  tp.o_st = shape->o_stride_tok;
+  tp.o_sh = shape->o_stride_head;
+  tp.lse_st = shape->lse_stride_tok;
+  tp.kv_ss = shape->kv_stride_slot;
+  tp.kv_sh = shape->kv_stride_head;
+  tp.Hkv = shape->num_kv_heads;
+  tp.G = shape->num_q_heads / shape->num_kv_heads;
+  tp.K = shape->topk;
+  tp.S = static_cast<int32_t>(shape->num_slots);
+  // an FP8 cache's K scale multiplies every score; its V scale the output
+  tp.scale_log2 = sc * (fp8 ? k_scale : 1.f) * 1.4426950408889634f;
+  tp.o_scale = fp8 ? v_scale : 1.f;
+  tp.splits = 1;
+  tp.chunk = shape->topk << shift;
+  tp.part_o = nullptr;
+  tp.part_lse = nullptr;
+  tp.block_shift = shift;
+  tp.last_slot = last_slot;
+  const bool plain = shift == 0 && last_slot == nullptr;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  if (fp8)
+    e = plain ? launch_tc<false, false, false, true>(tp, st) : launch_tc<false, false, true, true>(tp, st);
+  else
+    e = plain ? launch_tc<false>(tp, st) : launch_tc<false, false, true>(tp, st);
+  return e == cudaSuccess ? QSA_OK : QSA_ERR_CUDA;
 }
 
 }  // namespace
@@ -470,48 +530,18 @@ qsa_status_t qsa_sparse_prefill_block_fwd(const qsa_shape_t* shape, int32_t bloc
                                           const int32_t* topk_idx, const int32_t* n_valid,
                                           float scale, void* out, float* lse, int32_t* status,
                                           void* stream) {
-  qsa_status_t rc = validate(shape, q, k_cache, v_cache, topk_idx, out);
-  if (rc != QSA_OK) return rc;
-  int shift = -1;
-  for (int b = 0; b <= 4; ++b)
-    if (block_size == (1 << b)) shift = b;
-  if (shift < 0) return QSA_ERR_UNSUPPORTED;
-  if ((static_cast<int64_t>(shape->topk) << shift) > 0x7fffffffLL) return QSA_ERR_UNSUPPORTED;
-  if (shape->num_tokens == 0) return QSA_OK;
-  static thread_local qsa::tc::TcParams tp;
-  if (!make_tc_params(shape, q, &tp)) return QSA_ERR_UNSUPPORTED;
-  const float sc = scale > 0.f ? scale : 0.0625f;
-  tp.idx = topk_idx;
-  tp.n_valid = n_valid;
-  tp.kraw = k_cache;
-  tp.vraw = v_cache;
-  tp.out = static_cast<__nv_bfloat16*>(out);
-  tp.lse = lse;
-  tp.status = status;
-  tp.gathered = nullptr;
-  tp.T = shape->num_tokens;
-  tp.idx_st = shape->idx_stride_tok;
-  tp.idx_sh = shape->idx_stride_head;
-  tp.o_st = shape->o_stride_tok;
-  tp.o_sh = shape->o_stride_head;
-  tp.lse_st = shape->lse_stride_tok;
-  tp.kv_ss = shape->kv_stride_slot;
-  tp.kv_sh = shape->kv_stride_head;
-  tp.Hkv = shape->num_kv_heads;
-  tp.G = shape->num_q_heads / shape->num_kv_heads;
-  tp.K = shape->topk;
-  tp.S = static_cast<int32_t>(shape->num_slots);
-  tp.scale_log2 = sc * 1.4426950408889634f;
-  tp.splits = 1;
-  tp.chunk = shape->topk << shift;
-  tp.part_o = nullptr;
-  tp.part_lse = nullptr;
-  tp.block_shift = shift;
-  tp.last_slot = last_slot;
-  const cudaError_t e = shift == 0 && last_slot == nullptr
-                            ? launch_tc<false>(tp, static_cast<cudaStream_t>(stream))
-                            : launch_tc<false, false, true>(tp, static_cast<cudaStream_t>(stream));
-  return e == cudaSuccess ? QSA_OK : QSA_ERR_CUDA;
+  return run_lists(shape, block_size, last_slot, q, k_cache, v_cache, topk_idx, n_valid, scale, 1.f,
+                   1.f, false, out, lse, status, stream);
+}
+
+qsa_status_t qsa_sparse_prefill_fp8_fwd(const qsa_shape_t* shape, int32_t block_size,
+                                        const int32_t* last_slot, const void* q,
+                                        const void* k_cache, const void* v_cache,
+                                        const int32_t* topk_idx, const int32_t* n_valid,
+                                        float scale, float k_scale, float v_scale, void* out,
+                                        float* lse, int32_t* status, void* stream) {
+  return run_lists(shape, block_size, last_slot, q, k_cache, v_cache, topk_idx, n_valid, scale,
+                   k_scale, v_scale, true, out, lse, status, stream);
 }
 
 qsa_status_t qsa_test_stalled_pipeline(const qsa_shape_t* shape, const void* q,

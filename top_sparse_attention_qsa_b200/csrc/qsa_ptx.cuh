@@ -98,6 +98,22 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// Two FP32 values -> packed FP16x2 (round to nearest even), lo in bits 0-15.
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;\n" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// Two OCP FP8 E4M3 values (bits 0-7 and 8-15) -> FP16x2, exactly (every
+// E4M3 value is an FP16 value).
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two_bytes) {
+  uint32_t r;
+  const uint16_t v = static_cast<uint16_t>(two_bytes);
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;\n" : "=r"(r) : "h"(v));
+  return r;
+}
+
 __device__ __forceinline__ int ld_nc_s32(const int32_t* p) {
   int v;
   asm volatile("ld.global.nc.L1::no_allocate.s32 %0, [%1];\n" : "=r"(v) : "l"(p));
