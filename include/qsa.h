@@ -65,9 +65,7 @@ typedef enum {
 #define QSA_STATUS_TIMEOUT 2  /* a pipeline wait inside the kernel exceeded its
                                  2 s bound; the kernel stopped early and its
                                  outputs are not valid */
-#define QSA_STATUS_Q_RANGE 4  /* FP8-cache path: a query element lies outside
-                                 the FP16 range (|q| > 65504); that unit's
-                                 outputs are not valid */
+
 
 typedef struct {
   int64_t num_tokens;     /* T >= 0: query tokens, packed over all sequences
@@ -178,12 +176,15 @@ qsa_status_t qsa_sparse_prefill_block_fwd(const qsa_shape_t* shape,
  * (block_size 1, last_slot NULL) or microblock lists as in
  * qsa_sparse_prefill_block_fwd.
  *
- * The kernel is the tcgen05 kernel with the cache rows converted to FP16 in
- * shared memory (exact: every E4M3 value is an FP16 value); Q is converted to
- * FP16 too (exact for 2^-14 <= |q| <= 65504, rounded to a multiple of 2^-24
- * below that; beyond it QSA_STATUS_Q_RANGE is set) and the probabilities
- * enter the PV product as FP16.  k_scale multiplies the softmax scale and
- * v_scale the normalised output, both in FP32.
+ * The kernel's tensor cores read the FP8 cache tiles as gathered
+ * (tcgen05 kind::f8f6f4).  Both MMA operands are E4M3, so the query (scaled
+ * per head by a power of two that puts its largest |q| in [128, 256)) and
+ * the softmax probabilities are each written as the sum of two E4M3 terms,
+ * hi + lo / 16 (the query exactly; the probabilities to 8 significant bits,
+ * as the BF16 kernel rounds them), with separate FP32 accumulators for the
+ * two terms.  k_scale multiplies the softmax scale and v_scale the
+ * normalised output, both in FP32.  Non-finite query elements give
+ * unspecified results for their unit.
  *
  * Cache strides (slot and head) must be multiples of 16 elements and the
  * cache bases 16-byte aligned (QSA_ERR_ALIGN otherwise).  Other arguments

@@ -26,7 +26,6 @@ QSA_OK, QSA_ERR_NULL, QSA_ERR_SHAPE, QSA_ERR_UNSUPPORTED, QSA_ERR_ALIGN, QSA_ERR
 NOALLOC_SCRATCH_BYTES = 16 << 20
 STATUS_OOB_SLOT = 1
 STATUS_TIMEOUT = 2
-STATUS_Q_RANGE = 4
 KERNEL_AUTO, KERNEL_TCGEN05, KERNEL_WARP_MMA = 0, 1, 2
 KERNELS = {"auto": KERNEL_AUTO, "tcgen05": KERNEL_TCGEN05, "warp_mma": KERNEL_WARP_MMA}
 HEAD_DIM = 256

@@ -15,6 +15,7 @@
 #include "qsa_merge.cuh"
 #include "qsa_prefill_mma.cuh"
 #include "qsa_prefill_tc.cuh"
+#include "qsa_prefill_f8.cuh"
 
 namespace {
 
@@ -95,10 +96,24 @@ bool make_tc_params(const qsa_shape_t* s, const void* q, qsa::tc::TcParams* tp) 
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <bool kDump, bool kStall = false, bool kBlocks = false, bool kFp8 = false>
+template <bool kBlocks>
+cudaError_t launch_f8(const qsa::tc::TcParams& tp, cudaStream_t stream) {
+  static std::atomic<int> done[kMaxDevices];
+  auto kernel = qsa::f8::qsa_prefill_f8_kernel<kBlocks>;
+  cudaError_t e = set_smem_once(kernel, qsa::f8::F_SMEM, done);
+  if (e != cudaSuccess) return e;
+  const int64_t units = tp.T * tp.Hkv;
+  const int nsm = sm_count();
+  if (nsm <= 0) return cudaErrorInvalidDevice;
+  const unsigned grid = static_cast<unsigned>(units < nsm ? units : nsm);
+  kernel<<<grid, qsa::tc::kThreads, qsa::f8::F_SMEM, stream>>>(tp);
+  return cudaGetLastError();
+}
+
+template <bool kDump, bool kStall = false, bool kBlocks = false>
 cudaError_t launch_tc(const qsa::tc::TcParams& tp, cudaStream_t stream) {
   static std::atomic<int> done[kMaxDevices];
-  auto kernel = qsa::tc::qsa_prefill_tc_kernel<kDump, kStall, kBlocks, kFp8>;
+  auto kernel = qsa::tc::qsa_prefill_tc_kernel<kDump, kStall, kBlocks>;
   cudaError_t e = set_smem_once(kernel, qsa::tc::SMEM_BYTES, done);
   if (e != cudaSuccess) return e;
   const int64_t units = tp.T * tp.Hkv;
@@ -396,11 +411,14 @@ qsa_status_t run_lists(const qsa_shape_t* shape, int32_t block_size, const int32
   tp.part_lse = nullptr;
   tp.block_shift = shift;
   tp.last_slot = last_slot;
+  tp.q_ptr = q;
+  tp.q_st = shape->q_stride_tok;
+  tp.q_sh = shape->q_stride_head;
   const bool plain = shift == 0 && last_slot == nullptr;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaError_t e;
   if (fp8)
-    e = plain ? launch_tc<false, false, false, true>(tp, st) : launch_tc<false, false, true, true>(tp, st);
+    e = plain ? launch_f8<false>(tp, st) : launch_f8<true>(tp, st);
   else
     e = plain ? launch_tc<false>(tp, st) : launch_tc<false, false, true>(tp, st);
   return e == cudaSuccess ? QSA_OK : QSA_ERR_CUDA;

@@ -1,0 +1,530 @@
+// qsa_prefill_f8.cuh -- QSA top-K sparse-attention prefill over an FP8 E4M3
+// KV cache: tcgen05 kind::f8f6f4 kernel for sm_100a.
+//
+// The operation is the one of qsa_prefill_tc.cuh (page "Qwen4-Exp QSA llega
+// al Ascend de Huawei", section "Lo que realmente añade la pull request"),
+// with the cache elements stored as OCP FP8 E4M3 times a per-tensor scale
+// (same page, the observations on the NVIDIA side: an fp8_e4m3 KV cache).
+//
+// The tensor cores read the cache tiles as they were gathered: one 32 KB ring
+// slot holds a whole K or V tile (128 keys x 256 dims x 1 B), so six slots
+// keep three tiles in flight, twice the BF16 kernel's 1.5.  Both MMA operands
+// of kind::f8f6f4 are FP8, so the BF16 query and the FP32 probabilities are
+// each written as an exact-enough pair of E4M3 terms:
+//   q * 2^a_h = q_hi + q_lo / 16     (exact: a BF16 value has 8 significant
+//                                     bits, each E4M3 term 4; a_h puts the
+//                                     head's largest |q| in [128, 256))
+//   p         = p_hi + p_lo / 16     (8 significant bits, like the BF16 P of
+//                                     the BF16 kernel; p <= 2^8 by the lazy
+//                                     rescale)
+// with separate TMEM accumulators for the two terms: S_hi, S_lo per score
+// buffer and O_hi, O_lo per output half.  s = (S_hi + S_lo / 16) * 2^-a_h and
+// o = (O_hi + O_lo / 16) * v_scale / l.
+//
+// Warps (persistent CTAs, one per SM):
+//   warps 0-3   producers: list entries one tile ahead, 16-byte cp.async of
+//               the 256-byte K and V rows into the 128-byte-swizzled K-major
+//               layout (K slot, then V slot per tile)
+//   warp 4      all lanes: the unit's Q (BF16, from global memory) split into
+//               q_hi / q_lo E4M3 tiles with per-head scale; lane 0 issues the
+//               score MMAs (A = K tile, B = q_hi then q_lo; M=128, N=16, K=32)
+//   warp 5      lane 0 issues PV: O_{hi,lo}^T += V^T (MN-major) . P_{hi,lo}^T
+//               (MN-major) for the two 128-dim halves
+//   warps 6-9   softmax as in the BF16 kernel, reading both score terms and
+//               writing p_hi / p_lo
+// Every wait is bounded (2 s of %globaltimer) as in the BF16 kernel.
+#pragma once
+
+#include "qsa_prefill_tc.cuh"
+
+namespace qsa {
+namespace f8 {
+
+using namespace tc;
+
+constexpr int kSlots8 = 6;                    // 32 KB: one K or V tile
+constexpr int kQ8Bytes = kGp * 256;           // one E4M3 Q term: 16 heads x 256 dims
+constexpr int kP8Bytes = kKeys * kGp;         // one E4M3 P term: 128 keys x 16 heads
+constexpr int kTmemCols8 = 128;               // S: 2 buffers x {hi, lo} x 16; O: {hi, lo} x 2 halves x 16
+constexpr int kTS = 0, kTO = 64;              // TMEM column bases
+
+constexpr int F_RING = 0;
+constexpr int F_Q8 = F_RING + kSlots8 * kSlotBytes;   // 2 buffers x {hi, lo}
+constexpr int F_P8 = F_Q8 + 2 * 2 * kQ8Bytes;         // 2 buffers x {hi, lo}
+constexpr int F_QSC = F_P8 + 2 * 2 * kP8Bytes;        // 2 buffers x 16 per-head score factors
+constexpr int F_RED = F_QSC + 2 * kGp * 4;            // max[2][4][16] + sum[2][4][16]
+constexpr int F_BAR = F_RED + 1024;
+constexpr int G_FULL = 0, G_EMPTY = 6, G_SFULL = 12, G_SFREE = 14, G_PFULL = 16, G_PEMPTY = 18,
+              G_QFULL = 20, G_QEMPTY = 22, G_OFULL = 24, G_OEMPTY = 25, G_RMAX = 26, G_RSUM = 28,
+              G_DONE = 30, G_NUM = 32;
+constexpr int F_MISC = F_BAR + G_NUM * 8;             // tmem base, abort flag
+constexpr int F_SMEM = F_MISC + 16 + 1024;
+
+// kind::f8f6f4: FP32 accumulator, E4M3 A and B (format 0), N = 16, M = 128.
+constexpr uint32_t kIdescQK8 = (1u << 4) | (2u << 17) | (8u << 24);
+// PV: both operands MN-major.
+constexpr uint32_t kIdescPV8 = kIdescQK8 | (1u << 15) | (1u << 16);
+
+// ------------------------------------------------------------------ producers
+
+template <bool kBlocks>
+__device__ void producer8(const TcParams& p, const Sync& sy, uint32_t sb, int pw, int lane) {
+  uint32_t c_slot = 0;
+  const int64_t units = num_units(p);
+  const int cc = lane & 15;                          // 16-byte chunk of the 256-byte row
+  const int rsel = lane >> 4;                        // which of the two rows of an instruction
+  const uint32_t dchunk = static_cast<uint32_t>((cc >> 3) * kBlockBytes);
+  constexpr int rows_w = kKeys / kProducerWarps;
+  bool ok = true;
+  for (int64_t u = blockIdx.x; u < units && ok; u += gridDim.x) {
+    const Unit un = decode_unit(p, u);
+    const int32_t* list = p.idx + un.t * p.idx_st + static_cast<int64_t>(un.g) * p.idx_sh;
+    const int32_t last = kBlocks ? last_visible(p, un.t) : 0x7fffffff;
+    const char* kbase = reinterpret_cast<const char*>(p.kraw) + static_cast<int64_t>(un.g) * p.kv_sh + cc * 16;
+    const char* vbase = reinterpret_cast<const char*>(p.vraw) + static_cast<int64_t>(un.g) * p.kv_sh + cc * 16;
+    const int64_t row_bytes = p.kv_ss;
+    const int jr = rows_w * pw + lane;
+    const bool own = lane < rows_w;
+    int32_t entry_next = own ? key_entry<kBlocks>(p, list, un, jr) : -1;
+    for (int i = 0; i < un.n_tiles && ok; ++i) {
+      int32_t id = key_slot<kBlocks>(p, un, i * kKeys + jr, entry_next, last);
+      entry_next = (own && i + 1 < un.n_tiles) ? key_entry<kBlocks>(p, list, un, (i + 1) * kKeys + jr) : -1;
+      if (id == -2) {
+        id = -1;
+        if (p.status != nullptr) atomicOr(p.status, static_cast<int32_t>(kStatusOob));
+      }
+#pragma unroll 1
+      for (int h = 0; h < 2; ++h) {                  // K tile, then V tile
+        const uint32_t slot = c_slot % kSlots8;
+        ok = sy.wait_warp(G_EMPTY + slot, ((c_slot / kSlots8) & 1u) ^ 1u);
+        if (!ok) break;
+        const char* src0 = h == 0 ? kbase : vbase;
+        const uint32_t dst0 = sb + F_RING + slot * kSlotBytes + dchunk;
+#pragma unroll
+        for (int k = 0; k < rows_w / 2; ++k) {
+          const int r = rows_w * pw + 2 * k + rsel;
+          const int32_t rid = __shfl_sync(0xffffffffu, id, 2 * k + rsel);
+          const bool live = rid >= 0;
+          const char* src = live ? src0 + static_cast<int64_t>(rid) * row_bytes : src0;
+          cp_async_16(dst0 + r * 128 + (((cc & 7) ^ (r & 7)) << 4), src, live ? 16 : 0);
+        }
+        cp_async_mbar_arrive(sy.bar(G_FULL + slot));
+        ++c_slot;
+      }
+    }
+  }
+  asm volatile("cp.async.wait_all;\n" ::: "memory");
+}
+
+// ------------------------------------------------------------------ Q split
+
+// Lane l of warp 4 takes head l/2, dims [128*(l&1), +128): loads them from
+// global memory, finds the head's largest |q| (with its partner lane), and
+// writes q * 2^a = q_hi + q_lo / 16 into the two E4M3 tiles (K-major, 128-byte
+// swizzle: two 128-dim blocks of 16 rows x 128 B) and 2^-a * scale_log2 into
+// the score factors.  Heads past the group are zero.
+__device__ __forceinline__ void q_split(const TcParams& p, const Unit& un, uint32_t qhi, uint32_t qlo,
+                                        float* qsc, int lane) {
+  const int h = lane >> 1, half = lane & 1;
+  uint4 v[16];
+  if (h < p.G) {
+    const char* src = reinterpret_cast<const char*>(p.q_ptr) +
+                      (un.t * p.q_st + (static_cast<int64_t>(un.g) * p.G + h) * p.q_sh + half * 128) * 2;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = __ldg(reinterpret_cast<const uint4*>(src) + i);
+  } else {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = make_uint4(0u, 0u, 0u, 0u);
+  }
+  uint32_t mx = 0u;                                  // max |q| as BF16 bits widened (order = magnitude)
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) mx = max(mx, max((w[j] << 16) & 0x7fffffffu, w[j] & 0x7fff0000u));
+  }
+  mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+  // a = 7 - floor(log2 max): the largest |q| * 2^a lands in [128, 256)
+  int a = 0;
+  if (mx != 0u) a = 7 - (static_cast<int>(mx >> 23) - 127);
+  a = max(-126, min(a, 126));
+  const float up = __int_as_float((127 + a) << 23);
+  if (half == 0) qsc[h] = p.scale_log2 * __int_as_float((127 - a) << 23);
+#pragma unroll
+  for (int c8 = 0; c8 < 8; ++c8) {                   // 16 dims per 16-byte chunk
+    uint32_t hw[4], lw[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      // dims 4j..4j+3 of the chunk: bf16 words v[2*c8 + j/2], halves
+      const uint4 vv = v[2 * c8 + (j >> 1)];
+      const uint32_t w0 = (j & 1) ? vv.z : vv.x, w1 = (j & 1) ? vv.w : vv.y;
+      const float x0 = __uint_as_float(w0 << 16) * up, x1 = __uint_as_float(w0 & 0xffff0000u) * up;
+      const float x2 = __uint_as_float(w1 << 16) * up, x3 = __uint_as_float(w1 & 0xffff0000u) * up;
+      const uint32_t h01 = pack_e4m3x2(x0, x1), h23 = pack_e4m3x2(x2, x3);
+      float y0, y1, y2, y3;
+      f16x2_to_f32(e4m3x2_to_f16x2(h01), y0, y1);
+      f16x2_to_f32(e4m3x2_to_f16x2(h23), y2, y3);
+      const uint32_t l01 = pack_e4m3x2((x0 - y0) * 16.f, (x1 - y1) * 16.f);
+      const uint32_t l23 = pack_e4m3x2((x2 - y2) * 16.f, (x3 - y3) * 16.f);
+      hw[j] = h01 | (h23 << 16);
+      lw[j] = l01 | (l23 << 16);
+    }
+    const uint32_t off = half * 2048 + h * 128 + ((c8 ^ (h & 7)) << 4);
+    st_shared_v4(qhi + off, hw[0], hw[1], hw[2], hw[3]);
+    st_shared_v4(qlo + off, lw[0], lw[1], lw[2], lw[3]);
+  }
+}
+
+// ------------------------------------------------------------------ MMA issuers
+
+// Warp 4: per unit all lanes split Q into buffer (unit & 1) once the MMAs of
+// two units ago have released it; lane 0 then issues S_hi += K q_hi^T and
+// S_lo += K q_lo^T for every tile.
+__device__ void qk8(const TcParams& p, const Sync& sy, uint32_t sb, uint8_t* sp, uint32_t tmem, int lane) {
+  uint32_t c_tile = 0, c_unit = 0;
+  const int64_t units = num_units(p);
+  bool ok = true;
+  for (int64_t u = blockIdx.x; u < units && ok; u += gridDim.x) {
+    const Unit un = decode_unit(p, u);
+    const uint32_t qb = c_unit & 1u;
+    ok = sy.wait_warp(G_QEMPTY + qb, ((c_unit >> 1) & 1u) ^ 1u);
+    if (!ok) break;
+    ++c_unit;
+    const uint32_t qhi = sb + F_Q8 + qb * 2 * kQ8Bytes, qlo = qhi + kQ8Bytes;
+    if (un.n_tiles > 0) q_split(p, un, qhi, qlo, reinterpret_cast<float*>(sp + F_QSC) + qb * kGp, lane);
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+      mbar_arrive(sy.bar(G_QFULL + qb));             // the softmax reads the score factors
+      if (un.n_tiles == 0) mbar_arrive(sy.bar(G_QEMPTY + qb));
+      for (int i = 0; i < un.n_tiles && ok; ++i, ++c_tile) {
+        const uint32_t c = c_tile;
+        const uint32_t sbuf = c & 1u;
+        ok = sy.wait(G_SFREE + sbuf, ((c >> 1) & 1u) ^ 1u);
+        const uint32_t ck = 2u * c;
+        const uint32_t slot = ck % kSlots8;
+        if (ok) ok = sy.wait(G_FULL + slot, (ck / kSlots8) & 1u);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t kt = sb + F_RING + slot * kSlotBytes;
+#pragma unroll
+        for (int term = 0; term < 2; ++term) {
+          const uint32_t qa = term == 0 ? qhi : qlo;
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            // K-major, 128-byte swizzle: a 32-dim step advances 32 B inside
+            // the atom; dims 128-255 sit 16 KB (K) / 2 KB (Q) further
+            const uint64_t a = smem_desc(kt + (kk >> 2) * kBlockBytes + (kk & 3) * 32, 16, 1024, 2);
+            const uint64_t b = smem_desc(qa + (kk >> 2) * 2048 + (kk & 3) * 32, 16, 1024, 2);
+            umma_f8_ss(tmem + kTS + sbuf * 32 + term * 16, a, b, kIdescQK8, kk > 0 ? 1u : 0u);
+          }
+        }
+        umma_commit(sy.bar(G_EMPTY + slot));
+        umma_commit(sy.bar(G_SFULL + sbuf));
+        if (i == un.n_tiles - 1) umma_commit(sy.bar(G_QEMPTY + qb));
+      }
+    }
+    ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+  }
+  if (lane == 0) {
+    umma_commit(sy.bar(G_DONE));
+    sy.drain(G_DONE, 0);
+  }
+  __syncwarp();
+}
+
+// Warp 5, lane 0: O_{hi,lo}[mh] += V_half(mh)^T . P_{hi,lo}^T per tile.
+__device__ void pv8(const TcParams& p, const Sync& sy, uint32_t sb, uint32_t tmem) {
+  uint32_t c_tile = 0, c_unit = 0;
+  const int64_t units = num_units(p);
+  bool ok = true;
+  for (int64_t u = blockIdx.x; u < units && ok; u += gridDim.x) {
+    const Unit un = decode_unit(p, u);
+    const uint32_t ue = c_unit++;
+    ok = sy.wait(G_OEMPTY, (ue & 1u) ^ 1u);
+    if (!ok) break;
+    if (un.n_tiles == 0) {
+      mbar_arrive(sy.bar(G_OFULL));
+      continue;
+    }
+    for (int i = 0; i < un.n_tiles && ok; ++i, ++c_tile) {
+      const uint32_t c = c_tile;
+      const uint32_t pb = c & 1u;
+      ok = sy.wait(G_PFULL + pb, (c >> 1) & 1u);
+      const uint32_t cv = 2u * c + 1u;
+      const uint32_t slot = cv % kSlots8;
+      if (ok) ok = sy.wait(G_FULL + slot, (cv / kSlots8) & 1u);
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t vt = sb + F_RING + slot * kSlotBytes;
+      const uint32_t pt = sb + F_P8 + pb * 2 * kP8Bytes;
+#pragma unroll
+      for (int mh = 0; mh < 2; ++mh)
+#pragma unroll
+        for (int term = 0; term < 2; ++term)
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            // A = V^T: MN-major, 128-byte swizzle; the 128 dims of a half are
+            // one atom row, groups of 8 keys 1 KB apart, 32 keys per step
+            const uint64_t a = smem_desc(vt + mh * kBlockBytes + kk * 4096, kBlockBytes, 1024, 2);
+            // B = P^T: MN-major, no swizzle; 16 heads = one 16-byte core row per
+            // key, key groups of 8 128 B apart
+            const uint64_t b = smem_desc(pt + term * kP8Bytes + kk * 512, 128, 2048, 0);
+            umma_f8_ss(tmem + kTO + term * 32 + mh * 16, a, b, kIdescPV8, (i == 0 && kk == 0) ? 0u : 1u);
+          }
+      umma_commit(sy.bar(G_EMPTY + slot));
+      umma_commit(sy.bar(G_PEMPTY + pb));
+    }
+    if (ok) umma_commit(sy.bar(G_OFULL));
+  }
+  umma_commit(sy.bar(G_DONE + 1));
+  sy.drain(G_DONE + 1, 0);
+}
+
+// ------------------------------------------------------------------ softmax
+
+template <bool kBlocks>
+__device__ void softmax8(const TcParams& p, const Sync& sy, uint32_t sb, uint8_t* sp, uint32_t tmem, int warp,
+                         int lane) {
+  const int wq = warp & 3;
+  const int key = wq * 32 + lane;
+  const uint32_t tl = tmem + (static_cast<uint32_t>(wq * 32) << 16);
+  float* red_max = reinterpret_cast<float*>(sp + F_RED);
+  float* red_sum = red_max + 128;
+  const float* qsc_all = reinterpret_cast<const float*>(sp + F_QSC);
+  uint32_t c_tile = 0, c_unit = 0;
+  const int64_t units = num_units(p);
+  const int G = p.G;
+  bool ok = true;
+  for (int64_t u = blockIdx.x; u < units && ok; u += gridDim.x) {
+    const Unit un = decode_unit(p, u);
+    const int32_t* list = p.idx + un.t * p.idx_st + static_cast<int64_t>(un.g) * p.idx_sh;
+    const int32_t last = kBlocks ? last_visible(p, un.t) : 0x7fffffff;
+    const uint32_t qb = c_unit & 1u;
+    ok = sy.wait_warp(G_QFULL + qb, (c_unit >> 1) & 1u);
+    if (!ok) break;
+    float qs[kGp];
+#pragma unroll
+    for (int h = 0; h < kGp; ++h) qs[h] = qsc_all[qb * kGp + h];
+    float m_run[kGp], l_part[kGp];
+#pragma unroll
+    for (int h = 0; h < kGp; ++h) {
+      m_run[h] = -INFINITY;
+      l_part[h] = 0.f;
+    }
+    int32_t entry_next = un.n_tiles > 0 ? key_entry<kBlocks>(p, list, un, key) : -1;
+    for (int i = 0; i < un.n_tiles; ++i) {
+      const uint32_t c = c_tile + i;
+      const uint32_t buf = c & 1u;
+      const bool valid = key_slot<kBlocks>(p, un, i * kKeys + key, entry_next, last) >= 0;
+      entry_next = i + 1 < un.n_tiles ? key_entry<kBlocks>(p, list, un, (i + 1) * kKeys + key) : -1;
+      ok = sy.wait_warp(G_SFULL + buf, (c >> 1) & 1u);
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t rh[16], rl[16];
+      tmem_ld16(tl + kTS + buf * 32, rh);
+      tmem_ld16(tl + kTS + buf * 32 + 16, rl);
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(sy.bar(G_SFREE + buf));
+      float s[kGp];
+#pragma unroll
+      for (int h = 0; h < kGp; ++h)
+        s[h] = (valid && h < G) ? fmaf(__uint_as_float(rl[h]), 0.0625f, __uint_as_float(rh[h])) * qs[h]
+                                : -INFINITY;
+      const float wmax = xreduce16<true>(s, lane);
+      float* rm = red_max + buf * 64;
+      if ((lane & 1) == 0) rm[wq * 16 + ((lane >> 1) & 15)] = wmax;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(sy.bar(G_RMAX + buf));
+      ok = sy.wait_warp(G_RMAX + buf, (c >> 1) & 1u);
+      if (!ok) break;
+      float tmax[kGp];
+#pragma unroll
+      for (int h = 0; h < kGp; ++h)
+        tmax[h] = fmaxf(fmaxf(rm[h], rm[16 + h]), fmaxf(rm[32 + h], rm[48 + h]));
+      bool need = false;
+#pragma unroll
+      for (int h = 0; h < kGp; ++h)
+        need |= (m_run[h] != -INFINITY) && (tmax[h] > m_run[h] + kRescaleLog2);
+      if (need) {
+        if (i > 0) {
+          const uint32_t cp = c - 1;
+          ok = sy.wait_warp(G_PEMPTY + (cp & 1u), (cp >> 1) & 1u);
+          if (!ok) break;
+        }
+        tc_fence_after();
+        float alpha[kGp];
+#pragma unroll
+        for (int h = 0; h < kGp; ++h) {
+          const float mn = fmaxf(m_run[h], tmax[h]);
+          alpha[h] = m_run[h] == -INFINITY ? 1.f : ex2(m_run[h] - mn);
+          m_run[h] = mn;
+          l_part[h] *= alpha[h];
+        }
+        if (i > 0) {
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) {          // O_hi, O_lo x two halves
+            uint32_t o[16];
+            tmem_ld16(tl + kTO + q4 * 16, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int h = 0; h < kGp; ++h) o[h] = __float_as_uint(__uint_as_float(o[h]) * alpha[h]);
+            tmem_st16(tl + kTO + q4 * 16, o);
+          }
+          tmem_wait_st();
+        }
+      } else {
+#pragma unroll
+        for (int h = 0; h < kGp; ++h)
+          if (m_run[h] == -INFINITY) m_run[h] = tmax[h];
+      }
+      // p = p_hi + p_lo / 16, both E4M3 (p <= 2^8)
+      uint32_t ph[4], plo[4];
+#pragma unroll
+      for (int h4 = 0; h4 < 4; ++h4) {
+        float pv[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int h = 4 * h4 + j;
+          pv[j] = ex2(s[h] - (m_run[h] == -INFINITY ? 0.f : m_run[h]));
+          l_part[h] += pv[j];
+        }
+        const uint32_t h01 = pack_e4m3x2(pv[0], pv[1]), h23 = pack_e4m3x2(pv[2], pv[3]);
+        float y0, y1, y2, y3;
+        f16x2_to_f32(e4m3x2_to_f16x2(h01), y0, y1);
+        f16x2_to_f32(e4m3x2_to_f16x2(h23), y2, y3);
+        const uint32_t l01 = pack_e4m3x2((pv[0] - y0) * 16.f, (pv[1] - y1) * 16.f);
+        const uint32_t l23 = pack_e4m3x2((pv[2] - y2) * 16.f, (pv[3] - y3) * 16.f);
+        ph[h4] = h01 | (h23 << 16);
+        plo[h4] = l01 | (l23 << 16);
+      }
+      ok = sy.wait_warp(G_PEMPTY + buf, ((c >> 1) & 1u) ^ 1u);
+      if (!ok) break;
+      // P^T row of this key: 16 heads = 16 bytes, key k at 16 k
+      const uint32_t pa = sb + F_P8 + buf * 2 * kP8Bytes + key * 16;
+      st_shared_v4(pa, ph[0], ph[1], ph[2], ph[3]);
+      st_shared_v4(pa + kP8Bytes, plo[0], plo[1], plo[2], plo[3]);
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(sy.bar(G_PFULL + buf));
+    }
+    if (!ok) break;
+    const float wsum = xreduce16<false>(l_part, lane);
+    float* rs = red_sum + (c_unit & 1u) * 64;
+    if ((lane & 1) == 0) rs[wq * 16 + ((lane >> 1) & 15)] = wsum;
+    __syncwarp();
+    if (lane == 0) mbar_arrive(sy.bar(G_RSUM + (c_unit & 1u)));
+    ok = sy.wait_warp(G_RSUM + (c_unit & 1u), (c_unit >> 1) & 1u);
+    if (!ok) break;
+    float l_tot[kGp];
+#pragma unroll
+    for (int h = 0; h < kGp; ++h) l_tot[h] = (rs[h] + rs[16 + h]) + (rs[32 + h] + rs[48 + h]);
+    ok = sy.wait_warp(G_OFULL, c_unit & 1u);
+    if (!ok) break;
+    tc_fence_after();
+    uint32_t oh0[16] = {}, oh1[16] = {}, ol0[16] = {}, ol1[16] = {};
+    if (un.n_tiles > 0) {
+      tmem_ld16(tl + kTO, oh0);
+      tmem_ld16(tl + kTO + 16, oh1);
+      tmem_ld16(tl + kTO + 32, ol0);
+      tmem_ld16(tl + kTO + 48, ol1);
+      tmem_wait_ld();
+    }
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(sy.bar(G_OEMPTY));
+    __nv_bfloat16* orow = p.out + un.t * p.o_st + static_cast<int64_t>(un.g) * G * p.o_sh;
+#pragma unroll
+    for (int h = 0; h < kGp; ++h) {
+      if (h < G) {
+        const bool live = l_tot[h] > 0.f;
+        const float inv = live ? p.o_scale / l_tot[h] : 0.f;
+        const float v0 = live ? fmaf(__uint_as_float(ol0[h]), 0.0625f, __uint_as_float(oh0[h])) * inv : 0.f;
+        const float v1 = live ? fmaf(__uint_as_float(ol1[h]), 0.0625f, __uint_as_float(oh1[h])) * inv : 0.f;
+        orow[h * p.o_sh + key] = __float2bfloat16_rn(v0);
+        orow[h * p.o_sh + 128 + key] = __float2bfloat16_rn(v1);
+      }
+    }
+    if (key < G && p.lse != nullptr) {
+      float mk = 0.f, lk = 0.f;
+#pragma unroll
+      for (int h = 0; h < kGp; ++h)
+        if (h == key) {
+          mk = m_run[h];
+          lk = l_tot[h];
+        }
+      p.lse[un.t * p.lse_st + static_cast<int64_t>(un.g) * G + key] =
+          lk > 0.f ? (mk + lg2(lk)) * 0.69314718055994531f : -INFINITY;
+    }
+    c_tile += un.n_tiles;
+    ++c_unit;
+  }
+}
+
+// ------------------------------------------------------------------ kernel
+
+template <bool kBlocks>
+__global__ void __launch_bounds__(kThreads, 1) qsa_prefill_f8_kernel(const __grid_constant__ TcParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t sb = (raw + 1023u) & ~1023u;
+  uint8_t* sp = smem_raw + (sb - raw);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  Sync sy;
+  sy.bars = sb + F_BAR;
+  sy.abort_flag = reinterpret_cast<volatile uint32_t*>(sp + F_MISC + 4);
+  sy.status = p.status;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kSlots8; ++s) {
+      mbar_init(sy.bar(G_FULL + s), 32 * kProducerWarps);
+      mbar_init(sy.bar(G_EMPTY + s), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(sy.bar(G_SFULL + b), 1);
+      mbar_init(sy.bar(G_SFREE + b), 4);
+      mbar_init(sy.bar(G_PFULL + b), 4);
+      mbar_init(sy.bar(G_PEMPTY + b), 1);
+      mbar_init(sy.bar(G_QFULL + b), 1);
+      mbar_init(sy.bar(G_QEMPTY + b), 1);
+      mbar_init(sy.bar(G_RMAX + b), 4);
+      mbar_init(sy.bar(G_RSUM + b), 4);
+    }
+    mbar_init(sy.bar(G_OFULL), 1);
+    mbar_init(sy.bar(G_OEMPTY), 4);
+    mbar_init(sy.bar(G_DONE), 1);
+    mbar_init(sy.bar(G_DONE + 1), 1);
+    *sy.abort_flag = 0u;
+    mbar_fence_init();
+  }
+  if (warp == kWarpQK) {
+    tmem_alloc(sb + F_MISC, kTmemCols8);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(sp + F_MISC);
+
+  if (warp < kProducerWarps) {
+    producer8<kBlocks>(p, sy, sb, warp, lane);
+  } else if (warp == kWarpQK) {
+    qk8(p, sy, sb, sp, tmem, lane);
+  } else if (warp == kWarpPV) {
+    if (lane == 0) pv8(p, sy, sb, tmem);
+    __syncwarp();
+  } else {
+    softmax8<kBlocks>(p, sy, sb, sp, tmem, warp, lane);
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == kWarpQK) tmem_dealloc(tmem, kTmemCols8);
+}
+
+}  // namespace f8
+}  // namespace qsa

@@ -106,8 +106,11 @@ struct TcParams {
   int32_t block_shift;
   const int32_t* last_slot;
   // output scale applied with the 1/l normalisation (the V dequantisation
-  // scale of an FP8 cache; 1 otherwise)
+  // scale of an FP8 cache, in the FP8 kernel; 1 otherwise)
   float o_scale;
+  // Q in global memory (the FP8 kernel reads it directly; strides in elements)
+  const void* q_ptr;
+  int64_t q_st, q_sh;
 };
 
 // Instruction descriptors (kind::f16): FP32 accumulator, BF16 A and B,
@@ -115,11 +118,6 @@ struct TcParams {
 constexpr uint32_t kIdescQK = (1u << 4) | (1u << 7) | (1u << 10) | (2u << 17) | (8u << 24);
 // PV: both operands MN-major (bits 15 and 16).
 constexpr uint32_t kIdescPV = kIdescQK | (1u << 15) | (1u << 16);
-// The same with FP16 A and B (format fields 0): the FP8-cache variant, whose
-// K, V, Q and P tiles are FP16 in shared memory.
-constexpr uint32_t kIdescQK16 = (1u << 4) | (2u << 17) | (8u << 24);
-constexpr uint32_t kIdescPV16 = kIdescQK16 | (1u << 15) | (1u << 16);
-constexpr uint32_t kStatusQRange = 4u;   // a Q element outside the FP16 range (FP8 variant)
 
 
 struct Unit {
@@ -226,41 +224,7 @@ __device__ __forceinline__ float xreduce16(const float (&v)[16], int lane) {
 // the slot's full barrier when its own copies land (cp.async.mbarrier.arrive).
 // kStall (test hook): withhold the completion signal of the first ring slot,
 // so that every wait must expire and the kernel must stop with kStatusTimeout.
-// FP8 cache: the raw E4M3 half rows of a slot (128 rows x 128 B) sit in the
-// slot's upper 16 KB, row-major.  Lane l of producer warp pw converts row
-// 32*pw + l: it reads its 128 raw bytes first (the FP16 row's second 64-dim
-// block overwrites exactly those bytes), then writes the 128 FP16 values
-// into the 128-byte-swizzled K-major layout the BF16 path uses.
-__device__ __forceinline__ void convert_fp8_rows(uint32_t slot_base, int r) {
-  const uint32_t raw = slot_base + kBlockBytes + r * 128;
-  // step i handles raw chunk (i + r) & 7: the lanes of a warp (consecutive
-  // rows 128 B apart) then read different banks
-  uint32_t w[8][4];
-#pragma unroll
-  for (int i = 0; i < 8; ++i)
-    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];\n"
-                 : "=r"(w[i][0]), "=r"(w[i][1]), "=r"(w[i][2]), "=r"(w[i][3])
-                 : "r"(raw + ((i + r) & 7) * 16));
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    // raw chunk c = dims 16c .. 16c+15 -> FP16 chunks 2c and 2c+1 (8 dims each)
-    const int c = (i + r) & 7;
-    uint32_t h[8];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      h[2 * j] = e4m3x2_to_f16x2(w[i][j]);
-      h[2 * j + 1] = e4m3x2_to_f16x2(w[i][j] >> 16);
-    }
-#pragma unroll
-    for (int half = 0; half < 2; ++half) {
-      const int cc = 2 * c + half;
-      const uint32_t dst = slot_base + (cc >> 3) * kBlockBytes + r * 128 + (((cc & 7) ^ (r & 7)) << 4);
-      st_shared_v4(dst, h[4 * half], h[4 * half + 1], h[4 * half + 2], h[4 * half + 3]);
-    }
-  }
-}
-
-template <bool kDump, bool kStall, bool kBlocks, bool kFp8>
+template <bool kDump, bool kStall, bool kBlocks>
 __device__ void producer_role(const TcParams& p, const Sync& sy, uint32_t sb, int pw, int lane) {
   uint32_t c_slot = 0, c_unit = 0;
   const int64_t units = num_units(p);
@@ -291,19 +255,14 @@ __device__ void producer_role(const TcParams& p, const Sync& sy, uint32_t sb, in
     if (!ok) break;
     const int32_t* list = p.idx + un.t * p.idx_st + static_cast<int64_t>(un.g) * p.idx_sh;
     const int32_t last = kBlocks ? last_visible(p, un.t) : 0x7fffffff;
-    constexpr int kElem = kFp8 ? 1 : 2;                // bytes per cache element
-    // BF16: lane = (row of the pair, 16-byte chunk of the 256-byte half row);
-    // FP8: lane = (row of the quad, 16-byte chunk of the 128-byte half row)
-    const int lchunk = kFp8 ? (lane & 7) : cc;
-    const char* kbase = reinterpret_cast<const char*>(p.kraw) + static_cast<int64_t>(un.g) * p.kv_sh * kElem + lchunk * 16;
-    const char* vbase = reinterpret_cast<const char*>(p.vraw) + static_cast<int64_t>(un.g) * p.kv_sh * kElem + lchunk * 16;
-    const int64_t row_bytes = p.kv_ss * kElem;
+    const char* kbase = reinterpret_cast<const char*>(p.kraw) + static_cast<int64_t>(un.g) * p.kv_sh * 2 + cc * 16;
+    const char* vbase = reinterpret_cast<const char*>(p.vraw) + static_cast<int64_t>(un.g) * p.kv_sh * 2 + cc * 16;
+    const int64_t row_bytes = p.kv_ss * 2;
     // list entry of this lane's row (rows_w rows per warp; lanes >= rows_w idle), one tile ahead
     constexpr int rows_w = kKeys / kProducerWarps;
     const int jr = rows_w * pw + lane;
     const bool own = lane < rows_w;
     int32_t entry_next = own ? key_entry<kBlocks>(p, list, un, jr) : -1;
-    const uint32_t c_first = c_slot;   // FP8: slots of this unit are converted one step late
     for (int i = 0; i < un.n_tiles && ok; ++i) {
       int32_t id = key_slot<kBlocks>(p, un, i * kKeys + jr, entry_next, last);
       entry_next = (own && i + 1 < un.n_tiles) ? key_entry<kBlocks>(p, list, un, (i + 1) * kKeys + jr) : -1;
@@ -321,56 +280,18 @@ __device__ void producer_role(const TcParams& p, const Sync& sy, uint32_t sb, in
         const uint32_t round = c_slot / kSlots;
         ok = sy.wait_warp(B_EMPTY + slot, (round & 1u) ^ 1u);
         if (!ok) break;
-        if constexpr (kFp8) {
-          // raw E4M3 half rows into the slot's upper half; 4 rows per copy
-          const char* src0 = (h < 2 ? kbase : vbase) + (h & 1) * 128;
-          const uint32_t dst0 = sb + OFF_RING + slot * kSlotBytes + kBlockBytes + (lane & 7) * 16;
-          const int rq = lane >> 3;
+        const char* src0 = (h < 2 ? kbase : vbase) + (h & 1) * 256;
+        const uint32_t dst0 = sb + OFF_RING + slot * kSlotBytes + dchunk;
 #pragma unroll
-          for (int k = 0; k < rows_w / 4; ++k) {
-            const int r = rows_w * pw + 4 * k + rq;
-            const int32_t rid = __shfl_sync(0xffffffffu, id, 4 * k + rq);
-            const bool live = rid >= 0;
-            const char* src = live ? src0 + static_cast<int64_t>(rid) * row_bytes : src0;
-            cp_async_16(dst0 + r * 128, src, live ? 16 : 0);
-          }
-          cp_async_commit();
-          // the previous slot's raw rows have landed: convert them and signal it
-          if (c_slot > c_first) {
-            cp_async_wait<1>();
-            __syncwarp();
-            const uint32_t ps = (c_slot - 1) % kSlots;
-            convert_fp8_rows(sb + OFF_RING + ps * kSlotBytes, rows_w * pw + lane);
-            fence_proxy_async_smem();
-            __syncwarp();
-            mbar_arrive(sy.bar(B_FULL + ps));
-          }
-        } else {
-          const char* src0 = (h < 2 ? kbase : vbase) + (h & 1) * 256;
-          const uint32_t dst0 = sb + OFF_RING + slot * kSlotBytes + dchunk;
-#pragma unroll
-          for (int k = 0; k < rows_w / 2; ++k) {
-            const int r = rows_w * pw + 2 * k + rsel;               // row of the tile
-            const int32_t rid = __shfl_sync(0xffffffffu, id, 2 * k + rsel);
-            const bool live = rid >= 0;
-            const char* src = live ? src0 + static_cast<int64_t>(rid) * row_bytes : src0;
-            cp_async_16(dst0 + r * 128 + (((cc & 7) ^ (r & 7)) << 4), src, live ? 16 : 0);
-          }
-          if (!(kStall && c_slot == 0)) cp_async_mbar_arrive(sy.bar(B_FULL + slot));
+        for (int k = 0; k < rows_w / 2; ++k) {
+          const int r = rows_w * pw + 2 * k + rsel;               // row of the tile
+          const int32_t rid = __shfl_sync(0xffffffffu, id, 2 * k + rsel);
+          const bool live = rid >= 0;
+          const char* src = live ? src0 + static_cast<int64_t>(rid) * row_bytes : src0;
+          cp_async_16(dst0 + r * 128 + (((cc & 7) ^ (r & 7)) << 4), src, live ? 16 : 0);
         }
+        if (!(kStall && c_slot == 0)) cp_async_mbar_arrive(sy.bar(B_FULL + slot));
         ++c_slot;
-      }
-    }
-    if constexpr (kFp8) {
-      // the unit's last slot: its raw rows land, are converted and signalled
-      if (ok && c_slot > c_first) {
-        cp_async_wait<0>();
-        __syncwarp();
-        const uint32_t ps = (c_slot - 1) % kSlots;
-        convert_fp8_rows(sb + OFF_RING + ps * kSlotBytes, rows_w * pw + lane);
-        fence_proxy_async_smem();
-        __syncwarp();
-        mbar_arrive(sy.bar(B_FULL + ps));
       }
     }
   }
@@ -383,34 +304,8 @@ __device__ void producer_role(const TcParams& p, const Sync& sy, uint32_t sb, in
 
 // ------------------------------------------------------------------ MMA issuers
 
-// FP8 variant: the unit's Q tile (BF16, as the TMA wrote it) becomes FP16 in
-// place, one 16-byte chunk per lane and step; elements beyond the FP16 range
-// raise status bit 2.
-__device__ __forceinline__ void q_to_f16(uint32_t qaddr, int lane, int32_t* status) {
-  bool bad = false;
-#pragma unroll 4
-  for (int i = 0; i < kQBytes / (16 * 32); ++i) {
-    const uint32_t a = qaddr + (i * 32 + lane) * 16;
-    uint32_t w[4], o[4];
-    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];\n"
-                 : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3])
-                 : "r"(a));
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const float lo = __uint_as_float(w[j] << 16), hi = __uint_as_float(w[j] & 0xffff0000u);
-      bad |= fabsf(lo) > 65504.f || fabsf(hi) > 65504.f;
-      o[j] = pack_f16x2(lo, hi);
-    }
-    st_shared_v4(a, o[0], o[1], o[2], o[3]);
-  }
-  if (__any_sync(0xffffffffu, bad) && lane == 0 && status != nullptr)
-    atomicOr(status, static_cast<int32_t>(kStatusQRange));
-}
-
-// Scores: S^T[c & 1] = K_tile(c) . Q^T for every tile c of the CTA.  One
-// thread issues; in the FP8 variant the whole warp first converts Q.
-template <bool kFp8>
-__device__ void qk_role(const TcParams& p, const Sync& sy, uint32_t sb, uint32_t tmem, int lane) {
+// Scores: S^T[c & 1] = K_tile(c) . Q^T for every tile c of the CTA.
+__device__ void qk_role(const TcParams& p, const Sync& sy, uint32_t sb, uint32_t tmem) {
   uint32_t c_tile = 0, c_unit = 0;
   const int64_t units = num_units(p);
   bool ok = true;
@@ -420,19 +315,11 @@ __device__ void qk_role(const TcParams& p, const Sync& sy, uint32_t sb, uint32_t
     ok = sy.wait(B_QFULL + qb, (c_unit >> 1) & 1u);
     if (!ok) break;
     ++c_unit;
-    const uint32_t qaddr = sb + OFF_Q + qb * kQBytes;
-    if constexpr (kFp8) {
-      if (un.n_tiles > 0) {
-        q_to_f16(qaddr, lane, p.status);
-        fence_proxy_async_smem();
-        __syncwarp();
-      }
-    }
-    if (lane != 0) continue;
     if (un.n_tiles == 0) {
       mbar_arrive(sy.bar(B_QEMPTY + qb));
       continue;
     }
+    const uint32_t qaddr = sb + OFF_Q + qb * kQBytes;
     for (int i = 0; i < un.n_tiles && ok; ++i, ++c_tile) {
       const uint32_t c = c_tile;
       const uint32_t sbuf = c & 1u;
@@ -451,7 +338,7 @@ __device__ void qk_role(const TcParams& p, const Sync& sy, uint32_t sb, uint32_t
           const uint64_t a = smem_desc(
               sb + OFF_RING + slot * kSlotBytes + (kk >> 2) * kBlockBytes + (kk & 3) * 32, 16, 1024, 2);
           const uint64_t b = smem_desc(qaddr + (ks >> 2) * (kQBytes / 4) + (ks & 3) * 32, 16, 1024, 2);
-          umma_f16_ss(tmem + sbuf * 16, a, b, kFp8 ? kIdescQK16 : kIdescQK, ks > 0 ? 1u : 0u);
+          umma_f16_ss(tmem + sbuf * 16, a, b, kIdescQK, ks > 0 ? 1u : 0u);
         }
         umma_commit(sy.bar(B_EMPTY + slot));
       }
@@ -460,15 +347,12 @@ __device__ void qk_role(const TcParams& p, const Sync& sy, uint32_t sb, uint32_t
       if (i == un.n_tiles - 1) umma_commit(sy.bar(B_QEMPTY + qb));
     }
   }
-  if (lane == 0) {
-    // no tensor-core operation of this thread may still run when TMEM is released
-    umma_commit(sy.bar(B_DONE));
-    sy.drain(B_DONE, 0);
-  }
+  // no tensor-core operation of this thread may still run when TMEM is released
+  umma_commit(sy.bar(B_DONE));
+  sy.drain(B_DONE, 0);
 }
 
 // PV: O^T (two M=128 halves) += V_tile(c)^T . P^T(c) for every tile c.
-template <bool kFp8>
 __device__ void pv_role(const TcParams& p, const Sync& sy, uint32_t sb, uint32_t tmem) {
   uint32_t c_tile = 0, c_unit = 0;
   const int64_t units = num_units(p);
@@ -502,7 +386,7 @@ __device__ void pv_role(const TcParams& p, const Sync& sy, uint32_t sb, uint32_t
           // B = P^T: MN-major, no swizzle; 8x8 core matrices, key groups 128 B
           // apart (LBO), head groups 2 KB apart (SBO).
           const uint64_t b = smem_desc(sb + OFF_P + pb * kPBytes + kk * 256, 128, 2048, 0);
-          umma_f16_ss(t_o + mh * 16, a, b, kFp8 ? kIdescPV16 : kIdescPV, (i == 0 && kk == 0) ? 0u : 1u);
+          umma_f16_ss(t_o + mh * 16, a, b, kIdescPV, (i == 0 && kk == 0) ? 0u : 1u);
         }
         umma_commit(sy.bar(B_EMPTY + slot));
       }
@@ -517,7 +401,7 @@ __device__ void pv_role(const TcParams& p, const Sync& sy, uint32_t sb, uint32_t
 
 // ------------------------------------------------------------------ softmax
 
-template <bool kBlocks, bool kFp8>
+template <bool kBlocks>
 __device__ void softmax_role(const TcParams& p, const Sync& sy, uint32_t sb, uint8_t* sp,
                              uint32_t tmem, int warp, int lane) {
   const int wq = warp & 3;                       // TMEM lane quadrant of this warp
@@ -616,7 +500,7 @@ __device__ void softmax_role(const TcParams& p, const Sync& sy, uint32_t sb, uin
         const float p1 = ex2(s[h + 1] - (m_run[h + 1] == -INFINITY ? 0.f : m_run[h + 1]));
         l_part[h] += p0;
         l_part[h + 1] += p1;
-        pk[h >> 1] = kFp8 ? pack_f16x2(p0, p1) : pack_bf16x2(p0, p1);
+        pk[h >> 1] = pack_bf16x2(p0, p1);
       }
       ok = sy.wait_warp(B_PEMPTY + buf, ((c >> 1) & 1u) ^ 1u);
       if (!ok) break;
@@ -660,7 +544,7 @@ __device__ void softmax_role(const TcParams& p, const Sync& sy, uint32_t sb, uin
     for (int h = 0; h < kGp; ++h) {
       if (h < G) {
         const bool live = l_tot[h] > 0.f;
-        const float inv = live ? p.o_scale / l_tot[h] : 0.f;
+        const float inv = live ? 1.f / l_tot[h] : 0.f;
         const float v0 = live ? __uint_as_float(o0[h]) * inv : 0.f;
         const float v1 = live ? __uint_as_float(o1[h]) * inv : 0.f;
         if (p.part_o != nullptr) {
@@ -694,7 +578,7 @@ __device__ void softmax_role(const TcParams& p, const Sync& sy, uint32_t sb, uin
 
 // ------------------------------------------------------------------ kernel
 
-template <bool kDump, bool kStall = false, bool kBlocks = false, bool kFp8 = false>
+template <bool kDump, bool kStall = false, bool kBlocks = false>
 __global__ void __launch_bounds__(kThreads, 1) qsa_prefill_tc_kernel(const __grid_constant__ TcParams p) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -741,18 +625,15 @@ __global__ void __launch_bounds__(kThreads, 1) qsa_prefill_tc_kernel(const __gri
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(sp + OFF_MISC);
 
   if (warp < kProducerWarps) {
-    producer_role<kDump, kStall, kBlocks, kFp8>(p, sy, sb, warp, lane);
+    producer_role<kDump, kStall, kBlocks>(p, sy, sb, warp, lane);
   } else if (warp == kWarpQK) {
-    if (kFp8)
-      qk_role<true>(p, sy, sb, tmem, lane);
-    else if (lane == 0)
-      qk_role<false>(p, sy, sb, tmem, 0);
+    if (lane == 0) qk_role(p, sy, sb, tmem);
     __syncwarp();
   } else if (warp == kWarpPV) {
-    if (lane == 0) pv_role<kFp8>(p, sy, sb, tmem);
+    if (lane == 0) pv_role(p, sy, sb, tmem);
     __syncwarp();
   } else {
-    softmax_role<kBlocks, kFp8>(p, sy, sb, sp, tmem, warp, lane);
+    softmax_role<kBlocks>(p, sy, sb, sp, tmem, warp, lane);
   }
 
   tc_fence_before();

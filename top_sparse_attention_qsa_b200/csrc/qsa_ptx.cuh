@@ -114,6 +114,21 @@ __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two_bytes) {
   return r;
 }
 
+// Two FP32 values -> two OCP FP8 E4M3 bytes (round to nearest even,
+// saturating to +-448), lo in bits 0-7.
+__device__ __forceinline__ uint32_t pack_e4m3x2(float lo, float hi) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;\n" : "=h"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// FP16x2 -> the two FP32 values (lo = bits 0-15).
+__device__ __forceinline__ void f16x2_to_f32(uint32_t v, float& lo, float& hi) {
+  asm("{\n\t.reg .f16 a, b;\n\tmov.b32 {a, b}, %2;\n\tcvt.f32.f16 %0, a;\n\tcvt.f32.f16 %1, b;\n\t}\n"
+      : "=f"(lo), "=f"(hi)
+      : "r"(v));
+}
+
 __device__ __forceinline__ int ld_nc_s32(const int32_t* p) {
   int v;
   asm volatile("ld.global.nc.L1::no_allocate.s32 %0, [%1];\n" : "=r"(v) : "l"(p));
