@@ -79,6 +79,9 @@ def parse_args():
                     help="override the query-token count of c4/c5 (smaller ncu captures)")
     ap.add_argument("--profile", action="store_true",
                     help="minimal run for ncu: no clocks, e2e, cpu baseline or secondary")
+    ap.add_argument("--only", default="", choices=["", "fp8", "indexer", "blocks", "decode"],
+                    help="run one secondary leg alone (--steps / --warmup / --tokens apply), for "
+                         "profiling; prints that leg's JSON")
     return ap.parse_args()
 
 
@@ -143,10 +146,10 @@ def workload_accounting(w):
     return dict(entries=entries, gathered_bytes=gathered, algo_bytes=algo, flops=flops)
 
 
-# Sources the sparse-prefill kernels compile from (the launch code in
-# qsa_api.cu included); the indexer's file is not among them.
-PREFILL_SOURCES = ("qsa_api.cu", "qsa_host.cuh", "qsa_prefill_tc.cuh", "qsa_prefill_mma.cuh", "qsa_tc_ptx.cuh",
-                   "qsa_ptx.cuh", "qsa_merge.cuh")
+# Device sources of the default sparse-prefill kernel (qsa_prefill_tc_kernel);
+# its launch shape (persistent grid of min(units, SMs) CTAs of 320 threads)
+# is fixed in qsa_api.cu.
+PREFILL_SOURCES = ("qsa_prefill_tc.cuh", "qsa_tc_ptx.cuh", "qsa_ptx.cuh")
 
 
 def kernel_source_hash(files=PREFILL_SOURCES):
@@ -298,6 +301,11 @@ def time_oracle(w, budget_s, min_tokens=1):
                        f"{dt:.1f} s on {cores} threads")
 
 
+def W_make(name, device, **kw):
+    from top_sparse_attention_qsa_b200 import workloads as W
+    return W.make(name, device=device, **kw)
+
+
 def make_workload(name, device):
     from top_sparse_attention_qsa_b200 import workloads as W
     return W.make(name, device=device)
@@ -385,6 +393,24 @@ def run_cuda(args):
 
     from top_sparse_attention_qsa_b200 import _capi
     from top_sparse_attention_qsa_b200 import workloads as W
+
+    if args.only:
+        hbm, bf16, _ = measured_peaks()
+        kw = {"T": args.tokens} if args.tokens else {}
+        leg = {"fp8": lambda: run_fp8_bench("c5", dev, barrier, max_ranks, world, hbm, args.steps,
+                                            args.warmup, **kw),
+               "indexer": lambda: run_indexer_bench(dev, barrier, max_ranks, world, hbm, bf16, args.steps,
+                                                    args.warmup, **kw),
+               "blocks": lambda: run_blocks_bench("c5_block4", dev, barrier, max_ranks, world, hbm,
+                                                  args.steps, args.warmup, **kw),
+               "decode": lambda: run_decode_bench("decode", dev, barrier, max_ranks, world, hbm, args.steps,
+                                                  args.warmup)}[args.only]()
+        if rank == 0:
+            print(json.dumps({"leg": args.only, **leg}), flush=True)
+        if pg is not None:
+            pg.barrier()
+            pg.destroy_process_group()
+        return 0
 
     # weak scaling (default): every rank runs its own replica (own seed);
     # strong scaling (--shard tokens): the ranks split one workload's tokens
@@ -528,7 +554,7 @@ def run_secondary(name, dev, barrier, reduce_max, world, hbm, bf16, kernel="auto
             "frac_of_roofline_time": roof_ms / ms, "steps": steps}
 
 
-def run_decode_bench(name, dev, barrier, reduce_max, world, hbm):
+def run_decode_bench(name, dev, barrier, reduce_max, world, hbm, steps=50, warmup=5):
     """Split-K decode (one query token per sequence): two launches per step
     (chunk kernel + merge), workspace allocated once outside the timed loop."""
     from top_sparse_attention_qsa_b200 import _capi
@@ -544,23 +570,37 @@ def run_decode_bench(name, dev, barrier, reduce_max, world, hbm):
         _capi.sparse_decode_fwd(w.q, w.k_cache, w.v_cache, w.topk_idx, w.n_valid, w.scale,
                                 num_splits=0, workspace=ws, out=out, lse=lse)
 
-    steps = 50
-    total_ms, per_ms, _ = time_launches(step, steps, 5, barrier, "decode")
+    total_ms, per_ms, _ = time_launches(step, steps, warmup, barrier, "decode")
     total_ms = reduce_max(total_ms)
     ms = statistics.mean(per_ms)
     algo = acct["algo_bytes"] + need  # partial results are written once and read once by the merge
+    # the same decode over an FP8 E4M3 cache (k_scale 0.5, v_scale 2)
+    from top_sparse_attention_qsa_b200 import workloads as W
+    gen = torch.Generator(device=dev).manual_seed(78)
+    k8 = W.normal_fp8(tuple(w.k_cache.shape), gen, dev)
+    v8 = W.normal_fp8(tuple(w.v_cache.shape), gen, dev)
+
+    def step8():
+        _capi.sparse_decode_fp8_fwd(w.q, k8, v8, w.topk_idx, 0.5, 2.0, n_valid=w.n_valid, scale=w.scale,
+                                    num_splits=0, workspace=ws, out=out, lse=lse)
+
+    _, per8, _ = time_launches(step8, steps, warmup, barrier, "decode_fp8")
+    ms8 = statistics.mean(per8)
+    algo8 = acct["algo_bytes"] - acct["gathered_bytes"] // 2 + need
     return {"workload": w.name, "desc": w.description, "splits": splits,
             "workspace_bytes": need, "tokens_per_s": w.shape["T"] * steps * world / (total_ms / 1e3),
             "mean_step_ms": ms, "gathered_kv_gbs": acct["gathered_bytes"] / (ms / 1e3) / 1e9,
             "algo_gbs": algo / (ms / 1e3) / 1e9, "frac_of_hbm": algo / (ms / 1e3) / 1e9 / hbm,
-            "launches_per_step": 2 if need > 0 else 1, "steps": steps}
+            "launches_per_step": 2 if need > 0 else 1, "steps": steps,
+            "fp8": {"mean_step_ms": ms8, "tokens_per_s": w.shape["T"] * world / (ms8 / 1e3),
+                    "algo_gbs": algo8 / (ms8 / 1e3) / 1e9, "frac_of_hbm": algo8 / (ms8 / 1e3) / 1e9 / hbm}}
 
 
-def run_blocks_bench(name, dev, barrier, reduce_max, world, hbm):
+def run_blocks_bench(name, dev, barrier, reduce_max, world, hbm, steps=20, warmup=3, **kw):
     """Microblock lists on the c5 shape: the same 2048 keys per (token, KV
     head) as c5, named by 512 blocks of 4 slots."""
     from top_sparse_attention_qsa_b200 import _capi
-    w = make_workload(name, dev)
+    w = W_make(name, dev, **kw)
     out = torch.empty_like(w.q)
     lse = torch.empty(w.q.shape[:2], dtype=torch.float32, device=dev)
     bs = w.block_size
@@ -578,8 +618,7 @@ def run_blocks_bench(name, dev, barrier, reduce_max, world, hbm):
         _capi.sparse_prefill_block_fwd(w.q, w.k_cache, w.v_cache, w.topk_idx, bs, w.last_slot,
                                        w.n_valid, w.scale, out=out, lse=lse)
 
-    steps = 20
-    total_ms, per_ms, _ = time_launches(step, steps, 3, barrier, "blocks")
+    total_ms, per_ms, _ = time_launches(step, steps, warmup, barrier, "blocks")
     total_ms = reduce_max(total_ms)
     ms = statistics.mean(per_ms)
     return {"workload": w.name, "desc": w.description, "tokens_per_s": s["T"] * steps * world / (total_ms / 1e3),
@@ -588,12 +627,12 @@ def run_blocks_bench(name, dev, barrier, reduce_max, world, hbm):
             "steps": steps}
 
 
-def run_fp8_bench(name, dev, barrier, reduce_max, world, hbm):
+def run_fp8_bench(name, dev, barrier, reduce_max, world, hbm, steps=20, warmup=3, **kw):
     """The same lists and Q as `name`, with the K and V caches stored as FP8
     E4M3 (k_scale 0.5, v_scale 2): half the gathered bytes per key."""
     from top_sparse_attention_qsa_b200 import _capi
     from top_sparse_attention_qsa_b200 import workloads as W
-    w = make_workload(name, dev)
+    w = W_make(name, dev, **kw)
     entries = workload_accounting(w)["entries"]
     gen = torch.Generator(device=dev).manual_seed(77)
     k8 = W.normal_fp8(tuple(w.k_cache.shape), gen, dev)
@@ -609,8 +648,7 @@ def run_fp8_bench(name, dev, barrier, reduce_max, world, hbm):
         _capi.sparse_prefill_fp8_fwd(w.q, k8, v8, w.topk_idx, 0.5, 2.0, n_valid=w.n_valid, scale=w.scale,
                                      out=out, lse=lse)
 
-    steps = 20
-    total_ms, per_ms, _ = time_launches(step, steps, 3, barrier, "fp8")
+    total_ms, per_ms, _ = time_launches(step, steps, warmup, barrier, "fp8")
     total_ms = reduce_max(total_ms)
     ms = statistics.mean(per_ms)
     return {"workload": w.name + "_fp8e4m3", "tokens_per_s": T * steps * world / (total_ms / 1e3),
@@ -620,7 +658,7 @@ def run_fp8_bench(name, dev, barrier, reduce_max, world, hbm):
             "steps": steps}
 
 
-def run_indexer_bench(dev, barrier, reduce_max, world, hbm, bf16, **kw):
+def run_indexer_bench(dev, barrier, reduce_max, world, hbm, bf16, steps=20, warmup=3, **kw):
     """Indexer scores (tcgen05) then top-K selection on the c5 size: 8192
     tokens, 32768 block keys, 4 heads x 128, budget 2048 + causal tail.  Each
     kernel is timed on its own (events on the launching stream) and as the
@@ -649,10 +687,9 @@ def run_indexer_bench(dev, barrier, reduce_max, world, hbm, bf16, **kw):
         s_step()
         k_step()
 
-    steps = 20
-    _, s_per, _ = time_launches(s_step, steps, 3, barrier, "indexer_scores")
-    _, k_per, _ = time_launches(k_step, steps, 3, barrier, "topk_select")
-    total_ms, p_per, _ = time_launches(pair, steps, 3, barrier, "indexer_pair")
+    _, s_per, _ = time_launches(s_step, steps, warmup, barrier, "indexer_scores")
+    _, k_per, _ = time_launches(k_step, steps, warmup, barrier, "topk_select")
+    total_ms, p_per, _ = time_launches(pair, steps, warmup, barrier, "indexer_pair")
     total_ms = reduce_max(total_ms)
     s_ms, k_ms = statistics.mean(s_per), statistics.mean(k_per)
     flops = cand * H * Dh * 2

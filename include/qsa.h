@@ -232,6 +232,26 @@ qsa_status_t qsa_sparse_decode_fwd(const qsa_shape_t* shape, const void* q,
                                    int32_t num_splits, void* workspace,
                                    size_t workspace_bytes, void* stream);
 
+/*
+ * Split-K decode over an FP8 E4M3 KV cache: qsa_sparse_decode_fwd's chunking,
+ * workspace and LSE merge, with the chunks computed by the FP8 kernel of
+ * qsa_sparse_prefill_fp8_fwd (element value = stored byte * k_scale /
+ * v_scale; token lists).  The workspace size is what
+ * qsa_sparse_decode_workspace_bytes returns for the same shape and
+ * num_splits.  Cache strides must be multiples of 16 elements (QSA_ERR_ALIGN
+ * otherwise).  The pages measure decode over an fp8_e4m3 KV cache on
+ * NVIDIA hardware (page "Qwen4-Exp QSA llega al Ascend de Huawei", the
+ * observations on the NVIDIA side).
+ */
+qsa_status_t qsa_sparse_decode_fp8_fwd(const qsa_shape_t* shape, const void* q,
+                                       const void* k_cache, const void* v_cache,
+                                       const int32_t* topk_idx,
+                                       const int32_t* n_valid, float scale,
+                                       float k_scale, float v_scale, void* out,
+                                       float* lse, int32_t* status,
+                                       int32_t num_splits, void* workspace,
+                                       size_t workspace_bytes, void* stream);
+
 /* Workspace bytes qsa_sparse_decode_fwd needs for this shape and num_splits
  * (0: no workspace needed, or an invalid shape).  With num_splits <= 0 the
  * answer depends on the current device's SM count. */

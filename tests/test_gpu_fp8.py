@@ -113,3 +113,20 @@ def test_large_and_tiny_queries(C):
     torch.cuda.synchronize()
     ref_out, ref_lse, _ = oracle_fp8(w, k8, v8, 0.5, 2.0)
     compare(host(out), host(lse), ref_out, ref_lse, "fp8 query range")
+
+
+@pytest.mark.parametrize("splits", [0, 1, 4, 16])
+def test_split_k_decode(C, splits):
+    """Decode over an FP8 cache: 16 sequences of 8192 slots, one query token
+    each, 2048-entry lists, cut into chunks merged by their log-sum-exp."""
+    w = W.config_decode(device=DEV, seed=51, B=16, ctx=8192, heads=(24, 2), topk=2048, local=256)
+    gen = torch.Generator(device=DEV).manual_seed(52)
+    k8 = W.normal_fp8(tuple(w.k_cache.shape), gen, DEV, std=2.0)
+    v8 = W.normal_fp8(tuple(w.v_cache.shape), gen, DEV)
+    w.n_valid[3] = 0                              # an empty row
+    w.n_valid[5] = 700                            # a ragged one
+    out, lse = C.sparse_decode_fp8_fwd(w.q, k8, v8, w.topk_idx, 0.5, 2.0, n_valid=w.n_valid,
+                                       scale=w.scale, num_splits=splits)
+    torch.cuda.synchronize()
+    ref_out, ref_lse, _ = oracle_fp8(w, k8, v8, 0.5, 2.0)
+    compare(host(out), host(lse), ref_out, ref_lse, f"fp8 decode splits={splits}")

@@ -35,7 +35,7 @@ EXPORTS = ("qsa_sparse_prefill_fwd", "qsa_sparse_prefill_fwd_with", "qsa_sparse_
            "qsa_sparse_prefill_block_fwd",
            "qsa_sparse_prefill_fwd_host", "qsa_sparse_decode_fwd", "qsa_sparse_decode_workspace_bytes",
            "qsa_sparse_decode_num_splits", "qsa_sparse_decode_fwd_noalloc", "qsa_test_stalled_pipeline",
-           "qsa_sparse_prefill_fp8_fwd", "qsa_indexer_scores", "qsa_topk_select", "qsa_status_string",
+           "qsa_sparse_prefill_fp8_fwd", "qsa_sparse_decode_fp8_fwd", "qsa_indexer_scores", "qsa_topk_select", "qsa_status_string",
            "qsa_abi_version")
 
 
@@ -112,6 +112,9 @@ _lib.qsa_sparse_prefill_block_fwd.argtypes = [ctypes.POINTER(Shape), ctypes.c_in
 _lib.qsa_sparse_prefill_fp8_fwd.argtypes = [ctypes.POINTER(Shape), ctypes.c_int32, _vp, _vp, _vp, _vp, _vp,
                                             _vp, ctypes.c_float, ctypes.c_float, ctypes.c_float, _vp, _vp,
                                             _vp, _vp]
+_lib.qsa_sparse_decode_fp8_fwd.argtypes = [ctypes.POINTER(Shape), _vp, _vp, _vp, _vp, _vp, ctypes.c_float,
+                                           ctypes.c_float, ctypes.c_float, _vp, _vp, _vp, ctypes.c_int32,
+                                           _vp, ctypes.c_size_t, _vp]
 _lib.qsa_indexer_scores.argtypes = [ctypes.POINTER(IndexerShape), _vp, _vp, _vp, _vp, _vp, _vp, _vp]
 _lib.qsa_topk_select.argtypes = [ctypes.POINTER(IndexerShape), _vp, _vp, _vp, ctypes.c_int64, ctypes.c_int32,
                                  _vp, ctypes.c_int64, _vp, ctypes.c_int32, _vp, _vp]
@@ -467,6 +470,45 @@ def sparse_prefill_fp8_fwd(q, k_cache, v_cache, topk_idx, k_scale: float = 1.0, 
                                            _ptr(k_cache), _ptr(v_cache), _ptr(topk_idx), _ptr(n_valid),
                                            float(scale), float(k_scale), float(v_scale), _ptr(out),
                                            _ptr(lse), _ptr(status), stream))
+    return out, lse
+
+
+def sparse_decode_fp8_fwd(q, k_cache, v_cache, topk_idx, k_scale: float = 1.0, v_scale: float = 1.0,
+                          n_valid=None, scale: float = 0.0, num_splits: int = 0, workspace=None, out=None,
+                          lse=None, status=None, stream=None, want_lse: bool = True):
+    """Split-K decode over an FP8 E4M3 cache (torch.float8_e4m3fn).  A
+    workspace of decode_workspace_bytes(...) bytes is allocated when none is
+    given."""
+    dev = q.device
+    _need(q, "q", torch.bfloat16, dev)
+    _need(k_cache, "k_cache", torch.float8_e4m3fn, dev)
+    _need(v_cache, "v_cache", torch.float8_e4m3fn, dev)
+    _need(topk_idx, "topk_idx", torch.int32, dev)
+    _check_kv(k_cache, v_cache)
+    if n_valid is not None:
+        _need(n_valid, "n_valid", torch.int32, dev)
+        if not n_valid.is_contiguous() or tuple(n_valid.shape) != tuple(topk_idx.shape[:2]):
+            raise ValueError("n_valid must be a contiguous [T, Hkv] tensor")
+    if out is None:
+        out = torch.empty(q.shape, dtype=torch.bfloat16, device=dev)
+    _need(out, "out", torch.bfloat16, dev)
+    if lse is None and want_lse:
+        lse = torch.empty(q.shape[:2], dtype=torch.float32, device=dev)
+    if lse is not None:
+        _need(lse, "lse", torch.float32, dev)
+    if status is not None:
+        _need(status, "status", torch.int32, dev)
+    shape = make_shape(q, k_cache, topk_idx, out, lse)
+    need = int(_lib.qsa_sparse_decode_workspace_bytes(ctypes.byref(shape), int(num_splits)))
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    if stream is None:
+        stream = torch.cuda.current_stream(dev).cuda_stream
+    _raise(_lib.qsa_sparse_decode_fp8_fwd(ctypes.byref(shape), _ptr(q), _ptr(k_cache), _ptr(v_cache),
+                                          _ptr(topk_idx), _ptr(n_valid), float(scale), float(k_scale),
+                                          float(v_scale), _ptr(out), _ptr(lse), _ptr(status), int(num_splits),
+                                          _ptr(workspace), ws_bytes, stream))
     return out, lse
 
 

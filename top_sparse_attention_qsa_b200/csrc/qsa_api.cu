@@ -274,18 +274,31 @@ cudaError_t launch_merge(const qsa_shape_t* s, const float* part_o, const float*
 
 // Split-K forward: partial results of every chunk go to `workspace` (laid
 // out by plan_splits), then one merge launch writes out/lse.
+qsa_status_t run_lists(const qsa_shape_t* shape, int32_t block_size, const int32_t* last_slot,
+                       const void* q, const void* k_cache, const void* v_cache,
+                       const int32_t* topk_idx, const int32_t* n_valid, float scale,
+                       float k_scale, float v_scale, bool fp8, void* out, float* lse,
+                       int32_t* status, void* stream);
+
 qsa_status_t run_decode(const qsa_shape_t* s, const void* q, const void* k, const void* v,
                         const int32_t* idx, const int32_t* n_valid, float scale, void* out,
                         float* lse, int32_t* status, int32_t num_splits, void* workspace,
-                        size_t workspace_bytes, void* stream) {
+                        size_t workspace_bytes, void* stream, bool fp8 = false, float k_scale = 1.f,
+                        float v_scale = 1.f) {
   qsa_status_t rc = validate(s, q, k, v, idx, out);
   if (rc != QSA_OK) return rc;
+  if (fp8 && s->topk > 0 && (s->kv_stride_slot % 16 != 0 || s->kv_stride_head % 16 != 0))
+    return QSA_ERR_ALIGN;
   if (s->num_tokens == 0) return QSA_OK;
   SplitPlan pl;
   if (!plan_splits(s, num_splits, &pl)) return QSA_ERR_CUDA;
   static thread_local qsa::tc::TcParams tp;
-  if (pl.splits <= 1 || !make_tc_params(s, q, &tp))
+  if (pl.splits <= 1 || !make_tc_params(s, q, &tp)) {
+    if (fp8)
+      return run_lists(s, 1, nullptr, q, k, v, idx, n_valid, scale, k_scale, v_scale, true, out, lse,
+                       status, stream);
     return run_forward(s, q, k, v, idx, n_valid, scale, out, lse, status, nullptr, stream);
+  }
   if (workspace == nullptr) return QSA_ERR_NULL;
   if (workspace_bytes < pl.total_bytes) return QSA_ERR_SHAPE;
   if (reinterpret_cast<uintptr_t>(workspace) & 255u) return QSA_ERR_ALIGN;
@@ -312,16 +325,19 @@ qsa_status_t run_decode(const qsa_shape_t* s, const void* q, const void* k, cons
   tp.G = s->num_q_heads / s->num_kv_heads;
   tp.K = s->topk;
   tp.S = static_cast<int32_t>(s->num_slots);
-  tp.scale_log2 = sc * 1.4426950408889634f;
+  tp.scale_log2 = sc * (fp8 ? k_scale : 1.f) * 1.4426950408889634f;
   tp.splits = pl.splits;
   tp.chunk = pl.chunk;
   tp.part_o = part_o;
   tp.part_lse = part_lse;
   tp.block_shift = 0;
   tp.last_slot = nullptr;
-  tp.o_scale = 1.f;
+  tp.o_scale = fp8 ? v_scale : 1.f;
+  tp.q_ptr = q;
+  tp.q_st = s->q_stride_tok;
+  tp.q_sh = s->q_stride_head;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (launch_tc<false>(tp, st) != cudaSuccess) return QSA_ERR_CUDA;
+  if ((fp8 ? launch_f8<false>(tp, st) : launch_tc<false>(tp, st)) != cudaSuccess) return QSA_ERR_CUDA;
   if (launch_merge(s, part_o, part_lse, pl.splits, out, lse, st) != cudaSuccess) return QSA_ERR_CUDA;
   return QSA_OK;
 }
@@ -522,6 +538,16 @@ qsa_status_t qsa_sparse_decode_fwd(const qsa_shape_t* shape, const void* q, cons
                                    size_t workspace_bytes, void* stream) {
   return run_decode(shape, q, k_cache, v_cache, topk_idx, n_valid, scale, out, lse, status,
                     num_splits, workspace, workspace_bytes, stream);
+}
+
+qsa_status_t qsa_sparse_decode_fp8_fwd(const qsa_shape_t* shape, const void* q, const void* k_cache,
+                                       const void* v_cache, const int32_t* topk_idx,
+                                       const int32_t* n_valid, float scale, float k_scale,
+                                       float v_scale, void* out, float* lse, int32_t* status,
+                                       int32_t num_splits, void* workspace, size_t workspace_bytes,
+                                       void* stream) {
+  return run_decode(shape, q, k_cache, v_cache, topk_idx, n_valid, scale, out, lse, status, num_splits,
+                    workspace, workspace_bytes, stream, true, k_scale, v_scale);
 }
 
 qsa_status_t qsa_sparse_decode_fwd_noalloc(const qsa_shape_t* shape, const void* q,

@@ -306,6 +306,11 @@ __device__ void softmax8(const TcParams& p, const Sync& sy, uint32_t sb, uint8_t
     float qs[kGp];
 #pragma unroll
     for (int h = 0; h < kGp; ++h) qs[h] = qsc_all[qb * kGp + h];
+    // the score factors are read: the Q buffer may be refilled once the MMAs
+    // are done too (without this release, warp 4 could run two units ahead
+    // through empty units and complete a G_QFULL phase this warp never saw)
+    __syncwarp();
+    if (lane == 0) mbar_arrive(sy.bar(G_QEMPTY + qb));
     float m_run[kGp], l_part[kGp];
 #pragma unroll
     for (int h = 0; h < kGp; ++h) {
@@ -436,6 +441,7 @@ __device__ void softmax8(const TcParams& p, const Sync& sy, uint32_t sb, uint8_t
     tc_fence_before();
     __syncwarp();
     if (lane == 0) mbar_arrive(sy.bar(G_OEMPTY));
+    const int64_t row0 = un.t * static_cast<int64_t>(p.Hkv) * G + static_cast<int64_t>(un.g) * G;
     __nv_bfloat16* orow = p.out + un.t * p.o_st + static_cast<int64_t>(un.g) * G * p.o_sh;
 #pragma unroll
     for (int h = 0; h < kGp; ++h) {
@@ -444,11 +450,18 @@ __device__ void softmax8(const TcParams& p, const Sync& sy, uint32_t sb, uint8_t
         const float inv = live ? p.o_scale / l_tot[h] : 0.f;
         const float v0 = live ? fmaf(__uint_as_float(ol0[h]), 0.0625f, __uint_as_float(oh0[h])) * inv : 0.f;
         const float v1 = live ? fmaf(__uint_as_float(ol1[h]), 0.0625f, __uint_as_float(oh1[h])) * inv : 0.f;
-        orow[h * p.o_sh + key] = __float2bfloat16_rn(v0);
-        orow[h * p.o_sh + 128 + key] = __float2bfloat16_rn(v1);
+        if (p.part_o != nullptr) {
+          // split-K: this chunk's normalised partial output, for the merge
+          float* po = p.part_o + ((row0 + h) * p.splits + un.s) * 256;
+          po[key] = v0;
+          po[128 + key] = v1;
+        } else {
+          orow[h * p.o_sh + key] = __float2bfloat16_rn(v0);
+          orow[h * p.o_sh + 128 + key] = __float2bfloat16_rn(v1);
+        }
       }
     }
-    if (key < G && p.lse != nullptr) {
+    if (key < G && (p.lse != nullptr || p.part_lse != nullptr)) {
       float mk = 0.f, lk = 0.f;
 #pragma unroll
       for (int h = 0; h < kGp; ++h)
@@ -456,8 +469,11 @@ __device__ void softmax8(const TcParams& p, const Sync& sy, uint32_t sb, uint8_t
           mk = m_run[h];
           lk = l_tot[h];
         }
-      p.lse[un.t * p.lse_st + static_cast<int64_t>(un.g) * G + key] =
-          lk > 0.f ? (mk + lg2(lk)) * 0.69314718055994531f : -INFINITY;
+      const float lv = lk > 0.f ? (mk + lg2(lk)) * 0.69314718055994531f : -INFINITY;
+      if (p.part_lse != nullptr)
+        p.part_lse[(row0 + key) * p.splits + un.s] = lv;
+      else
+        p.lse[un.t * p.lse_st + static_cast<int64_t>(un.g) * G + key] = lv;
     }
     c_tile += un.n_tiles;
     ++c_unit;
@@ -489,7 +505,7 @@ __global__ void __launch_bounds__(kThreads, 1) qsa_prefill_f8_kernel(const __gri
       mbar_init(sy.bar(G_PFULL + b), 4);
       mbar_init(sy.bar(G_PEMPTY + b), 1);
       mbar_init(sy.bar(G_QFULL + b), 1);
-      mbar_init(sy.bar(G_QEMPTY + b), 1);
+      mbar_init(sy.bar(G_QEMPTY + b), 1 + 4);   // the MMAs, and each softmax warp
       mbar_init(sy.bar(G_RMAX + b), 4);
       mbar_init(sy.bar(G_RSUM + b), 4);
     }
