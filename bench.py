@@ -68,6 +68,8 @@ def parse_args():
                     help="microblock-list workload timed under 'blocks' ('' to skip)")
     ap.add_argument("--fp8", default="c5",
                     help="workload timed with an FP8 E4M3 KV cache under 'fp8' ('' to skip)")
+    ap.add_argument("--qsa-step", default="on", choices=["on", ""],
+                    help="time indexer -> top-K -> microblock attention as one step ('' to skip)")
     ap.add_argument("--indexer", default="indexer",
                     help="indexer + top-K workload timed under 'indexer' ('' to skip)")
     ap.add_argument("--e2e-steps", type=int, default=10)
@@ -79,7 +81,7 @@ def parse_args():
                     help="override the query-token count of c4/c5 (smaller ncu captures)")
     ap.add_argument("--profile", action="store_true",
                     help="minimal run for ncu: no clocks, e2e, cpu baseline or secondary")
-    ap.add_argument("--only", default="", choices=["", "fp8", "indexer", "blocks", "decode"],
+    ap.add_argument("--only", default="", choices=["", "fp8", "indexer", "blocks", "decode", "qsa_step"],
                     help="run one secondary leg alone (--steps / --warmup / --tokens apply), for "
                          "profiling; prints that leg's JSON")
     return ap.parse_args()
@@ -404,7 +406,9 @@ def run_cuda(args):
                "blocks": lambda: run_blocks_bench("c5_block4", dev, barrier, max_ranks, world, hbm,
                                                   args.steps, args.warmup, **kw),
                "decode": lambda: run_decode_bench("decode", dev, barrier, max_ranks, world, hbm, args.steps,
-                                                  args.warmup)}[args.only]()
+                                                  args.warmup),
+               "qsa_step": lambda: run_qsa_step_bench(dev, barrier, max_ranks, world, hbm, args.steps,
+                                                      args.warmup, **kw)}[args.only]()
         if rank == 0:
             print(json.dumps({"leg": args.only, **leg}), flush=True)
         if pg is not None:
@@ -490,6 +494,8 @@ def run_cuda(args):
         line["fp8"] = run_fp8_bench(args.fp8, dev, barrier, max_ranks, world, hbm)
     if args.indexer and not args.profile:
         line["indexer"] = run_indexer_bench(dev, barrier, max_ranks, world, hbm, bf16)
+    if args.qsa_step and not args.profile:
+        line["qsa_step"] = run_qsa_step_bench(dev, barrier, max_ranks, world, hbm)
     if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.profile:
         line["cpu_baseline"] = time_oracle(w, args.cpu_budget)
     elif not args.profile:
@@ -705,6 +711,58 @@ def run_indexer_bench(dev, barrier, reduce_max, world, hbm, bf16, steps=20, warm
             "topk": {"mean_launch_ms": k_ms, "algo_gbs": k_bytes / (k_ms / 1e3) / 1e9,
                      "frac_of_hbm": k_bytes / (k_ms / 1e3) / 1e9 / hbm},
             "launches_per_step": 2, "steps": steps}
+
+
+def run_qsa_step_bench(dev, barrier, reduce_max, world, hbm, steps=5, warmup=3, T=8192, S=131072,
+                       heads=(24, 2)):
+    """One whole QSA sparse-attention step on the c5 shape: indexer scores and
+    top-K select 2048 microblocks of 4 (+ the causal tail) per query token,
+    and the attention reads those 8196 keys per (token, KV head), both KV
+    heads sharing the token's list.  Timed with a BF16 and with an FP8 E4M3
+    KV cache; three launches per step."""
+    from top_sparse_attention_qsa_b200 import _capi
+    from top_sparse_attention_qsa_b200 import workloads as W
+    wi = W.config_indexer(device=dev, T=T, S=S)
+    gen = torch.Generator(device=dev).manual_seed(79)
+    Hq, Hkv = heads
+    q = W.normal_bf16((T, Hq, 256), gen, dev)
+    k = W.normal_bf16((S, Hkv, 256), gen, dev)
+    v = W.normal_bf16((S, Hkv, 256), gen, dev)
+    k8 = W.normal_fp8((S, Hkv, 256), gen, dev)
+    v8 = W.normal_fp8((S, Hkv, 256), gen, dev)
+    NB = wi.k_idx.shape[0]
+    width = wi.budget + 1
+    scores = torch.empty((T, NB), dtype=torch.float32, device=dev)
+    lists = torch.empty((T, width), dtype=torch.int32, device=dev)
+    nv = torch.empty((T, Hkv), dtype=torch.int32, device=dev)
+    idx = lists[:, None, :].expand(T, Hkv, width)
+    out = torch.empty_like(q)
+    lse = torch.empty((T, Hq), dtype=torch.float32, device=dev)
+
+    def select():
+        _capi.indexer_scores(wi.q_idx, wi.k_idx, wi.positions, wi.seq_start, 4, scores=scores)
+        _capi.topk_select(scores, wi.positions, wi.seq_start, NB, wi.budget, 4, True, lists=lists, n_valid=nv,
+                          copies=Hkv)
+
+    def step_bf16():
+        select()
+        _capi.sparse_prefill_block_fwd(q, k, v, idx, 4, wi.positions, nv, 0.0, out=out, lse=lse)
+
+    def step_fp8():
+        select()
+        _capi.sparse_prefill_fp8_fwd(q, k8, v8, idx, 0.5, 2.0, n_valid=nv, block_size=4, last_slot=wi.positions,
+                                     out=out, lse=lse)
+
+    res = {"workload": f"qsa_step_T{T}_S{S}_g{Hq}x{Hkv}_budget{wi.budget}x4",
+           "desc": f"indexer ({wi.q_idx.shape[1]}x128, {NB} block keys) + top-{wi.budget} blocks of 4 + tail, "
+                   f"then attention over <= {4 * width} keys per (token, KV head)", "launches_per_step": 3}
+    for name, fn in (("bf16", step_bf16), ("fp8", step_fp8)):
+        total_ms, per_ms, _ = time_launches(fn, steps, warmup, barrier, "qsa_step_" + name)
+        total_ms = reduce_max(total_ms)
+        res[name] = {"mean_step_ms": statistics.mean(per_ms), "tokens_per_s": T * steps * world / (total_ms / 1e3)}
+    res["keys_per_token_head"] = float(nv.float().mean().item()) * 4
+    res["steps"] = steps
+    return res
 
 
 def main():
