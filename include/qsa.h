@@ -315,14 +315,20 @@ typedef struct {
 } qsa_device_buffers_t;
 
 /*
- * Host-buffer variant: enqueues on `stream` one host->device cudaMemcpyAsync
- * per input (q, k_cache, v_cache, topk_idx, n_valid), the forward kernel,
- * and one device->host cudaMemcpyAsync per output (out, lse), then returns.
- * Host pointers address buffers laid out exactly like the device ones with
- * the strides of `shape` (each copied as one contiguous span from the first
- * to the last element); page-locked host memory keeps the copies
- * asynchronous.  The caller synchronises `stream` before reading out/lse.
- * The status word (dev->status) is zeroed on the stream before the launch.
+ * Host-buffer variant.  Host pointers address buffers laid out exactly like
+ * the device ones with the strides of `shape` (each part copied as one
+ * contiguous span from its first to its last element); page-locked host
+ * memory keeps the copies asynchronous.  The whole K and V caches go up
+ * first; the query tokens are then cut into chunks of about 1024 (at most 8
+ * chunks), and each chunk's Q / list / n_valid copies, forward kernel and
+ * out / lse copies form a pipeline: the copies up and down run on two
+ * streams the library keeps per device, overlapping the kernels on
+ * `stream` (one chunk and one stream when T < 2048).  Every copy is one
+ * cudaMemcpyAsync.  `stream` is ordered after all of it (events), so the
+ * caller synchronises `stream` before reading out/lse; the call itself
+ * never blocks on the device.  The status word (dev->status) is zeroed on
+ * `stream` before the first launch.  Calls on one device are serialised by
+ * a lock while they enqueue.
  */
 qsa_status_t qsa_sparse_prefill_fwd_host(
     const qsa_shape_t* shape, const void* q_host, const void* k_cache_host,

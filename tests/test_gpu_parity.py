@@ -260,6 +260,33 @@ def test_host_buffer_entry_point_matches_device():
     assert int(bufs["status"].item()) == 0
 
 
+def test_host_buffer_entry_point_pipelined_chunks():
+    """T = 4096 (c2): the host entry point cuts the tokens into 4 chunks whose
+    copies overlap the kernels on three streams; results equal the device
+    entry point's bit for bit, n_valid included, and the caller's stream is
+    ordered after the last copy down."""
+    from top_sparse_attention_qsa_b200 import _capi
+    w = W.make("c2", device=DEV)
+    ref_out, ref_lse = run_gpu(w)
+    torch.cuda.synchronize()
+    hq, hk, hv = host(w.q).pin_memory(), host(w.k_cache).pin_memory(), host(w.v_cache).pin_memory()
+    hi = host(w.topk_idx).pin_memory()
+    hn = host(w.n_valid).pin_memory() if w.n_valid is not None else None
+    ho = torch.full(w.q.shape, 3.0, dtype=torch.bfloat16).pin_memory()
+    hl = torch.full(w.q.shape[:2], 3.0, dtype=torch.float32).pin_memory()
+    bufs = dict(q=torch.empty_like(w.q), k_cache=torch.empty_like(w.k_cache),
+                v_cache=torch.empty_like(w.v_cache), topk_idx=torch.empty_like(w.topk_idx),
+                n_valid=torch.empty_like(w.n_valid) if hn is not None else None,
+                out=torch.empty_like(w.q), lse=torch.empty(w.q.shape[:2], device=DEV),
+                status=torch.ones(1, dtype=torch.int32, device=DEV))
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        _capi.sparse_prefill_fwd_host(hq, hk, hv, hi, hn, w.scale, ho, hl, bufs, stream=s.cuda_stream)
+    s.synchronize()                                        # the caller's stream alone
+    assert torch.equal(ho, host(ref_out)) and torch.equal(hl, host(ref_lse))
+    assert int(bufs["status"].item()) == 0
+
+
 def test_misaligned_pointer_rejected():
     from top_sparse_attention_qsa_b200 import _capi
     w = W.generic_case(T=4, S=64, Hq=3, Hkv=1, K=8, seed=1, device=DEV)

@@ -8,6 +8,7 @@
 #include <atomic>
 #include <cstdint>
 #include <cstring>
+#include <algorithm>
 #include <mutex>
 
 #include "qsa.h"
@@ -280,6 +281,38 @@ qsa_status_t run_lists(const qsa_shape_t* shape, int32_t block_size, const int32
                        float k_scale, float v_scale, bool fp8, void* out, float* lse,
                        int32_t* status, void* stream);
 
+// The host-buffer entry point cuts the query tokens into chunks of about
+// kHostChunkTokens (at most kHostMaxChunks) so that the copies of one chunk
+// overlap the kernel of the previous one.  Its copy streams and events are
+// made once per device and reused; a mutex serialises the calls that enqueue
+// on them.
+constexpr int64_t kHostChunkTokens = 1024;
+constexpr int kHostMaxChunks = 8;
+
+struct HostPipe {
+  std::mutex lock;
+  cudaStream_t up = nullptr, down = nullptr;
+  cudaEvent_t ev[2 + 2 * kHostMaxChunks] = {};
+};
+
+HostPipe* host_pipe() {
+  static HostPipe pipes[kMaxDevices];
+  static std::atomic<int> made[kMaxDevices];
+  static std::mutex make_lock;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  if (made[dev].load(std::memory_order_acquire) == 1) return &pipes[dev];
+  std::lock_guard<std::mutex> g(make_lock);
+  if (made[dev].load(std::memory_order_acquire) == 0) {
+    HostPipe& hp = pipes[dev];
+    bool ok = cudaStreamCreateWithFlags(&hp.up, cudaStreamNonBlocking) == cudaSuccess &&
+              cudaStreamCreateWithFlags(&hp.down, cudaStreamNonBlocking) == cudaSuccess;
+    for (auto& e : hp.ev) ok = ok && cudaEventCreateWithFlags(&e, cudaEventDisableTiming) == cudaSuccess;
+    made[dev].store(ok ? 1 : -1, std::memory_order_release);
+  }
+  return made[dev].load(std::memory_order_acquire) == 1 ? &pipes[dev] : nullptr;
+}
+
 qsa_status_t run_decode(const qsa_shape_t* s, const void* q, const void* k, const void* v,
                         const int32_t* idx, const int32_t* n_valid, float scale, void* out,
                         float* lse, int32_t* status, int32_t num_splits, void* workspace,
@@ -488,29 +521,70 @@ qsa_status_t qsa_sparse_prefill_fwd_host(const qsa_shape_t* s, const void* q_hos
   if ((n_valid_host != nullptr) != (dev->n_valid != nullptr)) return QSA_ERR_NULL;
   if (lse_host != nullptr && dev->lse == nullptr) return QSA_ERR_NULL;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  auto h2d = [&](void* d, const void* h, size_t n) {
-    return n == 0 || cudaMemcpyAsync(d, h, n, cudaMemcpyHostToDevice, st) == cudaSuccess;
+  const int chunks = static_cast<int>(std::min<int64_t>(std::max<int64_t>(T / kHostChunkTokens, 1), kHostMaxChunks));
+  HostPipe* hp = chunks > 1 ? host_pipe() : nullptr;
+  if (chunks > 1 && hp == nullptr) return QSA_ERR_CUDA;
+  std::unique_lock<std::mutex> hold;
+  if (hp != nullptr) hold = std::unique_lock<std::mutex>(hp->lock);
+  // one stream does everything for a single chunk; otherwise inputs go up on
+  // hp->up, the kernels run on `stream`, outputs come down on hp->down
+  cudaStream_t up = hp ? hp->up : st, down = hp ? hp->down : st;
+  auto copy = [](void* d, const void* h, size_t n, cudaMemcpyKind kind, cudaStream_t x) {
+    return n == 0 || cudaMemcpyAsync(d, h, n, kind, x) == cudaSuccess;
   };
-  auto d2h = [&](void* h, const void* d, size_t n) {
-    return n == 0 || cudaMemcpyAsync(h, d, n, cudaMemcpyDeviceToHost, st) == cudaSuccess;
+  auto at = [](const void* p, int64_t elems, int64_t bytes_per) {
+    return static_cast<const char*>(p) + elems * bytes_per;
   };
-  bool ok = h2d(dev->q, q_host, span_bytes(T, s->q_stride_tok, Hq, s->q_stride_head, D, 2));
-  if (K > 0) {
-    const size_t kv = span_bytes(S, s->kv_stride_slot, Hkv, s->kv_stride_head, D, 2);
-    ok = ok && h2d(dev->k_cache, k_cache_host, kv) && h2d(dev->v_cache, v_cache_host, kv);
-    ok = ok && h2d(dev->topk_idx, topk_idx_host,
-                   span_bytes(T, s->idx_stride_tok, Hkv, s->idx_stride_head, K, 4));
+  bool ok = true;
+  if (hp != nullptr) {
+    ok = cudaEventRecord(hp->ev[0], st) == cudaSuccess && cudaStreamWaitEvent(up, hp->ev[0], 0) == cudaSuccess &&
+         cudaStreamWaitEvent(down, hp->ev[0], 0) == cudaSuccess;
   }
-  if (n_valid_host != nullptr)
-    ok = ok && h2d(dev->n_valid, n_valid_host, static_cast<size_t>(T * Hkv) * 4);
-  if (dev->status != nullptr) ok = ok && cudaMemsetAsync(dev->status, 0, 4, st) == cudaSuccess;
-  if (!ok) return QSA_ERR_CUDA;
-  rc = run_forward(s, dev->q, dev->k_cache, dev->v_cache, dev->topk_idx, dev->n_valid, scale,
-                   dev->out, lse_host != nullptr ? dev->lse : nullptr, dev->status, nullptr, stream);
-  if (rc != QSA_OK) return rc;
-  ok = d2h(out_host, dev->out, span_bytes(T, s->o_stride_tok, Hq, s->o_stride_head, D, 2));
-  if (lse_host != nullptr)
-    ok = ok && d2h(lse_host, dev->lse, span_bytes(T, s->lse_stride_tok, 1, 0, Hq, 4));
+  if (ok && K > 0) {
+    const size_t kv = span_bytes(S, s->kv_stride_slot, Hkv, s->kv_stride_head, D, 2);
+    ok = copy(dev->k_cache, k_cache_host, kv, cudaMemcpyHostToDevice, up) &&
+         copy(dev->v_cache, v_cache_host, kv, cudaMemcpyHostToDevice, up);
+  }
+  if (ok && dev->status != nullptr) ok = cudaMemsetAsync(dev->status, 0, 4, st) == cudaSuccess;
+  for (int c = 0; c < chunks && ok; ++c) {
+    const int64_t t0 = T * c / chunks, tc = T * (c + 1) / chunks - t0;
+    // this chunk's inputs
+    ok = copy(const_cast<char*>(at(dev->q, t0 * s->q_stride_tok, 2)), at(q_host, t0 * s->q_stride_tok, 2),
+              span_bytes(tc, s->q_stride_tok, Hq, s->q_stride_head, D, 2), cudaMemcpyHostToDevice, up);
+    if (ok && K > 0)
+      ok = copy(const_cast<char*>(at(dev->topk_idx, t0 * s->idx_stride_tok, 4)),
+                at(topk_idx_host, t0 * s->idx_stride_tok, 4),
+                span_bytes(tc, s->idx_stride_tok, Hkv, s->idx_stride_head, K, 4), cudaMemcpyHostToDevice, up);
+    if (ok && n_valid_host != nullptr)
+      ok = copy(const_cast<char*>(at(dev->n_valid, t0 * Hkv, 4)), at(n_valid_host, t0 * Hkv, 4),
+                static_cast<size_t>(tc * Hkv) * 4, cudaMemcpyHostToDevice, up);
+    if (ok && hp != nullptr)
+      ok = cudaEventRecord(hp->ev[2 + c], up) == cudaSuccess && cudaStreamWaitEvent(st, hp->ev[2 + c], 0) == cudaSuccess;
+    if (!ok) break;
+    // its kernel
+    qsa_shape_t sc = *s;
+    sc.num_tokens = tc;
+    rc = run_forward(&sc, at(dev->q, t0 * s->q_stride_tok, 2), dev->k_cache, dev->v_cache,
+                     reinterpret_cast<const int32_t*>(at(dev->topk_idx, t0 * s->idx_stride_tok, 4)),
+                     dev->n_valid ? reinterpret_cast<const int32_t*>(at(dev->n_valid, t0 * Hkv, 4)) : nullptr,
+                     scale, const_cast<char*>(at(dev->out, t0 * s->o_stride_tok, 2)),
+                     lse_host != nullptr ? reinterpret_cast<float*>(const_cast<char*>(at(dev->lse, t0 * s->lse_stride_tok, 4)))
+                                         : nullptr,
+                     dev->status, nullptr, st);
+    if (rc != QSA_OK) return rc;
+    // its outputs
+    if (hp != nullptr)
+      ok = cudaEventRecord(hp->ev[2 + kHostMaxChunks + c], st) == cudaSuccess &&
+           cudaStreamWaitEvent(down, hp->ev[2 + kHostMaxChunks + c], 0) == cudaSuccess;
+    ok = ok && copy(const_cast<char*>(at(out_host, t0 * s->o_stride_tok, 2)), at(dev->out, t0 * s->o_stride_tok, 2),
+                    span_bytes(tc, s->o_stride_tok, Hq, s->o_stride_head, D, 2), cudaMemcpyDeviceToHost, down);
+    if (ok && lse_host != nullptr)
+      ok = copy(const_cast<char*>(at(lse_host, t0 * s->lse_stride_tok, 4)), at(dev->lse, t0 * s->lse_stride_tok, 4),
+                span_bytes(tc, s->lse_stride_tok, 1, 0, Hq, 4), cudaMemcpyDeviceToHost, down);
+  }
+  // `stream` ends after the last copy down
+  if (hp != nullptr)
+    ok = ok && cudaEventRecord(hp->ev[1], down) == cudaSuccess && cudaStreamWaitEvent(st, hp->ev[1], 0) == cudaSuccess;
   return ok ? QSA_OK : QSA_ERR_CUDA;
 }
 
