@@ -68,6 +68,8 @@ def parse_args():
                     help="microblock-list workload timed under 'blocks' ('' to skip)")
     ap.add_argument("--fp8", default="c5",
                     help="workload timed with an FP8 E4M3 KV cache under 'fp8' ('' to skip)")
+    ap.add_argument("--per-config", default="on", choices=["on", ""],
+                    help="also time the five configs (tiny, c2..c5) and report each one's absolute numbers")
     ap.add_argument("--qsa-step", default="on", choices=["on", ""],
                     help="time indexer -> top-K -> microblock attention as one step ('' to skip)")
     ap.add_argument("--indexer", default="indexer",
@@ -494,6 +496,8 @@ def run_cuda(args):
         line["fp8"] = run_fp8_bench(args.fp8, dev, barrier, max_ranks, world, hbm)
     if args.indexer and not args.profile:
         line["indexer"] = run_indexer_bench(dev, barrier, max_ranks, world, hbm, bf16)
+    if args.per_config and not args.profile:
+        line["per_config"] = run_per_config(dev, barrier, max_ranks, world, hbm, bf16)
     if args.qsa_step and not args.profile:
         line["qsa_step"] = run_qsa_step_bench(dev, barrier, max_ranks, world, hbm)
     if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.profile:
@@ -711,6 +715,36 @@ def run_indexer_bench(dev, barrier, reduce_max, world, hbm, bf16, steps=20, warm
             "topk": {"mean_launch_ms": k_ms, "algo_gbs": k_bytes / (k_ms / 1e3) / 1e9,
                      "frac_of_hbm": k_bytes / (k_ms / 1e3) / 1e9 / hbm},
             "launches_per_step": 2, "steps": steps}
+
+
+def run_per_config(dev, barrier, reduce_max, world, hbm, bf16, steps=20, warmup=3):
+    """Every config of the workload table with the default kernel: query
+    tokens/s, gathered-KV GB/s, effective TFLOP/s and the fraction of the
+    roofline time (gathered bytes at the HBM peak vs FLOPs at the BF16
+    peak, the slower of the two)."""
+    from top_sparse_attention_qsa_b200 import _capi
+    res = {}
+    for name in ("tiny", "c2", "c3", "c4", "c5"):
+        w = make_workload(name, dev)
+        acct = workload_accounting(w)
+        out = torch.empty_like(w.q)
+        lse = torch.empty(w.q.shape[:2], dtype=torch.float32, device=dev)
+
+        def step():
+            _capi.sparse_prefill_fwd(w.q, w.k_cache, w.v_cache, w.topk_idx, w.n_valid, w.scale, out=out, lse=lse)
+
+        total_ms, per_ms, _ = time_launches(step, steps, warmup, barrier, "config_" + name)
+        total_ms = reduce_max(total_ms)
+        ms = statistics.mean(per_ms)
+        roof_ms = 1e3 * max(acct["gathered_bytes"] / (hbm * 1e9), acct["flops"] / (bf16 * 1e12))
+        s = w.shape
+        res[name] = {"workload": w.name, "T": s["T"], "S": s["S"], "heads": [s["Hq"], s["Hkv"]], "topk": s["K"],
+                     "mean_launch_ms": ms, "tokens_per_s": s["T"] * steps * world / (total_ms / 1e3),
+                     "gathered_kv_gbs": acct["gathered_bytes"] / (ms / 1e3) / 1e9,
+                     "effective_tflops": acct["flops"] / (ms / 1e3) / 1e12,
+                     "frac_of_roofline_time": roof_ms / ms}
+        del w, out, lse
+    return res
 
 
 def run_qsa_step_bench(dev, barrier, reduce_max, world, hbm, steps=5, warmup=3, T=8192, S=131072,
