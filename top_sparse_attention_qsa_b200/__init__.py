@@ -8,8 +8,11 @@ libqsa.so raises ImportError (there is no fallback).
 """
 
 _API = ("sparse_prefill_fwd", "sparse_prefill_debug_gather", "sparse_prefill_fwd_host",
-        "sparse_decode_fwd", "decode_workspace_bytes", "decode_num_splits",
-        "status_string", "abi_version", "QSAError", "STATUS_OOB_SLOT")
+        "sparse_prefill_block_fwd", "sparse_prefill_fp8_fwd",
+        "sparse_decode_fwd", "sparse_decode_fwd_noalloc", "sparse_decode_fp8_fwd",
+        "decode_workspace_bytes", "decode_num_splits",
+        "indexer_scores", "topk_select", "indexer_select",
+        "status_string", "abi_version", "QSAError", "STATUS_OOB_SLOT", "STATUS_TIMEOUT")
 
 
 def __getattr__(name):

@@ -254,7 +254,9 @@ def sparse_prefill_fwd_host(q, k_cache, v_cache, topk_idx, n_valid, scale, out, 
                             dev_bufs: dict, stream=None):
     """Host-buffer entry point: host tensors in and out (pinned for async copies),
     device staging tensors in `dev_bufs` (keys as in qsa_device_buffers_t).
-    Enqueues copies + kernel + copies on `stream`; the caller synchronises."""
+    The library pipelines the copies of token chunks with their kernels on
+    its own copy streams and orders `stream` after the last copy down; the
+    caller synchronises `stream`."""
     for name, x, dt in (("q", q, torch.bfloat16), ("k_cache", k_cache, torch.bfloat16),
                         ("v_cache", v_cache, torch.bfloat16), ("topk_idx", topk_idx, torch.int32),
                         ("out", out, torch.bfloat16)):
