@@ -58,7 +58,7 @@ def parse_args():
     ap.add_argument("--secondary", default="c4",
                     help="second workload reported under 'secondary' ('' to skip)")
     ap.add_argument("--kernel", default="auto", choices=["auto", "tcgen05", "warp_mma"])
-    ap.add_argument("--shard", default="replicas", choices=["replicas", "tokens"],
+    ap.add_argument("--shard", default="replicas", choices=["replicas", "tokens", "heads"],
                     help="N>1: independent replicas (weak scaling) or one workload's tokens split (strong)")
     ap.add_argument("--compare", default="warp_mma",
                     help="second kernel timed on the same workload ('' to skip)")
@@ -122,6 +122,46 @@ def shard_workload(w, world, rank):
         w, q=w.q[t0:t1], topk_idx=w.topk_idx[t0:t1],
         n_valid=None if w.n_valid is None else w.n_valid[t0:t1],
         positions=w.positions[t0:t1], seq_start=w.seq_start[t0:t1])
+
+
+def shard_heads(w, world, rank):
+    """The rank's share of the KV heads (tensor-parallel split: the rank holds
+    only its heads' cache, as a compact copy), or None when the rank has no
+    head (more ranks than KV heads)."""
+    s = w.shape
+    g0, g1 = shard_range(s["Hkv"], world, rank)
+    if g1 <= g0:
+        return None
+    G = s["Hq"] // s["Hkv"]
+    import dataclasses
+    return dataclasses.replace(
+        w, q=w.q[:, g0 * G:g1 * G], k_cache=w.k_cache[:, g0:g1].contiguous(),
+        v_cache=w.v_cache[:, g0:g1].contiguous(), topk_idx=w.topk_idx[:, g0:g1],
+        n_valid=None if w.n_valid is None else w.n_valid[:, g0:g1].contiguous())
+
+
+def dataclasses_replace_empty(w):
+    """A workload with no query tokens (a rank with nothing to do)."""
+    import dataclasses
+    return dataclasses.replace(w, q=w.q[:0], topk_idx=w.topk_idx[:0],
+                               n_valid=None if w.n_valid is None else w.n_valid[:0],
+                               positions=w.positions[:0], seq_start=w.seq_start[:0])
+
+
+def compulsory_bytes(w):
+    """Bytes a launch cannot avoid moving: every cache row named by some list
+    once, plus Q, out, lse and the lists (context for the DRAM traffic)."""
+    s = w.shape
+    idx = w.topk_idx
+    live = (idx >= 0) & (idx < s["S"])
+    if w.n_valid is not None:
+        live &= torch.arange(s["K"], device=idx.device)[None, None, :] < w.n_valid[:, :, None]
+    rows = 0
+    for g in range(s["Hkv"]):
+        ids = idx[:, g][live[:, g]]
+        rows += int(torch.unique(ids).numel()) if ids.numel() else 0
+    return (rows * 2 * s["D"] * 2 + s["T"] * s["Hq"] * s["D"] * 2 * 2 + s["T"] * s["Hq"] * 4
+            + int(live.sum().item()) * 4)
 
 
 def measured_peaks():
@@ -279,6 +319,23 @@ def time_launches(fn, steps, warmup, barrier, label="timed"):
     return total, per, (t0, t1)
 
 
+def time_flushed(fn, n=5):
+    """Mean and median of n launches, each timed alone (CUDA events) after
+    writing a 256 MB buffer that evicts the 126 MB L2."""
+    flush = torch.empty(64 << 20, dtype=torch.float32, device="cuda")
+    per = []
+    for _ in range(n):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        fn()
+        b.record()
+        torch.cuda.synchronize()
+        per.append(a.elapsed_time(b))
+    del flush
+    return statistics.mean(per), statistics.median(per)
+
+
 def time_oracle(w, budget_s, min_tokens=1):
     """FP64 oracle over a bounded sample of the workload's tokens (host copies)."""
     import numpy as np
@@ -429,6 +486,10 @@ def run_cuda(args):
     T_job = w.shape["T"] * (world if args.shard == "replicas" else 1)
     if args.shard == "tokens":
         w = shard_workload(w, world, rank)
+    elif args.shard == "heads":
+        w_full, w = w, shard_heads(w, world, rank)
+        if w is None:                 # more ranks than KV heads: this rank idles
+            w = dataclasses_replace_empty(w_full)
     acct = workload_accounting(w)
     out = torch.empty_like(w.q)
     lse = torch.empty(w.q.shape[:2], dtype=torch.float32, device=dev)
@@ -469,6 +530,11 @@ def run_cuda(args):
             "gathered_kv_gbs": gathered_gbs, "effective_tflops": tflops,
             "roofline_time_ms": roof_time_ms, "frac_of_roofline_time": roof_time_ms / mean_launch_ms,
             "roofline": roof, "clocks": clocks}
+    if not args.profile:
+        fl_mean, fl_median = time_flushed(step)
+        line["timing"] = {"mean_launch_ms": mean_launch_ms, "median_launch_ms": statistics.median(per_ms),
+                          "l2_flushed_mean_ms": fl_mean, "l2_flushed_median_ms": fl_median,
+                          "compulsory_bytes": compulsory_bytes(w)}
     if int(status.item()) != 0:
         line["status_word"] = int(status.item())
 

@@ -38,7 +38,17 @@ def _rank_main(rank, world, port, queue):
         part = bench.shard_workload(w, world, rank)
         t0, t1 = bench.shard_range(w.shape["T"], world, rank)
         same = torch.equal(part.q, w.q[t0:t1]) and torch.equal(part.topk_idx, w.topk_idx[t0:t1])
-        queue.put((rank, m, (t0, t1), part.shape["T"], bool(same)))
+        # KV-head split: each rank's oracle result on its heads is the full
+        # result's head slice
+        import oracle
+        wh = W.generic_case(T=5, S=40, Hq=16, Hkv=2, K=9, seed=7)
+        wh.n_valid = torch.tensor([[9, 3], [0, 9], [5, 5], [9, 1], [2, 9]], dtype=torch.int32)
+        mine = bench.shard_heads(wh, world, rank)
+        full = oracle.sparse_prefill(wh.q, wh.k_cache, wh.v_cache, wh.topk_idx, wh.n_valid, 0.0)
+        part_res = oracle.sparse_prefill(mine.q, mine.k_cache, mine.v_cache, mine.topk_idx, mine.n_valid, 0.0)
+        h0 = rank * 8
+        heads_ok = bool((part_res[0] == full[0][:, h0:h0 + 8]).all() and (part_res[1] == full[1][:, h0:h0 + 8]).all())
+        queue.put((rank, m, (t0, t1), part.shape["T"], bool(same and heads_ok)))
         dist.barrier()
     finally:
         dist.destroy_process_group()
