@@ -107,7 +107,7 @@ cudaError_t launch_f8(const qsa::tc::TcParams& tp, cudaStream_t stream) {
   const int nsm = sm_count();
   if (nsm <= 0) return cudaErrorInvalidDevice;
   const unsigned grid = static_cast<unsigned>(units < nsm ? units : nsm);
-  kernel<<<grid, qsa::tc::kThreads, qsa::f8::F_SMEM, stream>>>(tp);
+  kernel<<<grid, qsa::f8::kThreads8, qsa::f8::F_SMEM, stream>>>(tp);
   return cudaGetLastError();
 }
 

@@ -26,11 +26,13 @@
 //               the 256-byte K and V rows into the 128-byte-swizzled K-major
 //               layout (K slot, then V slot per tile)
 //   warp 4      all lanes: the unit's Q (BF16, from global memory) split into
-//               q_hi / q_lo E4M3 tiles with per-head scale; lane 0 issues the
-//               score MMAs (A = K tile, B = q_hi then q_lo; M=128, N=16, K=32)
-//   warp 5      lane 0 issues PV: O_{hi,lo}^T += V^T (MN-major) . P_{hi,lo}^T
-//               (MN-major) for the two 128-dim halves
-//   warps 6-9   softmax as in the BF16 kernel, reading both score terms and
+//               q_hi / q_lo rows of one E4M3 tile with per-head scale; lane 0
+//               issues the score MMAs (A = K tile, B = [q_hi; q_lo];
+//               M=128, N=32, K=32)
+//   warp 5      lane 0 issues PV: [O_hi O_lo]^T += V^T (MN-major) .
+//               [P_hi P_lo]^T (MN-major, N=32) for the two 128-dim halves
+//   warps 6-13  softmax as in the BF16 kernel, two warps per TMEM lane
+//               quadrant (8 heads each), reading both score terms and
 //               writing p_hi / p_lo
 // Every wait is bounded (2 s of %globaltimer) as in the BF16 kernel.
 #pragma once
@@ -44,8 +46,9 @@ using namespace tc;
 
 constexpr int kSlots8 = 6;                    // 32 KB: one K or V tile
 constexpr int kQ8Bytes = kGp * 256;           // one E4M3 Q term: 16 heads x 256 dims
+constexpr int kQ8Block = 2 * kGp * 128;       // one 128-dim block of both terms: 32 rows x 128 B
 constexpr int kP8Bytes = kKeys * kGp;         // one E4M3 P term: 128 keys x 16 heads
-constexpr int kTmemCols8 = 128;               // S: 2 buffers x {hi, lo} x 16; O: {hi, lo} x 2 halves x 16
+constexpr int kTmemCols8 = 128;               // S: 2 buffers x {hi, lo} x 16; O: 2 halves x {hi, lo} x 16
 constexpr int kTS = 0, kTO = 64;              // TMEM column bases
 
 constexpr int F_RING = 0;
@@ -60,8 +63,9 @@ constexpr int G_FULL = 0, G_EMPTY = 6, G_SFULL = 12, G_SFREE = 14, G_PFULL = 16,
 constexpr int F_MISC = F_BAR + G_NUM * 8;             // tmem base, abort flag
 constexpr int F_SMEM = F_MISC + 16 + 1024;
 
-// kind::f8f6f4: FP32 accumulator, E4M3 A and B (format 0), N = 16, M = 128.
-constexpr uint32_t kIdescQK8 = (1u << 4) | (2u << 17) | (8u << 24);
+// kind::f8f6f4: FP32 accumulator, E4M3 A and B (format 0), M = 128, N = 32:
+// the hi and lo terms share one MMA (B rows / columns 0-15 hi, 16-31 lo).
+constexpr uint32_t kIdescQK8 = (1u << 4) | (4u << 17) | (8u << 24);
 // PV: both operands MN-major.
 constexpr uint32_t kIdescPV8 = kIdescQK8 | (1u << 15) | (1u << 16);
 
@@ -120,28 +124,26 @@ __device__ void producer8(const TcParams& p, const Sync& sy, uint32_t sb, int pw
 
 // Lane l of warp 4 takes head l/2, dims [128*(l&1), +128): loads them from
 // global memory, finds the head's largest |q| (with its partner lane), and
-// writes q * 2^a = q_hi + q_lo / 16 into the two E4M3 tiles (K-major, 128-byte
-// swizzle: two 128-dim blocks of 16 rows x 128 B) and 2^-a * scale_log2 into
-// the score factors.  Heads past the group are zero.
-__device__ __forceinline__ void q_split(const TcParams& p, const Unit& un, uint32_t qhi, uint32_t qlo,
-                                        float* qsc, int lane) {
+// writes q * 2^a = q_hi + q_lo / 16 as one E4M3 tile of 32 rows (K-major,
+// 128-byte swizzle: two 128-dim blocks of 32 rows x 128 B; row h holds the
+// hi term of head h, row 16 + h its lo term) and 2^-a * scale_log2 into the
+// score factors.  Heads past the group are zero.
+__device__ __forceinline__ void q_split(const TcParams& p, const Unit& un, uint32_t qt, float* qsc, int lane) {
   const int h = lane >> 1, half = lane & 1;
-  uint4 v[16];
-  if (h < p.G) {
-    const char* src = reinterpret_cast<const char*>(p.q_ptr) +
-                      (un.t * p.q_st + (static_cast<int64_t>(un.g) * p.G + h) * p.q_sh + half * 128) * 2;
+  const bool live = h < p.G;
+  const uint4* src = reinterpret_cast<const uint4*>(
+      reinterpret_cast<const char*>(p.q_ptr) +
+      (un.t * p.q_st + (static_cast<int64_t>(un.g) * p.G + (live ? h : 0)) * p.q_sh + half * 128) * 2);
+  // first read: the head's largest |q| (BF16 bits widened; order = magnitude)
+  uint32_t mx = 0u;
+  if (live) {
+#pragma unroll 4
+    for (int i = 0; i < 16; ++i) {
+      const uint4 v = __ldg(src + i);
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-    for (int i = 0; i < 16; ++i) v[i] = __ldg(reinterpret_cast<const uint4*>(src) + i);
-  } else {
-#pragma unroll
-    for (int i = 0; i < 16; ++i) v[i] = make_uint4(0u, 0u, 0u, 0u);
-  }
-  uint32_t mx = 0u;                                  // max |q| as BF16 bits widened (order = magnitude)
-#pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
-#pragma unroll
-    for (int j = 0; j < 4; ++j) mx = max(mx, max((w[j] << 16) & 0x7fffffffu, w[j] & 0x7fff0000u));
+      for (int j = 0; j < 4; ++j) mx = max(mx, max((w[j] << 16) & 0x7fffffffu, w[j] & 0x7fff0000u));
+    }
   }
   mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
   // a = 7 - floor(log2 max): the largest |q| * 2^a lands in [128, 256)
@@ -150,14 +152,17 @@ __device__ __forceinline__ void q_split(const TcParams& p, const Unit& un, uint3
   a = max(-126, min(a, 126));
   const float up = __int_as_float((127 + a) << 23);
   if (half == 0) qsc[h] = p.scale_log2 * __int_as_float((127 - a) << 23);
-#pragma unroll
-  for (int c8 = 0; c8 < 8; ++c8) {                   // 16 dims per 16-byte chunk
+  // second read (cached): the two E4M3 terms, 16 dims per 16-byte chunk
+#pragma unroll 2
+  for (int c8 = 0; c8 < 8; ++c8) {
+    const uint4 va = live ? __ldg(src + 2 * c8) : make_uint4(0u, 0u, 0u, 0u);
+    const uint4 vb = live ? __ldg(src + 2 * c8 + 1) : make_uint4(0u, 0u, 0u, 0u);
+    const uint32_t wv[8] = {va.x, va.y, va.z, va.w, vb.x, vb.y, vb.z, vb.w};
     uint32_t hw[4], lw[4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      // dims 4j..4j+3 of the chunk: bf16 words v[2*c8 + j/2], halves
-      const uint4 vv = v[2 * c8 + (j >> 1)];
-      const uint32_t w0 = (j & 1) ? vv.z : vv.x, w1 = (j & 1) ? vv.w : vv.y;
+      // dims 4j..4j+3 of the chunk: BF16 words wv[2j], wv[2j+1]
+      const uint32_t w0 = wv[2 * j], w1 = wv[2 * j + 1];
       const float x0 = __uint_as_float(w0 << 16) * up, x1 = __uint_as_float(w0 & 0xffff0000u) * up;
       const float x2 = __uint_as_float(w1 << 16) * up, x3 = __uint_as_float(w1 & 0xffff0000u) * up;
       const uint32_t h01 = pack_e4m3x2(x0, x1), h23 = pack_e4m3x2(x2, x3);
@@ -169,9 +174,9 @@ __device__ __forceinline__ void q_split(const TcParams& p, const Unit& un, uint3
       hw[j] = h01 | (h23 << 16);
       lw[j] = l01 | (l23 << 16);
     }
-    const uint32_t off = half * 2048 + h * 128 + ((c8 ^ (h & 7)) << 4);
-    st_shared_v4(qhi + off, hw[0], hw[1], hw[2], hw[3]);
-    st_shared_v4(qlo + off, lw[0], lw[1], lw[2], lw[3]);
+    const uint32_t off = half * kQ8Block + h * 128 + ((c8 ^ (h & 7)) << 4);   // rows h and 16 + h share the swizzle
+    st_shared_v4(qt + off, hw[0], hw[1], hw[2], hw[3]);
+    st_shared_v4(qt + off + 16 * 128, lw[0], lw[1], lw[2], lw[3]);
   }
 }
 
@@ -190,8 +195,8 @@ __device__ void qk8(const TcParams& p, const Sync& sy, uint32_t sb, uint8_t* sp,
     ok = sy.wait_warp(G_QEMPTY + qb, ((c_unit >> 1) & 1u) ^ 1u);
     if (!ok) break;
     ++c_unit;
-    const uint32_t qhi = sb + F_Q8 + qb * 2 * kQ8Bytes, qlo = qhi + kQ8Bytes;
-    if (un.n_tiles > 0) q_split(p, un, qhi, qlo, reinterpret_cast<float*>(sp + F_QSC) + qb * kGp, lane);
+    const uint32_t qt = sb + F_Q8 + qb * 2 * kQ8Bytes;
+    if (un.n_tiles > 0) q_split(p, un, qt, reinterpret_cast<float*>(sp + F_QSC) + qb * kGp, lane);
     fence_proxy_async_smem();
     __syncwarp();
     if (lane == 0) {
@@ -208,16 +213,13 @@ __device__ void qk8(const TcParams& p, const Sync& sy, uint32_t sb, uint8_t* sp,
         tc_fence_after();
         const uint32_t kt = sb + F_RING + slot * kSlotBytes;
 #pragma unroll
-        for (int term = 0; term < 2; ++term) {
-          const uint32_t qa = term == 0 ? qhi : qlo;
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            // K-major, 128-byte swizzle: a 32-dim step advances 32 B inside
-            // the atom; dims 128-255 sit 16 KB (K) / 2 KB (Q) further
-            const uint64_t a = smem_desc(kt + (kk >> 2) * kBlockBytes + (kk & 3) * 32, 16, 1024, 2);
-            const uint64_t b = smem_desc(qa + (kk >> 2) * 2048 + (kk & 3) * 32, 16, 1024, 2);
-            umma_f8_ss(tmem + kTS + sbuf * 32 + term * 16, a, b, kIdescQK8, kk > 0 ? 1u : 0u);
-          }
+        for (int kk = 0; kk < 8; ++kk) {
+          // K-major, 128-byte swizzle: a 32-dim step advances 32 B inside the
+          // atom; dims 128-255 sit 16 KB (K) / 4 KB (Q) further.  N = 32:
+          // S_hi in columns 0-15, S_lo in 16-31.
+          const uint64_t a = smem_desc(kt + (kk >> 2) * kBlockBytes + (kk & 3) * 32, 16, 1024, 2);
+          const uint64_t b = smem_desc(qt + (kk >> 2) * kQ8Block + (kk & 3) * 32, 16, 1024, 2);
+          umma_f8_ss(tmem + kTS + sbuf * 32, a, b, kIdescQK8, kk > 0 ? 1u : 0u);
         }
         umma_commit(sy.bar(G_EMPTY + slot));
         umma_commit(sy.bar(G_SFULL + sbuf));
@@ -261,17 +263,17 @@ __device__ void pv8(const TcParams& p, const Sync& sy, uint32_t sb, uint32_t tme
 #pragma unroll
       for (int mh = 0; mh < 2; ++mh)
 #pragma unroll
-        for (int term = 0; term < 2; ++term)
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            // A = V^T: MN-major, 128-byte swizzle; the 128 dims of a half are
-            // one atom row, groups of 8 keys 1 KB apart, 32 keys per step
-            const uint64_t a = smem_desc(vt + mh * kBlockBytes + kk * 4096, kBlockBytes, 1024, 2);
-            // B = P^T: MN-major, no swizzle; 16 heads = one 16-byte core row per
-            // key, key groups of 8 128 B apart
-            const uint64_t b = smem_desc(pt + term * kP8Bytes + kk * 512, 128, 2048, 0);
-            umma_f8_ss(tmem + kTO + term * 32 + mh * 16, a, b, kIdescPV8, (i == 0 && kk == 0) ? 0u : 1u);
-          }
+        for (int kk = 0; kk < 4; ++kk) {
+          // A = V^T: MN-major, 128-byte swizzle; the 128 dims of a half are
+          // one atom row, groups of 8 keys 1 KB apart, 32 keys per step
+          const uint64_t a = smem_desc(vt + mh * kBlockBytes + kk * 4096, kBlockBytes, 1024, 2);
+          // B = P^T: MN-major, no swizzle; per key one 16-byte core row of 16
+          // heads, key groups of 8 128 B apart (LBO); N = 32 spans P_hi and,
+          // one core-matrix column (SBO = 2 KB) further, P_lo: O_hi lands in
+          // columns 0-15 and O_lo in 16-31 of the half
+          const uint64_t b = smem_desc(pt + kk * 512, 128, kP8Bytes, 0);
+          umma_f8_ss(tmem + kTO + mh * 32, a, b, kIdescPV8, (i == 0 && kk == 0) ? 0u : 1u);
+        }
       umma_commit(sy.bar(G_EMPTY + slot));
       umma_commit(sy.bar(G_PEMPTY + pb));
     }
@@ -283,10 +285,46 @@ __device__ void pv8(const TcParams& p, const Sync& sy, uint32_t sb, uint32_t tme
 
 // ------------------------------------------------------------------ softmax
 
+constexpr int kSmWarps = 8;     // two per TMEM lane quadrant, 8 heads each
+constexpr int kHpw = kGp / 2;   // heads per softmax warp
+constexpr int kThreads8 = 32 * (kProducerWarps + 2 + kSmWarps);
+
+// Reduce 8 per-lane values across the 32 lanes of a warp by exchanging halves
+// (7 shuffles for the exchange, 2 for the rest).  Lane l ends with the result
+// for value (l >> 2) & 7.
+template <bool kMax>
+__device__ __forceinline__ float xreduce8(const float (&v)[8], int lane) {
+  auto op = [](float a, float b) { return kMax ? fmaxf(a, b) : a + b; };
+  float a[4], b[2];
+  bool up = (lane & 16) != 0;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const float send = up ? v[j] : v[4 + j];
+    const float keep = up ? v[4 + j] : v[j];
+    a[j] = op(keep, __shfl_xor_sync(0xffffffffu, send, 16));
+  }
+  up = (lane & 8) != 0;
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+    const float send = up ? a[j] : a[2 + j];
+    const float keep = up ? a[2 + j] : a[j];
+    b[j] = op(keep, __shfl_xor_sync(0xffffffffu, send, 8));
+  }
+  up = (lane & 4) != 0;
+  float c = op(up ? b[1] : b[0], __shfl_xor_sync(0xffffffffu, up ? b[0] : b[1], 4));
+  c = op(c, __shfl_xor_sync(0xffffffffu, c, 2));
+  c = op(c, __shfl_xor_sync(0xffffffffu, c, 1));
+  return c;
+}
+
+// Softmax warp w (6..13): TMEM lane quadrant q = w & 3 (thread = key of the
+// tile, and dim of an output half), heads [8 hh, 8 hh + 8) with hh = (w-6)/4.
 template <bool kBlocks>
 __device__ void softmax8(const TcParams& p, const Sync& sy, uint32_t sb, uint8_t* sp, uint32_t tmem, int warp,
                          int lane) {
   const int wq = warp & 3;
+  const int hh = (warp - kWarpSoftmax0) >> 2;
+  const int h0 = hh * kHpw;
   const int key = wq * 32 + lane;
   const uint32_t tl = tmem + (static_cast<uint32_t>(wq * 32) << 16);
   float* red_max = reinterpret_cast<float*>(sp + F_RED);
@@ -303,17 +341,17 @@ __device__ void softmax8(const TcParams& p, const Sync& sy, uint32_t sb, uint8_t
     const uint32_t qb = c_unit & 1u;
     ok = sy.wait_warp(G_QFULL + qb, (c_unit >> 1) & 1u);
     if (!ok) break;
-    float qs[kGp];
+    float qs[kHpw];
 #pragma unroll
-    for (int h = 0; h < kGp; ++h) qs[h] = qsc_all[qb * kGp + h];
+    for (int h = 0; h < kHpw; ++h) qs[h] = qsc_all[qb * kGp + h0 + h];
     // the score factors are read: the Q buffer may be refilled once the MMAs
     // are done too (without this release, warp 4 could run two units ahead
     // through empty units and complete a G_QFULL phase this warp never saw)
     __syncwarp();
     if (lane == 0) mbar_arrive(sy.bar(G_QEMPTY + qb));
-    float m_run[kGp], l_part[kGp];
+    float m_run[kHpw], l_part[kHpw];
 #pragma unroll
-    for (int h = 0; h < kGp; ++h) {
+    for (int h = 0; h < kHpw; ++h) {
       m_run[h] = -INFINITY;
       l_part[h] = 0.f;
     }
@@ -326,32 +364,32 @@ __device__ void softmax8(const TcParams& p, const Sync& sy, uint32_t sb, uint8_t
       ok = sy.wait_warp(G_SFULL + buf, (c >> 1) & 1u);
       if (!ok) break;
       tc_fence_after();
-      uint32_t rh[16], rl[16];
-      tmem_ld16(tl + kTS + buf * 32, rh);
-      tmem_ld16(tl + kTS + buf * 32 + 16, rl);
+      uint32_t rh[8], rl[8];
+      tmem_ld8(tl + kTS + buf * 32 + h0, rh);
+      tmem_ld8(tl + kTS + buf * 32 + 16 + h0, rl);
       tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(sy.bar(G_SFREE + buf));
-      float s[kGp];
+      float s[kHpw];
 #pragma unroll
-      for (int h = 0; h < kGp; ++h)
-        s[h] = (valid && h < G) ? fmaf(__uint_as_float(rl[h]), 0.0625f, __uint_as_float(rh[h])) * qs[h]
-                                : -INFINITY;
-      const float wmax = xreduce16<true>(s, lane);
+      for (int h = 0; h < kHpw; ++h)
+        s[h] = (valid && h0 + h < G) ? fmaf(__uint_as_float(rl[h]), 0.0625f, __uint_as_float(rh[h])) * qs[h]
+                                     : -INFINITY;
+      const float wmax = xreduce8<true>(s, lane);
       float* rm = red_max + buf * 64;
-      if ((lane & 1) == 0) rm[wq * 16 + ((lane >> 1) & 15)] = wmax;
+      if ((lane & 3) == 0) rm[wq * 16 + h0 + ((lane >> 2) & 7)] = wmax;
       __syncwarp();
       if (lane == 0) mbar_arrive(sy.bar(G_RMAX + buf));
       ok = sy.wait_warp(G_RMAX + buf, (c >> 1) & 1u);
       if (!ok) break;
-      float tmax[kGp];
+      float tmax[kHpw];
 #pragma unroll
-      for (int h = 0; h < kGp; ++h)
-        tmax[h] = fmaxf(fmaxf(rm[h], rm[16 + h]), fmaxf(rm[32 + h], rm[48 + h]));
+      for (int h = 0; h < kHpw; ++h)
+        tmax[h] = fmaxf(fmaxf(rm[h0 + h], rm[16 + h0 + h]), fmaxf(rm[32 + h0 + h], rm[48 + h0 + h]));
       bool need = false;
 #pragma unroll
-      for (int h = 0; h < kGp; ++h)
+      for (int h = 0; h < kHpw; ++h)
         need |= (m_run[h] != -INFINITY) && (tmax[h] > m_run[h] + kRescaleLog2);
       if (need) {
         if (i > 0) {
@@ -360,9 +398,9 @@ __device__ void softmax8(const TcParams& p, const Sync& sy, uint32_t sb, uint8_t
           if (!ok) break;
         }
         tc_fence_after();
-        float alpha[kGp];
+        float alpha[kHpw];
 #pragma unroll
-        for (int h = 0; h < kGp; ++h) {
+        for (int h = 0; h < kHpw; ++h) {
           const float mn = fmaxf(m_run[h], tmax[h]);
           alpha[h] = m_run[h] == -INFINITY ? 1.f : ex2(m_run[h] - mn);
           m_run[h] = mn;
@@ -370,25 +408,25 @@ __device__ void softmax8(const TcParams& p, const Sync& sy, uint32_t sb, uint8_t
         }
         if (i > 0) {
 #pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4) {          // O_hi, O_lo x two halves
-            uint32_t o[16];
-            tmem_ld16(tl + kTO + q4 * 16, o);
+          for (int q4 = 0; q4 < 4; ++q4) {          // O_hi, O_lo x two halves, this warp's heads
+            uint32_t o[8];
+            tmem_ld8(tl + kTO + q4 * 16 + h0, o);
             tmem_wait_ld();
 #pragma unroll
-            for (int h = 0; h < kGp; ++h) o[h] = __float_as_uint(__uint_as_float(o[h]) * alpha[h]);
-            tmem_st16(tl + kTO + q4 * 16, o);
+            for (int h = 0; h < kHpw; ++h) o[h] = __float_as_uint(__uint_as_float(o[h]) * alpha[h]);
+            tmem_st8(tl + kTO + q4 * 16 + h0, o);
           }
           tmem_wait_st();
         }
       } else {
 #pragma unroll
-        for (int h = 0; h < kGp; ++h)
+        for (int h = 0; h < kHpw; ++h)
           if (m_run[h] == -INFINITY) m_run[h] = tmax[h];
       }
       // p = p_hi + p_lo / 16, both E4M3 (p <= 2^8)
-      uint32_t ph[4], plo[4];
+      uint32_t ph[2], plo[2];
 #pragma unroll
-      for (int h4 = 0; h4 < 4; ++h4) {
+      for (int h4 = 0; h4 < 2; ++h4) {
         float pv[4];
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
@@ -407,35 +445,36 @@ __device__ void softmax8(const TcParams& p, const Sync& sy, uint32_t sb, uint8_t
       }
       ok = sy.wait_warp(G_PEMPTY + buf, ((c >> 1) & 1u) ^ 1u);
       if (!ok) break;
-      // P^T row of this key: 16 heads = 16 bytes, key k at 16 k
-      const uint32_t pa = sb + F_P8 + buf * 2 * kP8Bytes + key * 16;
-      st_shared_v4(pa, ph[0], ph[1], ph[2], ph[3]);
-      st_shared_v4(pa + kP8Bytes, plo[0], plo[1], plo[2], plo[3]);
+      // P^T row of this key: 16 heads = 16 bytes at 16 key; this warp's 8 heads at + 8 hh
+      const uint32_t pa = sb + F_P8 + buf * 2 * kP8Bytes + key * 16 + hh * 8;
+      asm volatile("st.shared.v2.b32 [%0], {%1, %2};\n" ::"r"(pa), "r"(ph[0]), "r"(ph[1]) : "memory");
+      asm volatile("st.shared.v2.b32 [%0], {%1, %2};\n" ::"r"(pa + kP8Bytes), "r"(plo[0]), "r"(plo[1]) : "memory");
       fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(sy.bar(G_PFULL + buf));
     }
     if (!ok) break;
-    const float wsum = xreduce16<false>(l_part, lane);
+    const float wsum = xreduce8<false>(l_part, lane);
     float* rs = red_sum + (c_unit & 1u) * 64;
-    if ((lane & 1) == 0) rs[wq * 16 + ((lane >> 1) & 15)] = wsum;
+    if ((lane & 3) == 0) rs[wq * 16 + h0 + ((lane >> 2) & 7)] = wsum;
     __syncwarp();
     if (lane == 0) mbar_arrive(sy.bar(G_RSUM + (c_unit & 1u)));
     ok = sy.wait_warp(G_RSUM + (c_unit & 1u), (c_unit >> 1) & 1u);
     if (!ok) break;
-    float l_tot[kGp];
+    float l_tot[kHpw];
 #pragma unroll
-    for (int h = 0; h < kGp; ++h) l_tot[h] = (rs[h] + rs[16 + h]) + (rs[32 + h] + rs[48 + h]);
+    for (int h = 0; h < kHpw; ++h)
+      l_tot[h] = (rs[h0 + h] + rs[16 + h0 + h]) + (rs[32 + h0 + h] + rs[48 + h0 + h]);
     ok = sy.wait_warp(G_OFULL, c_unit & 1u);
     if (!ok) break;
     tc_fence_after();
-    uint32_t oh0[16] = {}, oh1[16] = {}, ol0[16] = {}, ol1[16] = {};
+    uint32_t oh0[8] = {}, oh1[8] = {}, ol0[8] = {}, ol1[8] = {};
     if (un.n_tiles > 0) {
-      tmem_ld16(tl + kTO, oh0);
-      tmem_ld16(tl + kTO + 16, oh1);
-      tmem_ld16(tl + kTO + 32, ol0);
-      tmem_ld16(tl + kTO + 48, ol1);
+      tmem_ld8(tl + kTO + h0, oh0);          // half 0: O_hi, O_lo
+      tmem_ld8(tl + kTO + 16 + h0, ol0);
+      tmem_ld8(tl + kTO + 32 + h0, oh1);     // half 1
+      tmem_ld8(tl + kTO + 48 + h0, ol1);
       tmem_wait_ld();
     }
     tc_fence_before();
@@ -444,36 +483,37 @@ __device__ void softmax8(const TcParams& p, const Sync& sy, uint32_t sb, uint8_t
     const int64_t row0 = un.t * static_cast<int64_t>(p.Hkv) * G + static_cast<int64_t>(un.g) * G;
     __nv_bfloat16* orow = p.out + un.t * p.o_st + static_cast<int64_t>(un.g) * G * p.o_sh;
 #pragma unroll
-    for (int h = 0; h < kGp; ++h) {
-      if (h < G) {
+    for (int h = 0; h < kHpw; ++h) {
+      const int hg = h0 + h;
+      if (hg < G) {
         const bool live = l_tot[h] > 0.f;
         const float inv = live ? p.o_scale / l_tot[h] : 0.f;
         const float v0 = live ? fmaf(__uint_as_float(ol0[h]), 0.0625f, __uint_as_float(oh0[h])) * inv : 0.f;
         const float v1 = live ? fmaf(__uint_as_float(ol1[h]), 0.0625f, __uint_as_float(oh1[h])) * inv : 0.f;
         if (p.part_o != nullptr) {
           // split-K: this chunk's normalised partial output, for the merge
-          float* po = p.part_o + ((row0 + h) * p.splits + un.s) * 256;
+          float* po = p.part_o + ((row0 + hg) * p.splits + un.s) * 256;
           po[key] = v0;
           po[128 + key] = v1;
         } else {
-          orow[h * p.o_sh + key] = __float2bfloat16_rn(v0);
-          orow[h * p.o_sh + 128 + key] = __float2bfloat16_rn(v1);
+          orow[hg * p.o_sh + key] = __float2bfloat16_rn(v0);
+          orow[hg * p.o_sh + 128 + key] = __float2bfloat16_rn(v1);
         }
       }
     }
-    if (key < G && (p.lse != nullptr || p.part_lse != nullptr)) {
+    if (wq == 0 && lane < kHpw && h0 + lane < G && (p.lse != nullptr || p.part_lse != nullptr)) {
       float mk = 0.f, lk = 0.f;
 #pragma unroll
-      for (int h = 0; h < kGp; ++h)
-        if (h == key) {
+      for (int h = 0; h < kHpw; ++h)
+        if (h == lane) {
           mk = m_run[h];
           lk = l_tot[h];
         }
       const float lv = lk > 0.f ? (mk + lg2(lk)) * 0.69314718055994531f : -INFINITY;
       if (p.part_lse != nullptr)
-        p.part_lse[(row0 + key) * p.splits + un.s] = lv;
+        p.part_lse[(row0 + h0 + lane) * p.splits + un.s] = lv;
       else
-        p.lse[un.t * p.lse_st + static_cast<int64_t>(un.g) * G + key] = lv;
+        p.lse[un.t * p.lse_st + static_cast<int64_t>(un.g) * G + h0 + lane] = lv;
     }
     c_tile += un.n_tiles;
     ++c_unit;
@@ -483,7 +523,7 @@ __device__ void softmax8(const TcParams& p, const Sync& sy, uint32_t sb, uint8_t
 // ------------------------------------------------------------------ kernel
 
 template <bool kBlocks>
-__global__ void __launch_bounds__(kThreads, 1) qsa_prefill_f8_kernel(const __grid_constant__ TcParams p) {
+__global__ void __launch_bounds__(kThreads8, 1) qsa_prefill_f8_kernel(const __grid_constant__ TcParams p) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t sb = (raw + 1023u) & ~1023u;
@@ -501,16 +541,16 @@ __global__ void __launch_bounds__(kThreads, 1) qsa_prefill_f8_kernel(const __gri
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(sy.bar(G_SFULL + b), 1);
-      mbar_init(sy.bar(G_SFREE + b), 4);
-      mbar_init(sy.bar(G_PFULL + b), 4);
+      mbar_init(sy.bar(G_SFREE + b), kSmWarps);
+      mbar_init(sy.bar(G_PFULL + b), kSmWarps);
       mbar_init(sy.bar(G_PEMPTY + b), 1);
       mbar_init(sy.bar(G_QFULL + b), 1);
-      mbar_init(sy.bar(G_QEMPTY + b), 1 + 4);   // the MMAs, and each softmax warp
-      mbar_init(sy.bar(G_RMAX + b), 4);
-      mbar_init(sy.bar(G_RSUM + b), 4);
+      mbar_init(sy.bar(G_QEMPTY + b), 1 + kSmWarps);   // the MMAs, and each softmax warp
+      mbar_init(sy.bar(G_RMAX + b), kSmWarps);
+      mbar_init(sy.bar(G_RSUM + b), kSmWarps);
     }
     mbar_init(sy.bar(G_OFULL), 1);
-    mbar_init(sy.bar(G_OEMPTY), 4);
+    mbar_init(sy.bar(G_OEMPTY), kSmWarps);
     mbar_init(sy.bar(G_DONE), 1);
     mbar_init(sy.bar(G_DONE + 1), 1);
     *sy.abort_flag = 0u;
