@@ -55,11 +55,11 @@ constexpr int F_RING = 0;
 constexpr int F_Q8 = F_RING + kSlots8 * kSlotBytes;   // 2 buffers x {hi, lo}
 constexpr int F_P8 = F_Q8 + 2 * 2 * kQ8Bytes;         // 2 buffers x {hi, lo}
 constexpr int F_QSC = F_P8 + 2 * 2 * kP8Bytes;        // 2 buffers x 16 per-head score factors
-constexpr int F_RED = F_QSC + 2 * kGp * 4;            // max[2][4][16] + sum[2][4][16]
+constexpr int F_RED = F_QSC + 2 * kGp * 4;            // max[4][16], votes[2][8], sum[2][4][16]
 constexpr int F_BAR = F_RED + 1024;
 constexpr int G_FULL = 0, G_EMPTY = 6, G_SFULL = 12, G_SFREE = 14, G_PFULL = 16, G_PEMPTY = 18,
               G_QFULL = 20, G_QEMPTY = 22, G_OFULL = 24, G_OEMPTY = 25, G_RMAX = 26, G_RSUM = 28,
-              G_DONE = 30, G_NUM = 32;
+              G_DONE = 30, G_RMX2 = 32, G_NUM = 33;
 constexpr int F_MISC = F_BAR + G_NUM * 8;             // tmem base, abort flag
 constexpr int F_SMEM = F_MISC + 16 + 1024;
 
@@ -317,6 +317,29 @@ __device__ __forceinline__ float xreduce8(const float (&v)[8], int lane) {
   return c;
 }
 
+// p = 2^(s - m) for this thread's key and 8 heads as p = p_hi + p_lo / 16,
+// both E4M3 (p <= 2^8), packed 4 heads per word; pv gets the p themselves.
+__device__ __forceinline__ void form_p(const float (&s)[kHpw], const float (&m)[kHpw], uint32_t (&ph)[2],
+                                       uint32_t (&plo)[2], float (&pv)[kHpw]) {
+#pragma unroll
+  for (int h4 = 0; h4 < 2; ++h4) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int h = 4 * h4 + j;
+      pv[h] = ex2(s[h] - (m[h] == -INFINITY ? 0.f : m[h]));
+    }
+    const float* x = pv + 4 * h4;
+    const uint32_t h01 = pack_e4m3x2(x[0], x[1]), h23 = pack_e4m3x2(x[2], x[3]);
+    float y0, y1, y2, y3;
+    f16x2_to_f32(e4m3x2_to_f16x2(h01), y0, y1);
+    f16x2_to_f32(e4m3x2_to_f16x2(h23), y2, y3);
+    const uint32_t l01 = pack_e4m3x2((x[0] - y0) * 16.f, (x[1] - y1) * 16.f);
+    const uint32_t l23 = pack_e4m3x2((x[2] - y2) * 16.f, (x[3] - y3) * 16.f);
+    ph[h4] = h01 | (h23 << 16);
+    plo[h4] = l01 | (l23 << 16);
+  }
+}
+
 // Softmax warp w (6..13): TMEM lane quadrant q = w & 3 (thread = key of the
 // tile, and dim of an output half), heads [8 hh, 8 hh + 8) with hh = (w-6)/4.
 template <bool kBlocks>
@@ -328,9 +351,10 @@ __device__ void softmax8(const TcParams& p, const Sync& sy, uint32_t sb, uint8_t
   const int key = wq * 32 + lane;
   const uint32_t tl = tmem + (static_cast<uint32_t>(wq * 32) << 16);
   float* red_max = reinterpret_cast<float*>(sp + F_RED);
+  uint8_t* votes = sp + F_RED + 256;
   float* red_sum = red_max + 128;
   const float* qsc_all = reinterpret_cast<const float*>(sp + F_QSC);
-  uint32_t c_tile = 0, c_unit = 0;
+  uint32_t c_tile = 0, c_unit = 0, c_exact = 0;
   const int64_t units = num_units(p);
   const int G = p.G;
   bool ok = true;
@@ -372,77 +396,82 @@ __device__ void softmax8(const TcParams& p, const Sync& sy, uint32_t sb, uint8_t
       __syncwarp();
       if (lane == 0) mbar_arrive(sy.bar(G_SFREE + buf));
       float s[kHpw];
+      bool over = false;
 #pragma unroll
-      for (int h = 0; h < kHpw; ++h)
+      for (int h = 0; h < kHpw; ++h) {
         s[h] = (valid && h0 + h < G) ? fmaf(__uint_as_float(rl[h]), 0.0625f, __uint_as_float(rh[h])) * qs[h]
                                      : -INFINITY;
-      const float wmax = xreduce8<true>(s, lane);
-      float* rm = red_max + buf * 64;
-      if ((lane & 3) == 0) rm[wq * 16 + h0 + ((lane >> 2) & 7)] = wmax;
+        over |= s[h] > m_run[h] + kRescaleLog2;
+      }
+      // Most tiles hold no score above the running max plus the lazy-rescale
+      // bound.  Each warp votes on that, then forms P from the running max
+      // while the other warps' votes arrive; only a yes anywhere (the first
+      // tile of a unit, a real rescale) makes the warps combine the exact
+      // tile max and form P again.
+      const bool wover = __any_sync(0xffffffffu, over);
+      uint8_t* vt = votes + buf * 8;
+      if (lane == 0) vt[warp - kWarpSoftmax0] = wover ? 1 : 0;
       __syncwarp();
       if (lane == 0) mbar_arrive(sy.bar(G_RMAX + buf));
+      uint32_t ph[2], plo[2];
+      float pv[kHpw];
+      if (!wover) form_p(s, m_run, ph, plo, pv);
       ok = sy.wait_warp(G_RMAX + buf, (c >> 1) & 1u);
       if (!ok) break;
-      float tmax[kHpw];
-#pragma unroll
-      for (int h = 0; h < kHpw; ++h)
-        tmax[h] = fmaxf(fmaxf(rm[h0 + h], rm[16 + h0 + h]), fmaxf(rm[32 + h0 + h], rm[48 + h0 + h]));
-      bool need = false;
-#pragma unroll
-      for (int h = 0; h < kHpw; ++h)
-        need |= (m_run[h] != -INFINITY) && (tmax[h] > m_run[h] + kRescaleLog2);
-      if (need) {
-        if (i > 0) {
-          const uint32_t cp = c - 1;
-          ok = sy.wait_warp(G_PEMPTY + (cp & 1u), (cp >> 1) & 1u);
-          if (!ok) break;
-        }
-        tc_fence_after();
-        float alpha[kHpw];
-#pragma unroll
-        for (int h = 0; h < kHpw; ++h) {
-          const float mn = fmaxf(m_run[h], tmax[h]);
-          alpha[h] = m_run[h] == -INFINITY ? 1.f : ex2(m_run[h] - mn);
-          m_run[h] = mn;
-          l_part[h] *= alpha[h];
-        }
-        if (i > 0) {
-#pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4) {          // O_hi, O_lo x two halves, this warp's heads
-            uint32_t o[8];
-            tmem_ld8(tl + kTO + q4 * 16 + h0, o);
-            tmem_wait_ld();
-#pragma unroll
-            for (int h = 0; h < kHpw; ++h) o[h] = __float_as_uint(__uint_as_float(o[h]) * alpha[h]);
-            tmem_st8(tl + kTO + q4 * 16 + h0, o);
-          }
-          tmem_wait_st();
-        }
-      } else {
+      const uint2 vw = *reinterpret_cast<const uint2*>(vt);
+      if ((vw.x | vw.y) != 0u) {
+        const float wmax = xreduce8<true>(s, lane);
+        float* rm = red_max;
+        if ((lane & 3) == 0) rm[wq * 16 + h0 + ((lane >> 2) & 7)] = wmax;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(sy.bar(G_RMX2));
+        ok = sy.wait_warp(G_RMX2, c_exact & 1u);
+        ++c_exact;
+        if (!ok) break;
+        float tmax[kHpw];
 #pragma unroll
         for (int h = 0; h < kHpw; ++h)
-          if (m_run[h] == -INFINITY) m_run[h] = tmax[h];
-      }
-      // p = p_hi + p_lo / 16, both E4M3 (p <= 2^8)
-      uint32_t ph[2], plo[2];
+          tmax[h] = fmaxf(fmaxf(rm[h0 + h], rm[16 + h0 + h]), fmaxf(rm[32 + h0 + h], rm[48 + h0 + h]));
+        bool need = false;
 #pragma unroll
-      for (int h4 = 0; h4 < 2; ++h4) {
-        float pv[4];
+        for (int h = 0; h < kHpw; ++h)
+          need |= (m_run[h] != -INFINITY) && (tmax[h] > m_run[h] + kRescaleLog2);
+        if (need) {
+          if (i > 0) {
+            const uint32_t cp = c - 1;
+            ok = sy.wait_warp(G_PEMPTY + (cp & 1u), (cp >> 1) & 1u);
+            if (!ok) break;
+          }
+          tc_fence_after();
+          float alpha[kHpw];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int h = 4 * h4 + j;
-          pv[j] = ex2(s[h] - (m_run[h] == -INFINITY ? 0.f : m_run[h]));
-          l_part[h] += pv[j];
+          for (int h = 0; h < kHpw; ++h) {
+            const float mn = fmaxf(m_run[h], tmax[h]);
+            alpha[h] = m_run[h] == -INFINITY ? 1.f : ex2(m_run[h] - mn);
+            m_run[h] = mn;
+            l_part[h] *= alpha[h];
+          }
+          if (i > 0) {
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) {          // O_hi, O_lo x two halves, this warp's heads
+              uint32_t o[8];
+              tmem_ld8(tl + kTO + q4 * 16 + h0, o);
+              tmem_wait_ld();
+#pragma unroll
+              for (int h = 0; h < kHpw; ++h) o[h] = __float_as_uint(__uint_as_float(o[h]) * alpha[h]);
+              tmem_st8(tl + kTO + q4 * 16 + h0, o);
+            }
+            tmem_wait_st();
+          }
+        } else {
+#pragma unroll
+          for (int h = 0; h < kHpw; ++h)
+            if (m_run[h] == -INFINITY) m_run[h] = tmax[h];
         }
-        const uint32_t h01 = pack_e4m3x2(pv[0], pv[1]), h23 = pack_e4m3x2(pv[2], pv[3]);
-        float y0, y1, y2, y3;
-        f16x2_to_f32(e4m3x2_to_f16x2(h01), y0, y1);
-        f16x2_to_f32(e4m3x2_to_f16x2(h23), y2, y3);
-        const uint32_t l01 = pack_e4m3x2((pv[0] - y0) * 16.f, (pv[1] - y1) * 16.f);
-        const uint32_t l23 = pack_e4m3x2((pv[2] - y2) * 16.f, (pv[3] - y3) * 16.f);
-        ph[h4] = h01 | (h23 << 16);
-        plo[h4] = l01 | (l23 << 16);
+        form_p(s, m_run, ph, plo, pv);
       }
+#pragma unroll
+      for (int h = 0; h < kHpw; ++h) l_part[h] += pv[h];
       ok = sy.wait_warp(G_PEMPTY + buf, ((c >> 1) & 1u) ^ 1u);
       if (!ok) break;
       // P^T row of this key: 16 heads = 16 bytes at 16 key; this warp's 8 heads at + 8 hh
@@ -549,6 +578,7 @@ __global__ void __launch_bounds__(kThreads8, 1) qsa_prefill_f8_kernel(const __gr
       mbar_init(sy.bar(G_RMAX + b), kSmWarps);
       mbar_init(sy.bar(G_RSUM + b), kSmWarps);
     }
+    mbar_init(sy.bar(G_RMX2), kSmWarps);
     mbar_init(sy.bar(G_OFULL), 1);
     mbar_init(sy.bar(G_OEMPTY), kSmWarps);
     mbar_init(sy.bar(G_DONE), 1);
