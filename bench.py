@@ -552,6 +552,18 @@ def run_cuda(args):
                            "tokens_per_s": T * n_cmp * world / (cmp_ms / 1e3),
                            "mean_launch_ms": statistics.mean(cmp_per),
                            "algo_gbs": acct["algo_bytes"] / (statistics.mean(cmp_per) / 1e3) / 1e9}
+    if not args.profile and args.kernel in ("auto", "tcgen05"):
+        # the same lists through the kernel's gather step alone: the floor of
+        # the timed kernel on this workload
+        def step_gather():
+            _capi.sparse_prefill_fwd(w.q, w.k_cache, w.v_cache, w.topk_idx, w.n_valid, w.scale,
+                                     out=out, lse=lse, kernel="gather_only")
+        n_g = min(args.steps, 20)
+        g_ms, g_per, _ = time_launches(step_gather, n_g, 3, barrier, "gather_only")
+        g_mean = statistics.mean(g_per)
+        line["gather_floor"] = {"kernel": "qsa_gather_only_kernel", "mean_launch_ms": g_mean,
+                                "gathered_kv_gbs": acct["gathered_bytes"] / (g_mean / 1e3) / 1e9,
+                                "kernel_frac_of_floor": g_mean / mean_launch_ms, "launches": n_g}
     if not args.no_e2e and not args.profile:
         line["e2e"] = run_e2e(w, args, barrier, max_ranks, T_job, dev)
     if args.secondary and not args.profile and args.secondary != args.workload:

@@ -113,7 +113,13 @@ typedef enum {
                                0 < S < 2^31 - 1), otherwise the warp-MMA kernel */
   QSA_KERNEL_TCGEN05 = 1,   /* persistent warp-specialised cp.async-gather + tcgen05/TMEM
                                kernel only (QSA_ERR_UNSUPPORTED when the layout does not fit) */
-  QSA_KERNEL_WARP_MMA = 2   /* cp.async-gather + mma.sync kernel (any valid layout) */
+  QSA_KERNEL_WARP_MMA = 2,  /* cp.async-gather + mma.sync kernel (any valid layout) */
+  QSA_KERNEL_GATHER_ONLY = 3 /* measurement only: the KV gather of the tcgen05 kernel alone
+                               (its producer warps, ring and Q loads; the slots are handed
+                               back unread).  Writes neither out nor lse; the status word
+                               still receives out-of-range ids.  Its time is the floor of
+                               the tcgen05 kernel on the same lists.  QSA_ERR_UNSUPPORTED
+                               where QSA_KERNEL_TCGEN05 is. */
 } qsa_kernel_t;
 
 /* Same contract as qsa_sparse_prefill_fwd, with an explicit kernel choice.

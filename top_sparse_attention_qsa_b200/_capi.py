@@ -26,8 +26,9 @@ QSA_OK, QSA_ERR_NULL, QSA_ERR_SHAPE, QSA_ERR_UNSUPPORTED, QSA_ERR_ALIGN, QSA_ERR
 NOALLOC_SCRATCH_BYTES = 16 << 20
 STATUS_OOB_SLOT = 1
 STATUS_TIMEOUT = 2
-KERNEL_AUTO, KERNEL_TCGEN05, KERNEL_WARP_MMA = 0, 1, 2
-KERNELS = {"auto": KERNEL_AUTO, "tcgen05": KERNEL_TCGEN05, "warp_mma": KERNEL_WARP_MMA}
+KERNEL_AUTO, KERNEL_TCGEN05, KERNEL_WARP_MMA, KERNEL_GATHER_ONLY = 0, 1, 2, 3
+KERNELS = {"auto": KERNEL_AUTO, "tcgen05": KERNEL_TCGEN05, "warp_mma": KERNEL_WARP_MMA,
+           "gather_only": KERNEL_GATHER_ONLY}
 HEAD_DIM = 256
 
 # Every symbol include/qsa.h declares.
@@ -194,7 +195,8 @@ def sparse_prefill_fwd(q, k_cache, v_cache, topk_idx, n_valid=None, scale: float
                        out=None, lse=None, status=None, stream=None, want_lse: bool = True,
                        kernel: str = "auto"):
     """QSA sparse prefill on the GPU.  Returns (out [T,Hq,D] bf16, lse [T,Hq] fp32 or None).
-    kernel: "auto" | "tcgen05" | "warp_mma" (see qsa_kernel_t)."""
+    kernel: "auto" | "tcgen05" | "warp_mma" | "gather_only" (see qsa_kernel_t; the last
+    runs only the KV gather, for measurement, and leaves out and lse untouched)."""
     dev = q.device
     _need(q, "q", torch.bfloat16, dev)
     _need(k_cache, "k_cache", torch.bfloat16, dev)

@@ -13,6 +13,7 @@
 
 #include "qsa.h"
 #include "qsa_host.cuh"
+#include "qsa_gather_only.cuh"
 #include "qsa_merge.cuh"
 #include "qsa_prefill_mma.cuh"
 #include "qsa_prefill_tc.cuh"
@@ -111,6 +112,19 @@ cudaError_t launch_f8(const qsa::tc::TcParams& tp, cudaStream_t stream) {
   return cudaGetLastError();
 }
 
+cudaError_t launch_gather_only(const qsa::tc::TcParams& tp, cudaStream_t stream) {
+  static std::atomic<int> done[kMaxDevices];
+  auto kernel = qsa::tc::qsa_gather_only_kernel;
+  cudaError_t e = set_smem_once(kernel, qsa::tc::SMEM_BYTES, done);
+  if (e != cudaSuccess) return e;
+  const int64_t units = tp.T * tp.Hkv;
+  const int nsm = sm_count();
+  if (nsm <= 0) return cudaErrorInvalidDevice;
+  const unsigned grid = static_cast<unsigned>(units < nsm ? units : nsm);
+  kernel<<<grid, qsa::tc::kGatherOnlyThreads, qsa::tc::SMEM_BYTES, stream>>>(tp);
+  return cudaGetLastError();
+}
+
 template <bool kDump, bool kStall = false, bool kBlocks = false>
 cudaError_t launch_tc(const qsa::tc::TcParams& tp, cudaStream_t stream) {
   static std::atomic<int> done[kMaxDevices];
@@ -129,8 +143,10 @@ qsa_status_t run_forward(const qsa_shape_t* s, const void* q, const void* k, con
                          const int32_t* idx, const int32_t* n_valid, float scale, void* out,
                          float* lse, int32_t* status, int32_t* gathered, void* stream,
                          qsa_kernel_t which = QSA_KERNEL_AUTO, bool stall_test = false) {
-  if (which != QSA_KERNEL_AUTO && which != QSA_KERNEL_TCGEN05 && which != QSA_KERNEL_WARP_MMA)
+  if (which != QSA_KERNEL_AUTO && which != QSA_KERNEL_TCGEN05 && which != QSA_KERNEL_WARP_MMA &&
+      which != QSA_KERNEL_GATHER_ONLY)
     return QSA_ERR_UNSUPPORTED;
+  if (which == QSA_KERNEL_GATHER_ONLY && (gathered != nullptr || stall_test)) return QSA_ERR_UNSUPPORTED;
   qsa_status_t rc = validate(s, q, k, v, idx, out);
   if (rc != QSA_OK) return rc;
   if (gathered != nullptr && s->topk > 0 && (reinterpret_cast<uintptr_t>(gathered) & 3u))
@@ -171,7 +187,7 @@ qsa_status_t run_forward(const qsa_shape_t* s, const void* q, const void* k, con
   const bool dump = gathered != nullptr;
   static thread_local qsa::tc::TcParams tp;
   const bool use_tc = which != QSA_KERNEL_WARP_MMA && make_tc_params(s, q, &tp);
-  if (which == QSA_KERNEL_TCGEN05 && !use_tc) return QSA_ERR_UNSUPPORTED;
+  if ((which == QSA_KERNEL_TCGEN05 || which == QSA_KERNEL_GATHER_ONLY) && !use_tc) return QSA_ERR_UNSUPPORTED;
   if (use_tc) {
     tp.idx = idx;
     tp.n_valid = n_valid;
@@ -201,8 +217,11 @@ qsa_status_t run_forward(const qsa_shape_t* s, const void* q, const void* k, con
     tp.block_shift = 0;
     tp.last_slot = nullptr;
     tp.o_scale = 1.f;
-    e = stall_test ? launch_tc<false, true>(tp, st)
-                   : (dump ? launch_tc<true>(tp, st) : launch_tc<false>(tp, st));
+    if (which == QSA_KERNEL_GATHER_ONLY)
+      e = launch_gather_only(tp, st);
+    else
+      e = stall_test ? launch_tc<false, true>(tp, st)
+                     : (dump ? launch_tc<true>(tp, st) : launch_tc<false>(tp, st));
   } else if (p.G <= 8)
     e = dump ? launch_mma<1, true>(p, st) : launch_mma<1, false>(p, st);
   else

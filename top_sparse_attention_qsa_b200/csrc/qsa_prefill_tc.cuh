@@ -23,12 +23,14 @@
 //               (two M=128 halves, V read MN-major from the same slots) into
 //               TMEM.  Two issuers keep PV of tile i from queueing behind the
 //               scores of tile i+1.
-//   warps 6-9   softmax: thread k owns TMEM lane k = key k of the tile; tile
-//               max per head by a transposing shuffle reduction and a 4-warp
-//               exchange; exponentials in base 2; P^T written MN-major to
-//               shared memory; the running max is only raised (with an O
-//               rescale in TMEM) when a head's max grows by more than 2^8,
-//               which keeps every p <= 256 and the result exact up to rounding.
+//   warps 6-9   softmax: thread k owns TMEM lane k = key k of the tile;
+//               exponentials in base 2 from the running max; P^T written
+//               MN-major to shared memory; the running max is only raised
+//               (with an O rescale in TMEM) when a head's max grows by more
+//               than 2^8, which keeps every p <= 256 and the result exact up
+//               to rounding.  A warp vote per tile detects that case; only
+//               then is the tile max per head formed (a transposing shuffle
+//               reduction and a 4-warp exchange).
 //               Epilogue: lse = m + ln l, O / l -> BF16 rows, zeros for empty rows.
 // Every wait (all on mbarriers, including the exchanges inside the softmax
 // group) is bounded by 2 s of %globaltimer; on expiry the kernel raises status
@@ -68,12 +70,12 @@ constexpr float kRescaleLog2 = 8.f;        // lazy-rescale threshold (p <= 2^8)
 constexpr int OFF_RING = 0;
 constexpr int OFF_Q = OFF_RING + kSlots * kSlotBytes;
 constexpr int OFF_P = OFF_Q + 2 * kQBytes;
-constexpr int OFF_RED = OFF_P + 2 * kPBytes;     // max[2][4][16] + sum[2][4][16] floats
+constexpr int OFF_RED = OFF_P + 2 * kPBytes;     // max[4][16], votes[2][4], sum[2][4][16]
 constexpr int OFF_BAR = OFF_RED + 1024;
 // barrier indices
 constexpr int B_FULL = 0, B_EMPTY = 6, B_SFULL = 12, B_SFREE = 14, B_PFULL = 16, B_PEMPTY = 18,
               B_QFULL = 20, B_QEMPTY = 22, B_OFULL = 24, B_OEMPTY = 25, B_RMAX = 26, B_RSUM = 28,
-              B_DONE = 30, NUM_BARS = 32;
+              B_DONE = 30, B_RMX2 = 32, NUM_BARS = 33;
 constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;  // tmem base, abort flag
 constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + slack for 1024-byte alignment
 
@@ -401,15 +403,28 @@ __device__ void pv_role(const TcParams& p, const Sync& sy, uint32_t sb, uint32_t
 
 // ------------------------------------------------------------------ softmax
 
+// p = 2^(s - m) for this thread's key and 16 heads, as BF16 pairs; pv gets
+// the unrounded p for the running sums.
+__device__ __forceinline__ void form_p16(const float (&s)[kGp], const float (&m)[kGp], uint32_t (&pk)[8],
+                                         float (&pv)[kGp]) {
+#pragma unroll
+  for (int h = 0; h < kGp; h += 2) {
+    pv[h] = ex2(s[h] - (m[h] == -INFINITY ? 0.f : m[h]));
+    pv[h + 1] = ex2(s[h + 1] - (m[h + 1] == -INFINITY ? 0.f : m[h + 1]));
+    pk[h >> 1] = pack_bf16x2(pv[h], pv[h + 1]);
+  }
+}
+
 template <bool kBlocks>
 __device__ void softmax_role(const TcParams& p, const Sync& sy, uint32_t sb, uint8_t* sp,
                              uint32_t tmem, int warp, int lane) {
   const int wq = warp & 3;                       // TMEM lane quadrant of this warp
   const int key = wq * 32 + lane;                // TMEM lane = key row of the tile
   const uint32_t tl = tmem + (static_cast<uint32_t>(wq * 32) << 16);
-  float* red_max = reinterpret_cast<float*>(sp + OFF_RED);        // [2][4][16]
+  float* red_max = reinterpret_cast<float*>(sp + OFF_RED);        // [4][16]
+  uint8_t* votes = sp + OFF_RED + 256;                             // [2][4]
   float* red_sum = red_max + 128;                                  // [2][4][16]
-  uint32_t c_tile = 0, c_unit = 0;
+  uint32_t c_tile = 0, c_unit = 0, c_exact = 0;
   const int64_t units = num_units(p);
   const int G = p.G;
   bool ok = true;
@@ -441,67 +456,83 @@ __device__ void softmax_role(const TcParams& p, const Sync& sy, uint32_t sb, uin
       __syncwarp();
       if (lane == 0) mbar_arrive(sy.bar(B_SFREE + buf));
       float s[kGp];
+      bool over = false;
 #pragma unroll
-      for (int h = 0; h < kGp; ++h)
+      for (int h = 0; h < kGp; ++h) {
         s[h] = (valid && h < G) ? __uint_as_float(r[h]) * p.scale_log2 : -INFINITY;
-      // tile max per head over the 128 keys
-      const float wmax = xreduce16<true>(s, lane);
-      float* rm = red_max + buf * 64;
-      if ((lane & 1) == 0) rm[wq * 16 + ((lane >> 1) & 15)] = wmax;
+        over |= s[h] > m_run[h] + kRescaleLog2;
+      }
+      // Most tiles hold no score above the running max plus the lazy-rescale
+      // bound.  Each warp votes on that and forms P from the running max
+      // while the other votes arrive; only a yes anywhere (the first tile of
+      // a unit, a real rescale) makes the warps exchange exact tile maxima
+      // and form P again.  P always uses the running max, so the result is
+      // the same either way.
+      const bool wover = __any_sync(0xffffffffu, over);
+      uint8_t* vt = votes + buf * 4;
+      if (lane == 0) vt[wq] = wover ? 1 : 0;
       __syncwarp();
       if (lane == 0) mbar_arrive(sy.bar(B_RMAX + buf));
-      ok = sy.wait_warp(B_RMAX + buf, (c >> 1) & 1u);  // all four warps' maxima are in
+      uint32_t pk[8];
+      float pv[kGp];
+      if (!wover) form_p16(s, m_run, pk, pv);
+      ok = sy.wait_warp(B_RMAX + buf, (c >> 1) & 1u);  // all four votes are in
       if (!ok) break;
-      float tmax[kGp];
-#pragma unroll
-      for (int h = 0; h < kGp; ++h)
-        tmax[h] = fmaxf(fmaxf(rm[h], rm[16 + h]), fmaxf(rm[32 + h], rm[48 + h]));
-      bool need = false;
-#pragma unroll
-      for (int h = 0; h < kGp; ++h)
-        need |= (m_run[h] != -INFINITY) && (tmax[h] > m_run[h] + kRescaleLog2);
-      if (need) {
-        // raise the running max: O (TMEM) and the partial sums scale by 2^(m_old - m_new)
-        if (i > 0) {
-          const uint32_t cp = c - 1;
-          ok = sy.wait_warp(B_PEMPTY + (cp & 1u), (cp >> 1) & 1u);  // the previous PV has finished
-          if (!ok) break;
-        }
-        tc_fence_after();
-        float alpha[kGp];
-#pragma unroll
-        for (int h = 0; h < kGp; ++h) {
-          const float mn = fmaxf(m_run[h], tmax[h]);
-          alpha[h] = m_run[h] == -INFINITY ? 1.f : ex2(m_run[h] - mn);
-          m_run[h] = mn;
-          l_part[h] *= alpha[h];
-        }
-        if (i > 0) {
-#pragma unroll
-          for (int half = 0; half < 2; ++half) {
-            uint32_t o[16];
-            tmem_ld16(tl + 32 + half * 16, o);
-            tmem_wait_ld();
-#pragma unroll
-            for (int h = 0; h < kGp; ++h) o[h] = __float_as_uint(__uint_as_float(o[h]) * alpha[h]);
-            tmem_st16(tl + 32 + half * 16, o);
-          }
-          tmem_wait_st();
-        }
-      } else {
+      if (*reinterpret_cast<const uint32_t*>(vt) != 0u) {
+        // tile max per head over the 128 keys
+        const float wmax = xreduce16<true>(s, lane);
+        float* rm = red_max;
+        if ((lane & 1) == 0) rm[wq * 16 + ((lane >> 1) & 15)] = wmax;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(sy.bar(B_RMX2));
+        ok = sy.wait_warp(B_RMX2, c_exact & 1u);  // all four warps' maxima are in
+        ++c_exact;
+        if (!ok) break;
+        float tmax[kGp];
 #pragma unroll
         for (int h = 0; h < kGp; ++h)
-          if (m_run[h] == -INFINITY) m_run[h] = tmax[h];
-      }
-      uint32_t pk[8];
+          tmax[h] = fmaxf(fmaxf(rm[h], rm[16 + h]), fmaxf(rm[32 + h], rm[48 + h]));
+        bool need = false;
 #pragma unroll
-      for (int h = 0; h < kGp; h += 2) {
-        const float p0 = ex2(s[h] - (m_run[h] == -INFINITY ? 0.f : m_run[h]));
-        const float p1 = ex2(s[h + 1] - (m_run[h + 1] == -INFINITY ? 0.f : m_run[h + 1]));
-        l_part[h] += p0;
-        l_part[h + 1] += p1;
-        pk[h >> 1] = pack_bf16x2(p0, p1);
+        for (int h = 0; h < kGp; ++h)
+          need |= (m_run[h] != -INFINITY) && (tmax[h] > m_run[h] + kRescaleLog2);
+        if (need) {
+          // raise the running max: O (TMEM) and the partial sums scale by 2^(m_old - m_new)
+          if (i > 0) {
+            const uint32_t cp = c - 1;
+            ok = sy.wait_warp(B_PEMPTY + (cp & 1u), (cp >> 1) & 1u);  // the previous PV has finished
+            if (!ok) break;
+          }
+          tc_fence_after();
+          float alpha[kGp];
+#pragma unroll
+          for (int h = 0; h < kGp; ++h) {
+            const float mn = fmaxf(m_run[h], tmax[h]);
+            alpha[h] = m_run[h] == -INFINITY ? 1.f : ex2(m_run[h] - mn);
+            m_run[h] = mn;
+            l_part[h] *= alpha[h];
+          }
+          if (i > 0) {
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+              uint32_t o[16];
+              tmem_ld16(tl + 32 + half * 16, o);
+              tmem_wait_ld();
+#pragma unroll
+              for (int h = 0; h < kGp; ++h) o[h] = __float_as_uint(__uint_as_float(o[h]) * alpha[h]);
+              tmem_st16(tl + 32 + half * 16, o);
+            }
+            tmem_wait_st();
+          }
+        } else {
+#pragma unroll
+          for (int h = 0; h < kGp; ++h)
+            if (m_run[h] == -INFINITY) m_run[h] = tmax[h];
+        }
+        form_p16(s, m_run, pk, pv);
       }
+#pragma unroll
+      for (int h = 0; h < kGp; ++h) l_part[h] += pv[h];
       ok = sy.wait_warp(B_PEMPTY + buf, ((c >> 1) & 1u) ^ 1u);
       if (!ok) break;
       // P^T row of this key: heads 0-7 in the first 8x8 core-matrix column,
@@ -606,6 +637,7 @@ __global__ void __launch_bounds__(kThreads, 1) qsa_prefill_tc_kernel(const __gri
     for (int b = 0; b < 2; ++b) {
       mbar_init(sy.bar(B_RMAX + b), 4);
       mbar_init(sy.bar(B_RSUM + b), 4);
+      if (b == 0) mbar_init(sy.bar(B_RMX2), 4);
     }
     mbar_init(sy.bar(B_OFULL), 1);
     mbar_init(sy.bar(B_OEMPTY), 4);
