@@ -742,11 +742,21 @@ def run_fp8_bench(name, dev, barrier, reduce_max, world, hbm, steps=20, warmup=3
     total_ms, per_ms, _ = time_launches(step, steps, warmup, barrier, "fp8")
     total_ms = reduce_max(total_ms)
     ms = statistics.mean(per_ms)
+
+    def step_gather():
+        _capi.sparse_prefill_fp8_fwd(w.q, k8, v8, w.topk_idx, 0.5, 2.0, n_valid=w.n_valid, scale=w.scale,
+                                     out=out, lse=lse, kernel="gather_only")
+
+    _, g_per, _ = time_launches(step_gather, steps, warmup, barrier, "fp8_gather_only")
+    g_ms = statistics.mean(g_per)
     return {"workload": w.name + "_fp8e4m3", "tokens_per_s": T * steps * world / (total_ms / 1e3),
             "mean_launch_ms": ms, "live_entries": entries, "algo_bytes": algo,
             "gathered_kv_gbs": gathered / (ms / 1e3) / 1e9,
             "algo_gbs": algo / (ms / 1e3) / 1e9, "frac_of_hbm": algo / (ms / 1e3) / 1e9 / hbm,
-            "steps": steps}
+            "steps": steps,
+            "gather_floor": {"kernel": "qsa_gather_only_f8_kernel", "mean_launch_ms": g_ms,
+                             "gathered_kv_gbs": gathered / (g_ms / 1e3) / 1e9,
+                             "kernel_frac_of_floor": g_ms / ms}}
 
 
 def run_indexer_bench(dev, barrier, reduce_max, world, hbm, bf16, steps=20, warmup=3, **kw):

@@ -207,6 +207,24 @@ qsa_status_t qsa_sparse_prefill_fp8_fwd(const qsa_shape_t* shape,
                                         void* out, float* lse,
                                         int32_t* status, void* stream);
 
+/* Same contract as qsa_sparse_prefill_fp8_fwd, with an explicit kernel
+ * choice: QSA_KERNEL_AUTO or QSA_KERNEL_TCGEN05 run the FP8 kernel;
+ * QSA_KERNEL_GATHER_ONLY (token lists only: block_size 1, last_slot NULL)
+ * runs only that kernel's KV gather, for measurement, and writes neither out
+ * nor lse (the status word still receives out-of-range ids);
+ * QSA_KERNEL_WARP_MMA returns QSA_ERR_UNSUPPORTED. */
+qsa_status_t qsa_sparse_prefill_fp8_fwd_with(const qsa_shape_t* shape,
+                                             int32_t block_size,
+                                             const int32_t* last_slot,
+                                             const void* q, const void* k_cache,
+                                             const void* v_cache,
+                                             const int32_t* topk_idx,
+                                             const int32_t* n_valid, float scale,
+                                             float k_scale, float v_scale,
+                                             void* out, float* lse,
+                                             int32_t* status,
+                                             qsa_kernel_t kernel, void* stream);
+
 /*
  * Split-K sparse attention for decode-shaped calls: few query tokens per KV
  * head (one per sequence in decode) with long lists.  Each list is cut into

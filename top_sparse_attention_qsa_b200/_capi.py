@@ -36,7 +36,7 @@ EXPORTS = ("qsa_sparse_prefill_fwd", "qsa_sparse_prefill_fwd_with", "qsa_sparse_
            "qsa_sparse_prefill_block_fwd",
            "qsa_sparse_prefill_fwd_host", "qsa_sparse_decode_fwd", "qsa_sparse_decode_workspace_bytes",
            "qsa_sparse_decode_num_splits", "qsa_sparse_decode_fwd_noalloc", "qsa_test_stalled_pipeline",
-           "qsa_sparse_prefill_fp8_fwd", "qsa_sparse_decode_fp8_fwd", "qsa_indexer_scores", "qsa_topk_select", "qsa_status_string",
+           "qsa_sparse_prefill_fp8_fwd", "qsa_sparse_prefill_fp8_fwd_with", "qsa_sparse_decode_fp8_fwd", "qsa_indexer_scores", "qsa_topk_select", "qsa_status_string",
            "qsa_abi_version")
 
 
@@ -113,6 +113,10 @@ _lib.qsa_sparse_prefill_block_fwd.argtypes = [ctypes.POINTER(Shape), ctypes.c_in
 _lib.qsa_sparse_prefill_fp8_fwd.argtypes = [ctypes.POINTER(Shape), ctypes.c_int32, _vp, _vp, _vp, _vp, _vp,
                                             _vp, ctypes.c_float, ctypes.c_float, ctypes.c_float, _vp, _vp,
                                             _vp, _vp]
+_lib.qsa_sparse_prefill_fp8_fwd_with.restype = ctypes.c_int
+_lib.qsa_sparse_prefill_fp8_fwd_with.argtypes = [ctypes.POINTER(Shape), ctypes.c_int32, _vp, _vp, _vp, _vp, _vp,
+                                                 _vp, ctypes.c_float, ctypes.c_float, ctypes.c_float, _vp, _vp,
+                                                 _vp, ctypes.c_int, _vp]
 _lib.qsa_sparse_decode_fp8_fwd.argtypes = [ctypes.POINTER(Shape), _vp, _vp, _vp, _vp, _vp, ctypes.c_float,
                                            ctypes.c_float, ctypes.c_float, _vp, _vp, _vp, ctypes.c_int32,
                                            _vp, ctypes.c_size_t, _vp]
@@ -440,10 +444,13 @@ def sparse_prefill_block_fwd(q, k_cache, v_cache, block_idx, block_size: int, la
 
 def sparse_prefill_fp8_fwd(q, k_cache, v_cache, topk_idx, k_scale: float = 1.0, v_scale: float = 1.0,
                            n_valid=None, scale: float = 0.0, block_size: int = 1, last_slot=None,
-                           out=None, lse=None, status=None, stream=None, want_lse: bool = True):
+                           out=None, lse=None, status=None, stream=None, want_lse: bool = True,
+                           kernel: str = "auto"):
     """FP8 E4M3 KV cache (torch.float8_e4m3fn [S, Hkv, 256]); element value =
     stored value * k_scale (v_scale).  Token lists (block_size 1) or
-    microblock lists with an optional last_slot [T] int32."""
+    microblock lists with an optional last_slot [T] int32.  kernel: "auto" |
+    "tcgen05" | "gather_only" (the KV gather alone, for measurement; out and
+    lse untouched; token lists only)."""
     dev = q.device
     _need(q, "q", torch.bfloat16, dev)
     _need(k_cache, "k_cache", torch.float8_e4m3fn, dev)
@@ -470,10 +477,10 @@ def sparse_prefill_fp8_fwd(q, k_cache, v_cache, topk_idx, k_scale: float = 1.0, 
     shape = make_shape(q, k_cache, topk_idx, out, lse)
     if stream is None:
         stream = torch.cuda.current_stream(dev).cuda_stream
-    _raise(_lib.qsa_sparse_prefill_fp8_fwd(ctypes.byref(shape), int(block_size), _ptr(last_slot), _ptr(q),
-                                           _ptr(k_cache), _ptr(v_cache), _ptr(topk_idx), _ptr(n_valid),
-                                           float(scale), float(k_scale), float(v_scale), _ptr(out),
-                                           _ptr(lse), _ptr(status), stream))
+    _raise(_lib.qsa_sparse_prefill_fp8_fwd_with(ctypes.byref(shape), int(block_size), _ptr(last_slot), _ptr(q),
+                                                _ptr(k_cache), _ptr(v_cache), _ptr(topk_idx), _ptr(n_valid),
+                                                float(scale), float(k_scale), float(v_scale), _ptr(out),
+                                                _ptr(lse), _ptr(status), KERNELS[kernel], stream))
     return out, lse
 
 

@@ -125,6 +125,19 @@ cudaError_t launch_gather_only(const qsa::tc::TcParams& tp, cudaStream_t stream)
   return cudaGetLastError();
 }
 
+cudaError_t launch_f8_gather_only(const qsa::tc::TcParams& tp, cudaStream_t stream) {
+  static std::atomic<int> done[kMaxDevices];
+  auto kernel = qsa::f8::qsa_gather_only_f8_kernel;
+  cudaError_t e = set_smem_once(kernel, qsa::f8::F_SMEM, done);
+  if (e != cudaSuccess) return e;
+  const int64_t units = tp.T * tp.Hkv;
+  const int nsm = sm_count();
+  if (nsm <= 0) return cudaErrorInvalidDevice;
+  const unsigned grid = static_cast<unsigned>(units < nsm ? units : nsm);
+  kernel<<<grid, 32 * (qsa::tc::kProducerWarps + 1), qsa::f8::F_SMEM, stream>>>(tp);
+  return cudaGetLastError();
+}
+
 template <bool kDump, bool kStall = false, bool kBlocks = false>
 cudaError_t launch_tc(const qsa::tc::TcParams& tp, cudaStream_t stream) {
   static std::atomic<int> done[kMaxDevices];
@@ -298,7 +311,7 @@ qsa_status_t run_lists(const qsa_shape_t* shape, int32_t block_size, const int32
                        const void* q, const void* k_cache, const void* v_cache,
                        const int32_t* topk_idx, const int32_t* n_valid, float scale,
                        float k_scale, float v_scale, bool fp8, void* out, float* lse,
-                       int32_t* status, void* stream);
+                       int32_t* status, void* stream, bool gather_only = false);
 
 // The host-buffer entry point cuts the query tokens into chunks of about
 // kHostChunkTokens (at most kHostMaxChunks) so that the copies of one chunk
@@ -436,9 +449,10 @@ qsa_status_t run_lists(const qsa_shape_t* shape, int32_t block_size, const int32
                        const void* q, const void* k_cache, const void* v_cache,
                        const int32_t* topk_idx, const int32_t* n_valid, float scale,
                        float k_scale, float v_scale, bool fp8, void* out, float* lse,
-                       int32_t* status, void* stream) {
+                       int32_t* status, void* stream, bool gather_only) {
   qsa_status_t rc = validate(shape, q, k_cache, v_cache, topk_idx, out);
   if (rc != QSA_OK) return rc;
+  if (gather_only && (!fp8 || block_size != 1 || last_slot != nullptr)) return QSA_ERR_UNSUPPORTED;
   if (fp8 && shape->topk > 0 && (shape->kv_stride_slot % 16 != 0 || shape->kv_stride_head % 16 != 0))
     return QSA_ERR_ALIGN;   // FP8 rows move in 16-byte pieces of 16 elements
   int shift = -1;
@@ -485,7 +499,9 @@ qsa_status_t run_lists(const qsa_shape_t* shape, int32_t block_size, const int32
   const bool plain = shift == 0 && last_slot == nullptr;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaError_t e;
-  if (fp8)
+  if (gather_only)
+    e = launch_f8_gather_only(tp, st);
+  else if (fp8)
     e = plain ? launch_f8<false>(tp, st) : launch_f8<true>(tp, st);
   else
     e = plain ? launch_tc<false>(tp, st) : launch_tc<false, false, true>(tp, st);
@@ -679,6 +695,19 @@ qsa_status_t qsa_sparse_prefill_fp8_fwd(const qsa_shape_t* shape, int32_t block_
                                         float* lse, int32_t* status, void* stream) {
   return run_lists(shape, block_size, last_slot, q, k_cache, v_cache, topk_idx, n_valid, scale,
                    k_scale, v_scale, true, out, lse, status, stream);
+}
+
+qsa_status_t qsa_sparse_prefill_fp8_fwd_with(const qsa_shape_t* shape, int32_t block_size,
+                                             const int32_t* last_slot, const void* q,
+                                             const void* k_cache, const void* v_cache,
+                                             const int32_t* topk_idx, const int32_t* n_valid,
+                                             float scale, float k_scale, float v_scale, void* out,
+                                             float* lse, int32_t* status, qsa_kernel_t kernel,
+                                             void* stream) {
+  if (kernel != QSA_KERNEL_AUTO && kernel != QSA_KERNEL_TCGEN05 && kernel != QSA_KERNEL_GATHER_ONLY)
+    return QSA_ERR_UNSUPPORTED;
+  return run_lists(shape, block_size, last_slot, q, k_cache, v_cache, topk_idx, n_valid, scale,
+                   k_scale, v_scale, true, out, lse, status, stream, kernel == QSA_KERNEL_GATHER_ONLY);
 }
 
 qsa_status_t qsa_test_stalled_pipeline(const qsa_shape_t* shape, const void* q,

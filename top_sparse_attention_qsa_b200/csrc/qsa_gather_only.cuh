@@ -11,8 +11,10 @@
 // full.  It writes nothing to global memory.  Its time over a workload is
 // the floor the full kernel could reach with free compute, and the ratio of
 // the two times is the full kernel's efficiency against its own gather.
+// qsa_gather_only_f8_kernel does the same for the FP8-cache kernel.
 #pragma once
 
+#include "qsa_prefill_f8.cuh"
 #include "qsa_prefill_tc.cuh"
 
 namespace qsa {
@@ -77,4 +79,50 @@ __global__ void __launch_bounds__(kGatherOnlyThreads, 1)
 }
 
 }  // namespace tc
+
+namespace f8 {
+
+// The same for the FP8 kernel's gather: its producer warps (one 32 KB slot
+// per K or V tile of 256-byte rows), token lists; Q is not loaded, since the
+// FP8 kernel reads it from global memory in its own warp.
+__global__ void __launch_bounds__(32 * (kProducerWarps + 1), 1)
+    qsa_gather_only_f8_kernel(const __grid_constant__ TcParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t sb = (raw + 1023u) & ~1023u;
+  uint8_t* sp = smem_raw + (sb - raw);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  Sync sy;
+  sy.bars = sb + F_BAR;
+  sy.abort_flag = reinterpret_cast<volatile uint32_t*>(sp + F_MISC + 4);
+  sy.status = p.status;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kSlots8; ++s) {
+      mbar_init(sy.bar(G_FULL + s), 32 * kProducerWarps);
+      mbar_init(sy.bar(G_EMPTY + s), 1);
+    }
+    *sy.abort_flag = 0u;
+    mbar_fence_init();
+  }
+  __syncthreads();
+  if (warp < kProducerWarps) {
+    producer8<false>(p, sy, sb, warp, lane);
+  } else if (lane == 0) {
+    uint32_t c_slot = 0;
+    const int64_t units = num_units(p);
+    bool ok = true;
+    for (int64_t u = blockIdx.x; u < units && ok; u += gridDim.x) {
+      const Unit un = decode_unit(p, u);
+      for (int i = 0; i < 2 * un.n_tiles && ok; ++i, ++c_slot) {   // K tile, V tile
+        const uint32_t slot = c_slot % kSlots8;
+        ok = sy.wait(G_FULL + slot, (c_slot / kSlots8) & 1u);
+        if (ok) mbar_arrive(sy.bar(G_EMPTY + slot));
+      }
+    }
+  }
+  __syncwarp();
+  __syncthreads();
+}
+
+}  // namespace f8
 }  // namespace qsa

@@ -26,12 +26,13 @@
 //               the 256-byte K and V rows into the 128-byte-swizzled K-major
 //               layout (K slot, then V slot per tile)
 //   warp 4      all lanes: the unit's Q (BF16, from global memory) split into
-//               q_hi / q_lo rows of one E4M3 tile with per-head scale; lane 0
-//               issues the score MMAs (A = K tile, B = [q_hi; q_lo];
+//               q_hi / q_lo rows of one E4M3 tile with per-head scale, one
+//               unit ahead (double-buffered)
+//   warp 5      lane 0 issues the score MMAs (A = K tile, B = [q_hi; q_lo];
 //               M=128, N=32, K=32)
-//   warp 5      lane 0 issues PV: [O_hi O_lo]^T += V^T (MN-major) .
+//   warp 6      lane 0 issues PV: [O_hi O_lo]^T += V^T (MN-major) .
 //               [P_hi P_lo]^T (MN-major, N=32) for the two 128-dim halves
-//   warps 6-13  softmax as in the BF16 kernel, two warps per TMEM lane
+//   warps 7-14  softmax as in the BF16 kernel, two warps per TMEM lane
 //               quadrant (8 heads each), reading both score terms and
 //               writing p_hi / p_lo
 // Every wait is bounded (2 s of %globaltimer) as in the BF16 kernel.
@@ -185,8 +186,10 @@ __device__ __forceinline__ void q_split(const TcParams& p, const Unit& un, uint3
 // Warp 4: per unit all lanes split Q into buffer (unit & 1) once the MMAs of
 // two units ago have released it; lane 0 then issues S_hi += K q_hi^T and
 // S_lo += K q_lo^T for every tile.
-__device__ void qk8(const TcParams& p, const Sync& sy, uint32_t sb, uint8_t* sp, uint32_t tmem, int lane) {
-  uint32_t c_tile = 0, c_unit = 0;
+// Warp 4: each unit's Q tile and score factors, one unit ahead of the MMAs
+// (double-buffered), so that no unit waits for its Q to be read and split.
+__device__ void q8(const TcParams& p, const Sync& sy, uint32_t sb, uint8_t* sp, int lane) {
+  uint32_t c_unit = 0;
   const int64_t units = num_units(p);
   bool ok = true;
   for (int64_t u = blockIdx.x; u < units && ok; u += gridDim.x) {
@@ -200,8 +203,25 @@ __device__ void qk8(const TcParams& p, const Sync& sy, uint32_t sb, uint8_t* sp,
     fence_proxy_async_smem();
     __syncwarp();
     if (lane == 0) {
-      mbar_arrive(sy.bar(G_QFULL + qb));             // the softmax reads the score factors
+      mbar_arrive(sy.bar(G_QFULL + qb));             // the MMAs and the softmax read it
       if (un.n_tiles == 0) mbar_arrive(sy.bar(G_QEMPTY + qb));
+    }
+  }
+}
+
+// Warp 5, lane 0: the score MMAs of every tile.
+__device__ void qk8(const TcParams& p, const Sync& sy, uint32_t sb, uint32_t tmem) {
+  uint32_t c_tile = 0, c_unit = 0;
+  const int64_t units = num_units(p);
+  bool ok = true;
+  for (int64_t u = blockIdx.x; u < units && ok; u += gridDim.x) {
+    const Unit un = decode_unit(p, u);
+    const uint32_t qb = c_unit & 1u;
+    if (un.n_tiles > 0) ok = sy.wait(G_QFULL + qb, (c_unit >> 1) & 1u);
+    if (!ok) break;
+    ++c_unit;
+    const uint32_t qt = sb + F_Q8 + qb * 2 * kQ8Bytes;
+    {
       for (int i = 0; i < un.n_tiles && ok; ++i, ++c_tile) {
         const uint32_t c = c_tile;
         const uint32_t sbuf = c & 1u;
@@ -226,13 +246,9 @@ __device__ void qk8(const TcParams& p, const Sync& sy, uint32_t sb, uint8_t* sp,
         if (i == un.n_tiles - 1) umma_commit(sy.bar(G_QEMPTY + qb));
       }
     }
-    ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
   }
-  if (lane == 0) {
-    umma_commit(sy.bar(G_DONE));
-    sy.drain(G_DONE, 0);
-  }
-  __syncwarp();
+  umma_commit(sy.bar(G_DONE));
+  sy.drain(G_DONE, 0);
 }
 
 // Warp 5, lane 0: O_{hi,lo}[mh] += V_half(mh)^T . P_{hi,lo}^T per tile.
@@ -287,7 +303,9 @@ __device__ void pv8(const TcParams& p, const Sync& sy, uint32_t sb, uint32_t tme
 
 constexpr int kSmWarps = 8;     // two per TMEM lane quadrant, 8 heads each
 constexpr int kHpw = kGp / 2;   // heads per softmax warp
-constexpr int kThreads8 = 32 * (kProducerWarps + 2 + kSmWarps);
+constexpr int kWarpQ8 = kProducerWarps, kWarpQK8 = kProducerWarps + 1, kWarpPV8 = kProducerWarps + 2,
+              kWarpSm8 = kProducerWarps + 3;
+constexpr int kThreads8 = 32 * (kProducerWarps + 3 + kSmWarps);
 
 // Reduce 8 per-lane values across the 32 lanes of a warp by exchanging halves
 // (7 shuffles for the exchange, 2 for the rest).  Lane l ends with the result
@@ -340,13 +358,13 @@ __device__ __forceinline__ void form_p(const float (&s)[kHpw], const float (&m)[
   }
 }
 
-// Softmax warp w (6..13): TMEM lane quadrant q = w & 3 (thread = key of the
-// tile, and dim of an output half), heads [8 hh, 8 hh + 8) with hh = (w-6)/4.
+// Softmax warp w (7..14): TMEM lane quadrant q = w & 3 (thread = key of the
+// tile, and dim of an output half), heads [8 hh, 8 hh + 8) with hh = (w-7)/4.
 template <bool kBlocks>
 __device__ void softmax8(const TcParams& p, const Sync& sy, uint32_t sb, uint8_t* sp, uint32_t tmem, int warp,
                          int lane) {
   const int wq = warp & 3;
-  const int hh = (warp - kWarpSoftmax0) >> 2;
+  const int hh = (warp - kWarpSm8) >> 2;
   const int h0 = hh * kHpw;
   const int key = wq * 32 + lane;
   const uint32_t tl = tmem + (static_cast<uint32_t>(wq * 32) << 16);
@@ -410,7 +428,7 @@ __device__ void softmax8(const TcParams& p, const Sync& sy, uint32_t sb, uint8_t
       // tile max and form P again.
       const bool wover = __any_sync(0xffffffffu, over);
       uint8_t* vt = votes + buf * 8;
-      if (lane == 0) vt[warp - kWarpSoftmax0] = wover ? 1 : 0;
+      if (lane == 0) vt[warp - kWarpSm8] = wover ? 1 : 0;
       __syncwarp();
       if (lane == 0) mbar_arrive(sy.bar(G_RMAX + buf));
       uint32_t ph[2], plo[2];
@@ -586,7 +604,7 @@ __global__ void __launch_bounds__(kThreads8, 1) qsa_prefill_f8_kernel(const __gr
     *sy.abort_flag = 0u;
     mbar_fence_init();
   }
-  if (warp == kWarpQK) {
+  if (warp == kWarpQK8) {
     tmem_alloc(sb + F_MISC, kTmemCols8);
     tmem_relinquish();
   }
@@ -597,9 +615,12 @@ __global__ void __launch_bounds__(kThreads8, 1) qsa_prefill_f8_kernel(const __gr
 
   if (warp < kProducerWarps) {
     producer8<kBlocks>(p, sy, sb, warp, lane);
-  } else if (warp == kWarpQK) {
-    qk8(p, sy, sb, sp, tmem, lane);
-  } else if (warp == kWarpPV) {
+  } else if (warp == kWarpQ8) {
+    q8(p, sy, sb, sp, lane);
+  } else if (warp == kWarpQK8) {
+    if (lane == 0) qk8(p, sy, sb, tmem);
+    __syncwarp();
+  } else if (warp == kWarpPV8) {
     if (lane == 0) pv8(p, sy, sb, tmem);
     __syncwarp();
   } else {
@@ -609,7 +630,7 @@ __global__ void __launch_bounds__(kThreads8, 1) qsa_prefill_f8_kernel(const __gr
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == kWarpQK) tmem_dealloc(tmem, kTmemCols8);
+  if (warp == kWarpQK8) tmem_dealloc(tmem, kTmemCols8);
 }
 
 }  // namespace f8
