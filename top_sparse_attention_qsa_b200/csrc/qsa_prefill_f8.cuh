@@ -19,7 +19,10 @@
 //                                     rescale)
 // with separate TMEM accumulators for the two terms: S_hi, S_lo per score
 // buffer and O_hi, O_lo per output half.  s = (S_hi + S_lo / 16) * 2^-a_h and
-// o = (O_hi + O_lo / 16) * v_scale / l.
+// o = (O_hi + O_lo / 16) * v_scale / l.  The N dimension of Q, S, P and O runs
+// [hi of heads 0-7, lo of heads 0-7, hi of heads 8-15, lo of heads 8-15], so
+// that a softmax thread's 8 heads of both terms are 16 adjacent TMEM columns
+// and 16 adjacent bytes of P.
 //
 // Warps (persistent CTAs, one per SM):
 //   warps 0-3   producers: list entries one tile ahead, 16-byte cp.async of
@@ -126,8 +129,9 @@ __device__ void producer8(const TcParams& p, const Sync& sy, uint32_t sb, int pw
 // Lane l of warp 4 takes head l/2, dims [128*(l&1), +128): loads them from
 // global memory, finds the head's largest |q| (with its partner lane), and
 // writes q * 2^a = q_hi + q_lo / 16 as one E4M3 tile of 32 rows (K-major,
-// 128-byte swizzle: two 128-dim blocks of 32 rows x 128 B; row h holds the
-// hi term of head h, row 16 + h its lo term) and 2^-a * scale_log2 into the
+// 128-byte swizzle: two 128-dim blocks of 32 rows x 128 B; head h has its hi
+// term in row 16 (h / 8) + h % 8 and its lo term 8 rows further) and
+// 2^-a * scale_log2 into the
 // score factors.  Heads past the group are zero.
 __device__ __forceinline__ void q_split(const TcParams& p, const Unit& un, uint32_t qt, float* qsc, int lane) {
   const int h = lane >> 1, half = lane & 1;
@@ -175,9 +179,10 @@ __device__ __forceinline__ void q_split(const TcParams& p, const Unit& un, uint3
       hw[j] = h01 | (h23 << 16);
       lw[j] = l01 | (l23 << 16);
     }
-    const uint32_t off = half * kQ8Block + h * 128 + ((c8 ^ (h & 7)) << 4);   // rows h and 16 + h share the swizzle
+    // hi row 16 (h / 8) + h % 8 and lo row 8 further share the swizzle phase h % 8
+    const uint32_t off = half * kQ8Block + ((h >> 3) * 16 + (h & 7)) * 128 + ((c8 ^ (h & 7)) << 4);
     st_shared_v4(qt + off, hw[0], hw[1], hw[2], hw[3]);
-    st_shared_v4(qt + off + 16 * 128, lw[0], lw[1], lw[2], lw[3]);
+    st_shared_v4(qt + off + 8 * 128, lw[0], lw[1], lw[2], lw[3]);
   }
 }
 
@@ -235,8 +240,8 @@ __device__ void qk8(const TcParams& p, const Sync& sy, uint32_t sb, uint32_t tme
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           // K-major, 128-byte swizzle: a 32-dim step advances 32 B inside the
-          // atom; dims 128-255 sit 16 KB (K) / 4 KB (Q) further.  N = 32:
-          // S_hi in columns 0-15, S_lo in 16-31.
+          // atom; dims 128-255 sit 16 KB (K) / 4 KB (Q) further.  N = 32,
+          // columns in the interleaved hi / lo head order of the Q rows.
           const uint64_t a = smem_desc(kt + (kk >> 2) * kBlockBytes + (kk & 3) * 32, 16, 1024, 2);
           const uint64_t b = smem_desc(qt + (kk >> 2) * kQ8Block + (kk & 3) * 32, 16, 1024, 2);
           umma_f8_ss(tmem + kTS + sbuf * 32, a, b, kIdescQK8, kk > 0 ? 1u : 0u);
@@ -283,10 +288,10 @@ __device__ void pv8(const TcParams& p, const Sync& sy, uint32_t sb, uint32_t tme
           // A = V^T: MN-major, 128-byte swizzle; the 128 dims of a half are
           // one atom row, groups of 8 keys 1 KB apart, 32 keys per step
           const uint64_t a = smem_desc(vt + mh * kBlockBytes + kk * 4096, kBlockBytes, 1024, 2);
-          // B = P^T: MN-major, no swizzle; per key one 16-byte core row of 16
-          // heads, key groups of 8 128 B apart (LBO); N = 32 spans P_hi and,
-          // one core-matrix column (SBO = 2 KB) further, P_lo: O_hi lands in
-          // columns 0-15 and O_lo in 16-31 of the half
+          // B = P^T: MN-major, no swizzle; per key one 16-byte core row
+          // (hi then lo of heads 0-7), key groups of 8 128 B apart (LBO), and
+          // one core-matrix column (SBO = 2 KB) further the same for heads
+          // 8-15: O of the half lands in the same interleaved column order
           const uint64_t b = smem_desc(pt + kk * 512, 128, kP8Bytes, 0);
           umma_f8_ss(tmem + kTO + mh * 32, a, b, kIdescPV8, (i == 0 && kk == 0) ? 0u : 1u);
         }
@@ -406,9 +411,8 @@ __device__ void softmax8(const TcParams& p, const Sync& sy, uint32_t sb, uint8_t
       ok = sy.wait_warp(G_SFULL + buf, (c >> 1) & 1u);
       if (!ok) break;
       tc_fence_after();
-      uint32_t rh[8], rl[8];
-      tmem_ld8(tl + kTS + buf * 32 + h0, rh);
-      tmem_ld8(tl + kTS + buf * 32 + 16 + h0, rl);
+      uint32_t r16[16];                              // hi of this warp's 8 heads, then lo
+      tmem_ld16(tl + kTS + buf * 32 + 16 * hh, r16);
       tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
@@ -417,7 +421,7 @@ __device__ void softmax8(const TcParams& p, const Sync& sy, uint32_t sb, uint8_t
       bool over = false;
 #pragma unroll
       for (int h = 0; h < kHpw; ++h) {
-        s[h] = (valid && h0 + h < G) ? fmaf(__uint_as_float(rl[h]), 0.0625f, __uint_as_float(rh[h])) * qs[h]
+        s[h] = (valid && h0 + h < G) ? fmaf(__uint_as_float(r16[8 + h]), 0.0625f, __uint_as_float(r16[h])) * qs[h]
                                      : -INFINITY;
         over |= s[h] > m_run[h] + kRescaleLog2;
       }
@@ -473,11 +477,12 @@ __device__ void softmax8(const TcParams& p, const Sync& sy, uint32_t sb, uint8_t
 #pragma unroll
             for (int q4 = 0; q4 < 4; ++q4) {          // O_hi, O_lo x two halves, this warp's heads
               uint32_t o[8];
-              tmem_ld8(tl + kTO + q4 * 16 + h0, o);
+              const uint32_t col = kTO + (q4 >> 1) * 32 + 16 * hh + (q4 & 1) * 8;
+              tmem_ld8(tl + col, o);
               tmem_wait_ld();
 #pragma unroll
               for (int h = 0; h < kHpw; ++h) o[h] = __float_as_uint(__uint_as_float(o[h]) * alpha[h]);
-              tmem_st8(tl + kTO + q4 * 16 + h0, o);
+              tmem_st8(tl + col, o);
             }
             tmem_wait_st();
           }
@@ -492,10 +497,10 @@ __device__ void softmax8(const TcParams& p, const Sync& sy, uint32_t sb, uint8_t
       for (int h = 0; h < kHpw; ++h) l_part[h] += pv[h];
       ok = sy.wait_warp(G_PEMPTY + buf, ((c >> 1) & 1u) ^ 1u);
       if (!ok) break;
-      // P^T row of this key: 16 heads = 16 bytes at 16 key; this warp's 8 heads at + 8 hh
-      const uint32_t pa = sb + F_P8 + buf * 2 * kP8Bytes + key * 16 + hh * 8;
-      asm volatile("st.shared.v2.b32 [%0], {%1, %2};\n" ::"r"(pa), "r"(ph[0]), "r"(ph[1]) : "memory");
-      asm volatile("st.shared.v2.b32 [%0], {%1, %2};\n" ::"r"(pa + kP8Bytes), "r"(plo[0]), "r"(plo[1]) : "memory");
+      // P^T row of this key for this warp's 8 heads: p_hi then p_lo, 16 bytes
+      // at 16 key in core-matrix column hh
+      const uint32_t pa = sb + F_P8 + buf * 2 * kP8Bytes + hh * kP8Bytes + key * 16;
+      st_shared_v4(pa, ph[0], ph[1], plo[0], plo[1]);
       fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();
@@ -516,12 +521,10 @@ __device__ void softmax8(const TcParams& p, const Sync& sy, uint32_t sb, uint8_t
     ok = sy.wait_warp(G_OFULL, c_unit & 1u);
     if (!ok) break;
     tc_fence_after();
-    uint32_t oh0[8] = {}, oh1[8] = {}, ol0[8] = {}, ol1[8] = {};
+    uint32_t o0[16] = {}, o1[16] = {};     // per half: O_hi of the 8 heads, then O_lo
     if (un.n_tiles > 0) {
-      tmem_ld8(tl + kTO + h0, oh0);          // half 0: O_hi, O_lo
-      tmem_ld8(tl + kTO + 16 + h0, ol0);
-      tmem_ld8(tl + kTO + 32 + h0, oh1);     // half 1
-      tmem_ld8(tl + kTO + 48 + h0, ol1);
+      tmem_ld16(tl + kTO + 16 * hh, o0);
+      tmem_ld16(tl + kTO + 32 + 16 * hh, o1);
       tmem_wait_ld();
     }
     tc_fence_before();
@@ -535,8 +538,8 @@ __device__ void softmax8(const TcParams& p, const Sync& sy, uint32_t sb, uint8_t
       if (hg < G) {
         const bool live = l_tot[h] > 0.f;
         const float inv = live ? p.o_scale / l_tot[h] : 0.f;
-        const float v0 = live ? fmaf(__uint_as_float(ol0[h]), 0.0625f, __uint_as_float(oh0[h])) * inv : 0.f;
-        const float v1 = live ? fmaf(__uint_as_float(ol1[h]), 0.0625f, __uint_as_float(oh1[h])) * inv : 0.f;
+        const float v0 = live ? fmaf(__uint_as_float(o0[8 + h]), 0.0625f, __uint_as_float(o0[h])) * inv : 0.f;
+        const float v1 = live ? fmaf(__uint_as_float(o1[8 + h]), 0.0625f, __uint_as_float(o1[h])) * inv : 0.f;
         if (p.part_o != nullptr) {
           // split-K: this chunk's normalised partial output, for the merge
           float* po = p.part_o + ((row0 + hg) * p.splits + un.s) * 256;
