@@ -178,3 +178,18 @@ def test_pipeline_into_block_attention(C, orc):
     o = _host(out).double().numpy()
     assert np.all(np.abs(o - ref_o) <= 1e-2 + 1e-2 * np.abs(ref_o))
     assert np.all(np.abs(_host(lse).double().numpy() - ref_l) <= 1e-3)
+
+
+@pytest.mark.parametrize("bs", [1, 2, 8, 3])
+def test_other_block_sizes(C, orc, bs):
+    """Compression ratios other than 4 (the kernels take any block size >= 1):
+    the candidate ranges, the selection and the tail follow the block size;
+    two sequences starting on block boundaries."""
+    S = 1200 * bs
+    w = W.config_indexer(device=DEV, seed=60 + bs, T=150, S=S, heads=4, block_size=bs,
+                         seq_starts=[0, 600 * bs])
+    lists, nv, scores = C.indexer_select(w.q_idx, w.k_idx, w.positions, w.seq_start, 40, bs,
+                                         append_tail=True, copies=2)
+    torch.cuda.synchronize()
+    check_scores(orc, w, _host(scores))
+    check_selection(orc, w, scores, lists, nv, 40, True)

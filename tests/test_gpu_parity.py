@@ -66,6 +66,17 @@ def test_config_sampled(name, kernel):
     print(name, kernel, check_sampled(w, name, tokens, kernel))
 
 
+@pytest.mark.parametrize("kernel", KERNELS)
+def test_very_long_lists(kernel):
+    """40000 distinct entries per (token, KV head): 313 tiles per unit, long
+    runs of lazy rescales, heads (24,2); every row against the oracle."""
+    w = W.generic_case(T=6, S=50000, Hq=24, Hkv=2, K=40000, seed=71, device=DEV)
+    # a rising score trend along each list makes the running max move often
+    ramp = torch.linspace(0.0, 3.0, 50000, device=DEV)[:, None, None]
+    w.k_cache = (w.k_cache.float() * (1.0 + ramp)).to(torch.bfloat16)
+    print(check_all(w, "very long lists", kernel))
+
+
 def test_pages_long_prefill():
     """7810 query tokens x 65536-slot cache x 2051 slots, sampled rows + all finite."""
     w = W.make("pages_long", device=DEV)
