@@ -109,11 +109,11 @@ __device__ __forceinline__ void range_of(int32_t pos, int32_t s0, int32_t NB, in
   hi = static_cast<int>(h);
 }
 
-// Shared-memory add of 1 at `addr` when `pred` holds, without a branch.
-__device__ __forceinline__ void red_add_if(uint32_t addr, bool pred) {
+// Shared-memory add of 1 at `addr` when a == b, without a branch.
+__device__ __forceinline__ void red_add_if_eq(uint32_t addr, uint32_t a, uint32_t b) {
   asm volatile(
-      "{\n\t.reg .pred p;\n\tsetp.ne.u32 p, %1, 0;\n\t@p red.shared.add.u32 [%0], 1;\n\t}\n" ::"r"(addr),
-      "r"(static_cast<uint32_t>(pred))
+      "{\n\t.reg .pred p;\n\tsetp.eq.u32 p, %1, %2;\n\t@p red.shared.add.u32 [%0], 1;\n\t}\n" ::"r"(addr),
+      "r"(a), "r"(b)
       : "memory");
 }
 
@@ -385,45 +385,15 @@ struct TopkParams {
   int32_t NB, bs, budget, width, copies, append_tail;
 };
 
-// Order-preserving key: a > b as floats  <=>  key(a) > key(b) as unsigned;
-// -0.0 is first made +0.0 so that the two zeros tie.
+// Order-preserving key: a > b as floats  <=>  key(a) > key(b) as unsigned,
+// with -0.0 and +0.0 on the same key.  A negative float u maps to ~u, a
+// positive one to (u | 2^31) - 1: both zeros land on 0x7fffffff and every
+// other order is kept; -inf maps to 0x007fffff and only the negative NaN
+// 0xffffffff to 0.
 __device__ __forceinline__ uint32_t order_key(float f) {
-  uint32_t u = __float_as_uint(f);
-  if (u == 0x80000000u) u = 0u;
-  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-}
-
-// Inclusive scan over the CTA of one value per thread (thread order); the
-// CTA total lands in `total`.  wsum holds kNT/32 + 1 words; every thread
-// must call.
-template <int kNT>
-__device__ __forceinline__ uint32_t block_scan(uint32_t v, uint32_t* wsum, int warp, int lane,
-                                               uint32_t& total) {
-  constexpr int kW = kNT / 32;
-  uint32_t x = v;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
-    if (lane >= o) x += y;
-  }
-  if (lane == 31) wsum[warp] = x;
-  __syncthreads();
-  if (warp == 0) {
-    const uint32_t t = lane < kW ? wsum[lane] : 0u;
-    uint32_t ti = t;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const uint32_t y = __shfl_up_sync(0xffffffffu, ti, o);
-      if (lane >= o) ti += y;
-    }
-    if (lane < kW) wsum[lane] = ti - t;
-    if (lane == kW - 1) wsum[kW] = ti;
-  }
-  __syncthreads();
-  const uint32_t r = x + wsum[warp];
-  total = wsum[kW];
-  __syncthreads();
-  return r;
+  const uint32_t u = __float_as_uint(f);
+  const uint32_t sgn = static_cast<uint32_t>(static_cast<int32_t>(u) >> 31);   // 0 or ~0
+  return (u ^ (sgn | 0x80000000u)) + ~sgn;
 }
 
 __device__ __forceinline__ void bulk_copy_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
@@ -582,7 +552,7 @@ __global__ void __launch_bounds__(kTkThreads, 1) qsa_topk_kernel(const __grid_co
             const uint32_t hbase = smem_u32(hb);
 #pragma unroll
             for (int j = 0; j < kR; ++j)
-              red_add_if(hbase + 4u * ((key[j] >> shift) & dmask), (key[j] & mask) == prefix);
+              red_add_if_eq(hbase + 4u * ((key[j] >> shift) & dmask), key[j] & mask, prefix);
           }
           __syncthreads();
           // thread i owns bins 4095 - i*kBinsPer .. (high to low); warps in
