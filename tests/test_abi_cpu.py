@@ -173,3 +173,24 @@ def test_fp8_entry_validation(capi):
     assert fp8(ctypes.byref(s), 1, None, None, P, P, P, None, 0.0, 1.0, 1.0, P, None, None, None) == 1
     assert fp8(ctypes.byref(_shape(capi, head_dim=128)), 1, None, P, P, P, P, None, 0.0, 1.0, 1.0, P,
                None, None, None) == 3
+
+
+def test_kernel_choice_validation(capi):
+    """Kernel choices outside the enum, the warp-MMA choice for the FP8
+    cache, and the FP8 gather-only measurement on microblock lists are
+    refused before anything is enqueued."""
+    lib = capi.library()
+    s = _shape(capi)
+    fwd_with = lib.qsa_sparse_prefill_fwd_with
+    assert fwd_with(ctypes.byref(s), P, P, P, P, None, 0.0, P, None, None, 7, None) == 3
+    f8w = lib.qsa_sparse_prefill_fp8_fwd_with
+    args = (1, None, P, P, P, P, None, 0.0, 1.0, 1.0, P, None, None)
+    assert f8w(ctypes.byref(s), *args, capi.KERNEL_WARP_MMA, None) == 3
+    assert f8w(ctypes.byref(s), *args, 9, None) == 3
+    blk = (4,) + args[1:]
+    assert f8w(ctypes.byref(s), *blk, capi.KERNEL_GATHER_ONLY, None) == 3
+    last = (1, P) + args[2:]
+    assert f8w(ctypes.byref(s), *last, capi.KERNEL_GATHER_ONLY, None) == 3
+    # the same validation as the plain FP8 entry point comes first
+    odd = _shape(capi, kv_stride_slot=264, kv_stride_head=264)
+    assert f8w(ctypes.byref(odd), *args, capi.KERNEL_GATHER_ONLY, None) == 4
