@@ -1,4 +1,4 @@
-// qsa_prefill_tc.cuh -- QSA top-K sparse-attention prefill, TMA-gather +
+// qsa_prefill_tc.cuh -- QSA top-K sparse-attention prefill, cp.async-gather +
 // tcgen05 (TMEM) kernel for sm_100a.
 //
 // The operation (page "Qwen4-Exp QSA llega al Ascend de Huawei", section
