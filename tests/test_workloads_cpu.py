@@ -86,3 +86,31 @@ def test_c3_two_sequences_and_c5_positions():
     assert w5.k_cache.shape[0] == 131072 and w5.topk_idx.shape[1] == 2
     # the two KV heads draw independent random parts
     assert not torch.equal(w5.topk_idx[:, 0], w5.topk_idx[:, 1])
+
+
+def test_decode_lists_stay_in_their_sequence():
+    w = W.config_decode(device="cpu", B=4, ctx=4096, heads=(24, 2), topk=1024, local=64)
+    idx = w.topk_idx.long()
+    for b in range(4):
+        lo, hi = b * 4096, (b + 1) * 4096 - 1
+        assert int(w.positions[b]) == hi
+        assert bool(((idx[b] >= lo) & (idx[b] <= hi)).all())
+        for g in range(2):
+            row = idx[b, g]
+            assert row.unique().numel() == 1024
+            assert bool(((row > hi - 64) & (row <= hi)).sum() == 64)
+
+
+def test_block_lists_name_causal_blocks_with_a_masked_tail():
+    w = W.config_c5_block4(device="cpu", T=48, blocks=128, local_blocks=16)
+    idx = w.topk_idx.long()
+    pos = w.positions.long()
+    last_block = pos // 4
+    # every entry is a block that starts at or before the token's slot
+    assert bool((idx >= 0).all()) and bool((idx <= last_block[:, None, None]).all())
+    # the newest block is listed (its slots past the token are masked by last_slot)
+    assert bool((idx == last_block[:, None, None]).any(dim=2).all())
+    assert torch.equal(w.last_slot.long(), pos)
+    for t in range(0, 48, 7):
+        for g in range(2):
+            assert idx[t, g].unique().numel() == 128
