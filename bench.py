@@ -75,6 +75,8 @@ def parse_args():
                     help="time indexer -> top-K -> microblock attention as one step ('' to skip)")
     ap.add_argument("--indexer", default="indexer",
                     help="indexer + top-K workload timed under 'indexer' ('' to skip)")
+    ap.add_argument("--gather-peak", default="on", choices=["on", ""],
+                    help="measure the random-row gather rate (the roofline's gather ceiling)")
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -84,7 +86,8 @@ def parse_args():
                     help="override the query-token count of c4/c5 (smaller ncu captures)")
     ap.add_argument("--profile", action="store_true",
                     help="minimal run for ncu: no clocks, e2e, cpu baseline or secondary")
-    ap.add_argument("--only", default="", choices=["", "fp8", "indexer", "blocks", "decode", "qsa_step"],
+    ap.add_argument("--only", default="", choices=["", "fp8", "indexer", "blocks", "decode", "qsa_step",
+                                                    "gather_peak"],
                     help="run one secondary leg alone (--steps / --warmup / --tokens apply), for "
                          "profiling; prints that leg's JSON")
     return ap.parse_args()
@@ -470,7 +473,8 @@ def run_cuda(args):
                "decode": lambda: run_decode_bench("decode", dev, barrier, max_ranks, world, hbm, args.steps,
                                                   args.warmup),
                "qsa_step": lambda: run_qsa_step_bench(dev, barrier, max_ranks, world, hbm, args.steps,
-                                                      args.warmup, **kw)}[args.only]()
+                                                      args.warmup, **kw),
+               "gather_peak": lambda: run_gather_peak(dev)}[args.only]()
         if rank == 0:
             print(json.dumps({"leg": args.only, **leg}), flush=True)
         if pg is not None:
@@ -553,17 +557,33 @@ def run_cuda(args):
                            "mean_launch_ms": statistics.mean(cmp_per),
                            "algo_gbs": acct["algo_bytes"] / (statistics.mean(cmp_per) / 1e3) / 1e9}
     if not args.profile and args.kernel in ("auto", "tcgen05"):
-        # the same lists through the kernel's gather step alone: the floor of
-        # the timed kernel on this workload
+        # the same lists through the kernel's gather step alone (measurement
+        # kernel of libqsa_debug.so): the floor of the timed kernel here
+        from top_sparse_attention_qsa_b200 import _debug
+
         def step_gather():
-            _capi.sparse_prefill_fwd(w.q, w.k_cache, w.v_cache, w.topk_idx, w.n_valid, w.scale,
-                                     out=out, lse=lse, kernel="gather_only")
+            _debug.gather_only(w.q, w.k_cache, w.v_cache, w.topk_idx, w.n_valid)
         n_g = min(args.steps, 20)
         g_ms, g_per, _ = time_launches(step_gather, n_g, 3, barrier, "gather_only")
         g_mean = statistics.mean(g_per)
         line["gather_floor"] = {"kernel": "qsa_gather_only_kernel", "mean_launch_ms": g_mean,
                                 "gathered_kv_gbs": acct["gathered_bytes"] / (g_mean / 1e3) / 1e9,
                                 "kernel_frac_of_floor": g_mean / mean_launch_ms, "launches": n_g}
+    if args.gather_peak and not args.profile:
+        # the roofline's gather ceiling: the chip's random-row gather rate
+        peak = run_gather_peak(dev)
+        line["gather_peak"] = peak
+        l2 = peak["best"]["512B_32MB"]
+        ws = peak["best"]["512B_134MB"]
+        roof["l2_gather_peak"] = {"gbs": l2["gbs"], "method": l2["method"], "table_mb": 32,
+                                  "row_bytes": 512}
+        roof["gather_peak_working_set"] = {"gbs": ws["gbs"], "method": ws["method"], "table_mb": 134,
+                                           "row_bytes": 512,
+                                           "note": "table the size of one KV head's K+V rows of c5"}
+        roof["frac_gather"] = gathered_gbs / l2["gbs"]
+        roof["frac_gather_working_set"] = gathered_gbs / ws["gbs"]
+    if traffic is not None:
+        roof["frac_dram"] = traffic / (mean_launch_ms / 1e3) / 1e9 / hbm
     if not args.no_e2e and not args.profile:
         line["e2e"] = run_e2e(w, args, barrier, max_ranks, T_job, dev)
     if args.secondary and not args.profile and args.secondary != args.workload:
@@ -620,6 +640,67 @@ def run_e2e(w, args, barrier, reduce_max, T_job, dev):
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
             "ms_per_step": total_ms / steps, "steps": steps,
             "api": "qsa_sparse_prefill_fwd_host (pinned host buffers)"}
+
+
+# (method, depth, warps per CTA, CTAs per SM) of the gather probe, for 512-
+# and 256-byte rows: each fills a shared-memory ring of at most 192 KB per SM
+# (cp.async, bulk) or keeps 64-256 KB of loads in flight (ld.v4).
+PEAK_CONFIGS = {
+    512: [("cp_async", 2, 24, 1), ("cp_async", 4, 12, 1), ("cp_async", 8, 6, 1), ("cp_async", 4, 8, 1),
+          ("ld_v4", 4, 32, 1), ("ld_v4", 8, 32, 1), ("ld_v4", 16, 16, 1), ("ld_v4", 16, 16, 2),
+          ("bulk", 1, 12, 1), ("bulk", 2, 6, 1), ("bulk", 3, 4, 1)],
+    256: [("cp_async", 2, 24, 1), ("cp_async", 4, 12, 1), ("cp_async", 8, 6, 1),
+          ("ld_v4", 8, 32, 1), ("ld_v4", 16, 16, 1), ("ld_v4", 16, 16, 2),
+          ("bulk", 2, 12, 1), ("bulk", 3, 8, 1), ("bulk", 4, 6, 1)],
+}
+PEAK_TABLES_MB = (32, 134, 268)
+
+
+def run_gather_peak(dev, n_ids=1 << 23, launches=5, warmup=2):
+    """Random-row gather rate of this GPU, measured with libqsa_debug.so's
+    probe kernels (written independently of the prefill's producer code):
+    uniform random rows of 512 B (the BF16 cache row) and 256 B (the FP8
+    row) from tables of 32 MB (L2-resident), 134 MB (one KV head's K+V rows
+    of c5) and 268 MB (both heads), by each method and depth.  Reports every
+    configuration's GB/s (row bytes only; the 4-byte ids add 1-2 %) and the
+    best per (row size, table)."""
+    from top_sparse_attention_qsa_b200 import _debug
+    gen = torch.Generator(device=dev).manual_seed(31)
+    nsm = torch.cuda.get_device_properties(dev).multi_processor_count
+    sink = torch.zeros(nsm * 2 * 1024, dtype=torch.int32, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    res = {"n_ids": n_ids, "launches": launches, "configs": [], "best": {}}
+    for mb in PEAK_TABLES_MB:
+        table = torch.empty((mb << 20) // 512, 512, dtype=torch.uint8, device=dev)
+        table.random_(0, 255, generator=gen)
+        for row_bytes in (512, 256):
+            view = table.view(-1, row_bytes)
+            ids = torch.randint(0, view.shape[0], (n_ids,), generator=gen, device=dev, dtype=torch.int32)
+            best = None
+            for method, depth, warps, cps in PEAK_CONFIGS[row_bytes]:
+                def fn():
+                    _debug.gather_peak(view, ids, row_bytes, method, depth, warps, cps, sink=sink, status=status)
+                for _ in range(warmup):
+                    fn()
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                torch.cuda.synchronize()
+                a.record()
+                for _ in range(launches):
+                    fn()
+                b.record()
+                torch.cuda.synchronize()
+                ms = a.elapsed_time(b) / launches
+                gbs = n_ids * row_bytes / (ms / 1e3) / 1e9
+                entry = {"table_mb": mb, "row_bytes": row_bytes, "method": method, "depth": depth,
+                         "warps": warps, "ctas_per_sm": cps, "ms": ms, "gbs": gbs}
+                res["configs"].append(entry)
+                if best is None or gbs > best["gbs"]:
+                    best = entry
+            res["best"][f"{row_bytes}B_{mb}MB"] = best
+            del ids
+        del table
+    res["status_word"] = int(status.item())
+    return res
 
 
 def run_secondary(name, dev, barrier, reduce_max, world, hbm, bf16, kernel="auto"):
@@ -743,9 +824,10 @@ def run_fp8_bench(name, dev, barrier, reduce_max, world, hbm, steps=20, warmup=3
     total_ms = reduce_max(total_ms)
     ms = statistics.mean(per_ms)
 
+    from top_sparse_attention_qsa_b200 import _debug
+
     def step_gather():
-        _capi.sparse_prefill_fp8_fwd(w.q, k8, v8, w.topk_idx, 0.5, 2.0, n_valid=w.n_valid, scale=w.scale,
-                                     out=out, lse=lse, kernel="gather_only")
+        _debug.gather_only(w.q, k8, v8, w.topk_idx, w.n_valid)
 
     _, g_per, _ = time_launches(step_gather, steps, warmup, barrier, "fp8_gather_only")
     g_ms = statistics.mean(g_per)

@@ -47,7 +47,7 @@
 extern "C" {
 #endif
 
-#define QSA_ABI_VERSION 1
+#define QSA_ABI_VERSION 2
 
 typedef enum {
   QSA_OK = 0,
@@ -113,13 +113,7 @@ typedef enum {
                                0 < S < 2^31 - 1), otherwise the warp-MMA kernel */
   QSA_KERNEL_TCGEN05 = 1,   /* persistent warp-specialised cp.async-gather + tcgen05/TMEM
                                kernel only (QSA_ERR_UNSUPPORTED when the layout does not fit) */
-  QSA_KERNEL_WARP_MMA = 2,  /* cp.async-gather + mma.sync kernel (any valid layout) */
-  QSA_KERNEL_GATHER_ONLY = 3 /* measurement only: the KV gather of the tcgen05 kernel alone
-                               (its producer warps, ring and Q loads; the slots are handed
-                               back unread).  Writes neither out nor lse; the status word
-                               still receives out-of-range ids.  Its time is the floor of
-                               the tcgen05 kernel on the same lists.  QSA_ERR_UNSUPPORTED
-                               where QSA_KERNEL_TCGEN05 is. */
+  QSA_KERNEL_WARP_MMA = 2   /* cp.async-gather + mma.sync kernel (any valid layout) */
 } qsa_kernel_t;
 
 /* Same contract as qsa_sparse_prefill_fwd, with an explicit kernel choice.
@@ -144,6 +138,28 @@ qsa_status_t qsa_sparse_prefill_debug_gather(
     const qsa_shape_t* shape, const void* q, const void* k_cache,
     const void* v_cache, const int32_t* topk_idx, const int32_t* n_valid,
     float scale, void* out, float* lse, int32_t* status,
+    int32_t* gathered_ids, void* stream);
+
+/*
+ * Debug dump for every gather path: the kernel of qsa_sparse_prefill_block_fwd
+ * (cache_fp8 = 0, BF16 cache) or of qsa_sparse_prefill_fp8_fwd (cache_fp8 !=
+ * 0, FP8 E4M3 cache, k_scale / v_scale as there), for token lists
+ * (block_size 1, last_slot NULL) or microblock lists, computing out/lse as
+ * that call does and additionally writing, for every key, the slot its K and
+ * V rows were copied from.  Key j of the list of (t, g) is slot
+ * idx[t,g,j / block_size] * block_size + j % block_size; its dump entry is
+ * recovered from the source address of the copies the gather issued: the
+ * slot, or -1 where the key was masked and its rows zero-filled (entry past
+ * n_valid, negative, block or slot past the cache, slot past last_slot[t]),
+ * or -2 if the K and V copies of the key disagreed (never expected).
+ * gathered_ids is int32 device [T, Hkv, K * block_size] contiguous.  Other
+ * arguments and errors as those calls.
+ */
+qsa_status_t qsa_sparse_prefill_debug_gather_lists(
+    const qsa_shape_t* shape, int32_t block_size, const int32_t* last_slot,
+    int32_t cache_fp8, const void* q, const void* k_cache, const void* v_cache,
+    const int32_t* topk_idx, const int32_t* n_valid, float scale,
+    float k_scale, float v_scale, void* out, float* lse, int32_t* status,
     int32_t* gathered_ids, void* stream);
 
 /*
@@ -186,9 +202,12 @@ qsa_status_t qsa_sparse_prefill_block_fwd(const qsa_shape_t* shape,
  * (tcgen05 kind::f8f6f4).  Both MMA operands are E4M3, so the query (scaled
  * per head by a power of two that puts its largest |q| in [128, 256)) and
  * the softmax probabilities are each written as the sum of two E4M3 terms,
- * hi + lo / 16 (the query exactly; the probabilities to 8 significant bits,
- * as the BF16 kernel rounds them), with separate FP32 accumulators for the
- * two terms.  k_scale multiplies the softmax scale and v_scale the
+ * hi + lo / 16, with separate FP32 accumulators for the two terms.  The
+ * query pair is exact for every element within a factor of about 2^13 of
+ * its head's largest |q|; smaller elements lose low bits to E4M3's
+ * subnormal floor (an error below 2^-21 times that largest |q|, far below
+ * the rounding of the scores).  The probabilities keep 8
+ * significant bits, as the BF16 kernel's BF16 P does.  k_scale multiplies the softmax scale and v_scale the
  * normalised output, both in FP32.  Non-finite query elements give
  * unspecified results for their unit.
  *
@@ -206,24 +225,6 @@ qsa_status_t qsa_sparse_prefill_fp8_fwd(const qsa_shape_t* shape,
                                         float k_scale, float v_scale,
                                         void* out, float* lse,
                                         int32_t* status, void* stream);
-
-/* Same contract as qsa_sparse_prefill_fp8_fwd, with an explicit kernel
- * choice: QSA_KERNEL_AUTO or QSA_KERNEL_TCGEN05 run the FP8 kernel;
- * QSA_KERNEL_GATHER_ONLY (token lists only: block_size 1, last_slot NULL)
- * runs only that kernel's KV gather, for measurement, and writes neither out
- * nor lse (the status word still receives out-of-range ids);
- * QSA_KERNEL_WARP_MMA returns QSA_ERR_UNSUPPORTED. */
-qsa_status_t qsa_sparse_prefill_fp8_fwd_with(const qsa_shape_t* shape,
-                                             int32_t block_size,
-                                             const int32_t* last_slot,
-                                             const void* q, const void* k_cache,
-                                             const void* v_cache,
-                                             const int32_t* topk_idx,
-                                             const int32_t* n_valid, float scale,
-                                             float k_scale, float v_scale,
-                                             void* out, float* lse,
-                                             int32_t* status,
-                                             qsa_kernel_t kernel, void* stream);
 
 /*
  * Split-K sparse attention for decode-shaped calls: few query tokens per KV
@@ -359,24 +360,6 @@ qsa_status_t qsa_sparse_prefill_fwd_host(
     const void* v_cache_host, const int32_t* topk_idx_host,
     const int32_t* n_valid_host, float scale, void* out_host,
     float* lse_host, const qsa_device_buffers_t* dev, void* stream);
-
-/*
- * Failure-detection test hook (used by the test suite; not for production
- * calls).  Runs the tcgen05 kernel of qsa_sparse_prefill_fwd_with on the given
- * buffers with the producers' completion signal for the first shared-memory
- * slot of every CTA withheld, so that no pipeline stage can ever complete.
- * Every wait inside the kernel is bounded (2 s), so the kernel must end on
- * its own, with QSA_STATUS_TIMEOUT set in *status (required here) and the
- * CUDA context still usable; out/lse are left unspecified.  Same arguments
- * as qsa_sparse_prefill_fwd; QSA_ERR_UNSUPPORTED when the tcgen05 kernel
- * cannot take the layout.
- */
-qsa_status_t qsa_test_stalled_pipeline(const qsa_shape_t* shape, const void* q,
-                                       const void* k_cache, const void* v_cache,
-                                       const int32_t* topk_idx,
-                                       const int32_t* n_valid, float scale,
-                                       void* out, float* lse, int32_t* status,
-                                       void* stream);
 
 /*
  * QSA indexer and top-K microblock selection (page "Qwen4-Exp QSA llega al

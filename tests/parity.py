@@ -87,3 +87,25 @@ def expected_gather(w):
     if w.n_valid is not None:
         live &= torch.arange(K)[None, None, :] < host(w.n_valid).to(torch.int64)[:, :, None]
     return torch.where(live, idx, torch.full_like(idx, -1)).to(torch.int32)
+
+
+def expected_gather_lists(w, block_size=1, last_slot=None):
+    """The slot the gather must copy for every key of a token or microblock
+    list, [T, Hkv, K * block_size] int32: key j of (t, g) reads slot
+    idx[t,g,j // bs] * bs + j % bs when the entry is live (j // bs <
+    n_valid, id >= 0, its block starts inside the cache) and the slot is
+    inside the cache and at most last_slot[t]; -1 otherwise.  Integer work,
+    compared bit-exactly."""
+    idx = host(w.topk_idx).to(torch.int64)
+    T, Hkv, K = idx.shape
+    S = w.k_cache.shape[0]
+    bs = int(block_size)
+    live = idx >= 0
+    if w.n_valid is not None:
+        live &= torch.arange(K)[None, None, :] < host(w.n_valid).to(torch.int64)[:, :, None]
+    live &= idx * bs < S
+    slot = idx[..., None] * bs + torch.arange(bs)[None, None, None, :]          # [T, Hkv, K, bs]
+    ok = live[..., None] & (slot < S)
+    if last_slot is not None:
+        ok &= slot <= host(last_slot).to(torch.int64)[:, None, None, None]
+    return torch.where(ok, slot, torch.full_like(slot, -1)).reshape(T, Hkv, K * bs).to(torch.int32)

@@ -20,6 +20,12 @@ def capi():
     return _capi
 
 
+@pytest.fixture(scope="module")
+def dbg(capi):
+    from top_sparse_attention_qsa_b200 import _debug
+    return _debug
+
+
 def declared_functions():
     src = open(HEADER).read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
@@ -113,10 +119,10 @@ def test_binding_rejects_host_tensors(capi):
         capi.sparse_prefill_fwd(q.float(), k, k, idx)
 
 
-def test_stall_hook_needs_a_status_word(capi):
+def test_stall_hook_needs_a_status_word(dbg, capi):
     s = _shape(capi)
-    assert capi.library().qsa_test_stalled_pipeline(ctypes.byref(s), P, P, P, P, None, 0.0, P, None,
-                                                    None, None) == 1
+    assert dbg.library().qsa_test_stalled_pipeline(ctypes.byref(s), P, P, P, P, None, 0.0, P, None,
+                                                   None, None) == 1
 
 
 def _ishape(capi, **kw):
@@ -176,21 +182,74 @@ def test_fp8_entry_validation(capi):
 
 
 def test_kernel_choice_validation(capi):
-    """Kernel choices outside the enum, the warp-MMA choice for the FP8
-    cache, and the FP8 gather-only measurement on microblock lists are
-    refused before anything is enqueued."""
+    """Kernel choices outside the enum are refused before anything is
+    enqueued; the production library has no measurement-only choice."""
     lib = capi.library()
     s = _shape(capi)
     fwd_with = lib.qsa_sparse_prefill_fwd_with
     assert fwd_with(ctypes.byref(s), P, P, P, P, None, 0.0, P, None, None, 7, None) == 3
-    f8w = lib.qsa_sparse_prefill_fp8_fwd_with
-    args = (1, None, P, P, P, P, None, 0.0, 1.0, 1.0, P, None, None)
-    assert f8w(ctypes.byref(s), *args, capi.KERNEL_WARP_MMA, None) == 3
-    assert f8w(ctypes.byref(s), *args, 9, None) == 3
-    blk = (4,) + args[1:]
-    assert f8w(ctypes.byref(s), *blk, capi.KERNEL_GATHER_ONLY, None) == 3
-    last = (1, P) + args[2:]
-    assert f8w(ctypes.byref(s), *last, capi.KERNEL_GATHER_ONLY, None) == 3
-    # the same validation as the plain FP8 entry point comes first
+    assert fwd_with(ctypes.byref(s), P, P, P, P, None, 0.0, P, None, None, 3, None) == 3
+    assert "KERNEL_GATHER_ONLY" not in open(HEADER).read()
+
+
+def test_debug_gather_lists_validation(capi):
+    lib = capi.library()
+    s = _shape(capi)
+    dl = lib.qsa_sparse_prefill_debug_gather_lists
+    args = (P, P, P, P, None, 0.0, 1.0, 1.0, P, None, None)
+    assert dl(ctypes.byref(s), 1, None, 0, *args, None, None) == 1          # no dump buffer
+    assert dl(ctypes.byref(s), 3, None, 0, *args, P, None) == 3             # block size 3
     odd = _shape(capi, kv_stride_slot=264, kv_stride_head=264)
-    assert f8w(ctypes.byref(odd), *args, capi.KERNEL_GATHER_ONLY, None) == 4
+    assert dl(ctypes.byref(odd), 1, None, 1, *args, P, None) == 4           # FP8 strides
+    assert dl(ctypes.byref(s), 1, None, 0, *args, P + 2, None) == 4         # dump not 4-byte aligned
+
+
+# --- the debug library (measurement kernels, test hooks) ----------------------
+
+DEBUG_HEADER = os.path.join(ROOT, "include", "qsa_debug.h")
+
+
+def declared_debug_functions():
+    src = re.sub(r"/\*.*?\*/", "", open(DEBUG_HEADER).read(), flags=re.S)
+    return sorted(set(re.findall(r"\b(qsa_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_debug_library_exports_and_production_does_not(dbg, capi):
+    names = declared_debug_functions()
+    assert sorted(dbg.EXPORTS) == names
+    for name in names:
+        assert hasattr(dbg.library(), name), f"libqsa_debug.so does not export {name}"
+        assert name not in capi.EXPORTS
+        # the production library carries no test hook or measurement kernel
+        with pytest.raises(AttributeError):
+            getattr(ctypes.CDLL(capi.LIB_PATH), name)
+    m = re.search(r"#define QSA_DEBUG_ABI_VERSION (\d+)", open(DEBUG_HEADER).read())
+    assert dbg.abi_version() == int(m.group(1))
+
+
+def test_debug_gather_only_validation(dbg, capi):
+    lib = dbg.library()
+    s = _shape(capi)
+    assert lib.qsa_debug_gather_only(None, 0, P, P, P, P, None, None, None) == 1
+    odd = _shape(capi, kv_stride_slot=264, kv_stride_head=264)
+    assert lib.qsa_debug_gather_only(ctypes.byref(odd), 1, P, P, P, P, None, None, None) == 4
+    assert lib.qsa_debug_gather_only(ctypes.byref(_shape(capi, head_dim=128)), 0, P, P, P, P, None, None,
+                                     None) == 3
+
+
+@pytest.mark.parametrize("args,code", [
+    # table, rows, stride, row_bytes, ids, n_ids, method, depth, warps, ctas, sink, sink_words
+    ((None, 64, 512, 512, P, 64, 0, 4, 8, 1, None, 0), 1),
+    ((P, 64, 512, 384, P, 64, 0, 4, 8, 1, None, 0), 3),      # row bytes
+    ((P, 64, 512, 512, P, 64, 0, 3, 8, 1, None, 0), 3),      # cp.async depth 3
+    ((P, 64, 512, 512, P, 64, 1, 2, 8, 1, None, 0), 3),      # ld.v4 depth 2
+    ((P, 64, 512, 512, P, 64, 2, 5, 8, 1, None, 0), 3),      # bulk depth 5
+    ((P, 64, 512, 512, P, 64, 9, 4, 8, 1, None, 0), 3),      # method
+    ((P, 64, 504, 512, P, 64, 0, 4, 8, 1, None, 0), 2),      # stride < row
+    ((P, 64, 520, 512, P, 64, 0, 4, 8, 1, None, 0), 2),      # stride not 16-byte
+    ((P, 0, 512, 512, P, 64, 0, 4, 8, 1, None, 0), 2),       # no rows
+    ((P, 64, 512, 512, P, 64, 0, 4, 33, 1, None, 0), 2),     # warps
+    ((P + 8, 64, 512, 512, P, 64, 0, 4, 8, 1, None, 0), 4),  # table alignment
+])
+def test_debug_gather_peak_validation(dbg, args, code):
+    assert dbg.library().qsa_debug_gather_peak(*args, None, None) == code

@@ -23,10 +23,11 @@ DEV = "cuda"
 
 def test_stalled_pipeline_reports_timeout_and_context_survives():
     from top_sparse_attention_qsa_b200 import _capi as C
+    from top_sparse_attention_qsa_b200 import _debug as D
     w = W.generic_case(T=8, S=2000, Hq=12, Hkv=1, K=300, seed=3, device=DEV)
     status = torch.zeros(1, dtype=torch.int32, device=DEV)
     t0 = time.time()
-    C.run_stalled_pipeline_check(w.q, w.k_cache, w.v_cache, w.topk_idx, status)
+    D.run_stalled_pipeline_check(w.q, w.k_cache, w.v_cache, w.topk_idx, status)
     torch.cuda.synchronize()
     elapsed = time.time() - t0
     assert int(status.item()) & C.STATUS_TIMEOUT

@@ -130,29 +130,3 @@ def test_split_k_decode(C, splits):
     torch.cuda.synchronize()
     ref_out, ref_lse, _ = oracle_fp8(w, k8, v8, 0.5, 2.0)
     compare(host(out), host(lse), ref_out, ref_lse, f"fp8 decode splits={splits}")
-
-
-def test_gather_only_leaves_outputs(C):
-    """The FP8 gather-only choice (a measurement of the FP8 kernel's gather)
-    flags out-of-range ids and writes neither out nor lse."""
-    w = W.make("c2", device=DEV)
-    gen = torch.Generator(device=DEV).manual_seed(5)
-    k8 = W.normal_fp8(tuple(w.k_cache.shape), gen, DEV)
-    v8 = W.normal_fp8(tuple(w.v_cache.shape), gen, DEV)
-    out = torch.full_like(w.q, 3.0)
-    lse = torch.full(w.q.shape[:2], 5.0, dtype=torch.float32, device=DEV)
-    status = torch.zeros(1, dtype=torch.int32, device=DEV)
-    C.sparse_prefill_fp8_fwd(w.q, k8, v8, w.topk_idx, 0.5, 2.0, n_valid=w.n_valid, scale=w.scale, out=out,
-                             lse=lse, status=status, kernel="gather_only")
-    torch.cuda.synchronize()
-    assert int(status.item()) == 0
-    assert bool((out == 3.0).all()) and bool((lse == 5.0).all())
-    w.topk_idx[9, 0, 2] = w.k_cache.shape[0] + 5
-    C.sparse_prefill_fp8_fwd(w.q, k8, v8, w.topk_idx, 0.5, 2.0, n_valid=w.n_valid, scale=w.scale, out=out,
-                             lse=lse, status=status, kernel="gather_only")
-    torch.cuda.synchronize()
-    assert int(status.item()) & C.STATUS_OOB_SLOT
-    assert bool((out == 3.0).all()) and bool((lse == 5.0).all())
-    with pytest.raises(C.QSAError):
-        C.sparse_prefill_fp8_fwd(w.q, k8, v8, w.topk_idx, 0.5, 2.0, n_valid=w.n_valid, scale=w.scale,
-                                 block_size=4, kernel="gather_only")

@@ -236,28 +236,6 @@ def test_out_of_range_slots_flag_status():
     assert int(status.item()) == 0
 
 
-def test_gather_only_measurement_kernel():
-    """The gather-only choice (a measurement of the prefill's gather step)
-    reads the same lists and reports out-of-range ids like the full kernel,
-    but leaves out and lse exactly as they were."""
-    from top_sparse_attention_qsa_b200 import _capi
-    w = W.make("c2", device=DEV)
-    out = torch.full_like(w.q, 3.0)
-    lse = torch.full(w.q.shape[:2], 5.0, dtype=torch.float32, device=DEV)
-    status = torch.zeros(1, dtype=torch.int32, device=DEV)
-    _capi.sparse_prefill_fwd(w.q, w.k_cache, w.v_cache, w.topk_idx, w.n_valid, w.scale, out=out, lse=lse,
-                             status=status, kernel="gather_only")
-    torch.cuda.synchronize()
-    assert int(status.item()) == 0
-    assert bool((out == 3.0).all()) and bool((lse == 5.0).all())
-    w.topk_idx[7, 0, 3] = w.k_cache.shape[0] + 11
-    _capi.sparse_prefill_fwd(w.q, w.k_cache, w.v_cache, w.topk_idx, w.n_valid, w.scale, out=out, lse=lse,
-                             status=status, kernel="gather_only")
-    torch.cuda.synchronize()
-    assert int(status.item()) & _capi.STATUS_OOB_SLOT
-    assert bool((out == 3.0).all()) and bool((lse == 5.0).all())
-
-
 def test_permutation_and_determinism():
     w = W.generic_case(T=50, S=5000, Hq=12, Hkv=1, K=700, seed=9, device=DEV)
     a, la = run_gpu(w)

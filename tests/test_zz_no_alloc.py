@@ -64,3 +64,67 @@ def test_noalloc_refuses_oversized_calls(C):
         C.sparse_decode_fwd_noalloc(w.q, w.k_cache, w.v_cache, w.topk_idx, out,
                                     n_valid=w.n_valid, num_splits=64)
     assert e.value.code == C.QSA_ERR_SCRATCH
+
+
+def _pair(C, w, splits):
+    ref_out, ref_lse = C.sparse_decode_fwd(w.q, w.k_cache, w.v_cache, w.topk_idx, w.n_valid, w.scale,
+                                           num_splits=splits)
+    out = torch.full_like(w.q, 7.0)
+    lse = torch.full(w.q.shape[:2], 7.0, dtype=torch.float32, device=DEV)
+    C.sparse_decode_fwd_noalloc(w.q, w.k_cache, w.v_cache, w.topk_idx, out, lse, n_valid=w.n_valid,
+                                scale=w.scale, num_splits=splits)
+    torch.cuda.synchronize()
+    return out, lse, ref_out, ref_lse
+
+
+def test_noalloc_automatic_and_single_chunk_choices(C):
+    # few (token, KV head) units: the automatic choice splits the lists
+    w = W.config_decode(device=DEV, seed=303, B=2, ctx=8192, heads=(24, 2), topk=2048, local=256)
+    assert C.decode_num_splits(w.q, w.k_cache, w.topk_idx, 0) > 1
+    _close(*_pair(C, w, 0))
+    # one chunk: no scratch at all, the prefill kernel runs directly
+    assert C.decode_workspace_bytes(w.q, w.k_cache, w.topk_idx, 1) == 0
+    _close(*_pair(C, w, 1))
+
+
+def test_noalloc_smaller_call_after_larger(C):
+    # a large call leaves its partials in the shared array; a smaller one
+    # that follows must read only its own
+    big = W.config_decode(device=DEV, seed=404, B=16, ctx=8192, heads=(24, 2), topk=2048, local=256)
+    small = W.config_decode(device=DEV, seed=505, B=3, ctx=4096, heads=(12, 1), topk=1024, local=128)
+    _close(*_pair(C, big, 8))
+    _close(*_pair(C, small, 2))
+
+
+def test_noalloc_allocates_nothing(C):
+    w = W.config_decode(device=DEV, seed=606, B=8, ctx=8192, heads=(24, 2), topk=2048, local=256)
+    out = torch.empty_like(w.q)
+    lse = torch.empty(w.q.shape[:2], dtype=torch.float32, device=DEV)
+    C.sparse_decode_fwd_noalloc(w.q, w.k_cache, w.v_cache, w.topk_idx, out, lse, n_valid=w.n_valid,
+                                scale=w.scale, num_splits=4)                 # warm-up: module loaded
+    torch.cuda.synchronize()
+    alloc0, free0 = torch.cuda.memory_allocated(), torch.cuda.mem_get_info()[0]
+    for _ in range(3):
+        C.sparse_decode_fwd_noalloc(w.q, w.k_cache, w.v_cache, w.topk_idx, out, lse, n_valid=w.n_valid,
+                                    scale=w.scale, num_splits=4)
+    torch.cuda.synchronize()
+    assert torch.cuda.memory_allocated() == alloc0
+    assert torch.cuda.mem_get_info()[0] == free0
+
+
+def test_noalloc_against_the_oracle(C):
+    """The allocation-free path checked on its own against the FP64 oracle,
+    not only against the workspace path that shares its kernels."""
+    import oracle
+    w = W.config_decode(device=DEV, seed=707, B=6, ctx=8192, heads=(16, 2), topk=2048, local=256)
+    w.n_valid[2, 1] = 700
+    out = torch.empty_like(w.q)
+    lse = torch.empty(w.q.shape[:2], dtype=torch.float32, device=DEV)
+    C.sparse_decode_fwd_noalloc(w.q, w.k_cache, w.v_cache, w.topk_idx, out, lse, n_valid=w.n_valid,
+                                scale=w.scale, num_splits=4)
+    torch.cuda.synchronize()
+    ref_out, ref_lse, _ = oracle.sparse_prefill(w.q.cpu(), w.k_cache.cpu(), w.v_cache.cpu(), w.topk_idx.cpu(),
+                                                w.n_valid.cpu(), w.scale)
+    o = out.double().cpu().numpy()
+    assert np.all(np.abs(o - ref_out) <= 1e-2 + 1e-2 * np.abs(ref_out))
+    assert np.abs(lse.double().cpu().numpy() - ref_lse).max() <= 1e-3

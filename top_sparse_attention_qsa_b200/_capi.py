@@ -26,18 +26,17 @@ QSA_OK, QSA_ERR_NULL, QSA_ERR_SHAPE, QSA_ERR_UNSUPPORTED, QSA_ERR_ALIGN, QSA_ERR
 NOALLOC_SCRATCH_BYTES = 16 << 20
 STATUS_OOB_SLOT = 1
 STATUS_TIMEOUT = 2
-KERNEL_AUTO, KERNEL_TCGEN05, KERNEL_WARP_MMA, KERNEL_GATHER_ONLY = 0, 1, 2, 3
-KERNELS = {"auto": KERNEL_AUTO, "tcgen05": KERNEL_TCGEN05, "warp_mma": KERNEL_WARP_MMA,
-           "gather_only": KERNEL_GATHER_ONLY}
+KERNEL_AUTO, KERNEL_TCGEN05, KERNEL_WARP_MMA = 0, 1, 2
+KERNELS = {"auto": KERNEL_AUTO, "tcgen05": KERNEL_TCGEN05, "warp_mma": KERNEL_WARP_MMA}
 HEAD_DIM = 256
 
 # Every symbol include/qsa.h declares.
 EXPORTS = ("qsa_sparse_prefill_fwd", "qsa_sparse_prefill_fwd_with", "qsa_sparse_prefill_debug_gather",
-           "qsa_sparse_prefill_block_fwd",
+           "qsa_sparse_prefill_debug_gather_lists", "qsa_sparse_prefill_block_fwd",
            "qsa_sparse_prefill_fwd_host", "qsa_sparse_decode_fwd", "qsa_sparse_decode_workspace_bytes",
-           "qsa_sparse_decode_num_splits", "qsa_sparse_decode_fwd_noalloc", "qsa_test_stalled_pipeline",
-           "qsa_sparse_prefill_fp8_fwd", "qsa_sparse_prefill_fp8_fwd_with", "qsa_sparse_decode_fp8_fwd", "qsa_indexer_scores", "qsa_topk_select", "qsa_status_string",
-           "qsa_abi_version")
+           "qsa_sparse_decode_num_splits", "qsa_sparse_decode_fwd_noalloc",
+           "qsa_sparse_prefill_fp8_fwd", "qsa_sparse_decode_fp8_fwd", "qsa_indexer_scores",
+           "qsa_topk_select", "qsa_status_string", "qsa_abi_version")
 
 
 class Shape(ctypes.Structure):
@@ -104,19 +103,17 @@ _lib.qsa_sparse_decode_num_splits.argtypes = [ctypes.POINTER(Shape), ctypes.c_in
 _lib.qsa_sparse_decode_fwd_noalloc.restype = ctypes.c_int
 _lib.qsa_sparse_decode_fwd_noalloc.argtypes = [ctypes.POINTER(Shape), _vp, _vp, _vp, _vp, _vp,
                                                ctypes.c_float, _vp, _vp, _vp, ctypes.c_int32, _vp]
-_lib.qsa_test_stalled_pipeline.restype = ctypes.c_int
-_lib.qsa_test_stalled_pipeline.argtypes = [ctypes.POINTER(Shape), _vp, _vp, _vp, _vp, _vp,
-                                           ctypes.c_float, _vp, _vp, _vp, _vp]
+_lib.qsa_sparse_prefill_debug_gather_lists.restype = ctypes.c_int
+_lib.qsa_sparse_prefill_debug_gather_lists.argtypes = [ctypes.POINTER(Shape), ctypes.c_int32, _vp, ctypes.c_int32,
+                                                       _vp, _vp, _vp, _vp, _vp, ctypes.c_float, ctypes.c_float,
+                                                       ctypes.c_float, _vp, _vp, _vp, _vp, _vp]
 _lib.qsa_sparse_prefill_block_fwd.restype = ctypes.c_int
 _lib.qsa_sparse_prefill_block_fwd.argtypes = [ctypes.POINTER(Shape), ctypes.c_int32, _vp, _vp, _vp, _vp,
                                               _vp, _vp, ctypes.c_float, _vp, _vp, _vp, _vp]
+_lib.qsa_sparse_prefill_fp8_fwd.restype = ctypes.c_int
 _lib.qsa_sparse_prefill_fp8_fwd.argtypes = [ctypes.POINTER(Shape), ctypes.c_int32, _vp, _vp, _vp, _vp, _vp,
                                             _vp, ctypes.c_float, ctypes.c_float, ctypes.c_float, _vp, _vp,
                                             _vp, _vp]
-_lib.qsa_sparse_prefill_fp8_fwd_with.restype = ctypes.c_int
-_lib.qsa_sparse_prefill_fp8_fwd_with.argtypes = [ctypes.POINTER(Shape), ctypes.c_int32, _vp, _vp, _vp, _vp, _vp,
-                                                 _vp, ctypes.c_float, ctypes.c_float, ctypes.c_float, _vp, _vp,
-                                                 _vp, ctypes.c_int, _vp]
 _lib.qsa_sparse_decode_fp8_fwd.argtypes = [ctypes.POINTER(Shape), _vp, _vp, _vp, _vp, _vp, ctypes.c_float,
                                            ctypes.c_float, ctypes.c_float, _vp, _vp, _vp, ctypes.c_int32,
                                            _vp, ctypes.c_size_t, _vp]
@@ -199,8 +196,7 @@ def sparse_prefill_fwd(q, k_cache, v_cache, topk_idx, n_valid=None, scale: float
                        out=None, lse=None, status=None, stream=None, want_lse: bool = True,
                        kernel: str = "auto"):
     """QSA sparse prefill on the GPU.  Returns (out [T,Hq,D] bf16, lse [T,Hq] fp32 or None).
-    kernel: "auto" | "tcgen05" | "warp_mma" | "gather_only" (see qsa_kernel_t; the last
-    runs only the KV gather, for measurement, and leaves out and lse untouched)."""
+    kernel: "auto" | "tcgen05" | "warp_mma" (see qsa_kernel_t)."""
     dev = q.device
     _need(q, "q", torch.bfloat16, dev)
     _need(k_cache, "k_cache", torch.bfloat16, dev)
@@ -384,26 +380,6 @@ def sparse_decode_fwd_noalloc(q, k_cache, v_cache, topk_idx, out, lse=None, n_va
     return out, lse
 
 
-def run_stalled_pipeline_check(q, k_cache, v_cache, topk_idx, status, n_valid=None, scale: float = 0.0,
-                               stream=None):
-    """Failure-detection hook: runs the tcgen05 kernel with one pipeline signal
-    withheld; the kernel must stop on its own and set STATUS_TIMEOUT in `status`."""
-    dev = q.device
-    for name, x, dt in (("q", q, torch.bfloat16), ("k_cache", k_cache, torch.bfloat16),
-                        ("v_cache", v_cache, torch.bfloat16), ("topk_idx", topk_idx, torch.int32),
-                        ("status", status, torch.int32)):
-        _need(x, name, dt, dev)
-    _check_kv(k_cache, v_cache)
-    out = torch.empty(q.shape, dtype=torch.bfloat16, device=dev)
-    lse = torch.empty(q.shape[:2], dtype=torch.float32, device=dev)
-    shape = make_shape(q, k_cache, topk_idx, out, lse)
-    if stream is None:
-        stream = torch.cuda.current_stream(dev).cuda_stream
-    _raise(_lib.qsa_test_stalled_pipeline(ctypes.byref(shape), _ptr(q), _ptr(k_cache), _ptr(v_cache),
-                                          _ptr(topk_idx), _ptr(n_valid), float(scale), _ptr(out),
-                                          _ptr(lse), _ptr(status), stream))
-
-
 def sparse_prefill_block_fwd(q, k_cache, v_cache, block_idx, block_size: int, last_slot=None,
                              n_valid=None, scale: float = 0.0, out=None, lse=None, status=None,
                              stream=None, want_lse: bool = True):
@@ -444,13 +420,10 @@ def sparse_prefill_block_fwd(q, k_cache, v_cache, block_idx, block_size: int, la
 
 def sparse_prefill_fp8_fwd(q, k_cache, v_cache, topk_idx, k_scale: float = 1.0, v_scale: float = 1.0,
                            n_valid=None, scale: float = 0.0, block_size: int = 1, last_slot=None,
-                           out=None, lse=None, status=None, stream=None, want_lse: bool = True,
-                           kernel: str = "auto"):
+                           out=None, lse=None, status=None, stream=None, want_lse: bool = True):
     """FP8 E4M3 KV cache (torch.float8_e4m3fn [S, Hkv, 256]); element value =
     stored value * k_scale (v_scale).  Token lists (block_size 1) or
-    microblock lists with an optional last_slot [T] int32.  kernel: "auto" |
-    "tcgen05" | "gather_only" (the KV gather alone, for measurement; out and
-    lse untouched; token lists only)."""
+    microblock lists with an optional last_slot [T] int32."""
     dev = q.device
     _need(q, "q", torch.bfloat16, dev)
     _need(k_cache, "k_cache", torch.float8_e4m3fn, dev)
@@ -477,11 +450,48 @@ def sparse_prefill_fp8_fwd(q, k_cache, v_cache, topk_idx, k_scale: float = 1.0, 
     shape = make_shape(q, k_cache, topk_idx, out, lse)
     if stream is None:
         stream = torch.cuda.current_stream(dev).cuda_stream
-    _raise(_lib.qsa_sparse_prefill_fp8_fwd_with(ctypes.byref(shape), int(block_size), _ptr(last_slot), _ptr(q),
-                                                _ptr(k_cache), _ptr(v_cache), _ptr(topk_idx), _ptr(n_valid),
-                                                float(scale), float(k_scale), float(v_scale), _ptr(out),
-                                                _ptr(lse), _ptr(status), KERNELS[kernel], stream))
+    _raise(_lib.qsa_sparse_prefill_fp8_fwd(ctypes.byref(shape), int(block_size), _ptr(last_slot), _ptr(q),
+                                           _ptr(k_cache), _ptr(v_cache), _ptr(topk_idx), _ptr(n_valid),
+                                           float(scale), float(k_scale), float(v_scale), _ptr(out),
+                                           _ptr(lse), _ptr(status), stream))
     return out, lse
+
+
+def sparse_prefill_debug_gather_lists(q, k_cache, v_cache, topk_idx, block_size: int = 1, last_slot=None,
+                                      n_valid=None, scale: float = 0.0, k_scale: float = 1.0,
+                                      v_scale: float = 1.0, status=None, stream=None):
+    """The kernel of sparse_prefill_block_fwd (BF16 cache) or
+    sparse_prefill_fp8_fwd (float8_e4m3fn cache) with the gather dump:
+    returns (out, lse, gathered [T, Hkv, K * block_size] int32), the slot each
+    key's rows were copied from, -1 where masked."""
+    dev = q.device
+    fp8 = k_cache.dtype == torch.float8_e4m3fn
+    cdt = torch.float8_e4m3fn if fp8 else torch.bfloat16
+    _need(q, "q", torch.bfloat16, dev)
+    _need(k_cache, "k_cache", cdt, dev)
+    _need(v_cache, "v_cache", cdt, dev)
+    _need(topk_idx, "topk_idx", torch.int32, dev)
+    _check_kv(k_cache, v_cache)
+    if last_slot is not None:
+        _need_tok(last_slot, "last_slot", q.shape[0], dev)
+    if n_valid is not None:
+        _need(n_valid, "n_valid", torch.int32, dev)
+        if not n_valid.is_contiguous() or tuple(n_valid.shape) != tuple(topk_idx.shape[:2]):
+            raise ValueError("n_valid must be a contiguous [T, Hkv] tensor")
+    if status is not None:
+        _need(status, "status", torch.int32, dev)
+    out = torch.empty(q.shape, dtype=torch.bfloat16, device=dev)
+    lse = torch.empty(q.shape[:2], dtype=torch.float32, device=dev)
+    T, Hkv, K = topk_idx.shape
+    ids = torch.empty((T, Hkv, K * int(block_size)), dtype=torch.int32, device=dev)
+    shape = make_shape(q, k_cache, topk_idx, out, lse)
+    if stream is None:
+        stream = torch.cuda.current_stream(dev).cuda_stream
+    _raise(_lib.qsa_sparse_prefill_debug_gather_lists(
+        ctypes.byref(shape), int(block_size), _ptr(last_slot), 1 if fp8 else 0, _ptr(q), _ptr(k_cache),
+        _ptr(v_cache), _ptr(topk_idx), _ptr(n_valid), float(scale), float(k_scale), float(v_scale), _ptr(out),
+        _ptr(lse), _ptr(status), _ptr(ids), stream))
+    return out, lse, ids
 
 
 def sparse_decode_fp8_fwd(q, k_cache, v_cache, topk_idx, k_scale: float = 1.0, v_scale: float = 1.0,

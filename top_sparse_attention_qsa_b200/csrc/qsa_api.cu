@@ -12,154 +12,20 @@
 #include <mutex>
 
 #include "qsa.h"
-#include "qsa_host.cuh"
-#include "qsa_gather_only.cuh"
+#include "qsa_launch.cuh"
 #include "qsa_merge.cuh"
-#include "qsa_prefill_mma.cuh"
-#include "qsa_prefill_tc.cuh"
-#include "qsa_prefill_f8.cuh"
 
 namespace {
 
 using namespace qsa::host;
-
-// Validates `s` and the pointers of a forward call.  Returns QSA_OK or the
-// first error found; never touches device memory.
-qsa_status_t validate(const qsa_shape_t* s, const void* q, const void* k, const void* v,
-                      const int32_t* idx, const void* out) {
-  if (s == nullptr) return QSA_ERR_NULL;
-  if (s->num_tokens < 0 || s->topk < 0 || s->num_slots < 0 || s->num_q_heads <= 0 ||
-      s->num_kv_heads <= 0)
-    return QSA_ERR_SHAPE;
-  if (s->num_q_heads % s->num_kv_heads != 0) return QSA_ERR_SHAPE;
-  if (s->head_dim != qsa::kHeadDim) return QSA_ERR_UNSUPPORTED;
-  const int G = s->num_q_heads / s->num_kv_heads;
-  if (G > 16) return QSA_ERR_UNSUPPORTED;
-  if (s->num_kv_heads > 65535 || s->num_tokens > 0x7fffffffLL) return QSA_ERR_UNSUPPORTED;
-  if (s->num_tokens == 0) return QSA_OK;
-  if (q == nullptr || out == nullptr) return QSA_ERR_NULL;
-  const bool reads_cache = s->topk > 0;
-  if (reads_cache && (k == nullptr || v == nullptr || idx == nullptr)) return QSA_ERR_NULL;
-  // strides: non-negative, rows 16-byte aligned
-  const int64_t st[] = {s->q_stride_tok, s->q_stride_head, s->o_stride_tok, s->o_stride_head,
-                        s->kv_stride_slot, s->kv_stride_head};
-  for (int64_t x : st)
-    if (x < 0) return QSA_ERR_SHAPE;
-  if (s->idx_stride_tok < 0 || s->idx_stride_head < 0 || s->lse_stride_tok < 0) return QSA_ERR_SHAPE;
-  if (reads_cache && s->num_slots > 0 && s->kv_stride_slot == 0) return QSA_ERR_SHAPE;
-  for (int64_t x : st)
-    if (x % 8 != 0) return QSA_ERR_ALIGN;
-  if (!aligned16(q) || !aligned16(out)) return QSA_ERR_ALIGN;
-  if (reads_cache && (!aligned16(k) || !aligned16(v))) return QSA_ERR_ALIGN;
-  if (reads_cache && (reinterpret_cast<uintptr_t>(idx) & 3u)) return QSA_ERR_ALIGN;
-  if (s->num_slots > 0x80000000LL) return QSA_ERR_UNSUPPORTED;  // int32 slot ids
-  return QSA_OK;
-}
-
-template <int NT, bool kDump>
-cudaError_t launch_mma(const qsa::PrefillParams& p, cudaStream_t stream) {
-  using C = qsa::MmaCfg<NT>;
-  static std::atomic<int> done[kMaxDevices];
-  auto kernel = qsa::qsa_prefill_mma_kernel<NT, kDump>;
-  cudaError_t e = set_smem_once(kernel, C::SMEM, done);
-  if (e != cudaSuccess) return e;
-  dim3 grid(static_cast<unsigned>(p.T), static_cast<unsigned>(p.Hkv));
-  kernel<<<grid, C::THREADS, C::SMEM, stream>>>(p);
-  return cudaGetLastError();
-}
-
-// ---------------------------------------------------------------- TMA path
-
-// Fills the Q tensor map of the tcgen05 kernel.  Returns false when a TMA
-// descriptor cannot express the Q layout or there is nothing to gather (the
-// warp-MMA kernel takes those calls).
-bool make_tc_params(const qsa_shape_t* s, const void* q, qsa::tc::TcParams* tp) {
-  using namespace qsa::tc;
-  EncodeTiledFn enc = encode_fn();
-  if (enc == nullptr) return false;
-  if (s->topk <= 0 || s->num_slots <= 0 || s->num_slots >= 0x7fffffffLL) return false;
-  const cuuint32_t elem_str[3] = {1, 1, 1};
-  const uint64_t hq = static_cast<uint64_t>(s->num_q_heads);
-  uint64_t st_h = static_cast<uint64_t>(s->q_stride_head) * 2;
-  if (hq == 1 || st_h < 512) {
-    if (hq > 1) return false;
-    st_h = 512;
-  }
-  uint64_t st_t = static_cast<uint64_t>(s->q_stride_tok) * 2;
-  if (s->num_tokens == 1 || st_t < st_h * hq) {
-    if (s->num_tokens > 1) return false;
-    st_t = st_h * hq;
-  }
-  const cuuint64_t qdims[3] = {256, hq, static_cast<cuuint64_t>(s->num_tokens)};
-  const cuuint64_t qstr[2] = {st_h, st_t};
-  const cuuint32_t qbox[3] = {64, static_cast<cuuint32_t>(kGp), 1};
-  return enc(&tp->tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(q), qdims, qstr, qbox,
-             elem_str, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-template <bool kBlocks>
-cudaError_t launch_f8(const qsa::tc::TcParams& tp, cudaStream_t stream) {
-  static std::atomic<int> done[kMaxDevices];
-  auto kernel = qsa::f8::qsa_prefill_f8_kernel<kBlocks>;
-  cudaError_t e = set_smem_once(kernel, qsa::f8::F_SMEM, done);
-  if (e != cudaSuccess) return e;
-  const int64_t units = tp.T * tp.Hkv;
-  const int nsm = sm_count();
-  if (nsm <= 0) return cudaErrorInvalidDevice;
-  const unsigned grid = static_cast<unsigned>(units < nsm ? units : nsm);
-  kernel<<<grid, qsa::f8::kThreads8, qsa::f8::F_SMEM, stream>>>(tp);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_gather_only(const qsa::tc::TcParams& tp, cudaStream_t stream) {
-  static std::atomic<int> done[kMaxDevices];
-  auto kernel = qsa::tc::qsa_gather_only_kernel;
-  cudaError_t e = set_smem_once(kernel, qsa::tc::SMEM_BYTES, done);
-  if (e != cudaSuccess) return e;
-  const int64_t units = tp.T * tp.Hkv;
-  const int nsm = sm_count();
-  if (nsm <= 0) return cudaErrorInvalidDevice;
-  const unsigned grid = static_cast<unsigned>(units < nsm ? units : nsm);
-  kernel<<<grid, qsa::tc::kGatherOnlyThreads, qsa::tc::SMEM_BYTES, stream>>>(tp);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_f8_gather_only(const qsa::tc::TcParams& tp, cudaStream_t stream) {
-  static std::atomic<int> done[kMaxDevices];
-  auto kernel = qsa::f8::qsa_gather_only_f8_kernel;
-  cudaError_t e = set_smem_once(kernel, qsa::f8::F_SMEM, done);
-  if (e != cudaSuccess) return e;
-  const int64_t units = tp.T * tp.Hkv;
-  const int nsm = sm_count();
-  if (nsm <= 0) return cudaErrorInvalidDevice;
-  const unsigned grid = static_cast<unsigned>(units < nsm ? units : nsm);
-  kernel<<<grid, 32 * (qsa::tc::kProducerWarps + 1), qsa::f8::F_SMEM, stream>>>(tp);
-  return cudaGetLastError();
-}
-
-template <bool kDump, bool kStall = false, bool kBlocks = false>
-cudaError_t launch_tc(const qsa::tc::TcParams& tp, cudaStream_t stream) {
-  static std::atomic<int> done[kMaxDevices];
-  auto kernel = qsa::tc::qsa_prefill_tc_kernel<kDump, kStall, kBlocks>;
-  cudaError_t e = set_smem_once(kernel, qsa::tc::SMEM_BYTES, done);
-  if (e != cudaSuccess) return e;
-  const int64_t units = tp.T * tp.Hkv;
-  int nsm = sm_count();
-  if (nsm <= 0) return cudaErrorInvalidDevice;
-  const unsigned grid = static_cast<unsigned>(units < nsm ? units : nsm);
-  kernel<<<grid, qsa::tc::kThreads, qsa::tc::SMEM_BYTES, stream>>>(tp);
-  return cudaGetLastError();
-}
+using namespace qsa::launch;
 
 qsa_status_t run_forward(const qsa_shape_t* s, const void* q, const void* k, const void* v,
                          const int32_t* idx, const int32_t* n_valid, float scale, void* out,
                          float* lse, int32_t* status, int32_t* gathered, void* stream,
-                         qsa_kernel_t which = QSA_KERNEL_AUTO, bool stall_test = false) {
-  if (which != QSA_KERNEL_AUTO && which != QSA_KERNEL_TCGEN05 && which != QSA_KERNEL_WARP_MMA &&
-      which != QSA_KERNEL_GATHER_ONLY)
+                         qsa_kernel_t which = QSA_KERNEL_AUTO) {
+  if (which != QSA_KERNEL_AUTO && which != QSA_KERNEL_TCGEN05 && which != QSA_KERNEL_WARP_MMA)
     return QSA_ERR_UNSUPPORTED;
-  if (which == QSA_KERNEL_GATHER_ONLY && (gathered != nullptr || stall_test)) return QSA_ERR_UNSUPPORTED;
   qsa_status_t rc = validate(s, q, k, v, idx, out);
   if (rc != QSA_OK) return rc;
   if (gathered != nullptr && s->topk > 0 && (reinterpret_cast<uintptr_t>(gathered) & 3u))
@@ -169,6 +35,17 @@ qsa_status_t run_forward(const qsa_shape_t* s, const void* q, const void* k, con
   if (gathered != nullptr && s->topk > 0) {
     const size_t n = static_cast<size_t>(s->num_tokens) * s->num_kv_heads * s->topk;
     if (cudaMemsetAsync(gathered, 0xff, n * sizeof(int32_t), st) != cudaSuccess) return QSA_ERR_CUDA;
+  }
+  cudaError_t e;
+  const bool dump = gathered != nullptr;
+  static thread_local qsa::tc::TcParams tp;
+  const bool use_tc = which != QSA_KERNEL_WARP_MMA && make_tc_params(s, q, &tp);
+  if (which == QSA_KERNEL_TCGEN05 && !use_tc) return QSA_ERR_UNSUPPORTED;
+  if (use_tc) {
+    fill_tc_params(&tp, s, q, k, v, idx, n_valid, scale, 1.f, 1.f, out, lse, status, 0, nullptr);
+    tp.gathered = gathered;
+    e = dump ? launch_tc<true>(tp, st) : launch_tc<false>(tp, st);
+    return e == cudaSuccess ? QSA_OK : QSA_ERR_CUDA;
   }
   qsa::PrefillParams p;
   p.q = static_cast<const __nv_bfloat16*>(q);
@@ -196,46 +73,7 @@ qsa_status_t run_forward(const qsa_shape_t* s, const void* q, const void* k, con
   p.lse_st = s->lse_stride_tok;
   const float sc = scale > 0.f ? scale : 0.0625f;  // 1/sqrt(256)
   p.scale_log2 = sc * 1.4426950408889634f;
-  cudaError_t e;
-  const bool dump = gathered != nullptr;
-  static thread_local qsa::tc::TcParams tp;
-  const bool use_tc = which != QSA_KERNEL_WARP_MMA && make_tc_params(s, q, &tp);
-  if ((which == QSA_KERNEL_TCGEN05 || which == QSA_KERNEL_GATHER_ONLY) && !use_tc) return QSA_ERR_UNSUPPORTED;
-  if (use_tc) {
-    tp.idx = idx;
-    tp.n_valid = n_valid;
-    tp.kraw = k;
-    tp.vraw = v;
-    tp.kv_ss = s->kv_stride_slot;
-    tp.kv_sh = s->kv_stride_head;
-    tp.out = p.out;
-    tp.lse = lse;
-    tp.status = status;
-    tp.gathered = gathered;
-    tp.T = p.T;
-    tp.idx_st = p.idx_st;
-    tp.idx_sh = p.idx_sh;
-    tp.o_st = p.o_st;
-    tp.o_sh = p.o_sh;
-    tp.lse_st = p.lse_st;
-    tp.Hkv = p.Hkv;
-    tp.G = p.G;
-    tp.K = p.K;
-    tp.S = static_cast<int32_t>(p.S);
-    tp.scale_log2 = p.scale_log2;
-    tp.splits = 1;
-    tp.chunk = p.K;
-    tp.part_o = nullptr;
-    tp.part_lse = nullptr;
-    tp.block_shift = 0;
-    tp.last_slot = nullptr;
-    tp.o_scale = 1.f;
-    if (which == QSA_KERNEL_GATHER_ONLY)
-      e = launch_gather_only(tp, st);
-    else
-      e = stall_test ? launch_tc<false, true>(tp, st)
-                     : (dump ? launch_tc<true>(tp, st) : launch_tc<false>(tp, st));
-  } else if (p.G <= 8)
+  if (p.G <= 8)
     e = dump ? launch_mma<1, true>(p, st) : launch_mma<1, false>(p, st);
   else
     e = dump ? launch_mma<2, true>(p, st) : launch_mma<2, false>(p, st);
@@ -311,7 +149,7 @@ qsa_status_t run_lists(const qsa_shape_t* shape, int32_t block_size, const int32
                        const void* q, const void* k_cache, const void* v_cache,
                        const int32_t* topk_idx, const int32_t* n_valid, float scale,
                        float k_scale, float v_scale, bool fp8, void* out, float* lse,
-                       int32_t* status, void* stream, bool gather_only = false);
+                       int32_t* status, void* stream, int32_t* gathered = nullptr);
 
 // The host-buffer entry point cuts the query tokens into chunks of about
 // kHostChunkTokens (at most kHostMaxChunks) so that the copies of one chunk
@@ -369,38 +207,12 @@ qsa_status_t run_decode(const qsa_shape_t* s, const void* q, const void* k, cons
   if (reinterpret_cast<uintptr_t>(workspace) & 255u) return QSA_ERR_ALIGN;
   float* part_o = static_cast<float*>(workspace);
   float* part_lse = reinterpret_cast<float*>(static_cast<char*>(workspace) + pl.lse_offset);
-  const float sc = scale > 0.f ? scale : 0.0625f;
-  tp.idx = idx;
-  tp.n_valid = n_valid;
-  tp.kraw = k;
-  tp.vraw = v;
-  tp.out = static_cast<__nv_bfloat16*>(out);
-  tp.lse = lse;
-  tp.status = status;
-  tp.gathered = nullptr;
-  tp.T = s->num_tokens;
-  tp.idx_st = s->idx_stride_tok;
-  tp.idx_sh = s->idx_stride_head;
-  tp.o_st = s->o_stride_tok;
-  tp.o_sh = s->o_stride_head;
-  tp.lse_st = s->lse_stride_tok;
-  tp.kv_ss = s->kv_stride_slot;
-  tp.kv_sh = s->kv_stride_head;
-  tp.Hkv = s->num_kv_heads;
-  tp.G = s->num_q_heads / s->num_kv_heads;
-  tp.K = s->topk;
-  tp.S = static_cast<int32_t>(s->num_slots);
-  tp.scale_log2 = sc * (fp8 ? k_scale : 1.f) * 1.4426950408889634f;
+  fill_tc_params(&tp, s, q, k, v, idx, n_valid, scale, fp8 ? k_scale : 1.f, fp8 ? v_scale : 1.f, out, lse,
+                 status, 0, nullptr);
   tp.splits = pl.splits;
   tp.chunk = pl.chunk;
   tp.part_o = part_o;
   tp.part_lse = part_lse;
-  tp.block_shift = 0;
-  tp.last_slot = nullptr;
-  tp.o_scale = fp8 ? v_scale : 1.f;
-  tp.q_ptr = q;
-  tp.q_st = s->q_stride_tok;
-  tp.q_sh = s->q_stride_head;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if ((fp8 ? launch_f8<false>(tp, st) : launch_tc<false>(tp, st)) != cudaSuccess) return QSA_ERR_CUDA;
   if (launch_merge(s, part_o, part_lse, pl.splits, out, lse, st) != cudaSuccess) return QSA_ERR_CUDA;
@@ -421,26 +233,56 @@ size_t span_bytes(int64_t n0, int64_t s0, int64_t n1, int64_t s1, int64_t inner,
 // only a stand-in symbol); it passes the device address looked up below.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[QSA_NOALLOC_SCRATCH_BYTES];
 
-// Device address of g_noalloc_scratch on the current device, looked up once
-// per device (cudaGetSymbolAddress allocates nothing).
-cudaError_t noalloc_scratch_address(void** ptr) {
-  static std::atomic<void*> cache[kMaxDevices];
+// Device address of g_noalloc_scratch in the current context.  The lookup
+// (cudaGetSymbolAddress, which allocates nothing) is cached per device
+// together with the context it was made in, and redone when the current
+// context differs (after cudaDeviceReset, or under another context): the
+// module, and with it the array, may then sit at another address.  A lookup
+// that would have to happen while `stream` is being captured is refused
+// (cudaErrorStreamCaptureUnsupported), since it may load the module.
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+
+CtxGetCurrentFn ctx_get_current_fn() {
+  static CtxGetCurrentFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(f);
+  });
+  return fn;
+}
+
+cudaError_t noalloc_scratch_address(cudaStream_t stream, void** ptr) {
+  struct Entry {
+    CUcontext ctx = nullptr;
+    void* ptr = nullptr;
+  };
+  static Entry cache[kMaxDevices];
   static std::mutex lock;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-  void* p = cache[dev].load(std::memory_order_acquire);
-  if (p == nullptr) {
-    std::lock_guard<std::mutex> g(lock);
-    p = cache[dev].load(std::memory_order_acquire);
-    if (p == nullptr) {
-      e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-      if (e != cudaSuccess) return e;
-      cache[dev].store(p, std::memory_order_release);
-    }
+  CtxGetCurrentFn get_ctx = ctx_get_current_fn();
+  if (get_ctx == nullptr) return cudaErrorContextIsDestroyed;
+  CUcontext ctx = nullptr;
+  if (get_ctx(&ctx) != CUDA_SUCCESS) return cudaErrorContextIsDestroyed;
+  std::lock_guard<std::mutex> g(lock);
+  if (ctx == nullptr || cache[dev].ctx != ctx || cache[dev].ptr == nullptr) {
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    if ((e = cudaStreamIsCapturing(stream, &cap)) != cudaSuccess) return e;
+    if (cap != cudaStreamCaptureStatusNone) return cudaErrorStreamCaptureUnsupported;
+    void* p = nullptr;
+    // (this also makes the device's primary context current if none was)
+    if ((e = cudaGetSymbolAddress(&p, g_noalloc_scratch)) != cudaSuccess) return e;
+    if (get_ctx(&ctx) != CUDA_SUCCESS || ctx == nullptr) return cudaErrorContextIsDestroyed;
+    cache[dev].ctx = ctx;
+    cache[dev].ptr = p;
   }
-  *ptr = p;
+  *ptr = cache[dev].ptr;
   return cudaSuccess;
 }
 
@@ -449,62 +291,41 @@ qsa_status_t run_lists(const qsa_shape_t* shape, int32_t block_size, const int32
                        const void* q, const void* k_cache, const void* v_cache,
                        const int32_t* topk_idx, const int32_t* n_valid, float scale,
                        float k_scale, float v_scale, bool fp8, void* out, float* lse,
-                       int32_t* status, void* stream, bool gather_only) {
+                       int32_t* status, void* stream, int32_t* gathered) {
   qsa_status_t rc = validate(shape, q, k_cache, v_cache, topk_idx, out);
   if (rc != QSA_OK) return rc;
-  if (gather_only && (!fp8 || block_size != 1 || last_slot != nullptr)) return QSA_ERR_UNSUPPORTED;
   if (fp8 && shape->topk > 0 && (shape->kv_stride_slot % 16 != 0 || shape->kv_stride_head % 16 != 0))
     return QSA_ERR_ALIGN;   // FP8 rows move in 16-byte pieces of 16 elements
-  int shift = -1;
-  for (int b = 0; b <= 4; ++b)
-    if (block_size == (1 << b)) shift = b;
+  const int shift = block_shift_of(block_size);
   if (shift < 0) return QSA_ERR_UNSUPPORTED;
   if ((static_cast<int64_t>(shape->topk) << shift) > 0x7fffffffLL) return QSA_ERR_UNSUPPORTED;
+  if (gathered != nullptr && shape->topk > 0 && (reinterpret_cast<uintptr_t>(gathered) & 3u))
+    return QSA_ERR_ALIGN;
   if (shape->num_tokens == 0) return QSA_OK;
   static thread_local qsa::tc::TcParams tp;
   if (!make_tc_params(shape, q, &tp)) return QSA_ERR_UNSUPPORTED;
-  const float sc = scale > 0.f ? scale : 0.0625f;
-  tp.idx = topk_idx;
-  tp.n_valid = n_valid;
-  tp.kraw = k_cache;
-  tp.vraw = v_cache;
-  tp.out = static_cast<__nv_bfloat16*>(out);
-  tp.lse = lse;
-  tp.status = status;
-  tp.gathered = nullptr;
-  tp.T = shape->num_tokens;
-  tp.idx_st = shape->idx_stride_tok;
-  tp.idx_sh = shape->idx_stride_head;
-  tp.o_st = shape->o_stride_tok;
-  tp.o_sh = shape->o_stride_head;
-  tp.lse_st = shape->lse_stride_tok;
-  tp.kv_ss = shape->kv_stride_slot;
-  tp.kv_sh = shape->kv_stride_head;
-  tp.Hkv = shape->num_kv_heads;
-  tp.G = shape->num_q_heads / shape->num_kv_heads;
-  tp.K = shape->topk;
-  tp.S = static_cast<int32_t>(shape->num_slots);
-  // an FP8 cache's K scale multiplies every score; its V scale the output
-  tp.scale_log2 = sc * (fp8 ? k_scale : 1.f) * 1.4426950408889634f;
-  tp.o_scale = fp8 ? v_scale : 1.f;
-  tp.splits = 1;
-  tp.chunk = shape->topk << shift;
-  tp.part_o = nullptr;
-  tp.part_lse = nullptr;
-  tp.block_shift = shift;
-  tp.last_slot = last_slot;
-  tp.q_ptr = q;
-  tp.q_st = shape->q_stride_tok;
-  tp.q_sh = shape->q_stride_head;
-  const bool plain = shift == 0 && last_slot == nullptr;
+  fill_tc_params(&tp, shape, q, k_cache, v_cache, topk_idx, n_valid, scale, fp8 ? k_scale : 1.f,
+                 fp8 ? v_scale : 1.f, out, lse, status, shift, last_slot);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (gathered != nullptr) {
+    const size_t n = static_cast<size_t>(shape->num_tokens) * shape->num_kv_heads * (static_cast<size_t>(shape->topk) << shift);
+    if (cudaMemsetAsync(gathered, 0xff, n * sizeof(int32_t), st) != cudaSuccess) return QSA_ERR_CUDA;
+    tp.gathered = gathered;
+  }
+  const bool plain = shift == 0 && last_slot == nullptr;
+  const bool dump = gathered != nullptr;
   cudaError_t e;
-  if (gather_only)
-    e = launch_f8_gather_only(tp, st);
-  else if (fp8)
-    e = plain ? launch_f8<false>(tp, st) : launch_f8<true>(tp, st);
-  else
-    e = plain ? launch_tc<false>(tp, st) : launch_tc<false, false, true>(tp, st);
+  if (fp8) {
+    if (dump)
+      e = plain ? launch_f8<false, true>(tp, st) : launch_f8<true, true>(tp, st);
+    else
+      e = plain ? launch_f8<false>(tp, st) : launch_f8<true>(tp, st);
+  } else {
+    if (dump)
+      e = plain ? launch_tc<true>(tp, st) : launch_tc<true, false, true>(tp, st);
+    else
+      e = plain ? launch_tc<false>(tp, st) : launch_tc<false, false, true>(tp, st);
+  }
   return e == cudaSuccess ? QSA_OK : QSA_ERR_CUDA;
 }
 
@@ -606,7 +427,7 @@ qsa_status_t qsa_sparse_prefill_fwd_host(const qsa_shape_t* s, const void* q_hos
                      lse_host != nullptr ? reinterpret_cast<float*>(const_cast<char*>(at(dev->lse, t0 * s->lse_stride_tok, 4)))
                                          : nullptr,
                      dev->status, nullptr, st);
-    if (rc != QSA_OK) return rc;
+    if (rc != QSA_OK) break;
     // its outputs
     if (hp != nullptr)
       ok = cudaEventRecord(hp->ev[2 + kHostMaxChunks + c], st) == cudaSuccess &&
@@ -617,9 +438,17 @@ qsa_status_t qsa_sparse_prefill_fwd_host(const qsa_shape_t* s, const void* q_hos
       ok = copy(const_cast<char*>(at(lse_host, t0 * s->lse_stride_tok, 4)), at(dev->lse, t0 * s->lse_stride_tok, 4),
                 span_bytes(tc, s->lse_stride_tok, 1, 0, Hq, 4), cudaMemcpyDeviceToHost, down);
   }
-  // `stream` ends after the last copy down
-  if (hp != nullptr)
-    ok = ok && cudaEventRecord(hp->ev[1], down) == cudaSuccess && cudaStreamWaitEvent(st, hp->ev[1], 0) == cudaSuccess;
+  // `stream` ends after every copy enqueued on the two copy streams, on the
+  // error paths too: the caller may free or reuse the host buffers as soon
+  // as `stream` is done
+  if (hp != nullptr) {
+    const bool joined = cudaEventRecord(hp->ev[0], up) == cudaSuccess &&
+                        cudaStreamWaitEvent(st, hp->ev[0], 0) == cudaSuccess &&
+                        cudaEventRecord(hp->ev[1], down) == cudaSuccess &&
+                        cudaStreamWaitEvent(st, hp->ev[1], 0) == cudaSuccess;
+    ok = ok && joined;
+  }
+  if (rc != QSA_OK) return rc;
   return ok ? QSA_OK : QSA_ERR_CUDA;
 }
 
@@ -672,7 +501,11 @@ qsa_status_t qsa_sparse_decode_fwd_noalloc(const qsa_shape_t* shape, const void*
   const size_t need = pl.splits > 1 ? pl.total_bytes : 0;
   if (need > QSA_NOALLOC_SCRATCH_BYTES) return QSA_ERR_SCRATCH;
   void* scratch = nullptr;
-  if (need > 0 && noalloc_scratch_address(&scratch) != cudaSuccess) return QSA_ERR_CUDA;
+  if (need > 0) {
+    const cudaError_t e = noalloc_scratch_address(static_cast<cudaStream_t>(stream), &scratch);
+    if (e == cudaErrorStreamCaptureUnsupported) return QSA_ERR_UNSUPPORTED;
+    if (e != cudaSuccess) return QSA_ERR_CUDA;
+  }
   return run_decode(shape, q, k_cache, v_cache, topk_idx, n_valid, scale, out, lse, status,
                     num_splits, scratch, need, stream);
 }
@@ -697,27 +530,17 @@ qsa_status_t qsa_sparse_prefill_fp8_fwd(const qsa_shape_t* shape, int32_t block_
                    k_scale, v_scale, true, out, lse, status, stream);
 }
 
-qsa_status_t qsa_sparse_prefill_fp8_fwd_with(const qsa_shape_t* shape, int32_t block_size,
-                                             const int32_t* last_slot, const void* q,
-                                             const void* k_cache, const void* v_cache,
-                                             const int32_t* topk_idx, const int32_t* n_valid,
-                                             float scale, float k_scale, float v_scale, void* out,
-                                             float* lse, int32_t* status, qsa_kernel_t kernel,
-                                             void* stream) {
-  if (kernel != QSA_KERNEL_AUTO && kernel != QSA_KERNEL_TCGEN05 && kernel != QSA_KERNEL_GATHER_ONLY)
-    return QSA_ERR_UNSUPPORTED;
+qsa_status_t qsa_sparse_prefill_debug_gather_lists(const qsa_shape_t* shape, int32_t block_size,
+                                                   const int32_t* last_slot, int32_t cache_fp8,
+                                                   const void* q, const void* k_cache, const void* v_cache,
+                                                   const int32_t* topk_idx, const int32_t* n_valid,
+                                                   float scale, float k_scale, float v_scale, void* out,
+                                                   float* lse, int32_t* status, int32_t* gathered_ids,
+                                                   void* stream) {
+  if (gathered_ids == nullptr) return QSA_ERR_NULL;
   return run_lists(shape, block_size, last_slot, q, k_cache, v_cache, topk_idx, n_valid, scale,
-                   k_scale, v_scale, true, out, lse, status, stream, kernel == QSA_KERNEL_GATHER_ONLY);
-}
-
-qsa_status_t qsa_test_stalled_pipeline(const qsa_shape_t* shape, const void* q,
-                                       const void* k_cache, const void* v_cache,
-                                       const int32_t* topk_idx, const int32_t* n_valid,
-                                       float scale, void* out, float* lse, int32_t* status,
-                                       void* stream) {
-  if (status == nullptr) return QSA_ERR_NULL;
-  return run_forward(shape, q, k_cache, v_cache, topk_idx, n_valid, scale, out, lse, status,
-                     nullptr, stream, QSA_KERNEL_TCGEN05, true);
+                   cache_fp8 ? k_scale : 1.f, cache_fp8 ? v_scale : 1.f, cache_fp8 != 0, out, lse, status,
+                   stream, gathered_ids);
 }
 
 const char* qsa_status_string(qsa_status_t status) {

@@ -10,10 +10,17 @@
 // slot holds a whole K or V tile (128 keys x 256 dims x 1 B), so six slots
 // keep three tiles in flight, twice the BF16 kernel's 1.5.  Both MMA operands
 // of kind::f8f6f4 are FP8, so the BF16 query and the FP32 probabilities are
-// each written as an exact-enough pair of E4M3 terms:
-//   q * 2^a_h = q_hi + q_lo / 16     (exact: a BF16 value has 8 significant
-//                                     bits, each E4M3 term 4; a_h puts the
-//                                     head's largest |q| in [128, 256))
+// each written as a pair of E4M3 terms:
+//   q * 2^a_h = q_hi + q_lo / 16     (a_h puts the head's largest |q| in
+//                                     [128, 256); a BF16 value has 8
+//                                     significant bits, each E4M3 term 4, so
+//                                     the pair is exact for every element
+//                                     of magnitude >= 2^-6 after scaling,
+//                                     i.e. within about 2^13 of the head's
+//                                     largest; smaller ones lose low bits to
+//                                     E4M3's subnormal floor, an error below
+//                                     2^-14 after scaling, 2^-21 of the
+//                                     largest)
 //   p         = p_hi + p_lo / 16     (8 significant bits, like the BF16 P of
 //                                     the BF16 kernel; p <= 2^8 by the lazy
 //                                     rescale)
@@ -75,7 +82,9 @@ constexpr uint32_t kIdescPV8 = kIdescQK8 | (1u << 15) | (1u << 16);
 
 // ------------------------------------------------------------------ producers
 
-template <bool kBlocks>
+// kDump: also write, per key, the slot its K and V copies read (see the BF16
+// kernel's producer).
+template <bool kBlocks, bool kDump = false>
 __device__ void producer8(const TcParams& p, const Sync& sy, uint32_t sb, int pw, int lane) {
   uint32_t c_slot = 0;
   const int64_t units = num_units(p);
@@ -101,6 +110,7 @@ __device__ void producer8(const TcParams& p, const Sync& sy, uint32_t sb, int pw
         id = -1;
         if (p.status != nullptr) atomicOr(p.status, static_cast<int32_t>(kStatusOob));
       }
+      int32_t from_k[kDump ? rows_w / 2 : 1];
 #pragma unroll 1
       for (int h = 0; h < 2; ++h) {                  // K tile, then V tile
         const uint32_t slot = c_slot % kSlots8;
@@ -115,6 +125,17 @@ __device__ void producer8(const TcParams& p, const Sync& sy, uint32_t sb, int pw
           const bool live = rid >= 0;
           const char* src = live ? src0 + static_cast<int64_t>(rid) * row_bytes : src0;
           cp_async_16(dst0 + r * 128 + (((cc & 7) ^ (r & 7)) << 4), src, live ? 16 : 0);
+          if (kDump && cc == 0) {
+            const int32_t from = live ? static_cast<int32_t>((src - src0) / row_bytes) : -1;
+            if (h == 0) {
+              from_k[kDump ? k : 0] = from;
+            } else {
+              const int64_t key = un.j0 + static_cast<int64_t>(i) * kKeys + r;
+              const int64_t n_keys = static_cast<int64_t>(p.K) << p.block_shift;
+              if (key < n_keys)
+                p.gathered[(un.t * p.Hkv + un.g) * n_keys + key] = from == from_k[kDump ? k : 0] ? from : -2;
+            }
+          }
         }
         cp_async_mbar_arrive(sy.bar(G_FULL + slot));
         ++c_slot;
@@ -572,7 +593,7 @@ __device__ void softmax8(const TcParams& p, const Sync& sy, uint32_t sb, uint8_t
 
 // ------------------------------------------------------------------ kernel
 
-template <bool kBlocks>
+template <bool kBlocks, bool kDump = false>
 __global__ void __launch_bounds__(kThreads8, 1) qsa_prefill_f8_kernel(const __grid_constant__ TcParams p) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -617,7 +638,7 @@ __global__ void __launch_bounds__(kThreads8, 1) qsa_prefill_f8_kernel(const __gr
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(sp + F_MISC);
 
   if (warp < kProducerWarps) {
-    producer8<kBlocks>(p, sy, sb, warp, lane);
+    producer8<kBlocks, kDump>(p, sy, sb, warp, lane);
   } else if (warp == kWarpQ8) {
     q8(p, sy, sb, sp, lane);
   } else if (warp == kWarpQK8) {

@@ -89,7 +89,7 @@ struct TcParams {
   __nv_bfloat16* out;
   float* lse;
   int32_t* status;
-  int32_t* gathered;                // debug dump [T][Hkv][K] or nullptr
+  int32_t* gathered;                // debug dump [T][Hkv][K << block_shift] or nullptr
   int64_t T;
   int64_t idx_st, idx_sh, o_st, o_sh, lse_st, kv_ss, kv_sh;
   int32_t Hkv, G, K, S;
@@ -272,10 +272,7 @@ __device__ void producer_role(const TcParams& p, const Sync& sy, uint32_t sb, in
         id = -1;
         if (p.status != nullptr) atomicOr(p.status, static_cast<int32_t>(kStatusOob));
       }
-      if (kDump && own) {
-        const int j = un.j0 + i * kKeys + jr;
-        if (j < p.K) p.gathered[(un.t * p.Hkv + un.g) * static_cast<int64_t>(p.K) + j] = id < 0 ? -1 : id;
-      }
+      int32_t from_k[kDump ? rows_w / 2 : 1];       // kDump: slot behind each K copy of this lane
 #pragma unroll 1
       for (int h = 0; h < 4; ++h) {
         const uint32_t slot = c_slot % kSlots;
@@ -291,6 +288,20 @@ __device__ void producer_role(const TcParams& p, const Sync& sy, uint32_t sb, in
           const bool live = rid >= 0;
           const char* src = live ? src0 + static_cast<int64_t>(rid) * row_bytes : src0;
           cp_async_16(dst0 + r * 128 + (((cc & 7) ^ (r & 7)) << 4), src, live ? 16 : 0);
+          if (kDump && cc == 0 && (h & 1) == 0) {
+            // debug dump: the slot this copy read, recovered from its source
+            // address (-1 for a zero-filled row); the K and V copies of a key
+            // must agree, else -2 is recorded
+            const int32_t from = live ? static_cast<int32_t>((src - src0) / row_bytes) : -1;
+            if (h == 0) {
+              from_k[kDump ? k : 0] = from;
+            } else {
+              const int64_t key = un.j0 + static_cast<int64_t>(i) * kKeys + r;
+              const int64_t n_keys = static_cast<int64_t>(p.K) << p.block_shift;
+              if (key < n_keys)
+                p.gathered[(un.t * p.Hkv + un.g) * n_keys + key] = from == from_k[kDump ? k : 0] ? from : -2;
+            }
+          }
         }
         if (!(kStall && c_slot == 0)) cp_async_mbar_arrive(sy.bar(B_FULL + slot));
         ++c_slot;
