@@ -646,10 +646,12 @@ def run_e2e(w, args, barrier, reduce_max, T_job, dev):
 # and 256-byte rows: each fills a shared-memory ring of at most 192 KB per SM
 # (cp.async, bulk) or keeps 64-256 KB of loads in flight (ld.v4).
 PEAK_CONFIGS = {
-    512: [("cp_async", 2, 24, 1), ("cp_async", 4, 12, 1), ("cp_async", 8, 6, 1), ("cp_async", 4, 8, 1),
+    512: [("cp_async", 1, 32, 1), ("cp_async", 2, 16, 1), ("cp_async", 1, 24, 2), ("cp_async", 2, 12, 2),
+          ("cp_async", 2, 24, 1), ("cp_async", 4, 12, 1), ("cp_async", 8, 6, 1), ("cp_async", 4, 8, 1),
           ("ld_v4", 4, 32, 1), ("ld_v4", 8, 32, 1), ("ld_v4", 16, 16, 1), ("ld_v4", 16, 16, 2),
           ("bulk", 1, 12, 1), ("bulk", 2, 6, 1), ("bulk", 3, 4, 1)],
-    256: [("cp_async", 2, 24, 1), ("cp_async", 4, 12, 1), ("cp_async", 8, 6, 1),
+    256: [("cp_async", 1, 32, 1), ("cp_async", 1, 24, 2), ("cp_async", 2, 24, 1), ("cp_async", 4, 12, 1),
+          ("cp_async", 8, 6, 1),
           ("ld_v4", 8, 32, 1), ("ld_v4", 16, 16, 1), ("ld_v4", 16, 16, 2),
           ("bulk", 2, 12, 1), ("bulk", 3, 8, 1), ("bulk", 4, 6, 1)],
 }

@@ -41,7 +41,7 @@ qsa_status_t qsa_debug_gather_only(const qsa_shape_t* shape, int32_t cache_fp8,
 
 /* Methods of qsa_debug_gather_peak. */
 #define QSA_PEAK_CP_ASYNC 0 /* 16-byte cp.async per lane into a per-warp ring
-                               of `depth` groups of 4 KB (depth 2, 4 or 8) */
+                               of `depth` groups of 4 KB (depth 1, 2, 4 or 8) */
 #define QSA_PEAK_LD_V4 1    /* 16-byte ld.global.cg.v4 per lane, `depth`
                                loads in flight per lane (4, 8 or 16; at most
                                16 warps per CTA for 16) */

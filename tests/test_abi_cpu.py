@@ -242,6 +242,7 @@ def test_debug_gather_only_validation(dbg, capi):
     ((None, 64, 512, 512, P, 64, 0, 4, 8, 1, None, 0), 1),
     ((P, 64, 512, 384, P, 64, 0, 4, 8, 1, None, 0), 3),      # row bytes
     ((P, 64, 512, 512, P, 64, 0, 3, 8, 1, None, 0), 3),      # cp.async depth 3
+    ((P, 64, 512, 512, P, 64, 0, 16, 2, 1, None, 0), 3),     # cp.async depth 16
     ((P, 64, 512, 512, P, 64, 1, 2, 8, 1, None, 0), 3),      # ld.v4 depth 2
     ((P, 64, 512, 512, P, 64, 2, 5, 8, 1, None, 0), 3),      # bulk depth 5
     ((P, 64, 512, 512, P, 64, 9, 4, 8, 1, None, 0), 3),      # method

@@ -94,7 +94,7 @@ cudaError_t run_peak(int method, int depth, const PeakLaunch& L, cudaStream_t st
 bool peak_depth_ok(int method, int depth) {
   using namespace qsa::peak;
   switch (method) {
-    case kCpAsync: return depth == 2 || depth == 4 || depth == 8;
+    case kCpAsync: return depth == 1 || depth == 2 || depth == 4 || depth == 8;
     case kLdV4: return depth == 4 || depth == 8 || depth == 16;
     case kBulk: return depth >= 1 && depth <= 4;
     default: return false;

@@ -72,8 +72,12 @@ __global__ void gather_peak_cp_async(const __grid_constant__ PeakParams p) {
   const uint32_t ring = smem_u32(smem) + static_cast<uint32_t>(warp * kDepth * kGroupBytes);
   const int sub = lane / kChunks, cc = lane % kChunks;
   int k = 0;
+  // the ids of a group are loaded one group ahead, off the copies' critical path
+  auto ids_of = [&](int64_t g) { return (g < g1 && lane < kRowsPerGroup) ? __ldg(p.ids + g * kRowsPerGroup + lane) : 0; };
+  int32_t next = ids_of(g0 + warp);
   for (int64_t g = g0 + warp; g < g1; g += nw) {
-    const int32_t mine = lane < kRowsPerGroup ? __ldg(p.ids + g * kRowsPerGroup + lane) : 0;
+    const int32_t mine = next;
+    next = ids_of(g + nw);
     const uint32_t dst = ring + static_cast<uint32_t>(k * kGroupBytes);
 #pragma unroll
     for (int i = 0; i < kInstrPerGroup; ++i) {
@@ -99,13 +103,21 @@ __global__ void __launch_bounds__(kDepth >= 16 ? 512 : 1024) gather_peak_ld_v4(c
   cta_share(p.n_ids / kRowsPerGroup, g0, g1);
   const int sub = lane / kChunks, cc = lane % kChunks;
   uint32_t acc = 0;
-  for (int64_t g = g0 + warp; g < g1; g += nw) {
-    int32_t mine[(kRowsPerGroup + 31) / 32];
+  constexpr int kIdWords = (kRowsPerGroup + 31) / 32;
+  int32_t next[kIdWords];
+  auto load_ids = [&](int64_t g, int32_t (&dst)[kIdWords]) {
 #pragma unroll
-    for (int j = 0; j < (kRowsPerGroup + 31) / 32; ++j) {
+    for (int j = 0; j < kIdWords; ++j) {
       const int r = j * 32 + lane;
-      mine[j] = r < kRowsPerGroup ? __ldg(p.ids + g * kRowsPerGroup + r) : 0;
+      dst[j] = (g < g1 && r < kRowsPerGroup) ? __ldg(p.ids + g * kRowsPerGroup + r) : 0;
     }
+  };
+  load_ids(g0 + warp, next);
+  for (int64_t g = g0 + warp; g < g1; g += nw) {
+    int32_t mine[kIdWords];
+#pragma unroll
+    for (int j = 0; j < kIdWords; ++j) mine[j] = next[j];
+    load_ids(g + nw, next);
     uint4 v[kDepth];
 #pragma unroll
     for (int i = 0; i < kDepth; ++i) {
@@ -142,7 +154,10 @@ __global__ void gather_peak_bulk(const __grid_constant__ PeakParams p) {
   cta_share(p.n_ids / kBulkRows, g0, g1);
   uint32_t n_issued = 0;
   bool ok = true;
+  int32_t next = g0 + warp < g1 ? __ldg(p.ids + (g0 + warp) * kBulkRows + lane) : 0;
   for (int64_t g = g0 + warp; g < g1 && ok; g += nw, ++n_issued) {
+    const int32_t mine = next;
+    next = g + nw < g1 ? __ldg(p.ids + (g + nw) * kBulkRows + lane) : 0;
     const uint32_t st = n_issued % kDepth;
     const uint32_t bar = bars + 8 * st;
     if (n_issued >= static_cast<uint32_t>(kDepth)) {
@@ -160,7 +175,7 @@ __global__ void gather_peak_bulk(const __grid_constant__ PeakParams p) {
     }
     if (lane == 0) tc::mbar_arrive_expect_tx(bar, kStageBytes);
     __syncwarp();
-    const int64_t row = clamp_row(__ldg(p.ids + g * kBulkRows + lane), p.rows);
+    const int64_t row = clamp_row(mine, p.rows);
     bulk_copy_g2s(ring + st * kStageBytes + lane * kRowBytes, p.table + row * p.row_stride, kRowBytes, bar);
   }
   // drain: every stage that received copies completes before the CTA exits
