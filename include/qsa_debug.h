@@ -63,8 +63,9 @@ qsa_status_t qsa_debug_gather_only(const qsa_shape_t* shape, int32_t cache_fp8,
  *                loads live); may be NULL otherwise.
  *   status     : device int32 or NULL; bit 1 when a bounded wait of
  *                QSA_PEAK_BULK ran out (2 s).
- * QSA_ERR_UNSUPPORTED: an unsupported row_bytes / method / depth, or a
- * shared-memory ring larger than one SM holds.  One launch; no allocation.
+ * QSA_ERR_UNSUPPORTED: an unsupported row_bytes / method / depth, more than
+ * 1024 threads per SM (warps x 32 x ctas_per_sm), or a shared-memory ring
+ * larger than one SM holds.  One launch; no allocation.
  */
 qsa_status_t qsa_debug_gather_peak(const void* table, int64_t rows,
                                    int64_t row_stride_bytes, int32_t row_bytes,

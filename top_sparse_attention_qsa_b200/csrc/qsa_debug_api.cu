@@ -121,7 +121,7 @@ qsa_status_t qsa_debug_gather_only(const qsa_shape_t* shape, int32_t cache_fp8, 
   cudaError_t e;
   if (cache_fp8) {
     static std::atomic<int> done[kMaxDevices];
-    e = launch_persistent(qsa::f8::qsa_gather_only_f8_kernel, tp, 32 * (qsa::tc::kProducerWarps + 1),
+    e = launch_persistent(qsa::f8::qsa_gather_only_f8_kernel, tp, 32 * (qsa::f8::kProducerWarps8 + 1),
                           qsa::f8::F_SMEM, done, st);
   } else {
     static std::atomic<int> done[kMaxDevices];
@@ -156,6 +156,8 @@ qsa_status_t qsa_debug_gather_peak(const void* table, int64_t rows, int64_t row_
   }
   if (L.smem > 227 * 1024 || static_cast<int64_t>(L.smem) * ctas_per_sm > 228 * 1024) return QSA_ERR_UNSUPPORTED;
   if (method == kLdV4 && warps > (depth >= 16 ? 16 : 32)) return QSA_ERR_UNSUPPORTED;
+  // every kernel is built for at most 1024 threads per SM (64 registers each)
+  if (warps * 32 * ctas_per_sm > 1024) return QSA_ERR_UNSUPPORTED;
   if (method == kLdV4 && (sink == nullptr || sink_words < static_cast<int64_t>(L.grid) * L.threads))
     return QSA_ERR_SHAPE;
   if (n_ids == 0) return QSA_OK;

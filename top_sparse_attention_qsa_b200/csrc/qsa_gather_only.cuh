@@ -85,7 +85,7 @@ namespace f8 {
 // The same for the FP8 kernel's gather: its producer warps (one 32 KB slot
 // per K or V tile of 256-byte rows), token lists; Q is not loaded, since the
 // FP8 kernel reads it from global memory in its own warp.
-__global__ void __launch_bounds__(32 * (kProducerWarps + 1), 1)
+__global__ void __launch_bounds__(32 * (kProducerWarps8 + 1), 1)
     qsa_gather_only_f8_kernel(const __grid_constant__ TcParams p) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -98,14 +98,14 @@ __global__ void __launch_bounds__(32 * (kProducerWarps + 1), 1)
   sy.status = p.status;
   if (threadIdx.x == 0) {
     for (int s = 0; s < kSlots8; ++s) {
-      mbar_init(sy.bar(G_FULL + s), 32 * kProducerWarps);
+      mbar_init(sy.bar(G_FULL + s), 32 * kProducerWarps8);
       mbar_init(sy.bar(G_EMPTY + s), 1);
     }
     *sy.abort_flag = 0u;
     mbar_fence_init();
   }
   __syncthreads();
-  if (warp < kProducerWarps) {
+  if (warp < kProducerWarps8) {
     producer8<false>(p, sy, sb, warp, lane);
   } else if (lane == 0) {
     uint32_t c_slot = 0;

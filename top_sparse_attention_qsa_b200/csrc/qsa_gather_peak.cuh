@@ -61,7 +61,7 @@ __device__ __forceinline__ void cta_share(int64_t n, int64_t& begin, int64_t& en
 
 // cp.async into a per-warp ring of kDepth groups (kDepth x 4 KB per warp).
 template <int kRowBytes, int kDepth>
-__global__ void gather_peak_cp_async(const __grid_constant__ PeakParams p) {
+__global__ void __launch_bounds__(1024) gather_peak_cp_async(const __grid_constant__ PeakParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
   constexpr int kRowsPerInstr = 512 / kRowBytes;
   constexpr int kRowsPerGroup = kInstrPerGroup * kRowsPerInstr;
@@ -140,7 +140,7 @@ __device__ __forceinline__ void bulk_copy_g2s(uint32_t dst, const void* src, uin
 // One 1-d bulk copy per row: each warp owns kDepth stages of 32 rows and one
 // mbarrier per stage.  Waits are bounded (2 s) and set status bit 1 on expiry.
 template <int kRowBytes, int kDepth>
-__global__ void gather_peak_bulk(const __grid_constant__ PeakParams p) {
+__global__ void __launch_bounds__(1024) gather_peak_bulk(const __grid_constant__ PeakParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
   constexpr int kStageBytes = kBulkRows * kRowBytes;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;

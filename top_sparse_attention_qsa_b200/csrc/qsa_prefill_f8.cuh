@@ -56,6 +56,7 @@ namespace f8 {
 using namespace tc;
 
 constexpr int kSlots8 = 6;                    // 32 KB: one K or V tile
+constexpr int kProducerWarps8 = 4;            // 32 rows of every tile each
 constexpr int kQ8Bytes = kGp * 256;           // one E4M3 Q term: 16 heads x 256 dims
 constexpr int kQ8Block = 2 * kGp * 128;       // one 128-dim block of both terms: 32 rows x 128 B
 constexpr int kP8Bytes = kKeys * kGp;         // one E4M3 P term: 128 keys x 16 heads
@@ -91,7 +92,7 @@ __device__ void producer8(const TcParams& p, const Sync& sy, uint32_t sb, int pw
   const int cc = lane & 15;                          // 16-byte chunk of the 256-byte row
   const int rsel = lane >> 4;                        // which of the two rows of an instruction
   const uint32_t dchunk = static_cast<uint32_t>((cc >> 3) * kBlockBytes);
-  constexpr int rows_w = kKeys / kProducerWarps;
+  constexpr int rows_w = kKeys / kProducerWarps8;
   bool ok = true;
   for (int64_t u = blockIdx.x; u < units && ok; u += gridDim.x) {
     const Unit un = decode_unit(p, u);
@@ -329,9 +330,9 @@ __device__ void pv8(const TcParams& p, const Sync& sy, uint32_t sb, uint32_t tme
 
 constexpr int kSmWarps = 8;     // two per TMEM lane quadrant, 8 heads each
 constexpr int kHpw = kGp / 2;   // heads per softmax warp
-constexpr int kWarpQ8 = kProducerWarps, kWarpQK8 = kProducerWarps + 1, kWarpPV8 = kProducerWarps + 2,
-              kWarpSm8 = kProducerWarps + 3;
-constexpr int kThreads8 = 32 * (kProducerWarps + 3 + kSmWarps);
+constexpr int kWarpQ8 = kProducerWarps8, kWarpQK8 = kProducerWarps8 + 1, kWarpPV8 = kProducerWarps8 + 2,
+              kWarpSm8 = kProducerWarps8 + 3;
+constexpr int kThreads8 = 32 * (kProducerWarps8 + 3 + kSmWarps);
 
 // Reduce 8 per-lane values across the 32 lanes of a warp by exchanging halves
 // (7 shuffles for the exchange, 2 for the rest).  Lane l ends with the result
@@ -607,7 +608,7 @@ __global__ void __launch_bounds__(kThreads8, 1) qsa_prefill_f8_kernel(const __gr
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kSlots8; ++s) {
-      mbar_init(sy.bar(G_FULL + s), 32 * kProducerWarps);
+      mbar_init(sy.bar(G_FULL + s), 32 * kProducerWarps8);
       mbar_init(sy.bar(G_EMPTY + s), 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -637,7 +638,7 @@ __global__ void __launch_bounds__(kThreads8, 1) qsa_prefill_f8_kernel(const __gr
   tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(sp + F_MISC);
 
-  if (warp < kProducerWarps) {
+  if (warp < kProducerWarps8) {
     producer8<kBlocks, kDump>(p, sy, sb, warp, lane);
   } else if (warp == kWarpQ8) {
     q8(p, sy, sb, sp, lane);

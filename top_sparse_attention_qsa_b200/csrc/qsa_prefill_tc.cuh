@@ -56,14 +56,25 @@ constexpr int kSlots = 6;
 constexpr int kBlockBytes = 16384;         // 128 rows x 64 dims (one 128-byte swizzle column block)
 constexpr int kQBytes = kGp * 512;         // 16 rows x 256 dims x 2 B
 constexpr int kPBytes = kKeys * kGp * 2;   // 128 keys x 16 heads x 2 B
-#ifndef QSA_TC_PRODUCER_WARPS
-#define QSA_TC_PRODUCER_WARPS 4
-#endif
-constexpr int kProducerWarps = QSA_TC_PRODUCER_WARPS;  // must divide 128 rows into 2-row steps
+// Sixteen producer warps: many warps with few copies each in flight move
+// random rows faster than a few warps with many (the gather probe's finding).
+constexpr int kProducerWarps = 16;         // 8 rows of every tile each
 static_assert(kKeys % (2 * kProducerWarps) == 0 && kKeys / kProducerWarps <= 32,
               "each producer lane holds at most one row id; rows per warp must be even");
-constexpr int kWarpQK = kProducerWarps, kWarpPV = kProducerWarps + 1, kWarpSoftmax0 = kProducerWarps + 2;
-constexpr int kThreads = 32 * (kProducerWarps + 6);
+// Warp roles, in warpgroups of four (registers are rebalanced per warpgroup):
+//   warps 0-3     softmax (TMEM lane quadrants 0-3)
+//   warps 4-19    producers
+//   warp 20       score MMA issuer, warp 21 PV MMA issuer, warps 22-23 idle
+constexpr int kWarpSoftmax0 = 0, kWarpProducer0 = 4;
+constexpr int kWarpQK = kWarpProducer0 + kProducerWarps, kWarpPV = kWarpQK + 1;
+constexpr int kThreads = 32 * 24;
+// Registers per thread after setmaxnreg: softmax / producers / MMA warpgroup.
+// Their sum over the six warpgroups (x 128 threads) must stay within what the
+// block is launched with, 768 threads x 80 registers: 176 + 4 * 64 + 48 = 480
+// = 6 * 80.
+constexpr int kRegsSoftmax = 176, kRegsProducer = 64, kRegsMma = 48, kRegsLaunch = 80;
+static_assert(kRegsSoftmax + 4 * kRegsProducer + kRegsMma <= 6 * kRegsLaunch,
+              "the register split exceeds the launch allocation");
 constexpr int kTmemCols = 64;              // S double buffer (2 x 16) + O (2 halves x 16)
 constexpr float kRescaleLog2 = 8.f;        // lazy-rescale threshold (p <= 2^8)
 
@@ -657,7 +668,7 @@ __global__ void __launch_bounds__(kThreads, 1) qsa_prefill_tc_kernel(const __gri
     *sy.abort_flag = 0u;
     mbar_fence_init();
   }
-  if (warp == 0 && lane == 0) prefetch_tensormap(&p.tm_q);
+  if (warp == kWarpProducer0 && lane == 0) prefetch_tensormap(&p.tm_q);
   if (warp == kWarpQK) {
     tmem_alloc(sb + OFF_MISC, kTmemCols);
     tmem_relinquish();
@@ -667,16 +678,20 @@ __global__ void __launch_bounds__(kThreads, 1) qsa_prefill_tc_kernel(const __gri
   tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(sp + OFF_MISC);
 
-  if (warp < kProducerWarps) {
-    producer_role<kDump, kStall, kBlocks>(p, sy, sb, warp, lane);
-  } else if (warp == kWarpQK) {
-    if (lane == 0) qk_role(p, sy, sb, tmem);
-    __syncwarp();
-  } else if (warp == kWarpPV) {
-    if (lane == 0) pv_role(p, sy, sb, tmem);
-    __syncwarp();
-  } else {
+  if (warp < kWarpProducer0) {
+    setmaxnreg_inc<kRegsSoftmax>();
     softmax_role<kBlocks>(p, sy, sb, sp, tmem, warp, lane);
+  } else if (warp < kWarpQK) {
+    setmaxnreg_dec<kRegsProducer>();
+    producer_role<kDump, kStall, kBlocks>(p, sy, sb, warp - kWarpProducer0, lane);
+  } else {
+    setmaxnreg_dec<kRegsMma>();
+    if (warp == kWarpQK) {
+      if (lane == 0) qk_role(p, sy, sb, tmem);
+    } else if (warp == kWarpPV) {
+      if (lane == 0) pv_role(p, sy, sb, tmem);
+    }
+    __syncwarp();
   }
 
   tc_fence_before();
