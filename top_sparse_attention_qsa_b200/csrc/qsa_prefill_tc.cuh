@@ -7,23 +7,30 @@
 // heads of the group attend to the cache rows named by the token's list,
 // softmax(scale q K_sel^T) V_sel, -1 / n_valid masking, zeros for empty rows.
 //
-// Persistent CTAs (one per SM) walk the units in KV-head-major order.  Ten
-// warps with fixed roles, synchronised only through mbarriers:
-//   warps 0-3   producers: read each tile's 128 list entries one tile ahead
-//               and gather the K and V rows with 16-byte cp.async copies
-//               written straight into the 128-byte-swizzled layout the
-//               tensor core reads, into a ring of six 32 KB slots (K dims
-//               0-127, K dims 128-255, V dims 0-127, V dims 128-255); masked
-//               entries are zero-filled without a global read.  Warp 0 also
-//               loads the 16 Q rows of the unit (tiled TMA, double-buffered).
-//   warp 4      one thread issues the score MMAs (tcgen05.mma, kind::f16):
+// Persistent CTAs (one per SM) walk the units in KV-head-major order.
+// Twenty-four warps in six warpgroups with fixed roles, synchronised only
+// through mbarriers; registers are rebalanced per warpgroup (setmaxnreg) so
+// that the softmax keeps 176 per thread and each producer 64:
+//   warps 4-19  sixteen producers: read each tile's 128 list entries one
+//               tile ahead and gather the K and V rows (in the order K(0),
+//               K(1), V(0), K(2), V(1), ... within a unit, so that a tile's
+//               V rows land about when its probabilities are ready) with
+//               16-byte cp.async copies written straight into the
+//               128-byte-swizzled layout the tensor core reads, into a ring
+//               of six 32 KB slots (one half, dims 0-127 or 128-255, of a
+//               tile's K or V rows each); masked entries are zero-filled
+//               without a global read.  Warp 4 also loads the 16 Q rows of
+//               the unit (tiled TMA, double-buffered).  Many warps with few
+//               copies each in flight move random rows faster than a few
+//               warps with many.
+//   warp 20     one thread issues the score MMAs (tcgen05.mma, kind::f16):
 //               S^T[128 keys x 16 heads] = K_tile . Q^T (M=128, N=16, K-major
 //               operands) into a TMEM double buffer.
-//   warp 5      one thread issues the PV MMAs: O^T[256 x 16] += V_tile^T . P^T
+//   warp 21     one thread issues the PV MMAs: O^T[256 x 16] += V_tile^T . P^T
 //               (two M=128 halves, V read MN-major from the same slots) into
 //               TMEM.  Two issuers keep PV of tile i from queueing behind the
 //               scores of tile i+1.
-//   warps 6-9   softmax: thread k owns TMEM lane k = key k of the tile;
+//   warps 0-3   softmax: thread k owns TMEM lane k = key k of the tile;
 //               exponentials in base 2 from the running max; P^T written
 //               MN-major to shared memory; the running max is only raised
 //               (with an O rescale in TMEM) when a head's max grows by more
@@ -32,6 +39,12 @@
 //               then is the tile max per head formed (a transposing shuffle
 //               reduction and a 4-warp exchange).
 //               Epilogue: lse = m + ln l, O / l -> BF16 rows, zeros for empty rows.
+// The consumers of the ring take only their own slots (the score MMAs the K
+// slots, PV the V slots) and skip the others without waiting.  That is safe
+// because every lane's cp.async copies complete in issue order: when a
+// consumer's previous slot is full, every slot filled before it is full too,
+// including the one it skips to, so a parity wait can never see an older
+// phase of a slot as the one it waits for.
 // Every wait (all on mbarriers, including the exchanges inside the softmax
 // group) is bounded by 2 s of %globaltimer; on expiry the kernel raises status
 // bit 1, every role stops, in-flight copies and MMAs are drained and the TMEM
@@ -275,22 +288,17 @@ __device__ void producer_role(const TcParams& p, const Sync& sy, uint32_t sb, in
     constexpr int rows_w = kKeys / kProducerWarps;
     const int jr = rows_w * pw + lane;
     const bool own = lane < rows_w;
-    int32_t entry_next = own ? key_entry<kBlocks>(p, list, un, jr) : -1;
-    for (int i = 0; i < un.n_tiles && ok; ++i) {
-      int32_t id = key_slot<kBlocks>(p, un, i * kKeys + jr, entry_next, last);
-      entry_next = (own && i + 1 < un.n_tiles) ? key_entry<kBlocks>(p, list, un, (i + 1) * kKeys + jr) : -1;
-      if (id == -2) {
-        id = -1;
-        if (p.status != nullptr) atomicOr(p.status, static_cast<int32_t>(kStatusOob));
-      }
-      int32_t from_k[kDump ? rows_w / 2 : 1];       // kDump: slot behind each K copy of this lane
+    // the tile's two K or V ring slots (dims 0-127, 128-255) for this lane's
+    // share of the rows, `id` the lane's row slot (-1: masked, zero-filled)
+    auto issue = [&](int i, bool v, int32_t id) {
+      const char* base = v ? vbase : kbase;
 #pragma unroll 1
-      for (int h = 0; h < 4; ++h) {
+      for (int h = 0; h < 2; ++h) {
         const uint32_t slot = c_slot % kSlots;
         const uint32_t round = c_slot / kSlots;
         ok = sy.wait_warp(B_EMPTY + slot, (round & 1u) ^ 1u);
-        if (!ok) break;
-        const char* src0 = (h < 2 ? kbase : vbase) + (h & 1) * 256;
+        if (!ok) return;
+        const char* src0 = base + h * 256;
         const uint32_t dst0 = sb + OFF_RING + slot * kSlotBytes + dchunk;
 #pragma unroll
         for (int k = 0; k < rows_w / 2; ++k) {
@@ -299,24 +307,52 @@ __device__ void producer_role(const TcParams& p, const Sync& sy, uint32_t sb, in
           const bool live = rid >= 0;
           const char* src = live ? src0 + static_cast<int64_t>(rid) * row_bytes : src0;
           cp_async_16(dst0 + r * 128 + (((cc & 7) ^ (r & 7)) << 4), src, live ? 16 : 0);
-          if (kDump && cc == 0 && (h & 1) == 0) {
+          if (kDump && cc == 0 && h == 0) {
             // debug dump: the slot this copy read, recovered from its source
-            // address (-1 for a zero-filled row); the K and V copies of a key
-            // must agree, else -2 is recorded
+            // address (-1 for a zero-filled row); the V copy of a key (by the
+            // same lane, after the K copy) must agree, else -2 is recorded
             const int32_t from = live ? static_cast<int32_t>((src - src0) / row_bytes) : -1;
-            if (h == 0) {
-              from_k[kDump ? k : 0] = from;
-            } else {
-              const int64_t key = un.j0 + static_cast<int64_t>(i) * kKeys + r;
-              const int64_t n_keys = static_cast<int64_t>(p.K) << p.block_shift;
-              if (key < n_keys)
-                p.gathered[(un.t * p.Hkv + un.g) * n_keys + key] = from == from_k[kDump ? k : 0] ? from : -2;
+            const int64_t key = un.j0 + static_cast<int64_t>(i) * kKeys + r;
+            const int64_t n_keys = static_cast<int64_t>(p.K) << p.block_shift;
+            if (key < n_keys) {
+              int32_t* d = p.gathered + (un.t * p.Hkv + un.g) * n_keys + key;
+              if (!v)
+                *d = from;
+              else if (*d != from)
+                *d = -2;
             }
           }
         }
         if (!(kStall && c_slot == 0)) cp_async_mbar_arrive(sy.bar(B_FULL + slot));
         ++c_slot;
       }
+    };
+    // slot of this lane's row of tile i from its entry (loaded a tile ahead)
+    auto resolve = [&](int i, int32_t e) {
+      int32_t id = key_slot<kBlocks>(p, un, i * kKeys + jr, e, last);
+      if (id == -2) {
+        id = -1;
+        if (p.status != nullptr) atomicOr(p.status, static_cast<int32_t>(kStatusOob));
+      }
+      return id;
+    };
+    // Order within a unit: K(0), K(1), V(0), K(2), V(1), ..., V(n-1): a
+    // tile's V rows follow the next tile's K rows, so that they land about
+    // when the tile's probabilities are ready.
+    int32_t entry_next = own ? key_entry<kBlocks>(p, list, un, jr) : -1;
+    int32_t id0 = resolve(0, entry_next);
+    entry_next = (own && 1 < un.n_tiles) ? key_entry<kBlocks>(p, list, un, kKeys + jr) : -1;
+    if (un.n_tiles > 0) issue(0, false, id0);
+    for (int i = 0; i < un.n_tiles && ok; ++i) {
+      int32_t id1 = -1;
+      if (i + 1 < un.n_tiles) {
+        id1 = resolve(i + 1, entry_next);
+        entry_next = (own && i + 2 < un.n_tiles) ? key_entry<kBlocks>(p, list, un, (i + 2) * kKeys + jr) : -1;
+        issue(i + 1, false, id1);
+        if (!ok) break;
+      }
+      issue(i, true, id0);
+      id0 = id1;
     }
   }
   // every copy this lane issued has landed before the CTA can exit
@@ -348,8 +384,10 @@ __device__ void qk_role(const TcParams& p, const Sync& sy, uint32_t sb, uint32_t
       const uint32_t c = c_tile;
       const uint32_t sbuf = c & 1u;
       ok = sy.wait(B_SFREE + sbuf, ((c >> 1) & 1u) ^ 1u);
+      // the unit's items in the producers' order: K(0), K(1), V(0), K(2), ...
+      const uint32_t item = 2u * (c - i) + (i == 0 ? 0u : 2u * i - 1u);
       for (int h = 0; h < 2 && ok; ++h) {
-        const uint32_t ck = 4u * c + h;
+        const uint32_t ck = 2u * item + h;
         const uint32_t slot = ck % kSlots;
         ok = sy.wait(B_FULL + slot, (ck / kSlots) & 1u);
         if (!ok) break;
@@ -396,8 +434,9 @@ __device__ void pv_role(const TcParams& p, const Sync& sy, uint32_t sb, uint32_t
       const uint32_t c = c_tile;
       const uint32_t pb = c & 1u;
       ok = sy.wait(B_PFULL + pb, (c >> 1) & 1u);
+      const uint32_t item = 2u * (c - i) + (i + 1 < un.n_tiles ? 2u * i + 2u : 2u * un.n_tiles - 1u);
       for (int mh = 0; mh < 2 && ok; ++mh) {
-        const uint32_t cv = 4u * c + 2 + mh;
+        const uint32_t cv = 2u * item + mh;
         const uint32_t slot = cv % kSlots;
         ok = sy.wait(B_FULL + slot, (cv / kSlots) & 1u);
         if (!ok) break;
