@@ -41,10 +41,13 @@
 //               Epilogue: lse = m + ln l, O / l -> BF16 rows, zeros for empty rows.
 // The consumers of the ring take only their own slots (the score MMAs the K
 // slots, PV the V slots) and skip the others without waiting.  That is safe
-// because every lane's cp.async copies complete in issue order: when a
-// consumer's previous slot is full, every slot filled before it is full too,
-// including the one it skips to, so a parity wait can never see an older
-// phase of a slot as the one it waits for.
+// because every lane's cp.async copies complete in issue order and, in this
+// gather order, the previous fill of the slot a consumer waits on was always
+// issued before the last slot that consumer waited on: when that one is
+// full, so is the older fill, and a parity wait can never take an older
+// phase of the slot for the one it waits for.  (Running the K rows two or
+// more tiles ahead breaks this at unit boundaries, where the V rows of the
+// last tiles follow each other.)
 // Every wait (all on mbarriers, including the exchanges inside the softmax
 // group) is bounded by 2 s of %globaltimer; on expiry the kernel raises status
 // bit 1, every role stops, in-flight copies and MMAs are drained and the TMEM
