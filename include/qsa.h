@@ -408,6 +408,29 @@ qsa_status_t qsa_indexer_scores(const qsa_indexer_shape_t* shape,
                                 int32_t* status, void* stream);
 
 /*
+ * Head folding of the indexer query (optional step before
+ * qsa_indexer_scores).  The score is linear in the query, so
+ * sum_h <q_idx[t,h], k> = <s_t, k> with s_t = sum_h q_idx[t,h] (page "Qwen4-
+ * Exp QSA llega al Ascend de Huawei", section "Por qué QSA es la parte
+ * incómoda, en cifras": several indexer heads per token over one key head).
+ * Writes, per token t and dim d, the FP32 head sum s (heads added in order
+ * 0..H-1) as two BF16 values: q_folded[t][0][d] = hi = bf16(s) and
+ * q_folded[t][1][d] = lo = bf16(s - hi), round to nearest, so that
+ * |s - hi - lo| <= 2^-16 |s| (BF16 keeps 8 significant bits, so each
+ * rounding is within 2^-8 of its argument).  q_folded: BF16 device
+ * [T, 2, 128] contiguous,
+ * caller-owned, 16-byte aligned.  Calling qsa_indexer_scores on it with
+ * num_heads = 2 (strides 256 and 128) gives the scores of the H-head query
+ * with half the tensor-core work; folding moves a score by at most
+ * 2^-16 sum_d |s_d k[b,d]| <= 2^-16 sum_h sum_d |q_idx[t,h,d] k[b,d]|.  Uses num_tokens,
+ * num_heads, head_dim and the q strides of `shape` (validated as for
+ * qsa_indexer_scores).  One launch; no allocation.
+ */
+qsa_status_t qsa_indexer_fold_heads(const qsa_indexer_shape_t* shape,
+                                    const void* q_idx, void* q_folded,
+                                    void* stream);
+
+/*
  * Top-K selection over scores laid out as qsa_indexer_scores writes them
  * (only the candidate columns of each row are read).
  *   budget      : blocks chosen per token, >= 0 (2048 in the model).

@@ -168,6 +168,21 @@ def test_indexer_nulls_and_topk_limits(capi):
     assert sel(ctypes.byref(odd), P, P, P, 8, 0, P, 8, P, 1, None, None) == 4   # row stride not 4 floats
 
 
+def test_indexer_fold_validation(capi):
+    lib = capi.library()
+    fold = lib.qsa_indexer_fold_heads
+    s = _ishape(capi)
+    assert fold(None, P, P, None) == 1
+    assert fold(ctypes.byref(s), None, P, None) == 1
+    assert fold(ctypes.byref(s), P, None, None) == 1
+    assert fold(ctypes.byref(s), P + 8, P, None) == 4            # q not 16-byte aligned
+    assert fold(ctypes.byref(s), P, P + 8, None) == 4            # output not 16-byte aligned
+    assert fold(ctypes.byref(_ishape(capi, q_stride_head=132)), P, P, None) == 4
+    assert fold(ctypes.byref(_ishape(capi, num_heads=3)), P, P, None) == 3
+    assert fold(ctypes.byref(_ishape(capi, head_dim=64)), P, P, None) == 3
+    assert fold(ctypes.byref(_ishape(capi, num_tokens=0)), None, None, None) == 0
+
+
 def test_fp8_entry_validation(capi):
     lib = capi.library()
     s = _shape(capi)

@@ -65,15 +65,41 @@ def check_selection(orc, w, scores, lists, nv, budget, tail, rows=None):
         np.testing.assert_array_equal(gnv[:, c], cnt)
 
 
-@pytest.mark.parametrize("H", [4, 1, 2, 8])
-def test_scores_small_ragged(C, orc, H):
+@pytest.mark.parametrize("H,fold", [(4, True), (4, False), (1, False), (2, False), (8, True), (8, False)])
+def test_scores_small_ragged(C, orc, H, fold):
     # 300 tokens (several 256/H-token tiles and a ragged one), 700 block keys
-    # (several 128-block tiles and a ragged one), two sequences, tails 0..3
+    # (several 128-block tiles and a ragged one), two sequences, tails 0..3;
+    # H >= 4 with and without the head folding
     w = W.config_indexer(device=DEV, seed=5 + H, T=300, S=2800, heads=H, budget=64,
                          seq_starts=[0, 1400])
-    scores = C.indexer_scores(w.q_idx, w.k_idx, w.positions, w.seq_start, w.block_size)
+    scores = C.indexer_scores(w.q_idx, w.k_idx, w.positions, w.seq_start, w.block_size, fold=fold)
     torch.cuda.synchronize()
     check_scores(orc, w, _host(scores))
+
+
+@pytest.mark.parametrize("H", [1, 2, 4, 8])
+def test_fold_heads(C, H):
+    """hi + lo against the FP64 head sum: |s - hi - lo| <= 2^-16 |s| (two
+    roundings to 8 significant bits) plus the
+    FP32 sum's own error (at most (H - 1) 2^-24 sum_h |q_h|, taken as H
+    2^-24 sum_h |q_h| to cover the 2^-16 term's argument too); hi is the
+    BF16 rounding of the FP32 sum, so |lo| <= half an ulp of hi <= 2^-8 |hi|;
+    a strided q (head stride 256) and T = 33."""
+    g = torch.Generator(device=DEV).manual_seed(70 + H)
+    base = W.normal_bf16((33, H, 256), g, DEV)
+    q = base[:, :, :128]
+    assert q.stride(1) == 256
+    k = W.normal_bf16((8, 128), g, DEV)
+    f = C.indexer_fold_heads(q, k)
+    torch.cuda.synchronize()
+    qd = _host(q).double()
+    s = qd.sum(1)
+    hi, lo = _host(f[:, 0]).double(), _host(f[:, 1]).double()
+    bound = 2.0 ** -16 * s.abs() + H * 2.0 ** -24 * qd.abs().sum(1)
+    assert bool(((hi + lo - s).abs() <= bound).all())
+    assert bool((lo.abs() <= 2.0 ** -8 * hi.abs()).all())
+    if H == 1:
+        assert torch.equal(hi, qd[:, 0]) and bool((lo == 0).all())
 
 
 @pytest.mark.parametrize("budget,tail", [(0, True), (1, False), (37, True), (128, False), (2048, True)])
@@ -127,6 +153,25 @@ def test_ties_and_signed_zeros(C, orc):
     sc[2, 100:4000] = 7.0
     scores = sc.to(DEV)
     for budget in (1, 10, 1000, 3900):
+        lists, nv = C.topk_select(scores, w.positions, w.seq_start, NB, budget, w.block_size,
+                                  append_tail=True)
+        torch.cuda.synchronize()
+        check_selection(orc, w, scores, lists, nv, budget, True)
+
+
+@pytest.mark.parametrize("NB,step", [(32768, 1 / 16), (32768, 1 / 1024), (12000, 1 / 8)])
+def test_ties_inside_threshold_bin(C, orc, NB, step):
+    """Normal scores on a grid of `step`: the bin that holds the budget-th
+    score has a few hundred keys (the lists' path) and the exact threshold
+    value is shared by many of them, which are taken in block order; rows
+    of 32768 and 12000 candidates."""
+    T = 24
+    w = W.config_indexer(device=DEV, seed=47, T=T, S=4 * NB, heads=4)
+    g = torch.Generator().manual_seed(int(1 / step))
+    sc = torch.round(torch.randn(T, NB, generator=g) / step) * step
+    sc[5] = -sc[5]
+    scores = sc.to(DEV)
+    for budget in (2048, 777):
         lists, nv = C.topk_select(scores, w.positions, w.seq_start, NB, budget, w.block_size,
                                   append_tail=True)
         torch.cuda.synchronize()

@@ -36,7 +36,7 @@ EXPORTS = ("qsa_sparse_prefill_fwd", "qsa_sparse_prefill_fwd_with", "qsa_sparse_
            "qsa_sparse_prefill_fwd_host", "qsa_sparse_decode_fwd", "qsa_sparse_decode_workspace_bytes",
            "qsa_sparse_decode_num_splits", "qsa_sparse_decode_fwd_noalloc",
            "qsa_sparse_prefill_fp8_fwd", "qsa_sparse_decode_fp8_fwd", "qsa_indexer_scores",
-           "qsa_topk_select", "qsa_status_string", "qsa_abi_version")
+           "qsa_indexer_fold_heads", "qsa_topk_select", "qsa_status_string", "qsa_abi_version")
 
 
 class Shape(ctypes.Structure):
@@ -118,6 +118,7 @@ _lib.qsa_sparse_decode_fp8_fwd.argtypes = [ctypes.POINTER(Shape), _vp, _vp, _vp,
                                            ctypes.c_float, ctypes.c_float, _vp, _vp, _vp, ctypes.c_int32,
                                            _vp, ctypes.c_size_t, _vp]
 _lib.qsa_indexer_scores.argtypes = [ctypes.POINTER(IndexerShape), _vp, _vp, _vp, _vp, _vp, _vp, _vp]
+_lib.qsa_indexer_fold_heads.argtypes = [ctypes.POINTER(IndexerShape), _vp, _vp, _vp]
 _lib.qsa_topk_select.argtypes = [ctypes.POINTER(IndexerShape), _vp, _vp, _vp, ctypes.c_int64, ctypes.c_int32,
                                  _vp, ctypes.c_int64, _vp, ctypes.c_int32, _vp, _vp]
 _lib.qsa_status_string.restype = ctypes.c_char_p
@@ -565,14 +566,38 @@ def _need_tok(x, name, T, dev):
         raise ValueError(f"{name} must be a contiguous [T] int32 tensor")
 
 
+def indexer_fold_heads(q_idx, k_idx, out=None, stream=None):
+    """The head sum of q_idx [T, H, 128] as two BF16 terms: [T, 2, 128]
+    (hi = bf16(s), lo = bf16(s - hi)), a two-head query with the same scores."""
+    dev = q_idx.device
+    _need(q_idx, "q_idx", torch.bfloat16, dev)
+    T = q_idx.shape[0]
+    if out is None:
+        out = torch.empty((T, 2, q_idx.shape[2]), dtype=torch.bfloat16, device=dev)
+    _need(out, "q_folded", torch.bfloat16, dev)
+    if not out.is_contiguous() or tuple(out.shape) != (T, 2, q_idx.shape[2]):
+        raise ValueError("q_folded must be a contiguous [T, 2, Dh] tensor")
+    shape = make_indexer_shape(q_idx, k_idx, 1)
+    if stream is None:
+        stream = torch.cuda.current_stream(dev).cuda_stream
+    _raise(_lib.qsa_indexer_fold_heads(ctypes.byref(shape), _ptr(q_idx), _ptr(out), stream))
+    return out
+
+
 def indexer_scores(q_idx, k_idx, positions, seq_start, block_size: int = 4, scores=None, status=None,
-                   stream=None):
+                   stream=None, fold=None, q_folded=None):
     """FP32 scores [T, NB]: sum over the H indexer heads of <q_idx[t,h], k_idx[b]>
     at the complete causal microblocks of each token (other entries untouched;
-    a new buffer starts as -inf)."""
+    a new buffer starts as -inf).  With `fold` (default: H >= 4) the heads
+    are first summed into a two-term BF16 query (qsa_indexer_fold_heads,
+    into `q_folded` when given) and the scores computed from that."""
     dev = q_idx.device
     _need(q_idx, "q_idx", torch.bfloat16, dev)
     _need(k_idx, "k_idx", torch.bfloat16, dev)
+    if fold is None:
+        fold = q_idx.dim() == 3 and q_idx.shape[1] >= 4
+    if fold:
+        q_idx = indexer_fold_heads(q_idx, k_idx, out=q_folded, stream=stream)
     T = q_idx.shape[0]
     _need_tok(positions, "positions", T, dev)
     _need_tok(seq_start, "seq_start", T, dev)

@@ -372,6 +372,57 @@ __global__ void __launch_bounds__(kThreads, 1) qsa_indexer_scores_kernel(const _
   if (warp == 1) tmem_dealloc(tmem, kTmemCols);
 }
 
+// ------------------------------------------------------------ head folding
+
+// The score is linear in the query, sum_h <q[t,h], k[b]> = <sum_h q[t,h], k[b]>,
+// so the H indexer heads of a token can be summed once per token instead of
+// once per (token, block).  The FP32 head sum s of each dim (heads added in
+// order 0..H-1) is stored as two BF16 terms, hi = bf16(s) and
+// lo = bf16(s - hi) (round to nearest; s - hi is exact in FP32; BF16 keeps
+// 8 significant bits, so each rounding is within 2^-8), so
+// |s - hi - lo| <= 2^-16 |s|; the score kernel then takes (hi, lo) as a
+// query of two heads, which halves its tensor-core work and its accumulator
+// reads.  One thread per (token, 8-dim chunk): H 16-byte loads, two 16-byte
+// stores into folded[t][0..1][128].
+struct FoldParams {
+  const __nv_bfloat16* q;     // [T][H][128], strides in elements (multiples of 8)
+  __nv_bfloat16* folded;      // [T][2][128] contiguous
+  int64_t T, q_st, q_sh;
+};
+
+template <int kH>
+__global__ void __launch_bounds__(256) qsa_indexer_fold_kernel(const __grid_constant__ FoldParams p) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x;
+  if (i >= p.T * 16) return;
+  const int64_t t = i >> 4;
+  const int c = static_cast<int>(i & 15);
+  float s[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) s[e] = 0.f;
+#pragma unroll
+  for (int h = 0; h < kH; ++h) {
+    const uint4 v = __ldg(reinterpret_cast<const uint4*>(p.q + t * p.q_st + h * p.q_sh + c * 8));
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      s[2 * e] += __uint_as_float(w[e] << 16);
+      s[2 * e + 1] += __uint_as_float(w[e] & 0xffff0000u);
+    }
+  }
+  uint32_t hi[4], lo[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const __nv_bfloat162 h2 = __floats2bfloat162_rn(s[2 * e], s[2 * e + 1]);
+    const float2 hf = __bfloat1622float2(h2);
+    const __nv_bfloat162 l2 = __floats2bfloat162_rn(s[2 * e] - hf.x, s[2 * e + 1] - hf.y);
+    hi[e] = *reinterpret_cast<const uint32_t*>(&h2);
+    lo[e] = *reinterpret_cast<const uint32_t*>(&l2);
+  }
+  uint4* dst = reinterpret_cast<uint4*>(p.folded + t * 256 + c * 8);
+  dst[0] = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+  dst[16] = make_uint4(lo[0], lo[1], lo[2], lo[3]);        // 128 elements further
+}
+
 // ------------------------------------------------------------------ top-K
 
 struct TopkParams {
@@ -405,11 +456,14 @@ __device__ __forceinline__ void bulk_copy_g2s(uint32_t dst, const void* src, uin
 
 constexpr int kTkThreads = 512;
 constexpr int kTkMax = 32768;                      // candidates per row
+constexpr int kTkSlots = 16;                       // threshold-bin list entries per thread
 constexpr int TK_OFF_ROW = 0;                      // row copy, 16-byte aligned span
 constexpr int TK_OFF_HIST = ((kTkMax + 4) * 4 + 127) / 128 * 128;
 constexpr int TK_OFF_GT = TK_OFF_HIST + 2 * 4096 * 4;  // two histograms, then the bitmaps
 constexpr int TK_OFF_EQ = TK_OFF_GT + kTkMax / 8;
-constexpr int TK_OFF_MISC = TK_OFF_EQ + kTkMax / 8;  // warp totals[16], results[4], mbarrier
+constexpr int TK_OFF_LK = TK_OFF_EQ + kTkMax / 8;  // per-thread lists: keys, then candidate ids
+constexpr int TK_OFF_LE = TK_OFF_LK + kTkSlots * kTkThreads * 4;
+constexpr int TK_OFF_MISC = TK_OFF_LE + kTkSlots * kTkThreads * 2;  // warp totals[16], results[4], mbarrier
 constexpr int TK_SMEM = TK_OFF_MISC + 256;
 
 // Persistent CTAs (one per SM) walk the rows t = blockIdx.x + i * gridDim.x.
@@ -417,24 +471,32 @@ constexpr int TK_SMEM = TK_OFF_MISC + 256;
 // one bulk copy (cp.async.bulk, completion on an mbarrier) while the CTA
 // works on the current row from registers: candidate e = j * 512 + tid
 // (j < kR) sits in a register of thread tid as its order-preserving key.
-// Radix select in three passes over key bits 31-20, 19-8 and 7-0 with a
-// 4096-bin shared histogram (12 bits spread the few exponent values of real
-// scores over many bins, which keeps the shared atomics nearly
-// conflict-free; two histograms alternate so that clearing the next one
-// costs no barrier); after each pass `prefix` and `mask` name the bin that
-// holds the budget-th largest key and `need` how many keys of that bin are
-// still to take; a pass that finds the whole bin taken ends the search.
-// Keys above the bin are all taken, keys in it in block order until `need`
-// runs out: two bitmaps (above / in the bin; one warp ballot is one word)
-// and one packed scan of their word popcounts place every chosen block in
-// ascending order.  Every phase costs at most three CTA barriers.
+// Radix select over key bits 31-20, 19-8 and 7-0 with 4096-bin shared
+// histograms (12 bits spread the few exponent values of real scores over
+// many bins, which keeps the shared atomics nearly conflict-free); after
+// each pass `prefix` and `mask` name the bin that holds the budget-th
+// largest key and `need` how many keys of that bin are still to take; a pass
+// that finds the whole bin taken ends the search.  The first pass counts
+// the keys as they come out of the row copy.
+// One sweep over the keys then writes the bitmap of the keys above the
+// threshold bin (one warp ballot is one word) and appends the few keys in
+// that bin (a few percent of the row for any smooth score distribution) to
+// a per-thread list in shared memory, so that the remaining passes and the
+// in-bin decisions touch only the list; each chosen list entry then sets its
+// bit in the "above" or the "tied" bitmap.  A row whose bin does not fit the
+// lists (heavy ties) finishes the same passes over the register keys
+// instead.  Keys above the final bin are all taken, keys in it in block
+// order until `need` runs out: one packed scan of the two bitmaps' word
+// popcounts places every chosen block in ascending order.
 template <int kR>
 __global__ void __launch_bounds__(kTkThreads, 1) qsa_topk_kernel(const __grid_constant__ TopkParams p) {
   constexpr int kNT = kTkThreads, kW = kNT / 32;
   static_assert(kR % 32 == 0 && kR * kNT <= kTkMax, "bitmap words per thread = kR / 32");
+  static_assert(kR * kNT <= 65536, "list candidate ids are 16-bit");
   constexpr int kWords = kR * kW;                   // bitmap words in use
   constexpr int kWPer = kWords / kNT;               // words per thread
   constexpr int kBins = 4096, kBinsPer = kBins / kNT;
+  constexpr int kCap = kTkSlots;
   extern __shared__ __align__(128) uint8_t tk_smem[];
   const float* row_s = reinterpret_cast<const float*>(tk_smem + TK_OFF_ROW);
   uint32_t* hist = reinterpret_cast<uint32_t*>(tk_smem + TK_OFF_HIST);
@@ -445,6 +507,9 @@ __global__ void __launch_bounds__(kTkThreads, 1) qsa_topk_kernel(const __grid_co
   const uint32_t row_addr = smem_u32(tk_smem + TK_OFF_ROW);
   const uint32_t bar = smem_u32(tk_smem + TK_OFF_MISC + 128);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  // this thread's list: entry i at [i * kNT] (consecutive threads, consecutive words)
+  uint32_t* lk = reinterpret_cast<uint32_t*>(tk_smem + TK_OFF_LK) + tid;
+  uint16_t* le = reinterpret_cast<uint16_t*>(tk_smem + TK_OFF_LE) + tid;
 
   if (tid == 0) {
     mbar_init(bar, 1);
@@ -464,6 +529,47 @@ __global__ void __launch_bounds__(kTkThreads, 1) qsa_topk_kernel(const __grid_co
     mbar_arrive_expect_tx(bar, bytes);
     for (uint32_t off = 0; off < bytes; off += 32768u)
       bulk_copy_g2s(row_addr + off, p.scores + a0 + off / 4, min(32768u, bytes - off), bar);
+  };
+
+  // The bin of histogram hb (bins high to low) that holds the need-th
+  // largest counted key: its index, the count above it and its own count.
+  // Thread i owns bins 4095 - i*kBinsPer .. ; warps in thread order cover the
+  // bins from the top.  Two CTA barriers; hb may be cleared after it.
+  auto find_bin = [&](const uint32_t* hb, int need, uint32_t& d, uint32_t& above, uint32_t& cnt) {
+    uint32_t c[kBinsPer], own = 0u;
+#pragma unroll
+    for (int i = 0; i < kBinsPer; ++i) {
+      c[i] = hb[kBins - 1 - tid * kBinsPer - i];
+      own += c[i];
+    }
+    uint32_t x = own;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    if (lane == 31) wtot[warp] = x;
+    __syncthreads();
+    uint32_t before = 0u;
+    for (int w = 0; w < warp; ++w) before += wtot[w];
+    const uint32_t incl = before + x, excl = incl - own;
+    if (excl < static_cast<uint32_t>(need) && static_cast<uint32_t>(need) <= incl) {
+      uint32_t cum = excl;
+#pragma unroll
+      for (int i = 0; i < kBinsPer; ++i) {
+        if (cum + c[i] >= static_cast<uint32_t>(need)) {
+          shv[0] = kBins - 1u - tid * kBinsPer - i;
+          shv[1] = cum;
+          shv[3] = c[i];
+          break;
+        }
+        cum += c[i];
+      }
+    }
+    __syncthreads();
+    d = shv[0];
+    above = shv[1];
+    cnt = shv[3];
   };
 
   uint32_t it = 0;
@@ -509,15 +615,29 @@ __global__ void __launch_bounds__(kTkThreads, 1) qsa_topk_kernel(const __grid_co
     const int jn = n > tid ? (n - tid + kNT - 1) / kNT : 0;
     // key 0 marks "no candidate": a real score's key is at least 0x007fffff
     // (-inf), so 0 shares histogram bin 0 only with negative NaNs and never
-    // reaches the selection threshold while n > k
+    // reaches the selection threshold while n > k (it also sorts after every
+    // real candidate in block order)
     // (reads past n stay inside the buffer, which holds kTkMax + 4 floats)
     const int jv = k > 0 ? jn : 0;
+    const bool select = n > k;                         // else every candidate is taken
     uint32_t key[kR];
+    if (select) {
+      // the first radix pass counts bits 31-20 as the keys come in
 #pragma unroll
-    for (int j = 0; j < kR; ++j) {
-      const uint32_t kk = order_key(row_s[off + j * kNT + tid]);
-      key[j] = j < jv ? kk : 0u;
+      for (int j = 0; j < kR; ++j) {
+        const uint32_t kk = order_key(row_s[off + j * kNT + tid]);
+        key[j] = j < jv ? kk : 0u;
+        atomicAdd(&hist[key[j] >> 20], 1u);
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < kR; ++j) {
+        const uint32_t kk = order_key(row_s[off + j * kNT + tid]);
+        key[j] = j < jv ? kk : 0u;
+      }
     }
+#pragma unroll
+    for (int i = 0; i < kBinsPer; ++i) hist[kBins + i * kNT + tid] = 0u;   // the second pass's
     __syncthreads();                                   // the row buffer is free again
     if (tid == 0 && tn < p.T) {
       int l1, h1;
@@ -527,75 +647,10 @@ __global__ void __launch_bounds__(kTkThreads, 1) qsa_topk_kernel(const __grid_co
       pending = true;
     }
 
-    if (k > 0) {
-      // every candidate is taken when n <= k: all keys > 1, none equal
-      uint32_t prefix = 1u, mask = 0xffffffffu;
-      int need = 0;
-      if (n > k) {
-        prefix = 0u;
-        mask = 0u;
-        need = k;
-#pragma unroll 1
-        for (int pass = 0; pass < 3; ++pass) {
-          const int shift = pass == 0 ? 20 : (pass == 1 ? 8 : 0);
-          const uint32_t dmask = pass == 2 ? 0xffu : 0xfffu;
-          uint32_t* hb = hist + (pass & 1) * kBins;
-          if (pass < 2) {
-            uint32_t* hz = hist + ((pass + 1) & 1) * kBins;   // the next pass's
-#pragma unroll
-            for (int i = 0; i < kBinsPer; ++i) hz[i * kNT + tid] = 0u;
-          }
-          if (pass == 0) {
-#pragma unroll
-            for (int j = 0; j < kR; ++j) atomicAdd(&hb[key[j] >> 20], 1u);
-          } else {
-            const uint32_t hbase = smem_u32(hb);
-#pragma unroll
-            for (int j = 0; j < kR; ++j)
-              red_add_if_eq(hbase + 4u * ((key[j] >> shift) & dmask), key[j] & mask, prefix);
-          }
-          __syncthreads();
-          // thread i owns bins 4095 - i*kBinsPer .. (high to low); warps in
-          // thread order cover the bins from the top
-          uint32_t c[kBinsPer], own = 0u;
-#pragma unroll
-          for (int i = 0; i < kBinsPer; ++i) {
-            c[i] = hb[kBins - 1 - tid * kBinsPer - i];
-            own += c[i];
-          }
-          uint32_t x = own;
-#pragma unroll
-          for (int o = 1; o < 32; o <<= 1) {
-            const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
-            if (lane >= o) x += y;
-          }
-          if (lane == 31) wtot[warp] = x;
-          __syncthreads();
-          uint32_t before = 0u;
-          for (int w = 0; w < warp; ++w) before += wtot[w];
-          const uint32_t incl = before + x, excl = incl - own;
-          if (excl < static_cast<uint32_t>(need) && static_cast<uint32_t>(need) <= incl) {
-            uint32_t cum = excl;
-#pragma unroll
-            for (int i = 0; i < kBinsPer; ++i) {
-              if (cum + c[i] >= static_cast<uint32_t>(need)) {
-                shv[0] = kBins - 1u - tid * kBinsPer - i;
-                shv[1] = cum;
-                shv[3] = c[i];
-                break;
-              }
-              cum += c[i];
-            }
-          }
-          __syncthreads();
-          const uint32_t d = shv[0];
-          need -= static_cast<int>(shv[1]);
-          prefix |= d << shift;
-          mask |= dmask << shift;
-          if (static_cast<uint32_t>(need) == shv[3]) break;   // the whole bin is taken
-        }
-      }
-      // bitmaps: word j*kW + warp, bit lane = candidate j*kNT + warp*32 + lane
+    // bitmaps from the register keys: word j*kW + warp, bit lane =
+    // candidate j*kNT + warp*32 + lane (each path below that still holds the
+    // keys calls it last, so that no key outlives it)
+    auto key_bitmaps = [&](uint32_t mask, uint32_t prefix) {
 #pragma unroll
       for (int j = 0; j < kR; ++j) {
         const uint32_t km = key[j] & mask;
@@ -604,6 +659,110 @@ __global__ void __launch_bounds__(kTkThreads, 1) qsa_topk_kernel(const __grid_co
         if (lane == 0) {
           gtw[j * kW + warp] = bg;
           eqw[j * kW + warp] = be;
+        }
+      }
+    };
+
+    if (k > 0) {
+      // every candidate is taken when n <= k: all keys > 1, none equal
+      uint32_t prefix = 1u, mask = 0xffffffffu;
+      int need = 0;
+      if (!select) {
+        key_bitmaps(mask, prefix);
+      } else {
+        uint32_t d, above, cnt;
+        find_bin(hist, k, d, above, cnt);
+        need = k - static_cast<int>(above);
+        prefix = d << 20;
+        mask = 0xfff00000u;
+        if (static_cast<uint32_t>(need) != cnt) {
+          // one sweep: the "above" bitmap, and the bin's keys into the lists
+          // (an entry past the last slot overwrites it; such a row takes the
+          // fallback below)
+          uint32_t nl = 0u;                            // this thread's list length
+#pragma unroll
+          for (int j = 0; j < kR; ++j) {
+            const uint32_t b = key[j] >> 20;
+            const uint32_t bg = __ballot_sync(0xffffffffu, b > d);
+            if (lane == 0) gtw[j * kW + warp] = bg;
+            if (b == d) {
+              const uint32_t slot = min(nl, static_cast<uint32_t>(kCap - 1));
+              lk[slot * kNT] = key[j];
+              le[slot * kNT] = static_cast<uint16_t>(j * kNT + warp * 32 + lane);
+              ++nl;
+            }
+          }
+#pragma unroll
+          for (int i = 0; i < kWPer; ++i) eqw[tid * kWPer + i] = 0u;
+#pragma unroll
+          for (int i = 0; i < kBinsPer; ++i) hist[i * kNT + tid] = 0u;   // the third pass's
+          if (!__syncthreads_or(nl > static_cast<uint32_t>(kCap))) {
+            // bits 19-8, then 7-0, of the listed keys
+            for (uint32_t i = 0; i < nl; ++i) atomicAdd(&hist[kBins + ((lk[i * kNT] >> 8) & 0xfffu)], 1u);
+            __syncthreads();
+            find_bin(hist + kBins, need, d, above, cnt);
+            need -= static_cast<int>(above);
+            prefix |= d << 8;
+            mask |= 0xfffu << 8;
+            if (static_cast<uint32_t>(need) != cnt) {
+              const uint32_t hbase = smem_u32(hist);
+              for (uint32_t i = 0; i < nl; ++i) {
+                const uint32_t kk = lk[i * kNT];
+                red_add_if_eq(hbase + 4u * (kk & 0xffu), kk & mask, prefix);
+              }
+              __syncthreads();
+              find_bin(hist, need, d, above, cnt);
+              need -= static_cast<int>(above);
+              prefix |= d;
+              mask = 0xffffffffu;
+            }
+            // chosen list entries into the two bitmaps
+            for (uint32_t i = 0; i < nl; ++i) {
+              const uint32_t km = lk[i * kNT] & mask;
+              const uint32_t e = le[i * kNT];
+              if (km > prefix) atomicOr(&gtw[e >> 5], 1u << (e & 31u));
+              else if (km == prefix) atomicOr(&eqw[e >> 5], 1u << (e & 31u));
+            }
+          } else {
+            // heavy ties: the last two passes and the bitmaps over the
+            // row's keys read again from global memory (the registers are
+            // free by now, and the row has just been read, so it sits in L2)
+            const float* srow = p.scores + t * p.ld + lo;
+            auto gkey = [&](int j) -> uint32_t {
+              const int e = j * kNT + tid;
+              return e < n ? order_key(__ldg(srow + e)) : 0u;
+            };
+#pragma unroll 1
+            for (int pass = 1; pass < 3; ++pass) {
+              const int shift = pass == 1 ? 8 : 0;
+              const uint32_t dmask = pass == 2 ? 0xffu : 0xfffu;
+              uint32_t* hb = hist + (pass & 1) * kBins;   // both cleared before the sweep's barrier
+              const uint32_t hbase = smem_u32(hb);
+#pragma unroll 4
+              for (int j = 0; j < kR; ++j) {
+                const uint32_t kk = gkey(j);
+                red_add_if_eq(hbase + 4u * ((kk >> shift) & dmask), kk & mask, prefix);
+              }
+              __syncthreads();
+              find_bin(hb, need, d, above, cnt);
+              need -= static_cast<int>(above);
+              prefix |= d << shift;
+              mask |= dmask << shift;
+              if (static_cast<uint32_t>(need) == cnt) break;   // the whole bin is taken
+            }
+#pragma unroll 4
+            for (int j = 0; j < kR; ++j) {
+              const uint32_t km = gkey(j) & mask;
+              const uint32_t bg = __ballot_sync(0xffffffffu, km > prefix);
+              const uint32_t be = __ballot_sync(0xffffffffu, km == prefix);
+              if (lane == 0) {
+                gtw[j * kW + warp] = bg;
+                eqw[j * kW + warp] = be;
+              }
+            }
+          }
+        } else {
+          key_bitmaps(mask, prefix);                   // the whole bin is taken
         }
       }
       __syncthreads();

@@ -131,6 +131,31 @@ qsa_status_t qsa_indexer_scores(const qsa_indexer_shape_t* shape, const void* q_
   return e == cudaSuccess ? QSA_OK : QSA_ERR_CUDA;
 }
 
+qsa_status_t qsa_indexer_fold_heads(const qsa_indexer_shape_t* shape, const void* q_idx, void* q_folded,
+                                    void* stream) {
+  qsa_status_t rc = validate_indexer(shape);
+  if (rc != QSA_OK) return rc;
+  if (shape->num_tokens == 0) return QSA_OK;
+  if (q_idx == nullptr || q_folded == nullptr) return QSA_ERR_NULL;
+  if (shape->q_stride_tok % 8 || shape->q_stride_head % 8 || !aligned16(q_idx) || !aligned16(q_folded))
+    return QSA_ERR_ALIGN;
+  qsa::ix::FoldParams p;
+  p.q = static_cast<const __nv_bfloat16*>(q_idx);
+  p.folded = static_cast<__nv_bfloat16*>(q_folded);
+  p.T = shape->num_tokens;
+  p.q_st = shape->q_stride_tok;
+  p.q_sh = shape->q_stride_head;
+  const unsigned grid = static_cast<unsigned>((p.T * 16 + 255) / 256);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  switch (shape->num_heads) {
+    case 1: qsa::ix::qsa_indexer_fold_kernel<1><<<grid, 256, 0, st>>>(p); break;
+    case 2: qsa::ix::qsa_indexer_fold_kernel<2><<<grid, 256, 0, st>>>(p); break;
+    case 4: qsa::ix::qsa_indexer_fold_kernel<4><<<grid, 256, 0, st>>>(p); break;
+    default: qsa::ix::qsa_indexer_fold_kernel<8><<<grid, 256, 0, st>>>(p); break;
+  }
+  return cudaGetLastError() == cudaSuccess ? QSA_OK : QSA_ERR_CUDA;
+}
+
 qsa_status_t qsa_topk_select(const qsa_indexer_shape_t* shape, const float* scores,
                              const int32_t* positions, const int32_t* seq_start, int64_t budget,
                              int32_t append_tail, int32_t* lists, int64_t list_stride_tok,
