@@ -99,9 +99,16 @@ __device__ __forceinline__ void candidates(const int32_t* positions, const int32
 }
 
 // The same range from a token's position and sequence start.
+// Non-negative inputs take 32-bit unsigned divisions (pos + 1 <= 2^31).
 __device__ __forceinline__ void range_of(int32_t pos, int32_t s0, int32_t NB, int32_t bs, int& lo, int& hi) {
-  int64_t l = static_cast<int64_t>(s0) / bs;
-  int64_t h = (static_cast<int64_t>(pos) + 1) / bs;
+  int64_t l, h;
+  if ((pos | s0) >= 0) {
+    l = static_cast<uint32_t>(s0) / static_cast<uint32_t>(bs);
+    h = (static_cast<uint32_t>(pos) + 1u) / static_cast<uint32_t>(bs);
+  } else {
+    l = static_cast<int64_t>(s0) / bs;
+    h = (static_cast<int64_t>(pos) + 1) / bs;
+  }
   if (l < 0) l = 0;
   if (h > NB) h = NB;
   if (h < l) h = l;
@@ -810,10 +817,20 @@ __global__ void __launch_bounds__(kTkThreads, 1) qsa_topk_kernel(const __grid_co
     }
     // causal tail, padding, counts
     int cnt = k;
-    const int64_t pos = pos_t;
-    const bool tail = p.append_tail != 0 && (pos + 1) % p.bs != 0;
+    bool tail;
+    int32_t tail_blk;
+    if (pos_t >= 0) {
+      // pos / bs == (pos + 1) / bs whenever bs does not divide pos + 1
+      const uint32_t p1 = static_cast<uint32_t>(pos_t) + 1u, q1 = p1 / static_cast<uint32_t>(p.bs);
+      tail = p.append_tail != 0 && q1 * static_cast<uint32_t>(p.bs) != p1;
+      tail_blk = static_cast<int32_t>(q1);
+    } else {
+      const int64_t pos = pos_t;
+      tail = p.append_tail != 0 && (pos + 1) % p.bs != 0;
+      tail_blk = static_cast<int32_t>(pos / p.bs);
+    }
     if (tail) {
-      if (tid == 0) out[k] = static_cast<int32_t>(pos / p.bs);
+      if (tid == 0) out[k] = tail_blk;
       ++cnt;
     }
     for (int j = cnt + tid; j < p.width; j += kNT) out[j] = -1;
