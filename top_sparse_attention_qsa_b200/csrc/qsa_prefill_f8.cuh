@@ -400,6 +400,7 @@ __device__ void softmax8(const TcParams& p, const Sync& sy, uint32_t sb, uint8_t
   float* red_sum = red_max + 128;
   const float* qsc_all = reinterpret_cast<const float*>(sp + F_QSC);
   uint32_t c_tile = 0, c_unit = 0, c_exact = 0;
+  uint32_t c_vote[2] = {0u, 0u};                     // votes taken per score buffer
   const int64_t units = num_units(p);
   const int G = p.G;
   bool ok = true;
@@ -449,21 +450,28 @@ __device__ void softmax8(const TcParams& p, const Sync& sy, uint32_t sb, uint8_t
       }
       // Most tiles hold no score above the running max plus the lazy-rescale
       // bound.  Each warp votes on that, then forms P from the running max
-      // while the other warps' votes arrive; only a yes anywhere (the first
-      // tile of a unit, a real rescale) makes the warps combine the exact
-      // tile max and form P again.
-      const bool wover = __any_sync(0xffffffffu, over);
-      uint8_t* vt = votes + buf * 8;
-      if (lane == 0) vt[warp - kWarpSm8] = wover ? 1 : 0;
-      __syncwarp();
-      if (lane == 0) mbar_arrive(sy.bar(G_RMAX + buf));
+      // while the other warps' votes arrive; only a yes anywhere (a real
+      // rescale) makes the warps combine the exact tile max and form P
+      // again.  The first tile of a unit always takes that path (the
+      // running max is -inf), without a vote; the votes of each score buffer
+      // are counted apart, as the barrier's phases are.
       uint32_t ph[2], plo[2];
       float pv[kHpw];
-      if (!wover) form_p(s, m_run, ph, plo, pv);
-      ok = sy.wait_warp(G_RMAX + buf, (c >> 1) & 1u);
-      if (!ok) break;
-      const uint2 vw = *reinterpret_cast<const uint2*>(vt);
-      if ((vw.x | vw.y) != 0u) {
+      bool exact = true;
+      if (i > 0) {
+        const bool wover = __any_sync(0xffffffffu, over);
+        uint8_t* vt = votes + buf * 8;
+        if (lane == 0) vt[warp - kWarpSm8] = wover ? 1 : 0;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(sy.bar(G_RMAX + buf));
+        if (!wover) form_p(s, m_run, ph, plo, pv);
+        ok = sy.wait_warp(G_RMAX + buf, c_vote[buf] & 1u);
+        ++c_vote[buf];
+        if (!ok) break;
+        const uint2 vw = *reinterpret_cast<const uint2*>(vt);
+        exact = (vw.x | vw.y) != 0u;
+      }
+      if (exact) {
         const float wmax = xreduce8<true>(s, lane);
         float* rm = red_max;
         if ((lane & 3) == 0) rm[wq * 16 + h0 + ((lane >> 2) & 7)] = wmax;
