@@ -304,9 +304,12 @@ int32_t qsa_sparse_decode_num_splits(const qsa_shape_t* shape,
  *  - Calls whose chunks need more than the array holds (see
  *    qsa_sparse_decode_workspace_bytes with the same shape and num_splits)
  *    return QSA_ERR_SCRATCH before anything is enqueued.
- *  - The first call on each device looks up the array's device address (no
- *    allocation); make that first call before any stream capture on that
- *    device.
+ *  - The first call on each device (and again after the current context
+ *    changes, e.g. after cudaDeviceReset) looks up the array's device
+ *    address, which allocates nothing, and caches it with the context.  A
+ *    call that needs that lookup while `stream` is being captured returns
+ *    QSA_ERR_UNSUPPORTED without enqueuing anything: make one call outside
+ *    capture first; captured calls after it are fine.
  *  - All calls in the process share the one array per device: two calls
  *    whose work overlaps on the GPU (different streams, or host threads that
  *    do not order their streams) race on it.  Serialise them.  Nothing in the
