@@ -400,7 +400,7 @@ __device__ void softmax8(const TcParams& p, const Sync& sy, uint32_t sb, uint8_t
   float* red_sum = red_max + 128;
   const float* qsc_all = reinterpret_cast<const float*>(sp + F_QSC);
   uint32_t c_tile = 0, c_unit = 0, c_exact = 0;
-  uint32_t c_vote[2] = {0u, 0u};                     // votes taken per score buffer
+  uint32_t vote_par = 0u;                            // bit b: parity of the votes taken on score buffer b
   const int64_t units = num_units(p);
   const int G = p.G;
   bool ok = true;
@@ -465,8 +465,8 @@ __device__ void softmax8(const TcParams& p, const Sync& sy, uint32_t sb, uint8_t
         __syncwarp();
         if (lane == 0) mbar_arrive(sy.bar(G_RMAX + buf));
         if (!wover) form_p(s, m_run, ph, plo, pv);
-        ok = sy.wait_warp(G_RMAX + buf, c_vote[buf] & 1u);
-        ++c_vote[buf];
+        ok = sy.wait_warp(G_RMAX + buf, (vote_par >> buf) & 1u);
+        vote_par ^= 1u << buf;
         if (!ok) break;
         const uint2 vw = *reinterpret_cast<const uint2*>(vt);
         exact = (vw.x | vw.y) != 0u;
