@@ -291,9 +291,27 @@ __device__ void producer_role(const TcParams& p, const Sync& sy, uint32_t sb, in
     constexpr int rows_w = kKeys / kProducerWarps;
     const int jr = rows_w * pw + lane;
     const bool own = lane < rows_w;
+    // this lane's copies: one 16-byte chunk of rows_w / 2 rows per half tile;
+    // their places in a slot never change, their sources change per tile
+    constexpr int kCopies = rows_w / 2;
+    uint32_t dofs[kCopies];
+#pragma unroll
+    for (int k = 0; k < kCopies; ++k) {
+      const int r = rows_w * pw + 2 * k + rsel;                   // row of the tile
+      dofs[k] = dchunk + r * 128 + (((cc & 7) ^ (r & 7)) << 4);
+    }
+    // byte offsets in the cache of the rows this lane copies for one tile,
+    // from the row slots the owning lanes resolved (-1: masked, zero-filled)
+    auto row_offsets = [&](int32_t id, int64_t (&off)[kCopies]) {
+#pragma unroll
+      for (int k = 0; k < kCopies; ++k) {
+        const int32_t rid = __shfl_sync(0xffffffffu, id, 2 * k + rsel);
+        off[k] = rid >= 0 ? static_cast<int64_t>(rid) * row_bytes : int64_t(-1);
+      }
+    };
     // the tile's two K or V ring slots (dims 0-127, 128-255) for this lane's
-    // share of the rows, `id` the lane's row slot (-1: masked, zero-filled)
-    auto issue = [&](int i, bool v, int32_t id) {
+    // share of the rows
+    auto issue = [&](int i, bool v, const int64_t (&off)[kCopies]) {
       const char* base = v ? vbase : kbase;
 #pragma unroll 1
       for (int h = 0; h < 2; ++h) {
@@ -302,14 +320,13 @@ __device__ void producer_role(const TcParams& p, const Sync& sy, uint32_t sb, in
         ok = sy.wait_warp(B_EMPTY + slot, (round & 1u) ^ 1u);
         if (!ok) return;
         const char* src0 = base + h * 256;
-        const uint32_t dst0 = sb + OFF_RING + slot * kSlotBytes + dchunk;
+        const uint32_t dst0 = sb + OFF_RING + slot * kSlotBytes;
 #pragma unroll
-        for (int k = 0; k < rows_w / 2; ++k) {
+        for (int k = 0; k < kCopies; ++k) {
           const int r = rows_w * pw + 2 * k + rsel;               // row of the tile
-          const int32_t rid = __shfl_sync(0xffffffffu, id, 2 * k + rsel);
-          const bool live = rid >= 0;
-          const char* src = live ? src0 + static_cast<int64_t>(rid) * row_bytes : src0;
-          cp_async_16(dst0 + r * 128 + (((cc & 7) ^ (r & 7)) << 4), src, live ? 16 : 0);
+          const bool live = off[k] >= 0;
+          const char* src = src0 + (live ? off[k] : int64_t(0));
+          cp_async_16(dst0 + dofs[k], src, live ? 16 : 0);
           if (kDump && cc == 0 && h == 0) {
             // debug dump: the slot this copy read, recovered from its source
             // address (-1 for a zero-filled row); the V copy of a key (by the
@@ -343,19 +360,20 @@ __device__ void producer_role(const TcParams& p, const Sync& sy, uint32_t sb, in
     // tile's V rows follow the next tile's K rows, so that they land about
     // when the tile's probabilities are ready.
     int32_t entry_next = own ? key_entry<kBlocks>(p, list, un, jr) : -1;
-    int32_t id0 = resolve(0, entry_next);
+    int64_t off0[kCopies], off1[kCopies];
+    row_offsets(resolve(0, entry_next), off0);
     entry_next = (own && 1 < un.n_tiles) ? key_entry<kBlocks>(p, list, un, kKeys + jr) : -1;
-    if (un.n_tiles > 0) issue(0, false, id0);
+    if (un.n_tiles > 0) issue(0, false, off0);
     for (int i = 0; i < un.n_tiles && ok; ++i) {
-      int32_t id1 = -1;
       if (i + 1 < un.n_tiles) {
-        id1 = resolve(i + 1, entry_next);
+        row_offsets(resolve(i + 1, entry_next), off1);
         entry_next = (own && i + 2 < un.n_tiles) ? key_entry<kBlocks>(p, list, un, (i + 2) * kKeys + jr) : -1;
-        issue(i + 1, false, id1);
+        issue(i + 1, false, off1);
         if (!ok) break;
       }
-      issue(i, true, id0);
-      id0 = id1;
+      issue(i, true, off0);
+#pragma unroll
+      for (int k = 0; k < kCopies; ++k) off0[k] = off1[k];
     }
   }
   // every copy this lane issued has landed before the CTA can exit
