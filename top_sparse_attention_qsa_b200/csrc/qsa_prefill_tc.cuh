@@ -8,10 +8,10 @@
 // softmax(scale q K_sel^T) V_sel, -1 / n_valid masking, zeros for empty rows.
 //
 // Persistent CTAs (one per SM) walk the units in KV-head-major order.
-// Twenty-four warps in six warpgroups with fixed roles, synchronised only
+// Sixteen warps in four warpgroups with fixed roles, synchronised only
 // through mbarriers; registers are rebalanced per warpgroup (setmaxnreg) so
-// that the softmax keeps 176 per thread and each producer 64:
-//   warps 4-19  sixteen producers: read each tile's 128 list entries one
+// that the softmax keeps 176 per thread and each producer 120:
+//   warps 4-11  eight producers: read each tile's 128 list entries one
 //               tile ahead and gather the K and V rows (in the order K(0),
 //               K(1), V(0), K(2), V(1), ... within a unit, so that a tile's
 //               V rows land about when its probabilities are ready) with
@@ -20,13 +20,14 @@
 //               of six 32 KB slots (one half, dims 0-127 or 128-255, of a
 //               tile's K or V rows each); masked entries are zero-filled
 //               without a global read.  Warp 4 also loads the 16 Q rows of
-//               the unit (tiled TMA, double-buffered).  Many warps with few
-//               copies each in flight move random rows faster than a few
-//               warps with many.
-//   warp 20     one thread issues the score MMAs (tcgen05.mma, kind::f16):
+//               the unit (tiled TMA, double-buffered).  Each lane computes
+//               where its copies land in a slot once, and where its rows
+//               sit in the cache once per tile (for the K and the V copies
+//               of both halves): per copy only an add and the copy remain.
+//   warp 12     one thread issues the score MMAs (tcgen05.mma, kind::f16):
 //               S^T[128 keys x 16 heads] = K_tile . Q^T (M=128, N=16, K-major
 //               operands) into a TMEM double buffer.
-//   warp 21     one thread issues the PV MMAs: O^T[256 x 16] += V_tile^T . P^T
+//   warp 13     one thread issues the PV MMAs: O^T[256 x 16] += V_tile^T . P^T
 //               (two M=128 halves, V read MN-major from the same slots) into
 //               TMEM.  Two issuers keep PV of tile i from queueing behind the
 //               scores of tile i+1.
@@ -72,24 +73,26 @@ constexpr int kSlots = 6;
 constexpr int kBlockBytes = 16384;         // 128 rows x 64 dims (one 128-byte swizzle column block)
 constexpr int kQBytes = kGp * 512;         // 16 rows x 256 dims x 2 B
 constexpr int kPBytes = kKeys * kGp * 2;   // 128 keys x 16 heads x 2 B
-// Sixteen producer warps: many warps with few copies each in flight move
-// random rows faster than a few warps with many (the gather probe's finding).
-constexpr int kProducerWarps = 16;         // 8 rows of every tile each
+// Eight producer warps, each lane with its copies' addresses computed once:
+// more warps with fewer copies each in flight move random rows faster (the
+// gather probe's finding), up to where their instructions crowd the issue
+// slots of the softmax and MMA warps.
+constexpr int kProducerWarps = 8;          // 16 rows of every tile each
 static_assert(kKeys % (2 * kProducerWarps) == 0 && kKeys / kProducerWarps <= 32,
               "each producer lane holds at most one row id; rows per warp must be even");
 // Warp roles, in warpgroups of four (registers are rebalanced per warpgroup):
 //   warps 0-3     softmax (TMEM lane quadrants 0-3)
-//   warps 4-19    producers
-//   warp 20       score MMA issuer, warp 21 PV MMA issuer, warps 22-23 idle
+//   warps 4-11    producers
+//   warp 12       score MMA issuer, warp 13 PV MMA issuer, warps 14-15 idle
 constexpr int kWarpSoftmax0 = 0, kWarpProducer0 = 4;
 constexpr int kWarpQK = kWarpProducer0 + kProducerWarps, kWarpPV = kWarpQK + 1;
-constexpr int kThreads = 32 * 24;
+constexpr int kThreads = 32 * 16;
 // Registers per thread after setmaxnreg: softmax / producers / MMA warpgroup.
-// Their sum over the six warpgroups (x 128 threads) must stay within what the
-// block is launched with, 768 threads x 80 registers: 176 + 4 * 64 + 48 = 480
-// = 6 * 80.
-constexpr int kRegsSoftmax = 176, kRegsProducer = 64, kRegsMma = 48, kRegsLaunch = 80;
-static_assert(kRegsSoftmax + 4 * kRegsProducer + kRegsMma <= 6 * kRegsLaunch,
+// Their sum over the four warpgroups (x 128 threads) must stay within what the
+// block is launched with, 512 threads x 128 registers: 176 + 2 * 120 + 64 =
+// 480 <= 4 * 128.
+constexpr int kRegsSoftmax = 176, kRegsProducer = 120, kRegsMma = 64, kRegsLaunch = 128;
+static_assert(kRegsSoftmax + 2 * kRegsProducer + kRegsMma <= 4 * kRegsLaunch,
               "the register split exceeds the launch allocation");
 constexpr int kTmemCols = 64;              // S double buffer (2 x 16) + O (2 halves x 16)
 constexpr float kRescaleLog2 = 8.f;        // lazy-rescale threshold (p <= 2^8)
