@@ -161,7 +161,7 @@ cudaError_t check_register_split(Kernel kernel, std::atomic<int>* done) {
   cudaError_t e = cudaFuncGetAttributes(&attr, kernel);
   if (e != cudaSuccess) return e;
   using namespace qsa::tc;
-  const long need = 128L * (kRegsSoftmax + 2L * kRegsProducer + kRegsMma);
+  const long need = 128L * (kRegsSoftmax + long(kProducerGroups) * kRegsProducer + kRegsMma);
   if (static_cast<long>(attr.numRegs) * kThreads < need) return cudaErrorInvalidConfiguration;
   done->store(1, std::memory_order_release);
   return cudaSuccess;

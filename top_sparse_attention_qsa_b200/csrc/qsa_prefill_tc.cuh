@@ -86,13 +86,15 @@ static_assert(kKeys % (2 * kProducerWarps) == 0 && kKeys / kProducerWarps <= 32,
 //   warp 12       score MMA issuer, warp 13 PV MMA issuer, warps 14-15 idle
 constexpr int kWarpSoftmax0 = 0, kWarpProducer0 = 4;
 constexpr int kWarpQK = kWarpProducer0 + kProducerWarps, kWarpPV = kWarpQK + 1;
-constexpr int kThreads = 32 * 16;
+constexpr int kProducerGroups = kProducerWarps / 4;   // warpgroups of producers
+constexpr int kThreads = 32 * (kProducerWarps + 8);
 // Registers per thread after setmaxnreg: softmax / producers / MMA warpgroup.
 // Their sum over the four warpgroups (x 128 threads) must stay within what the
 // block is launched with, 512 threads x 128 registers: 176 + 2 * 120 + 64 =
 // 480 <= 4 * 128.
 constexpr int kRegsSoftmax = 176, kRegsProducer = 120, kRegsMma = 64, kRegsLaunch = 128;
-static_assert(kRegsSoftmax + 2 * kRegsProducer + kRegsMma <= 4 * kRegsLaunch,
+static_assert(kProducerWarps % 4 == 0 &&
+                  kRegsSoftmax + kProducerGroups * kRegsProducer + kRegsMma <= (kProducerGroups + 2) * kRegsLaunch,
               "the register split exceeds the launch allocation");
 constexpr int kTmemCols = 64;              // S double buffer (2 x 16) + O (2 halves x 16)
 constexpr float kRescaleLog2 = 8.f;        // lazy-rescale threshold (p <= 2^8)
