@@ -150,19 +150,18 @@ inline cudaError_t persistent_grid(const qsa::tc::TcParams& tp, unsigned* grid) 
   return cudaSuccess;
 }
 
-// The BF16 kernel rebalances registers between its warpgroups with
+// The attention kernels rebalance registers between their warpgroups with
 // setmaxnreg, which draws on the registers the block was launched with: a
 // split larger than that would make a warpgroup wait for registers forever.
-// Checked once per kernel against the compiled launch register count.
+// Checked once per kernel against the compiled launch register count;
+// `need` = 128 x the sum over the warpgroups of their registers per thread.
 template <typename Kernel>
-cudaError_t check_register_split(Kernel kernel, std::atomic<int>* done) {
+cudaError_t check_register_split(Kernel kernel, int threads, long need, std::atomic<int>* done) {
   if (done->load(std::memory_order_acquire)) return cudaSuccess;
   cudaFuncAttributes attr;
   cudaError_t e = cudaFuncGetAttributes(&attr, kernel);
   if (e != cudaSuccess) return e;
-  using namespace qsa::tc;
-  const long need = 128L * (kRegsSoftmax + long(kProducerGroups) * kRegsProducer + kRegsMma);
-  if (static_cast<long>(attr.numRegs) * kThreads < need) return cudaErrorInvalidConfiguration;
+  if (static_cast<long>(attr.numRegs) * threads < need) return cudaErrorInvalidConfiguration;
   done->store(1, std::memory_order_release);
   return cudaSuccess;
 }
@@ -172,7 +171,9 @@ cudaError_t launch_tc(const qsa::tc::TcParams& tp, cudaStream_t stream) {
   static std::atomic<int> done[kMaxDevices];
   static std::atomic<int> regs_ok;
   auto kernel = qsa::tc::qsa_prefill_tc_kernel<kDump, kStall, kBlocks>;
-  cudaError_t e = check_register_split(kernel, &regs_ok);
+  using namespace qsa::tc;
+  cudaError_t e = check_register_split(
+      kernel, kThreads, 128L * (kRegsSoftmax + long(kProducerGroups) * kRegsProducer + kRegsMma), &regs_ok);
   if (e != cudaSuccess) return e;
   e = set_smem_once(kernel, qsa::tc::SMEM_BYTES, done);
   if (e != cudaSuccess) return e;
