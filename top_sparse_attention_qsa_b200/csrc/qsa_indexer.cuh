@@ -17,8 +17,10 @@
 // block tiles of 128 blocks).  Swap-AB so that one TMEM lane is one block and
 // the head sum stays inside a thread: D^T[128 blocks x 256 token-heads] =
 // K_tile[128 x 128] . Q_tile[256 x 128]^T, kind::f16, M=128, N=256.
-//   warp 0      TMA: the unit's Q tile once (3-d map, 64 KB), K tiles through
-//               a 4-stage ring (2-d map, 32 KB each), 128-byte swizzle
+//   warp 0      TMA: the unit's Q tile once (3-d map, 64 KB, two buffers so
+//               that the next unit's Q loads while this one's last MMAs
+//               run), K tiles through a 2-stage ring (2-d map, 32 KB each;
+//               the 8 MB key table stays in L2), 128-byte swizzle
 //   warp 1      one thread issues the MMAs into a TMEM double buffer (2 x 256
 //               FP32 columns)
 //   warps 2-9   epilogue: thread = block row, two warps per TMEM lane quarter
@@ -51,7 +53,7 @@ using namespace tc;
 constexpr int kBlk = 128;                    // microblocks per tile (M)
 constexpr int kRows = 256;                   // token-head rows per tile (N)
 constexpr int kDh = 128;                     // indexer head dim
-constexpr int kStages = 4;
+constexpr int kStages = 2;
 constexpr int kTilesPerUnit = 16;            // block tiles per unit
 constexpr int kKBytes = kBlk * kDh * 2;      // 32 KB
 constexpr int kKHalf = kKBytes / 2;          // 128 rows x 64 dims
@@ -63,9 +65,9 @@ constexpr int kTmemCols = 512;
 
 constexpr int OFF_K = 0;
 constexpr int OFF_Q = OFF_K + kStages * kKBytes;
-constexpr int OFF_BAR = OFF_Q + kQBytes;
-constexpr int B_KFULL = 0, B_KEMPTY = 4, B_QFULL = 8, B_QEMPTY = 9, B_TFULL = 10, B_TEMPTY = 12,
-              B_DONE = 14, NUM_BARS = 16;
+constexpr int OFF_BAR = OFF_Q + 2 * kQBytes;            // two Q buffers
+constexpr int B_KFULL = 0, B_KEMPTY = 4, B_QFULL = 8, B_TFULL = 10, B_TEMPTY = 12, B_DONE = 14,
+              B_QEMPTY = 16, NUM_BARS = 18;
 constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;       // tmem base, abort flag
 constexpr int OFF_TOK = OFF_MISC + 16;                 // [8 warps][2][256] int32
 constexpr int SMEM_BYTES = OFF_TOK + kEpiWarps * 2 * kRows * 4 + 1024;
@@ -187,12 +189,13 @@ __device__ void ix_producer(const IxParams& p, const Sync& sy, uint32_t sb, int 
     const IxUnit un = ix_unit(p, u, lane, nullptr, nullptr);
     if (un.n_tiles == 0) continue;
     if (lane == 0) {
-      ok = sy.wait(B_QEMPTY, (c_q & 1u) ^ 1u);
+      const uint32_t qb = c_q & 1u;
+      ok = sy.wait(B_QEMPTY + qb, ((c_q >> 1) & 1u) ^ 1u);
       if (ok) {
-        mbar_arrive_expect_tx(sy.bar(B_QFULL), kQBytes);
+        mbar_arrive_expect_tx(sy.bar(B_QFULL + qb), kQBytes);
         const int32_t t0 = static_cast<int32_t>(un.tok0);
-        tc::tma_load_3d(sb + OFF_Q, &p.tm_q, 0, 0, t0, sy.bar(B_QFULL));
-        tc::tma_load_3d(sb + OFF_Q + kQHalf, &p.tm_q, 64, 0, t0, sy.bar(B_QFULL));
+        tc::tma_load_3d(sb + OFF_Q + qb * kQBytes, &p.tm_q, 0, 0, t0, sy.bar(B_QFULL + qb));
+        tc::tma_load_3d(sb + OFF_Q + qb * kQBytes + kQHalf, &p.tm_q, 64, 0, t0, sy.bar(B_QFULL + qb));
         ++c_q;
       }
       for (int i = 0; i < un.n_tiles && ok; ++i, ++c_tile) {
@@ -212,7 +215,7 @@ __device__ void ix_producer(const IxParams& p, const Sync& sy, uint32_t sb, int 
   if (lane == 0) {
     for (uint32_t c = c_tile > kStages ? c_tile - kStages : 0; c < c_tile; ++c)
       sy.drain(B_KFULL + c % kStages, (c / kStages) & 1u);
-    if (c_q > 0) sy.drain(B_QFULL, (c_q - 1) & 1u);
+    for (uint32_t c = c_q > 2 ? c_q - 2 : 0; c < c_q; ++c) sy.drain(B_QFULL + (c & 1u), (c >> 1) & 1u);
   }
   __syncwarp();
 }
@@ -225,7 +228,8 @@ __device__ void ix_mma(const IxParams& p, const Sync& sy, uint32_t sb, uint32_t 
     const IxUnit un = ix_unit(p, u, lane, nullptr, nullptr);
     if (un.n_tiles == 0) continue;
     if (lane == 0) {
-      ok = sy.wait(B_QFULL, c_q & 1u);
+      const uint32_t qb = c_q & 1u;
+      ok = sy.wait(B_QFULL + qb, (c_q >> 1) & 1u);
       ++c_q;
       for (int i = 0; i < un.n_tiles && ok; ++i, ++c_tile) {
         const uint32_t buf = c_tile & 1u;
@@ -240,13 +244,13 @@ __device__ void ix_mma(const IxParams& p, const Sync& sy, uint32_t sb, uint32_t 
           // K-major, 128-byte swizzle, 8-row groups 1 KB apart; a 16-dim step
           // advances 32 B inside the swizzle atom, dims 64-127 in the second half
           const uint64_t a = smem_desc(ka + (kk >> 2) * kKHalf + (kk & 3) * 32, 16, 1024, 2);
-          const uint64_t b = smem_desc(sb + OFF_Q + (kk >> 2) * kQHalf + (kk & 3) * 32, 16, 1024, 2);
+          const uint64_t b = smem_desc(sb + OFF_Q + qb * kQBytes + (kk >> 2) * kQHalf + (kk & 3) * 32, 16, 1024, 2);
           umma_f16_ss(tmem + buf * kRows, a, b, kIdesc, kk > 0 ? 1u : 0u);
         }
         umma_commit(sy.bar(B_KEMPTY + st));
         umma_commit(sy.bar(B_TFULL + buf));
       }
-      if (ok) umma_commit(sy.bar(B_QEMPTY));
+      if (ok) umma_commit(sy.bar(B_QEMPTY + qb));
     }
     ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
   }
@@ -343,8 +347,10 @@ __global__ void __launch_bounds__(kThreads, 1) qsa_indexer_scores_kernel(const _
       mbar_init(sy.bar(B_KFULL + s), 1);
       mbar_init(sy.bar(B_KEMPTY + s), 1);
     }
-    mbar_init(sy.bar(B_QFULL), 1);
-    mbar_init(sy.bar(B_QEMPTY), 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(sy.bar(B_QFULL + b), 1);
+      mbar_init(sy.bar(B_QEMPTY + b), 1);
+    }
     for (int b = 0; b < 2; ++b) {
       mbar_init(sy.bar(B_TFULL + b), 1);
       mbar_init(sy.bar(B_TEMPTY + b), kEpiWarps);
