@@ -195,7 +195,7 @@ def workload_accounting(w):
 
 
 # Device sources of the default sparse-prefill kernel (qsa_prefill_tc_kernel);
-# its launch shape (persistent grid of min(units, SMs) CTAs of 768 threads)
+# its launch shape (persistent grid of min(units, SMs) CTAs of 512 threads)
 # is fixed in qsa_launch.cuh.
 PREFILL_SOURCES = ("qsa_prefill_tc.cuh", "qsa_tc_ptx.cuh", "qsa_ptx.cuh")
 
