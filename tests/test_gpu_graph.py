@@ -112,8 +112,9 @@ def test_fp8_prefill_graph(C):
 
 
 def test_indexer_selection_attention_graph(C):
-    """The three launches of one QSA step (indexer scores, top-K microblocks,
-    microblock attention) captured as one graph."""
+    """The launches of one QSA step (head folding and indexer scores, top-K
+    microblocks, microblock attention) captured as one graph; the folded
+    query buffer is allocated inside the capture, from the graph's pool."""
     T, S, budget = 64, 4096, 96
     wi = W.config_indexer(device=DEV, seed=51, T=T, S=S, heads=4, seq_starts=[0, 2048])
     gen = torch.Generator(device=DEV).manual_seed(52)
