@@ -186,8 +186,13 @@ cudaError_t launch_tc(const qsa::tc::TcParams& tp, cudaStream_t stream) {
 template <bool kBlocks, bool kDump = false>
 cudaError_t launch_f8(const qsa::tc::TcParams& tp, cudaStream_t stream) {
   static std::atomic<int> done[kMaxDevices];
+  static std::atomic<int> regs_ok;
   auto kernel = qsa::f8::qsa_prefill_f8_kernel<kBlocks, kDump>;
-  cudaError_t e = set_smem_once(kernel, qsa::f8::F_SMEM, done);
+  using namespace qsa::f8;
+  cudaError_t e = check_register_split(kernel, kThreads8,
+                                       128L * (kRegsProd8 + kRegsMisc8 + 2L * kRegsSm8 + kRegsEpi8), &regs_ok);
+  if (e != cudaSuccess) return e;
+  e = set_smem_once(kernel, qsa::f8::F_SMEM, done);
   if (e != cudaSuccess) return e;
   unsigned grid = 0;
   if ((e = persistent_grid(tp, &grid)) != cudaSuccess) return e;

@@ -25,7 +25,7 @@
 //                                     the BF16 kernel; p <= 2^8 by the lazy
 //                                     rescale)
 // with separate TMEM accumulators for the two terms: S_hi, S_lo per score
-// buffer and O_hi, O_lo per output half.  s = (S_hi + S_lo / 16) * 2^-a_h and
+// buffer and O_hi, O_lo per output half (two O buffers, by unit parity).  s = (S_hi + S_lo / 16) * 2^-a_h and
 // o = (O_hi + O_lo / 16) * v_scale / l.  The N dimension of Q, S, P and O runs
 // [hi of heads 0-7, lo of heads 0-7, hi of heads 8-15, lo of heads 8-15], so
 // that a softmax thread's 8 heads of both terms are 16 adjacent TMEM columns
@@ -41,10 +41,17 @@
 //   warp 5      lane 0 issues the score MMAs (A = K tile, B = [q_hi; q_lo];
 //               M=128, N=32, K=32)
 //   warp 6      lane 0 issues PV: [O_hi O_lo]^T += V^T (MN-major) .
-//               [P_hi P_lo]^T (MN-major, N=32) for the two 128-dim halves
-//   warps 7-14  softmax as in the BF16 kernel, two warps per TMEM lane
+//               [P_hi P_lo]^T (MN-major, N=32) for the two 128-dim halves,
+//               into the O buffer of the unit's parity
+//   warp 7      idle (keeps the softmax warpgroups aligned)
+//   warps 8-15  softmax as in the BF16 kernel, two warps per TMEM lane
 //               quadrant (8 heads each), reading both score terms and
-//               writing p_hi / p_lo
+//               writing p_hi / p_lo; at the end of a unit they hand l and m
+//               to the epilogue warps through shared memory and go on
+//   warps 16-19 epilogue: once the unit's last PV is done, O from TMEM
+//               (the buffer then goes back to warp 6), normalised, stored
+//               with lse -- the next unit's scores and softmax overlap it
+// The warpgroups take their registers with setmaxnreg (kRegs*8 below).
 // Every wait is bounded (2 s of %globaltimer) as in the BF16 kernel.
 #pragma once
 
@@ -60,18 +67,19 @@ constexpr int kProducerWarps8 = 4;            // 32 rows of every tile each
 constexpr int kQ8Bytes = kGp * 256;           // one E4M3 Q term: 16 heads x 256 dims
 constexpr int kQ8Block = 2 * kGp * 128;       // one 128-dim block of both terms: 32 rows x 128 B
 constexpr int kP8Bytes = kKeys * kGp;         // one E4M3 P term: 128 keys x 16 heads
-constexpr int kTmemCols8 = 128;               // S: 2 buffers x {hi, lo} x 16; O: 2 halves x {hi, lo} x 16
-constexpr int kTS = 0, kTO = 64;              // TMEM column bases
+constexpr int kTmemCols8 = 256;               // S: 2 buffers x {hi, lo} x 16; O: 2 units x 2 halves x {hi, lo} x 16
+constexpr int kTS = 0, kTO = 64;              // TMEM column bases (O of unit parity b at kTO + 64 b)
 
 constexpr int F_RING = 0;
 constexpr int F_Q8 = F_RING + kSlots8 * kSlotBytes;   // 2 buffers x {hi, lo}
 constexpr int F_P8 = F_Q8 + 2 * 2 * kQ8Bytes;         // 2 buffers x {hi, lo}
 constexpr int F_QSC = F_P8 + 2 * 2 * kP8Bytes;        // 2 buffers x 16 per-head score factors
 constexpr int F_RED = F_QSC + 2 * kGp * 4;            // max[4][16], votes[2][8], sum[2][4][16]
-constexpr int F_BAR = F_RED + 1024;
+constexpr int F_LM = F_RED + 1024;                    // per unit parity: l[16], m[16] for the epilogue warps
+constexpr int F_BAR = F_LM + 256;
 constexpr int G_FULL = 0, G_EMPTY = 6, G_SFULL = 12, G_SFREE = 14, G_PFULL = 16, G_PEMPTY = 18,
-              G_QFULL = 20, G_QEMPTY = 22, G_OFULL = 24, G_OEMPTY = 25, G_RMAX = 26, G_RSUM = 28,
-              G_DONE = 30, G_RMX2 = 32, G_NUM = 33;
+              G_QFULL = 20, G_QEMPTY = 22, G_RMAX = 24, G_RSUM = 26, G_DONE = 28, G_RMX2 = 30,
+              G_OFULL2 = 32, G_OEMPTY2 = 34, G_LFULL = 36, G_LEMPTY = 38, G_NUM = 40;
 constexpr int F_MISC = F_BAR + G_NUM * 8;             // tmem base, abort flag
 constexpr int F_SMEM = F_MISC + 16 + 1024;
 
@@ -286,10 +294,11 @@ __device__ void pv8(const TcParams& p, const Sync& sy, uint32_t sb, uint32_t tme
   for (int64_t u = blockIdx.x; u < units && ok; u += gridDim.x) {
     const Unit un = decode_unit(p, u);
     const uint32_t ue = c_unit++;
-    ok = sy.wait(G_OEMPTY, (ue & 1u) ^ 1u);
+    const uint32_t ob = ue & 1u;                     // O buffer of this unit
+    ok = sy.wait(G_OEMPTY2 + ob, ((ue >> 1) & 1u) ^ 1u);
     if (!ok) break;
     if (un.n_tiles == 0) {
-      mbar_arrive(sy.bar(G_OFULL));
+      mbar_arrive(sy.bar(G_OFULL2 + ob));
       continue;
     }
     for (int i = 0; i < un.n_tiles && ok; ++i, ++c_tile) {
@@ -315,12 +324,12 @@ __device__ void pv8(const TcParams& p, const Sync& sy, uint32_t sb, uint32_t tme
           // one core-matrix column (SBO = 2 KB) further the same for heads
           // 8-15: O of the half lands in the same interleaved column order
           const uint64_t b = smem_desc(pt + kk * 512, 128, kP8Bytes, 0);
-          umma_f8_ss(tmem + kTO + mh * 32, a, b, kIdescPV8, (i == 0 && kk == 0) ? 0u : 1u);
+          umma_f8_ss(tmem + kTO + ob * 64 + mh * 32, a, b, kIdescPV8, (i == 0 && kk == 0) ? 0u : 1u);
         }
       umma_commit(sy.bar(G_EMPTY + slot));
       umma_commit(sy.bar(G_PEMPTY + pb));
     }
-    if (ok) umma_commit(sy.bar(G_OFULL));
+    if (ok) umma_commit(sy.bar(G_OFULL2 + ob));
   }
   umma_commit(sy.bar(G_DONE + 1));
   sy.drain(G_DONE + 1, 0);
@@ -330,9 +339,15 @@ __device__ void pv8(const TcParams& p, const Sync& sy, uint32_t sb, uint32_t tme
 
 constexpr int kSmWarps = 8;     // two per TMEM lane quadrant, 8 heads each
 constexpr int kHpw = kGp / 2;   // heads per softmax warp
+// warpgroups: producers, {Q, score MMA, PV MMA, idle}, softmax (two), epilogue
 constexpr int kWarpQ8 = kProducerWarps8, kWarpQK8 = kProducerWarps8 + 1, kWarpPV8 = kProducerWarps8 + 2,
-              kWarpSm8 = kProducerWarps8 + 3;
-constexpr int kThreads8 = 32 * (kProducerWarps8 + 3 + kSmWarps);
+              kWarpSm8 = kProducerWarps8 + 4, kWarpEpi8 = kWarpSm8 + kSmWarps;
+constexpr int kThreads8 = 32 * (kWarpEpi8 + 4);
+// Registers per thread after setmaxnreg (the block is launched with 640 x 96):
+// producers 80, Q / MMA warpgroup 64, softmax 128, epilogue 80:
+// 80 + 64 + 2*128 + 80 = 480 = 5 * 96.
+constexpr int kRegsProd8 = 80, kRegsMisc8 = 64, kRegsSm8 = 128, kRegsEpi8 = 80, kRegsLaunch8 = 96;
+static_assert(kRegsProd8 + kRegsMisc8 + 2 * kRegsSm8 + kRegsEpi8 <= 5 * kRegsLaunch8, "register split");
 
 // Reduce 8 per-lane values across the 32 lanes of a warp by exchanging halves
 // (7 shuffles for the exchange, 2 for the rest).  Lane l ends with the result
@@ -385,8 +400,8 @@ __device__ __forceinline__ void form_p(const float (&s)[kHpw], const float (&m)[
   }
 }
 
-// Softmax warp w (7..14): TMEM lane quadrant q = w & 3 (thread = key of the
-// tile, and dim of an output half), heads [8 hh, 8 hh + 8) with hh = (w-7)/4.
+// Softmax warp w (8..15): TMEM lane quadrant q = w & 3 (thread = key of the
+// tile), heads [8 hh, 8 hh + 8) with hh = (w-8)/4.
 template <bool kBlocks>
 __device__ void softmax8(const TcParams& p, const Sync& sy, uint32_t sb, uint8_t* sp, uint32_t tmem, int warp,
                          int lane) {
@@ -507,7 +522,7 @@ __device__ void softmax8(const TcParams& p, const Sync& sy, uint32_t sb, uint8_t
 #pragma unroll
             for (int q4 = 0; q4 < 4; ++q4) {          // O_hi, O_lo x two halves, this warp's heads
               uint32_t o[8];
-              const uint32_t col = kTO + (q4 >> 1) * 32 + 16 * hh + (q4 & 1) * 8;
+              const uint32_t col = kTO + (c_unit & 1u) * 64 + (q4 >> 1) * 32 + 16 * hh + (q4 & 1) * 8;
               tmem_ld8(tl + col, o);
               tmem_wait_ld();
 #pragma unroll
@@ -548,55 +563,95 @@ __device__ void softmax8(const TcParams& p, const Sync& sy, uint32_t sb, uint8_t
 #pragma unroll
     for (int h = 0; h < kHpw; ++h)
       l_tot[h] = (rs[h0 + h] + rs[16 + h0 + h]) + (rs[32 + h0 + h] + rs[48 + h0 + h]);
-    ok = sy.wait_warp(G_OFULL, c_unit & 1u);
-    if (!ok) break;
-    tc_fence_after();
-    uint32_t o0[16] = {}, o1[16] = {};     // per half: O_hi of the 8 heads, then O_lo
-    if (un.n_tiles > 0) {
-      tmem_ld16(tl + kTO + 16 * hh, o0);
-      tmem_ld16(tl + kTO + 32 + 16 * hh, o1);
-      tmem_wait_ld();
-    }
-    tc_fence_before();
-    __syncwarp();
-    if (lane == 0) mbar_arrive(sy.bar(G_OEMPTY));
-    const int64_t row0 = un.t * static_cast<int64_t>(p.Hkv) * G + static_cast<int64_t>(un.g) * G;
-    __nv_bfloat16* orow = p.out + un.t * p.o_st + static_cast<int64_t>(un.g) * G * p.o_sh;
+    // hand l and m of the unit to the epilogue warps, which write the output
+    // once the last PV is done, while these warps go on to the next unit
+    const uint32_t lb = c_unit & 1u;
+    if (wq == 0) {
+      ok = sy.wait_warp(G_LEMPTY + lb, ((c_unit >> 1) & 1u) ^ 1u);
+      if (!ok) break;
+      float* lm = reinterpret_cast<float*>(sp + F_LM) + lb * 32;
+      if (lane < kHpw) {
+        float mk = 0.f, lk = 0.f;
 #pragma unroll
-    for (int h = 0; h < kHpw; ++h) {
-      const int hg = h0 + h;
-      if (hg < G) {
-        const bool live = l_tot[h] > 0.f;
-        const float inv = live ? p.o_scale / l_tot[h] : 0.f;
-        const float v0 = live ? fmaf(__uint_as_float(o0[8 + h]), 0.0625f, __uint_as_float(o0[h])) * inv : 0.f;
-        const float v1 = live ? fmaf(__uint_as_float(o1[8 + h]), 0.0625f, __uint_as_float(o1[h])) * inv : 0.f;
-        if (p.part_o != nullptr) {
-          // split-K: this chunk's normalised partial output, for the merge
-          float* po = p.part_o + ((row0 + hg) * p.splits + un.s) * 256;
-          po[key] = v0;
-          po[128 + key] = v1;
-        } else {
-          orow[hg * p.o_sh + key] = __float2bfloat16_rn(v0);
-          orow[hg * p.o_sh + 128 + key] = __float2bfloat16_rn(v1);
-        }
+        for (int h = 0; h < kHpw; ++h)
+          if (h == lane) {
+            mk = m_run[h];
+            lk = l_tot[h];
+          }
+        lm[h0 + lane] = lk;
+        lm[16 + h0 + lane] = mk;
       }
-    }
-    if (wq == 0 && lane < kHpw && h0 + lane < G && (p.lse != nullptr || p.part_lse != nullptr)) {
-      float mk = 0.f, lk = 0.f;
-#pragma unroll
-      for (int h = 0; h < kHpw; ++h)
-        if (h == lane) {
-          mk = m_run[h];
-          lk = l_tot[h];
-        }
-      const float lv = lk > 0.f ? (mk + lg2(lk)) * 0.69314718055994531f : -INFINITY;
-      if (p.part_lse != nullptr)
-        p.part_lse[(row0 + h0 + lane) * p.splits + un.s] = lv;
-      else
-        p.lse[un.t * p.lse_st + static_cast<int64_t>(un.g) * G + h0 + lane] = lv;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(sy.bar(G_LFULL + lb));
     }
     c_tile += un.n_tiles;
     ++c_unit;
+  }
+}
+
+// Epilogue warp w (16..19, TMEM lane quadrant w & 3: thread = dim of an
+// output half): for every unit, l and m from the softmax warps, O from TMEM
+// once the unit's last PV is done (the O buffer then goes back to the PV
+// issuer), then o = (O_hi + O_lo / 16) * v_scale / l as BF16 rows (or the
+// normalised partial output of a split-K chunk) and lse.
+__device__ void epilogue8(const TcParams& p, const Sync& sy, uint8_t* sp, uint32_t tmem, int warp, int lane) {
+  const int wq = warp & 3;
+  const int key = wq * 32 + lane;
+  const uint32_t tl = tmem + (static_cast<uint32_t>(wq * 32) << 16);
+  uint32_t c_unit = 0;
+  const int64_t units = num_units(p);
+  const int G = p.G;
+  bool ok = true;
+  for (int64_t u = blockIdx.x; u < units && ok; u += gridDim.x) {
+    const Unit un = decode_unit(p, u);
+    const uint32_t ub = c_unit & 1u, par = (c_unit >> 1) & 1u;
+    ++c_unit;
+    ok = sy.wait_warp(G_LFULL + ub, par);
+    if (!ok) break;
+    const float* lm = reinterpret_cast<const float*>(sp + F_LM) + ub * 32;
+    const int64_t row0 = un.t * static_cast<int64_t>(p.Hkv) * G + static_cast<int64_t>(un.g) * G;
+    if (wq == 0 && lane < G && (p.lse != nullptr || p.part_lse != nullptr)) {
+      const float lk = lm[lane], mk = lm[16 + lane];
+      const float lv = lk > 0.f ? (mk + lg2(lk)) * 0.69314718055994531f : -INFINITY;
+      if (p.part_lse != nullptr)
+        p.part_lse[(row0 + lane) * p.splits + un.s] = lv;
+      else
+        p.lse[un.t * p.lse_st + static_cast<int64_t>(un.g) * G + lane] = lv;
+    }
+    float inv[kGp];
+#pragma unroll
+    for (int h = 0; h < kGp; ++h) inv[h] = lm[h] > 0.f ? p.o_scale / lm[h] : 0.f;
+    __syncwarp();
+    if (lane == 0) mbar_arrive(sy.bar(G_LEMPTY + ub));
+    ok = sy.wait_warp(G_OFULL2 + ub, par);
+    if (!ok) break;
+    tc_fence_after();
+    __nv_bfloat16* orow = p.out + un.t * p.o_st + static_cast<int64_t>(un.g) * G * p.o_sh;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {                   // O columns: half (q >> 1), heads 8 (q & 1) ..
+      uint32_t o[16] = {};                          // hi of 8 heads, then lo of the same 8
+      if (un.n_tiles > 0) {
+        tmem_ld16(tl + kTO + ub * 64 + q * 16, o);
+        tmem_wait_ld();
+      }
+      if (q == 3) {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(sy.bar(G_OEMPTY2 + ub));
+      }
+      const int dim = (q >> 1) * 128 + key;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int h = (q & 1) * 8 + j;
+        if (h < G) {
+          const float v = inv[h] != 0.f ? fmaf(__uint_as_float(o[8 + j]), 0.0625f, __uint_as_float(o[j])) * inv[h] : 0.f;
+          if (p.part_o != nullptr)
+            p.part_o[((row0 + h) * p.splits + un.s) * 256 + dim] = v;
+          else
+            orow[h * p.o_sh + dim] = __float2bfloat16_rn(v);
+        }
+      }
+    }
   }
 }
 
@@ -630,8 +685,12 @@ __global__ void __launch_bounds__(kThreads8, 1) qsa_prefill_f8_kernel(const __gr
       mbar_init(sy.bar(G_RSUM + b), kSmWarps);
     }
     mbar_init(sy.bar(G_RMX2), kSmWarps);
-    mbar_init(sy.bar(G_OFULL), 1);
-    mbar_init(sy.bar(G_OEMPTY), kSmWarps);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(sy.bar(G_OFULL2 + b), 1);
+      mbar_init(sy.bar(G_OEMPTY2 + b), 4);          // the epilogue warps
+      mbar_init(sy.bar(G_LFULL + b), 2);            // the quadrant-0 softmax warps
+      mbar_init(sy.bar(G_LEMPTY + b), 4);
+    }
     mbar_init(sy.bar(G_DONE), 1);
     mbar_init(sy.bar(G_DONE + 1), 1);
     *sy.abort_flag = 0u;
@@ -647,17 +706,25 @@ __global__ void __launch_bounds__(kThreads8, 1) qsa_prefill_f8_kernel(const __gr
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(sp + F_MISC);
 
   if (warp < kProducerWarps8) {
+    setmaxnreg_dec<kRegsProd8>();
     producer8<kBlocks, kDump>(p, sy, sb, warp, lane);
-  } else if (warp == kWarpQ8) {
-    q8(p, sy, sb, sp, lane);
-  } else if (warp == kWarpQK8) {
-    if (lane == 0) qk8(p, sy, sb, tmem);
-    __syncwarp();
-  } else if (warp == kWarpPV8) {
-    if (lane == 0) pv8(p, sy, sb, tmem);
-    __syncwarp();
-  } else {
+  } else if (warp < kWarpSm8) {
+    setmaxnreg_dec<kRegsMisc8>();
+    if (warp == kWarpQ8) {
+      q8(p, sy, sb, sp, lane);
+    } else if (warp == kWarpQK8) {
+      if (lane == 0) qk8(p, sy, sb, tmem);
+      __syncwarp();
+    } else if (warp == kWarpPV8) {
+      if (lane == 0) pv8(p, sy, sb, tmem);
+      __syncwarp();
+    }
+  } else if (warp < kWarpEpi8) {
+    setmaxnreg_inc<kRegsSm8>();
     softmax8<kBlocks>(p, sy, sb, sp, tmem, warp, lane);
+  } else {
+    setmaxnreg_dec<kRegsEpi8>();
+    epilogue8(p, sy, sp, tmem, warp, lane);
   }
 
   tc_fence_before();
