@@ -767,13 +767,70 @@ def run_decode_bench(name, dev, barrier, reduce_max, world, hbm, steps=50, warmu
     _, per8, _ = time_launches(step8, steps, warmup, barrier, "decode_fp8")
     ms8 = statistics.mean(per8)
     algo8 = acct["algo_bytes"] - acct["gathered_bytes"] // 2 + need
+    del k8, v8
+    small = run_decode_small_batch(dev)
     return {"workload": w.name, "desc": w.description, "splits": splits,
             "workspace_bytes": need, "tokens_per_s": w.shape["T"] * steps * world / (total_ms / 1e3),
             "mean_step_ms": ms, "gathered_kv_gbs": acct["gathered_bytes"] / (ms / 1e3) / 1e9,
             "algo_gbs": algo / (ms / 1e3) / 1e9, "frac_of_hbm": algo / (ms / 1e3) / 1e9 / hbm,
             "launches_per_step": 2 if need > 0 else 1, "steps": steps,
             "fp8": {"mean_step_ms": ms8, "tokens_per_s": w.shape["T"] * world / (ms8 / 1e3),
-                    "algo_gbs": algo8 / (ms8 / 1e3) / 1e9, "frac_of_hbm": algo8 / (ms8 / 1e3) / 1e9 / hbm}}
+                    "algo_gbs": algo8 / (ms8 / 1e3) / 1e9, "frac_of_hbm": algo8 / (ms8 / 1e3) / 1e9 / hbm},
+            "small_batch": small}
+
+
+def graph_call_us(fn, calls=20, replays=5):
+    """Device time of one call, from CUDA-graph replays of `calls` calls (a
+    call of a few microseconds is otherwise timed together with the host's
+    launch overhead)."""
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        for _ in range(3):
+            fn()
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for _ in range(calls):
+            fn()
+    g.replay()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(replays):
+        g.replay()
+    b.record()
+    torch.cuda.synchronize()
+    del g
+    return a.elapsed_time(b) * 1e3 / (calls * replays)
+
+
+def run_decode_small_batch(dev, B=16):
+    """Decode with few (token, KV head) units: 16 sequences x 32 K context,
+    heads (24,2), K = 2048 (32 units on the SMs).  The automatic chunk count
+    against a single chunk, BF16 and FP8 caches, CUDA-graph timed."""
+    from top_sparse_attention_qsa_b200 import _capi
+    from top_sparse_attention_qsa_b200 import workloads as W
+    w = W.config_decode(device=dev, B=B)
+    gen = torch.Generator(device=dev).manual_seed(79)
+    k8 = W.normal_fp8(tuple(w.k_cache.shape), gen, dev)
+    v8 = W.normal_fp8(tuple(w.v_cache.shape), gen, dev)
+    out = torch.empty_like(w.q)
+    lse = torch.empty(w.q.shape[:2], dtype=torch.float32, device=dev)
+    auto = _capi.decode_num_splits(w.q, w.k_cache, w.topk_idx, 0)
+    res = {"workload": w.name, "units": w.shape["T"] * w.shape["Hkv"], "auto_splits": auto}
+    for splits, key in ((0, "auto"), (1, "one_chunk")):
+        need = _capi.decode_workspace_bytes(w.q, w.k_cache, w.topk_idx, splits, out, lse)
+        ws = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+        res[key + "_us"] = graph_call_us(
+            lambda: _capi.sparse_decode_fwd(w.q, w.k_cache, w.v_cache, w.topk_idx, w.n_valid, w.scale,
+                                            num_splits=splits, workspace=ws, out=out, lse=lse))
+        res[key + "_fp8_us"] = graph_call_us(
+            lambda: _capi.sparse_decode_fp8_fwd(w.q, k8, v8, w.topk_idx, 0.5, 2.0, n_valid=w.n_valid,
+                                                scale=w.scale, num_splits=splits, workspace=ws, out=out,
+                                                lse=lse))
+    return res
 
 
 def run_blocks_bench(name, dev, barrier, reduce_max, world, hbm, steps=20, warmup=3, **kw):

@@ -238,9 +238,10 @@ qsa_status_t qsa_sparse_prefill_fp8_fwd(const qsa_shape_t* shape,
  * encaja esto en el despliegue del servicio de Qwen4Exp", vLLM #59279).
  * Same operation, arguments and conventions as qsa_sparse_prefill_fwd, plus:
  *   num_splits      : chunks per list (never shorter than 128 entries); <= 0
- *                     picks one chunk unless the (token, KV head) units are
- *                     fewer than SMs / 8, then about one unit per SM with
- *                     chunks of at least 256 entries.
+ *                     picks floor(SMs / units) chunks for the (token, KV
+ *                     head) units (one wave over the SMs; one chunk once
+ *                     the units exceed half the SMs), with chunks of at
+ *                     least 256 entries.
  *   workspace       : caller-owned device scratch, 256-byte aligned, of at
  *                     least qsa_sparse_decode_workspace_bytes(shape,
  *                     num_splits) bytes (FP32 partial outputs and lse).  It

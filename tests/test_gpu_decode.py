@@ -54,6 +54,21 @@ def test_decode_few_units_auto_splits():
     check(C, w, "decode_auto")
 
 
+@pytest.mark.parametrize("units", [1, 8, 16, 32, 48, 64, 74, 75, 96, 128, 300])
+def test_decode_auto_splits_fill_one_wave(C, units):
+    """The automatic chunk count: floor(SMs / units) chunks (all chunks in one
+    wave of one CTA per SM), never chunks under 256 entries, one chunk once
+    the units exceed half the SMs.  Shapes only: nothing is launched."""
+    nsm = torch.cuda.get_device_properties(0).multi_processor_count
+    K = 2048
+    q = torch.empty((units, 2, 256), dtype=torch.bfloat16, device=DEV)
+    k = torch.empty((16, 1, 256), dtype=torch.bfloat16, device=DEV)
+    idx = torch.empty((units, 1, K), dtype=torch.int32, device=DEV)
+    want = min(nsm // units, K // 256) if 2 * units <= nsm else 1
+    assert C.decode_num_splits(q, k, idx, 0) == max(want, 1)
+    assert C.decode_num_splits(q, k, idx, 4) == 4
+
+
 @pytest.mark.parametrize("splits", [0, 1, 2, 3, 7, 16, 100])
 def test_decode_splits(C, splits):
     w = W.config_decode(device=DEV, B=6, ctx=4096, heads=(12, 1), topk=2051, local=64)
