@@ -87,21 +87,10 @@ struct IxParams {
   int32_t NB, H, tpt, bs, n_chunks;
 };
 
-// Candidate blocks [lo, hi) of token t: the complete causal microblocks of
-// its sequence (integer division truncating like C, clamped to [0, NB]).
-__device__ __forceinline__ void candidates(const int32_t* positions, const int32_t* seq_start,
-                                           int32_t NB, int32_t bs, int64_t t, int& lo, int& hi) {
-  int64_t l = static_cast<int64_t>(__ldg(seq_start + t)) / bs;
-  int64_t h = (static_cast<int64_t>(__ldg(positions + t)) + 1) / bs;
-  if (l < 0) l = 0;
-  if (h > NB) h = NB;
-  if (h < l) h = l;
-  lo = static_cast<int>(l);
-  hi = static_cast<int>(h);
-}
-
-// The same range from a token's position and sequence start.
-// Non-negative inputs take 32-bit unsigned divisions (pos + 1 <= 2^31).
+// Candidate blocks [lo, hi) of a token from its position and sequence
+// start: the complete causal microblocks of its sequence (integer division
+// truncating like C, clamped to [0, NB]).  Non-negative inputs take 32-bit
+// unsigned divisions (pos + 1 <= 2^31).
 __device__ __forceinline__ void range_of(int32_t pos, int32_t s0, int32_t NB, int32_t bs, int& lo, int& hi) {
   int64_t l, h;
   if ((pos | s0) >= 0) {
@@ -136,16 +125,40 @@ struct IxUnit {
 // Unit u (token tile outer, chunk of block tiles inner) as seen by one warp:
 // every lane returns the same tile range; with `lo_s` set, the candidate range
 // of each of the tile's tokens is written there (tokens past T: empty).
+// Every role calls this at each unit start, so it is kept short: a lane
+// loads the positions and sequence starts of all its tokens (at most
+// kRows / 32) before any arithmetic, paying one global-memory latency per
+// unit, and the divisions are 32-bit wherever the values allow.
 __device__ IxUnit ix_unit(const IxParams& p, int64_t u, int lane, int* lo_s, int* hi_s) {
+  constexpr int kIt = kRows / 32;                  // tokens per lane at most (tpt <= kRows)
   IxUnit r;
-  const int64_t tt = u / p.n_chunks;
-  const int c = static_cast<int>(u - tt * p.n_chunks);
+  int64_t tt;
+  int c;
+  if (u <= 0xffffffffLL) {
+    const uint32_t uu = static_cast<uint32_t>(u), nc = static_cast<uint32_t>(p.n_chunks);
+    const uint32_t q = uu / nc;
+    tt = q;
+    c = static_cast<int>(uu - q * nc);
+  } else {
+    tt = u / p.n_chunks;
+    c = static_cast<int>(u - tt * p.n_chunks);
+  }
   r.tok0 = tt * p.tpt;
+  int32_t pos[kIt], s0[kIt];
+#pragma unroll
+  for (int k = 0; k < kIt; ++k) {
+    const int i = lane + 32 * k;
+    const bool in = i < p.tpt && r.tok0 + i < p.T;
+    pos[k] = in ? __ldg(p.positions + r.tok0 + i) : 0;
+    s0[k] = in ? __ldg(p.seq_start + r.tok0 + i) : 0;
+  }
   int mn = INT_MAX, mx = -1, flo = 0, fhi = INT_MAX;
-  for (int i = lane; i < p.tpt; i += 32) {
-    const int64_t t = r.tok0 + i;
+#pragma unroll
+  for (int k = 0; k < kIt; ++k) {
+    const int i = lane + 32 * k;
+    if (i >= p.tpt) break;
     int lo = 0, hi = 0;
-    if (t < p.T) candidates(p.positions, p.seq_start, p.NB, p.bs, t, lo, hi);
+    if (r.tok0 + i < p.T) range_of(pos[k], s0[k], p.NB, p.bs, lo, hi);
     if (lo_s != nullptr) {
       lo_s[i] = lo;
       hi_s[i] = hi;

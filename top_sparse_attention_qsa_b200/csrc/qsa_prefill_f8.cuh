@@ -644,7 +644,8 @@ __device__ void epilogue8(const TcParams& p, const Sync& sy, uint8_t* sp, uint32
       for (int j = 0; j < 8; ++j) {
         const int h = (q & 1) * 8 + j;
         if (h < G) {
-          const float v = inv[h] != 0.f ? fmaf(__uint_as_float(o[8 + j]), 0.0625f, __uint_as_float(o[j])) * inv[h] : 0.f;
+          const float oh = fmaf(__uint_as_float(o[8 + j]), 0.0625f, __uint_as_float(o[j]));
+          const float v = inv[h] != 0.f ? oh * inv[h] : 0.f;
           if (p.part_o != nullptr)
             p.part_o[((row0 + h) * p.splits + un.s) * 256 + dim] = v;
           else
