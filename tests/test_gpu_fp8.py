@@ -71,6 +71,27 @@ def test_masks_empty_rows_and_out_of_range(C):
     assert st["empty_rows"] >= 16
 
 
+def test_runs_of_empty_units(C):
+    """Ten units per CTA (one KV head: unit = token, CTA b takes tokens b,
+    b + SMs, ...), the rounds alternating full, empty (runs of three), short
+    and one-key units, so that the two O buffers and the hand-off of l and m
+    to the epilogue warps wrap their barrier phases on empty units too."""
+    nsm = torch.cuda.get_device_properties(0).multi_processor_count
+    pattern = [256, 0, 0, 0, 200, 0, 1, 256, 0, 130]
+    T = nsm * len(pattern)
+    w, k8, v8 = fp8_case(T=T, S=4096, heads=(16, 1), K=256, seed=23)
+    nv = torch.tensor([pattern[t // nsm] for t in range(T)], dtype=torch.int32, device=DEV)
+    w.n_valid = nv.reshape(T, 1).contiguous()
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    out, lse = C.sparse_prefill_fp8_fwd(w.q, k8, v8, w.topk_idx, 0.75, 1.5, n_valid=w.n_valid,
+                                        scale=w.scale, status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    ref_out, ref_lse, _ = oracle_fp8(w, k8, v8, 0.75, 1.5)
+    st = compare(host(out), host(lse), ref_out, ref_lse, "fp8 empty-unit runs")
+    assert st["empty_rows"] >= 16 * nsm * pattern.count(0)
+
+
 def test_block_lists_with_tail(C):
     T, S, bs = 25, 4001, 4
     w, k8, v8 = fp8_case(T=T, S=S, heads=(24, 2), K=1, seed=11)
